@@ -1,0 +1,245 @@
+/*
+ * foursight.h — C ABI of the SpliceGEMM hot path for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow FourSight (arXiv 2611.04887, "FourSight: Stable FP4 RL
+ * Post-Training via Sequence Filtering and Sparse Channel Compensation"):
+ *   - a W4A4 NVFP4 linear layer Y = X W^T in which a small protected set S of
+ *     input channels (64 by default) stays in BF16 (§4.2 Eq. 5, §5.1);
+ *   - running channel moments and per-step top-s reselection (§5.2);
+ *   - the TIM-aware dual-gate sequence filter with advantage masking (§4.1 Eq. 3-4).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument is a DEVICE pointer owned by the caller unless its
+ *   comment says "host".  The library never keeps a pointer past the call.
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream).  Apart from fs_plan_create, fs_plan_destroy, fs_plan_check and
+ *   fs_stats_check, no call allocates, frees or synchronises, so a sequence of
+ *   calls can be captured into a CUDA graph.
+ * - Argument errors are found on the host before anything is launched and are
+ *   returned as FS_ERR_INVALID_ARGUMENT (bad pointer, size, alignment) or
+ *   FS_ERR_UNSUPPORTED (a legal shape this build has no kernel for); nothing
+ *   is written in that case.  A launch failure returns FS_ERR_CUDA.
+ *   fs_last_error() gives a readable detail string for the calling thread.
+ * - Conditions only the device can see are recorded in a caller-visible word and
+ *   reported by the *_check calls: FS_ERR_RANGE (a statistics input out of range)
+ *   and FS_ERR_TIMEOUT (a bounded wait inside a kernel gave up; the kernel
+ *   returned early and its output is undefined).
+ * - dtype codes: FS_DTYPE_BF16 (row-major bf16), FS_DTYPE_F32 (row-major fp32).
+ * - Leading dimensions (ldx, ldw, ldy) are in elements and must make every row
+ *   start on a 16-byte boundary; base pointers must be 16-byte aligned (256-byte
+ *   for the packed operands of fs_splice_gemm, which are read by TMA).
+ *
+ * Packed NVFP4 operand layout (written by fs_quantize_splice / fs_prepare_weights,
+ * read by fs_splice_gemm):
+ *   q    [R][K/2] bytes: E2M1 codes, two per byte, the even-K element in the low
+ *        nibble; protected lanes hold code 0.
+ *   sf   UE4M3 block scales (one per 16 elements along K) in the MMA-ready tiled
+ *        layout: 512-byte atoms of 128 rows x 4 blocks, atoms running first along K
+ *        then along rows; inside an atom row r sits at byte (r%32)*16 + ((r%128)/32)*4
+ *        and its 4 blocks are consecutive bytes.  Size: roundup(R,128) * roundup(K/16,4)
+ *        bytes; padding bytes are written as 0.
+ *   side [R][Pp] bf16 with Pp = roundup(p,16): the protected columns in ascending
+ *        channel order (X_S for activations, W'_S = BF16(W_S/alpha) for weights),
+ *        columns p..Pp-1 zero.
+ * fs_side_cols(p) returns Pp; fs_sf_bytes(R, K) returns the sf size.
+ */
+#ifndef FOURSIGHT_H
+#define FOURSIGHT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fs_status {
+  FS_OK = 0,
+  FS_ERR_INVALID_ARGUMENT = 1,
+  FS_ERR_UNSUPPORTED = 2,
+  FS_ERR_CUDA = 3,
+  FS_ERR_RANGE = 4,
+  FS_ERR_TIMEOUT = 5
+} fs_status;
+
+enum { FS_DTYPE_BF16 = 0, FS_DTYPE_F32 = 1 };
+
+/* Option bits (the `opts` arguments). */
+enum {
+  FS_RESIDUAL = 1u << 0,   /* residual-correction form: block scales and gains are taken with the
+                              protected lanes present, then only their codes are zeroed (the
+                              "auxiliary residual" prior art FourSight contrasts with, §1, §7.1) */
+  FS_KEY_M2 = 1u << 1,     /* select by second moment E[x^2] instead of variance (§9.3 Prop. 2) */
+  FS_GAIN_EXACT = 1u << 2, /* encode gain fl32(2688/amax) instead of the power-of-two gain */
+  FS_OUT_BF16 = 1u << 3    /* fs_splice_gemm writes bf16 Y instead of fp32 */
+};
+
+/* Readable name of a status code (static storage). */
+const char* fs_status_string(fs_status s);
+/* Detail of the last non-FS_OK status returned on the calling host thread ("" if none). */
+const char* fs_last_error(void);
+/* Library version string (static storage). */
+const char* fs_version(void);
+
+/* Pp = roundup(p, 16): the column count of the packed side buffers. */
+int32_t fs_side_cols(int32_t p);
+/* Bytes of the tiled scale array for R rows and K channels. */
+int64_t fs_sf_bytes(int64_t R, int32_t K);
+
+/* ------------------------------------------------------------------------------------------
+ * Running channel moments — FourSight §5.2 "System Implementation": a forward hook uniformly
+ * subsamples token rows, before masking, and accumulates running channel moments in a GPU buffer.
+ *
+ * Adds rows 0, row_stride, 2*row_stride, ... of X [M][K] (row-major, leading dimension ldx,
+ * dtype FS_DTYPE_BF16 or FS_DTYPE_F32) to the state of ONE input group:
+ *   n     [1] int64   += number of rows taken
+ *   s1    [K] int64   += sum rint(x * 2^16)          (exact integer fixed point)
+ *   s2    [K] int64   += sum rint(x^2 * 2^14)        (x^2 formed exactly)
+ *   amax  [K] uint32  = bits of max(|x|) as float32
+ *   flags [1] uint32  |= 1 if some |x| >= 2^16 or x is not finite (read by fs_stats_check)
+ * Integer sums make the state independent of the reduction order.  The state must be
+ * zeroed before the first call (e.g. cudaMemsetAsync or fs_select_topk with reset=1).
+ * Requirements: K % 8 == 0, M >= 0, row_stride >= 1; the state must hold fewer than 2^17
+ * rows of values near the range limit for s2 not to overflow.
+ * ---------------------------------------------------------------------------------------- */
+fs_status fs_channel_stats(const void* X, int32_t dtype, int64_t M, int32_t K, int64_t ldx,
+                           int32_t row_stride, int64_t* n, int64_t* s1, int64_t* s2,
+                           uint32_t* amax, uint32_t* flags, void* stream);
+
+/* Synchronises `stream` and returns FS_ERR_RANGE if any of the nprob flag words is non-zero. */
+fs_status fs_stats_check(const uint32_t* flags, int32_t nprob, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Protected-channel reselection — FourSight §5.2: after each optimizer step the protected set is
+ * reselected as the top-s channels by the variance gathered in the previous step; §9.3 Prop. 2 /
+ * Cor. 1 for the key; §6.1 for s = 64.
+ *
+ * Batched over nprob problems that share K; state arrays are stacked: n [nprob], s1/s2/amax
+ * [nprob][K], flags [nprob].  For each problem:
+ *   key_j = m2 - m1*m1 (or m2 with FS_KEY_M2), m1 = s1/65536/n, m2 = s2/16384/n in float64
+ *           (key 0 when n == 0);
+ *   P     [nprob][p] int32: the p channels with the largest key (ties: lower index first),
+ *         written in ascending channel order;
+ *   mask  [nprob][ceil(K/32)] uint32: bit j%32 of word j/32 set for every j in P;
+ *   gA    [nprob] float: next-step activation encode gain from max amax over channels not in P
+ *         (over all channels with FS_RESIDUAL): the largest power of two g with amax*g <= 2688
+ *         (exponent clamped to [-126,127]; 1 when amax == 0), or fl32(2688/amax) with FS_GAIN_EXACT.
+ * reset != 0 zeroes the state after it has been read (start of the next window).
+ * Requirements: 0 <= p <= K <= 16384, p <= 256.  Runs one CTA per problem.
+ * ---------------------------------------------------------------------------------------- */
+fs_status fs_select_topk(int32_t nprob, int32_t K, int64_t* n, int64_t* s1, int64_t* s2,
+                         uint32_t* amax, uint32_t* flags, int32_t p, uint32_t opts,
+                         int32_t* P, uint32_t* mask, float* gA, int32_t reset, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Weight pre-split — FourSight §5.1 "Data preparation": after each policy update W is split into
+ * an NVFP4 pack of W_{~S} and a pre-scaled BF16 pack W'_S = BF16(W_S / alpha) (Eq. 5), fixed for
+ * one rollout step.
+ *
+ * W [N][K] (leading dimension ldw, dtype bf16 or fp32); mask as written by fs_select_topk
+ * (ceil(K/32) words; may be NULL when p == 0); gA: device float, the activation gain of this
+ * projection's input.  Writes
+ *   wq  [N][K/2], sfw (tiled, fs_sf_bytes(N,K)), ws [N][Pp] bf16 (the packed layout above);
+ *   gW  [1] float: the weight encode gain from max |W| over unprotected columns (all columns with
+ *       FS_RESIDUAL), same rule as gA;
+ *   alpha [1] float: fl32(1 / fl32(gA*gW)).
+ * Protected lanes are zeroed before the block scales are computed (split form) unless
+ * FS_RESIDUAL.  Block quantisation: t = fl32(fl32(a_b*g)/6), sf = UE4M3 round-to-nearest-even
+ * (saturating at 448), v = fl32(fl32(w*g)/sf), code = E2M1 round-to-nearest-even (saturating at
+ * 6, sign kept; sf == 0 gives code 0 with the sign of w).
+ * Requirements: K % 64 == 0, 0 <= p <= min(K, 256), N >= 1.
+ * ---------------------------------------------------------------------------------------- */
+fs_status fs_prepare_weights(const void* W, int32_t dtype, int32_t N, int32_t K, int64_t ldw,
+                             const uint32_t* mask, int32_t p, uint32_t opts, const float* gA,
+                             uint8_t* wq, uint8_t* sfw, uint16_t* ws, float* gW, float* alpha,
+                             void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Activation preparation — FourSight §5.1 "Data preparation": one pass over X that zeroes the
+ * protected lanes with a register bitmask (Mask S->0), quantises the rest to NVFP4 (FP4 Quant)
+ * and copies the protected columns to a compact BF16 side buffer X_S (Extract X_S).
+ *
+ * X [M][K] (ldx, bf16 or fp32); mask/p as for fs_prepare_weights; gA: device float (frozen gain).
+ * Writes xq [M][K/2], sfx (tiled, fs_sf_bytes(M,K)), xs [M][Pp] bf16 (bf16 of X_S, rounded to
+ * nearest even for fp32 input).  Same block rule as fs_prepare_weights.
+ * Requirements: K % 64 == 0, M >= 0, 0 <= p <= min(K, 256).
+ * ---------------------------------------------------------------------------------------- */
+fs_status fs_quantize_splice(const void* X, int32_t dtype, int64_t M, int32_t K, int64_t ldx,
+                             const uint32_t* mask, int32_t p, const float* gA, uint32_t opts,
+                             uint8_t* xq, uint8_t* sfx, uint16_t* xs, void* stream);
+
+/* Grouped (mixture-of-experts) form: E experts, expert e owning rows
+ * [row_offsets[e], row_offsets[e+1]) of X (row_offsets: device int64 [E+1], row_offsets[0] == 0,
+ * non-decreasing, row_offsets[E] <= max_rows).  Each expert has its own mask [E][ceil(K/32)] and
+ * gain gA [E]; all share p.  Expert e's packed rows start at the padded offset
+ * pad_e = sum_{e'<e} roundup(rows_e', 128) in xq [.][K/2], sfx and xs [.][Pp]; size the buffers
+ * with fs_grouped_rows(max_rows, E) rows.  Rows of the padding are zero. */
+fs_status fs_quantize_splice_grouped(const void* X, int32_t dtype, int32_t E, const int64_t* row_offsets,
+                                     int64_t max_rows, int32_t K, int64_t ldx, const uint32_t* masks,
+                                     int32_t p, const float* gA, uint32_t opts, uint8_t* xq,
+                                     uint8_t* sfx, uint16_t* xs, void* stream);
+/* Upper bound of the padded row count for max_rows routed rows over E experts. */
+int64_t fs_grouped_rows(int64_t max_rows, int32_t E);
+
+/* ------------------------------------------------------------------------------------------
+ * SpliceGEMM — FourSight §4.2 Eq. 5 and §5.1 "Dual-path execution":
+ *   Y = alpha * ( sum_k (q sf)_x (q sf)_w  +  X_S W'_S^T )
+ * the NVFP4 product over all K lanes (protected lanes hold code 0) and the BF16 product over the
+ * protected slice accumulated into the same FP32 accumulator, scaled once by alpha.
+ *
+ * A plan caches the kernel choice for one weight shape (N, K, p_max) and owns a device error
+ * word; creating it is the only call that allocates.  fs_plan_check synchronises `stream` and
+ * returns FS_ERR_TIMEOUT if a kernel launched with the plan gave up a bounded wait (the word is
+ * then cleared).  A plan may be used from one stream at a time.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct fs_plan_s* fs_plan;
+fs_status fs_plan_create(fs_plan* out, int32_t N, int32_t K, int32_t p_max, uint32_t opts);
+fs_status fs_plan_destroy(fs_plan plan);
+fs_status fs_plan_check(fs_plan plan, void* stream);
+
+/* Packed operands as written above (activation rows M; weight rows N = the plan's N), p <= the
+ * plan's p_max; alpha: device float.  Y [M][ldy] fp32 (bf16 with FS_OUT_BF16 in the plan's
+ * opts), ldy >= N.  M <= 16 runs the weight-streaming decode kernel, larger M the tcgen05
+ * tensor-core kernel.  Requirements: K % 256 == 0 or K % 64 == 0 with the decode path
+ * (FS_ERR_UNSUPPORTED otherwise), N % 16 == 0, 256-byte aligned q/sf/side pointers. */
+fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, const uint8_t* sfx,
+                         const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
+                         const float* alpha, void* Y, int64_t ldy, void* stream);
+
+/* Grouped SpliceGEMM over E experts (the mixture-of-experts projections).  Activations are the
+ * padded-row outputs of fs_quantize_splice_grouped (row_offsets as given there); expert e's
+ * weights are rows [e*N, (e+1)*N) of stacked wq [E*N][K/2], sfw (tiled over E*N rows) and
+ * ws [E*N][Pp]; alpha [E].  Y [row_offsets[E]][ldy] in the original (unpadded) row order. */
+fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64_t* row_offsets, int64_t max_rows,
+                                 int32_t p, const uint8_t* xq, const uint8_t* sfx, const uint16_t* xs,
+                                 const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
+                                 const float* alpha, void* Y, int64_t ldy, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * TIM-aware sequence filter — FourSight §4.1 "The dual-gate mechanism" and Eq. 3-4; §2.1 for the
+ * group advantage; §6.1 for tau = 1e-4, K1 = 0.01 x output_len, K2 = 5.
+ *
+ * logp [S][ld] fp32 train-engine log-probs; lengths [S] int32 (NULL: every sequence has T tokens;
+ * positions >= length are ignored).  A token is a tail token when logp <= log_tau or logp is NaN
+ * (log_tau = fl32(ln tau), formed by the caller).  Per sequence:
+ *   tail_count [S] int32, max_run [S] int32 (longest run of consecutive tail tokens),
+ *   keep [S] uint8 = (tail_count < K1 && max_run < K2).
+ * Advantages (optional):
+ *   rewards != NULL: adv [S] is written with keep ? (r - mu)/sigma : 0, mu and population sigma
+ *     over each group of G consecutive sequences (all of them, dropped ones included), float64
+ *     sequential sums rounded to float32, sigma == 0 giving 0; S % G == 0 is required;
+ *   rewards == NULL and adv != NULL: adv is masked in place (adv = keep ? adv : 0).
+ * The loss denominator stays G: nothing is renormalised by the number of kept sequences.
+ * Requirements: S >= 0, T >= 0, ld >= T, K1 >= 1, K2 >= 1, logp 4-byte aligned (rows are read with
+ * 16-byte loads when logp is 16-byte aligned and ld % 4 == 0).
+ * ---------------------------------------------------------------------------------------- */
+fs_status fs_seq_filter(const float* logp, int64_t ld, const int32_t* lengths, int32_t S, int32_t T,
+                        float log_tau, int32_t K1, int32_t K2, int32_t G, const float* rewards,
+                        float* adv, uint8_t* keep, int32_t* tail_count, int32_t* max_run, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FOURSIGHT_H */

@@ -1,0 +1,128 @@
+// Shared host/device helpers of the SpliceGEMM library (sm_100a).
+//
+// Host side: status/last-error bookkeeping and argument checks.
+// Device side: the NVFP4 block-quantiser arithmetic of FourSight §9.3.1 Eq. 9 and §5.1
+// "Data preparation", written so that every rounding decision matches the IEEE fp32
+// operation order the library documents (t = fl32(fl32(a_b*g)/6), v = fl32(fl32(x*g)/sf)).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+#include <algorithm>
+
+#include "../../include/foursight.h"
+
+namespace fs {
+
+// ------------------------------------------------------------------------------------------
+// Host: status handling
+// ------------------------------------------------------------------------------------------
+void set_last_error(const char* fmt, ...);
+fs_status fail(fs_status s, const char* fmt, ...);
+fs_status cuda_status(cudaError_t e, const char* what);
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+inline int side_cols(int p) { return (p + 15) / 16 * 16; }
+inline int64_t sf_bytes(int64_t rows, int K) { return round_up(rows, 128) * round_up(K / 16, 4); }
+
+#define FS_CHECK_LAUNCH(what)                                         \
+  do {                                                                \
+    cudaError_t e_ = cudaGetLastError();                              \
+    if (e_ != cudaSuccess) return ::fs::cuda_status(e_, what);        \
+  } while (0)
+
+// Device error words written by kernels whose bounded waits gave up.
+enum : uint32_t { ERR_NONE = 0, ERR_TIMEOUT = 1 };
+
+// ------------------------------------------------------------------------------------------
+// Device: small numeric helpers
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Round-to-nearest-even float -> bf16 bits.
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
+  __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// UE4M3 code of a finite t >= 0: round to nearest, ties to the even code, saturating at 448.
+// Subnormals are multiples of 2^-9 below 2^-6; normals carry 3 mantissa bits, exponent bias 7.
+__device__ __forceinline__ uint32_t ue4m3_rne(float t) {
+  if (t >= 448.0f) return 0x7Eu;
+  if (t < 0.015625f) return static_cast<uint32_t>(__float2int_rn(t * 512.0f));  // 0..8 (8 == 2^-6)
+  uint32_t b = __float_as_uint(t);
+  b += 0x7FFFFu + ((b >> 20) & 1u);            // round the 23-bit fraction to 3 bits, ties to even
+  const uint32_t c = (((b >> 23) - 120u) << 3) | ((b >> 20) & 7u);
+  return c > 0x7Eu ? 0x7Eu : c;
+}
+
+// Value of a UE4M3 code (0x00..0x7E).
+__device__ __forceinline__ float ue4m3_value(uint32_t c) {
+  const uint32_t e = c >> 3, m = c & 7u;
+  if (e == 0) return static_cast<float>(m) * 0.001953125f;                       // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));                        // (1+m/8) 2^(e-7)
+}
+
+// Exact quotient rounding for divisors with at most 4 significant bits.
+//
+// For q = y / d with y an fp32 value and d = o * 2^k (o odd, o <= 15), RN32(q) equals
+// RN32(RN64(y * RN64(1/d))).  Reason: the float64 product is within 2^-52 |q| of q, while q
+// either is exactly an fp32 value or lies at least 2^-28 |q| away from every fp32 rounding
+// midpoint (y has 24 significant bits, so y - M*d, for an fp32 midpoint M with 25 bits, is a
+// non-zero multiple of M's last unit unless y/d == M, which would need y to span more than
+// 24 bits).  The fp64 error therefore never moves the result across a rounding boundary.
+// Both block-scale steps divide by such a d: 6 = 3*2 and any UE4M3 value.
+__device__ __forceinline__ float div_small_divisor(float y, double inv_d) {
+  return __double2float_rn(__dmul_rn(static_cast<double>(y), inv_d));
+}
+constexpr double kInvSix = 1.0 / 6.0;   // RN64(1/6): compile-time IEEE division
+
+// Packs two fp32 values into one byte of E2M1 codes (round to nearest even, saturating at 6),
+// `lo` into the low nibble.  The PTX conversion places its first source in the high nibble.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Power-of-two encode gain: largest g = 2^E with amax*g <= 2688 = 0.65625*2^12, E clamped to
+// [-126,127]; 1 for amax == 0 or non-finite.  With amax = f*2^e, f in [0.5,1): E = 12-e when
+// f <= 0.65625, else 11-e.
+__device__ __forceinline__ float gain_pow2(float amax) {
+  if (!(amax > 0.0f) || !isfinite(amax)) return 1.0f;
+  uint32_t b = __float_as_uint(amax);
+  int bias = 0;
+  if ((b >> 23) == 0) {                         // subnormal: scale by 2^64 first (exact)
+    b = __float_as_uint(amax * 18446744073709551616.0f);
+    bias = 64;
+  }
+  const int e = static_cast<int>(b >> 23) - 126 - bias;     // amax = f * 2^e, f in [0.5, 1)
+  const uint32_t frac = b & 0x7FFFFFu;                       // f = (1 + frac/2^23) / 2
+  int E = (frac <= 0x280000u) ? 12 - e : 11 - e;             // f <= 0.65625 <=> frac <= 0.3125*2^23
+  E = E < -126 ? -126 : (E > 127 ? 127 : E);
+  return __uint_as_float(static_cast<uint32_t>(E + 127) << 23);
+}
+
+__device__ __forceinline__ float gain_exact(float amax) {
+  if (!(amax > 0.0f) || !isfinite(amax)) return 1.0f;
+  return __fdiv_rn(2688.0f, amax);
+}
+
+// Byte offset of (row r, 16-block b) in the tiled scale array; kb4 = roundup(K/16,4)/4.
+__device__ __host__ __forceinline__ int64_t sf_offset(int64_t r, int b, int kb4) {
+  return ((r >> 7) * kb4 + (b >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (b & 3);
+}
+
+// Bounded spin limit shared by the kernels that wait on barriers (about a second at 2 GHz).
+constexpr uint32_t kSpinLimit = 1u << 28;
+
+}  // namespace fs

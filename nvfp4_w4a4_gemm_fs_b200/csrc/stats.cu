@@ -1,0 +1,358 @@
+// Running channel moments and top-s protected-channel reselection.
+//
+// FourSight §5.2 "System Implementation": a forward hook subsamples token rows before masking
+// and accumulates running channel moments in a GPU buffer; after each optimizer step the
+// protected set is reselected as the top-s channels by the variance of the previous step
+// (§9.3 Prop. 2 / Cor. 1 justify variance and second moment as the key; §6.1: s = 64).
+//
+// Moments are exact integers (s1 = sum rint(x 2^16), s2 = sum rint(x^2 2^14)), so every
+// reduction order gives the same state and the selection is reproducible bit for bit.
+#include "common.cuh"
+
+namespace fs {
+namespace {
+
+constexpr int kStatsWarps = 8;
+constexpr double kS1Scale = 65536.0;
+constexpr double kS2Scale = 16384.0;
+constexpr float kRangeLimit = 65536.0f;
+
+struct ChanAcc {
+  long long s1, s2;
+  float amax;
+  bool bad;
+};
+
+__device__ __forceinline__ void add_value(ChanAcc& a, float x, bool f32_input) {
+  const float ax = fabsf(x);
+  if (!(ax < kRangeLimit)) {     // also catches NaN
+    a.bad = true;
+    return;
+  }
+  a.amax = fmaxf(a.amax, ax);
+  a.s1 += __float2ll_rn(x * 65536.0f);               // exact scaling, round half even
+  if (f32_input) {
+    const double xd = static_cast<double>(x);
+    a.s2 += __double2ll_rn(__dmul_rn(__dmul_rn(xd, xd), kS2Scale));
+  } else {
+    a.s2 += __float2ll_rn(__fmul_rn(x, x) * 16384.0f);   // bf16 x: x^2 exact in fp32
+  }
+}
+
+// Grid: x = channel chunks (a warp-width of channels each), y = row groups.
+// Block: kStatsWarps warps; warp w takes rows (blockIdx.y*W + w) * stride + i*gridDim.y*W*stride.
+// Lane l holds VEC consecutive channels.  Per-CTA partial sums are reduced across warps in
+// shared memory and added to the global state with integer atomics.
+template <typename T, int VEC>
+__global__ void __launch_bounds__(kStatsWarps * 32)
+channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int row_stride,
+                     unsigned long long* n, unsigned long long* s1, unsigned long long* s2,
+                     uint32_t* amax, uint32_t* flags) {
+  constexpr bool kF32 = sizeof(T) == 4;
+  __shared__ long long sh_s1[kStatsWarps][32 * VEC];
+  __shared__ long long sh_s2[kStatsWarps][32 * VEC];
+  __shared__ float sh_am[kStatsWarps][32 * VEC];
+  __shared__ int sh_bad;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c0 = blockIdx.x * 32 * VEC + lane * VEC;
+  const bool active = c0 < K;
+  if (threadIdx.x == 0) sh_bad = 0;
+
+  ChanAcc acc[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) acc[v] = ChanAcc{0, 0, 0.0f, false};
+
+  const int64_t taken = (M + row_stride - 1) / row_stride;     // rows 0, s, 2s, ...
+  const int64_t step = static_cast<int64_t>(gridDim.y) * kStatsWarps;
+  if (active) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.y) * kStatsWarps + warp; i < taken; i += step) {
+      const T* row = X + i * row_stride * ldx + c0;
+      if constexpr (kF32) {
+        const float4 q = __ldg(reinterpret_cast<const float4*>(row));
+        add_value(acc[0], q.x, true); add_value(acc[1], q.y, true);
+        add_value(acc[2], q.z, true); add_value(acc[3], q.w, true);
+      } else {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(row));
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          add_value(acc[2 * j], bf16_lo(w[j]), false);
+          add_value(acc[2 * j + 1], bf16_hi(w[j]), false);
+        }
+      }
+    }
+  }
+  bool bad = false;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    sh_s1[warp][lane * VEC + v] = acc[v].s1;
+    sh_s2[warp][lane * VEC + v] = acc[v].s2;
+    sh_am[warp][lane * VEC + v] = acc[v].amax;
+    bad |= acc[v].bad;
+  }
+  if (bad) atomicOr(&sh_bad, 1);
+  __syncthreads();
+  for (int c = threadIdx.x; c < 32 * VEC; c += blockDim.x) {
+    const int ch = blockIdx.x * 32 * VEC + c;
+    if (ch >= K) continue;
+    long long a = 0, b = 0;
+    float m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kStatsWarps; ++w) {
+      a += sh_s1[w][c];
+      b += sh_s2[w][c];
+      m = fmaxf(m, sh_am[w][c]);
+    }
+    if (a) atomicAdd(s1 + ch, static_cast<unsigned long long>(a));    // two's complement wraps
+    if (b) atomicAdd(s2 + ch, static_cast<unsigned long long>(b));
+    if (m > 0.0f) atomicMax(amax + ch, __float_as_uint(m));             // non-negative floats order as uints
+  }
+  if (threadIdx.x == 0) {
+    if (sh_bad) atomicOr(flags, 1u);
+    if (blockIdx.x == 0 && blockIdx.y == 0) atomicAdd(n, static_cast<unsigned long long>(taken));
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Reselection: one CTA per problem.
+// ------------------------------------------------------------------------------------------
+constexpr int kSelThreads = 1024;
+constexpr int kMaxK = 16384;
+
+// Map a double key to an unsigned integer with the same order (-0 folded onto +0 first).
+__device__ __forceinline__ unsigned long long order_bits(double k) {
+  if (k == 0.0) k = 0.0;
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(k));
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ double channel_key(long long n, long long s1, long long s2, bool m2_only) {
+  if (n == 0) return 0.0;
+  const double dn = __ll2double_rn(n);
+  const double m2 = __ddiv_rn(__ll2double_rn(s2) / kS2Scale, dn);   // /2^14 exact
+  if (m2_only) return m2;
+  const double m1 = __ddiv_rn(__ll2double_rn(s1) / kS1Scale, dn);   // /2^16 exact
+  return __dsub_rn(m2, __dmul_rn(m1, m1));
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_topk_kernel(int K, long long* n_all, long long* s1_all, long long* s2_all, uint32_t* amax_all,
+                   uint32_t* flags_all, int p, uint32_t opts, int32_t* P_all, uint32_t* mask_all,
+                   float* gA_all, int reset) {
+  extern __shared__ unsigned long long sh_keys[];         // [K]
+  __shared__ unsigned int hist[256];
+  __shared__ unsigned long long sh_prefix;
+  __shared__ int sh_need;
+  __shared__ int sh_scan[kSelThreads / 32];
+  __shared__ uint32_t sh_amax[kSelThreads / 32];
+
+  const int prob = blockIdx.x;
+  const long long n = n_all[prob];
+  const long long* s1 = s1_all + static_cast<int64_t>(prob) * K;
+  const long long* s2 = s2_all + static_cast<int64_t>(prob) * K;
+  const uint32_t* amax = amax_all + static_cast<int64_t>(prob) * K;
+  int32_t* P = P_all + static_cast<int64_t>(prob) * p;
+  const int words = (K + 31) / 32;
+  uint32_t* mask = mask_all + static_cast<int64_t>(prob) * words;
+  const bool m2_only = opts & FS_KEY_M2;
+  const int tid = threadIdx.x;
+
+  for (int j = tid; j < K; j += blockDim.x) sh_keys[j] = order_bits(channel_key(n, s1[j], s2[j], m2_only));
+  if (tid == 0) { sh_prefix = 0; sh_need = p; }
+  __syncthreads();
+
+  // Radix select of the p-th largest ordered key, 8 bits at a time from the top.
+  unsigned long long prefix = 0;
+  int need = p;
+  if (p > 0) {
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+      __syncthreads();
+      const unsigned long long hi_mask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
+      for (int j = tid; j < K; j += blockDim.x) {
+        const unsigned long long k = sh_keys[j];
+        if ((k & hi_mask) == prefix) atomicAdd(&hist[(k >> shift) & 0xFF], 1u);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int rem = need;
+        int d = 255;
+        for (; d > 0; --d) {
+          if (static_cast<int>(hist[d]) >= rem) break;
+          rem -= hist[d];
+        }
+        sh_prefix = prefix | (static_cast<unsigned long long>(d) << shift);
+        sh_need = rem;
+      }
+      __syncthreads();
+      prefix = sh_prefix;
+      need = sh_need;
+      __syncthreads();
+    }
+  }
+  // Selected: key > T, plus the `need` lowest-index channels with key == T (T = prefix).
+  // Channels are visited in index order, chunk per thread, with block-wide exclusive scans.
+  const int per = (K + blockDim.x - 1) / blockDim.x;
+  const int j0 = tid * per, j1 = min(K, j0 + per);
+  int n_gt = 0, n_eq = 0;
+  if (p > 0) {
+    for (int j = j0; j < j1; ++j) {
+      n_gt += sh_keys[j] > prefix;
+      n_eq += sh_keys[j] == prefix;
+    }
+  }
+  // exclusive scan of n_eq over threads (to rank ties by index)
+  auto block_exclusive_scan = [&](int v) -> int {
+    const int lane = tid & 31, warp = tid >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) sh_scan[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int s = (lane < (int)(blockDim.x >> 5)) ? sh_scan[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      if (lane < (int)(blockDim.x >> 5)) sh_scan[lane] = s;
+    }
+    __syncthreads();
+    const int excl = x - v + (warp > 0 ? sh_scan[warp - 1] : 0);
+    __syncthreads();
+    return excl;
+  };
+  const int eq_before = block_exclusive_scan(n_eq);
+  // count selected in this chunk
+  int n_sel = 0;
+  if (p > 0) {
+    int eq_seen = eq_before;
+    for (int j = j0; j < j1; ++j) {
+      const unsigned long long k = sh_keys[j];
+      if (k > prefix || (k == prefix && eq_seen++ < need)) ++n_sel;
+    }
+  }
+  const int sel_before = block_exclusive_scan(n_sel);
+  // write P (ascending) and the mask; unselected amax feed the gain
+  float am_unprot = 0.0f;
+  {
+    int eq_seen = eq_before, out = sel_before;
+    for (int j = j0; j < j1; ++j) {
+      const unsigned long long k = sh_keys[j];
+      const bool sel = p > 0 && (k > prefix || (k == prefix && eq_seen++ < need));
+      if (sel) P[out++] = j;
+      const float a = __uint_as_float(amax[j]);
+      if (!sel || (opts & FS_RESIDUAL)) am_unprot = fmaxf(am_unprot, a);
+      sh_keys[j] = sel ? 1ull : 0ull;       // reuse as the selection flag
+    }
+  }
+  __syncthreads();
+  for (int w = tid; w < words; w += blockDim.x) {
+    uint32_t bits = 0;
+    for (int b = 0; b < 32; ++b) {
+      const int j = w * 32 + b;
+      if (j < K && sh_keys[j]) bits |= 1u << b;
+    }
+    mask[w] = bits;
+  }
+  // block max of the unprotected amax
+  uint32_t am = __float_as_uint(am_unprot);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if ((tid & 31) == 0) sh_amax[tid >> 5] = am;
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t m = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = max(m, sh_amax[w]);
+    const float a = __uint_as_float(m);
+    gA_all[prob] = (opts & FS_GAIN_EXACT) ? gain_exact(a) : gain_pow2(a);
+  }
+  if (reset) {
+    __syncthreads();
+    for (int j = tid; j < K; j += blockDim.x) {
+      s1_all[static_cast<int64_t>(prob) * K + j] = 0;
+      s2_all[static_cast<int64_t>(prob) * K + j] = 0;
+      amax_all[static_cast<int64_t>(prob) * K + j] = 0;
+    }
+    if (tid == 0) { n_all[prob] = 0; flags_all[prob] = 0; }
+  }
+}
+
+}  // namespace
+}  // namespace fs
+
+using namespace fs;
+
+extern "C" fs_status fs_channel_stats(const void* X, int32_t dtype, int64_t M, int32_t K, int64_t ldx,
+                                      int32_t row_stride, int64_t* n, int64_t* s1, int64_t* s2,
+                                      uint32_t* amax, uint32_t* flags, void* stream) {
+  if (M < 0 || K <= 0 || K % 8 != 0) return fail(FS_ERR_INVALID_ARGUMENT, "fs_channel_stats: need M >= 0, K > 0, K %% 8 == 0 (M=%lld K=%d)", (long long)M, K);
+  if (row_stride < 1) return fail(FS_ERR_INVALID_ARGUMENT, "fs_channel_stats: row_stride must be >= 1");
+  if (dtype != FS_DTYPE_BF16 && dtype != FS_DTYPE_F32) return fail(FS_ERR_INVALID_ARGUMENT, "fs_channel_stats: bad dtype %d", dtype);
+  if (!n || !s1 || !s2 || !amax || !flags || (M > 0 && !X)) return fail(FS_ERR_INVALID_ARGUMENT, "fs_channel_stats: null pointer");
+  const int esz = dtype == FS_DTYPE_BF16 ? 2 : 4;
+  if (ldx < K || (ldx * esz) % 16 != 0 || !aligned(X, 16)) return fail(FS_ERR_INVALID_ARGUMENT, "fs_channel_stats: X rows must be 16-byte aligned and ldx >= K");
+  if (!aligned(s1, 8) || !aligned(s2, 8) || !aligned(n, 8) || !aligned(amax, 4) || !aligned(flags, 4)) return fail(FS_ERR_INVALID_ARGUMENT, "fs_channel_stats: misaligned state");
+  if (M == 0) return FS_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int vec = dtype == FS_DTYPE_BF16 ? 8 : 4;
+  const int chunks = static_cast<int>(ceil_div(K, 32 * vec));
+  const int64_t taken = ceil_div(M, row_stride);
+  // Enough CTAs for ~4 per SM, each reading at least 64 rows.
+  int64_t gy = ceil_div(148 * 4, chunks);
+  gy = std::min<int64_t>(gy, std::max<int64_t>(1, ceil_div(taken, 64)));
+  gy = std::min<int64_t>(gy, 65535);
+  dim3 grid(chunks, static_cast<unsigned>(gy));
+  auto* un = reinterpret_cast<unsigned long long*>(n);
+  auto* u1 = reinterpret_cast<unsigned long long*>(s1);
+  auto* u2 = reinterpret_cast<unsigned long long*>(s2);
+  if (dtype == FS_DTYPE_BF16)
+    channel_stats_kernel<uint16_t, 8><<<grid, kStatsWarps * 32, 0, s>>>(static_cast<const uint16_t*>(X), M, K, ldx, row_stride, un, u1, u2, amax, flags);
+  else
+    channel_stats_kernel<float, 4><<<grid, kStatsWarps * 32, 0, s>>>(static_cast<const float*>(X), M, K, ldx, row_stride, un, u1, u2, amax, flags);
+  FS_CHECK_LAUNCH("fs_channel_stats");
+  return FS_OK;
+}
+
+extern "C" fs_status fs_stats_check(const uint32_t* flags, int32_t nprob, void* stream) {
+  if (nprob < 0 || (nprob > 0 && !flags)) return fail(FS_ERR_INVALID_ARGUMENT, "fs_stats_check: bad arguments");
+  if (nprob == 0) return FS_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t host[64];
+  for (int32_t i0 = 0; i0 < nprob; i0 += 64) {
+    const int cnt = std::min(64, nprob - i0);
+    cudaError_t e = cudaMemcpyAsync(host, flags + i0, cnt * sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_status(e, "fs_stats_check");
+    for (int i = 0; i < cnt; ++i)
+      if (host[i]) return fail(FS_ERR_RANGE, "statistics input out of range (|x| >= 2^16 or not finite) in problem %d", i0 + i);
+  }
+  return FS_OK;
+}
+
+extern "C" fs_status fs_select_topk(int32_t nprob, int32_t K, int64_t* n, int64_t* s1, int64_t* s2,
+                                    uint32_t* amax, uint32_t* flags, int32_t p, uint32_t opts,
+                                    int32_t* P, uint32_t* mask, float* gA, int32_t reset, void* stream) {
+  if (nprob < 0 || K <= 0 || K > kMaxK) return fail(FS_ERR_INVALID_ARGUMENT, "fs_select_topk: need 0 < K <= %d", kMaxK);
+  if (p < 0 || p > K || p > 256) return fail(FS_ERR_INVALID_ARGUMENT, "fs_select_topk: need 0 <= p <= min(K, 256)");
+  if (nprob == 0) return FS_OK;
+  if (!n || !s1 || !s2 || !amax || !flags || !mask || !gA || (p > 0 && !P)) return fail(FS_ERR_INVALID_ARGUMENT, "fs_select_topk: null pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t smem = static_cast<size_t>(K) * sizeof(unsigned long long);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxK * 8);
+    if (e != cudaSuccess) return cuda_status(e, "fs_select_topk: smem attribute");
+    attr_set = true;
+  }
+  select_topk_kernel<<<nprob, kSelThreads, smem, s>>>(K, reinterpret_cast<long long*>(n), reinterpret_cast<long long*>(s1),
+                                                     reinterpret_cast<long long*>(s2), amax, flags, p, opts,
+                                                     P, mask, gA, reset);
+  FS_CHECK_LAUNCH("fs_select_topk");
+  return FS_OK;
+}

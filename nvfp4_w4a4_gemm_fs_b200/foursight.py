@@ -1,0 +1,210 @@
+"""Thin torch-tensor wrappers with the names of the C ABI (argument marshalling only).
+
+All tensors must already live on the current CUDA device; outputs are caller-allocated
+(helpers ``alloc_*`` allocate them with torch, outside any timed or captured region).
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import torch
+
+from . import _lib
+from ._lib import FS_DTYPE_BF16, FS_DTYPE_F32, check
+
+__all__ = [
+    "fs_channel_stats", "fs_stats_check", "fs_select_topk", "fs_prepare_weights",
+    "fs_quantize_splice", "fs_quantize_splice_grouped", "fs_splice_gemm", "fs_splice_gemm_grouped",
+    "fs_seq_filter", "Plan", "StatsState", "Packed", "side_cols", "sf_bytes", "grouped_rows",
+    "alloc_packed", "stream_handle",
+]
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def stream_handle(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FS_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return FS_DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def side_cols(p: int) -> int:
+    return _lib.load().fs_side_cols(p)
+
+
+def sf_bytes(rows: int, K: int) -> int:
+    return _lib.load().fs_sf_bytes(rows, K)
+
+
+def grouped_rows(max_rows: int, E: int) -> int:
+    return _lib.load().fs_grouped_rows(max_rows, E)
+
+
+class StatsState:
+    """Device state of fs_channel_stats for nprob input groups that share K."""
+
+    def __init__(self, nprob: int, K: int, device="cuda"):
+        self.nprob, self.K = nprob, K
+        self.n = torch.zeros(nprob, dtype=torch.int64, device=device)
+        self.s1 = torch.zeros(nprob, K, dtype=torch.int64, device=device)
+        self.s2 = torch.zeros(nprob, K, dtype=torch.int64, device=device)
+        self.amax = torch.zeros(nprob, K, dtype=torch.int32, device=device)
+        self.flags = torch.zeros(nprob, dtype=torch.int32, device=device)
+
+    def group(self, i: int):
+        return self.n[i:i + 1], self.s1[i], self.s2[i], self.amax[i], self.flags[i:i + 1]
+
+
+class Packed:
+    """Packed NVFP4 operand: q [R,K/2] u8, sf (tiled) u8, side [R,Pp] bf16."""
+
+    def __init__(self, q, sf, side, rows, K, p):
+        self.q, self.sf, self.side, self.rows, self.K, self.p = q, sf, side, rows, K, p
+
+
+def alloc_packed(rows: int, K: int, p: int, device="cuda") -> Packed:
+    pp = side_cols(p)
+    q = torch.empty(max(rows, 1), K // 2, dtype=torch.uint8, device=device)
+    sf = torch.empty(sf_bytes(rows, K), dtype=torch.uint8, device=device)
+    side = torch.empty(max(rows, 1), max(pp, 8), dtype=torch.bfloat16, device=device)[:, :pp]
+    return Packed(q, sf, side if pp else side, rows, K, p)
+
+
+def fs_channel_stats(X: torch.Tensor, state: StatsState, group: int = 0, row_stride: int = 1, stream=None):
+    lib = _lib.load()
+    n, s1, s2, amax, flags = state.group(group)
+    M, K = X.shape
+    check(lib.fs_channel_stats(_ptr(X), _dtype_code(X), M, K, X.stride(0), row_stride, _ptr(n), _ptr(s1),
+                               _ptr(s2), _ptr(amax), _ptr(flags), stream_handle(stream)), "fs_channel_stats")
+
+
+def fs_stats_check(state: StatsState, stream=None):
+    check(_lib.load().fs_stats_check(_ptr(state.flags), state.nprob, stream_handle(stream)), "fs_stats_check")
+
+
+def fs_select_topk(state: StatsState, p: int, opts: int = 0, reset: bool = False, P=None, mask=None, gA=None,
+                   stream=None):
+    lib = _lib.load()
+    dev = state.s1.device
+    nprob, K = state.nprob, state.K
+    P = torch.empty(nprob, max(p, 1), dtype=torch.int32, device=dev)[:, :p] if P is None else P
+    mask = torch.empty(nprob, (K + 31) // 32, dtype=torch.int32, device=dev) if mask is None else mask
+    gA = torch.empty(nprob, dtype=torch.float32, device=dev) if gA is None else gA
+    check(lib.fs_select_topk(nprob, K, _ptr(state.n), _ptr(state.s1), _ptr(state.s2), _ptr(state.amax),
+                             _ptr(state.flags), p, opts, _ptr(P), _ptr(mask), _ptr(gA), int(reset),
+                             stream_handle(stream)), "fs_select_topk")
+    return P, mask, gA
+
+
+def fs_prepare_weights(W: torch.Tensor, mask, p: int, gA: torch.Tensor, opts: int = 0, out: Packed | None = None,
+                       gW=None, alpha=None, stream=None):
+    lib = _lib.load()
+    N, K = W.shape
+    out = alloc_packed(N, K, p, W.device) if out is None else out
+    gW = torch.empty(1, dtype=torch.float32, device=W.device) if gW is None else gW
+    alpha = torch.empty(1, dtype=torch.float32, device=W.device) if alpha is None else alpha
+    check(lib.fs_prepare_weights(_ptr(W), _dtype_code(W), N, K, W.stride(0), _ptr(mask) if p else None, p, opts,
+                                 _ptr(gA), _ptr(out.q), _ptr(out.sf), _ptr(out.side) if p else None, _ptr(gW),
+                                 _ptr(alpha), stream_handle(stream)), "fs_prepare_weights")
+    return out, gW, alpha
+
+
+def fs_quantize_splice(X: torch.Tensor, mask, p: int, gA: torch.Tensor, opts: int = 0, out: Packed | None = None,
+                       stream=None):
+    lib = _lib.load()
+    M, K = X.shape
+    out = alloc_packed(M, K, p, X.device) if out is None else out
+    check(lib.fs_quantize_splice(_ptr(X), _dtype_code(X), M, K, X.stride(0), _ptr(mask) if p else None, p,
+                                 _ptr(gA), opts, _ptr(out.q), _ptr(out.sf), _ptr(out.side) if p else None,
+                                 stream_handle(stream)), "fs_quantize_splice")
+    return out
+
+
+def fs_quantize_splice_grouped(X: torch.Tensor, row_offsets: torch.Tensor, masks, p: int, gA: torch.Tensor,
+                               opts: int = 0, out: Packed | None = None, max_rows: int | None = None, stream=None):
+    lib = _lib.load()
+    rows, K = X.shape
+    E = row_offsets.numel() - 1
+    max_rows = rows if max_rows is None else max_rows
+    out = alloc_packed(grouped_rows(max_rows, E), K, p, X.device) if out is None else out
+    check(lib.fs_quantize_splice_grouped(_ptr(X), _dtype_code(X), E, _ptr(row_offsets), max_rows, K, X.stride(0),
+                                         _ptr(masks) if p else None, p, _ptr(gA), opts, _ptr(out.q), _ptr(out.sf),
+                                         _ptr(out.side) if p else None, stream_handle(stream)),
+          "fs_quantize_splice_grouped")
+    return out
+
+
+class Plan:
+    """Owns an fs_plan (kernel choice for one weight shape plus a device error word)."""
+
+    def __init__(self, N: int, K: int, p_max: int, opts: int = 0):
+        self._lib = _lib.load()
+        h = C.c_void_p()
+        check(self._lib.fs_plan_create(C.byref(h), N, K, p_max, opts), "fs_plan_create")
+        self.handle, self.N, self.K, self.p_max, self.opts = h, N, K, p_max, opts
+
+    def check(self, stream=None):
+        check(self._lib.fs_plan_check(self.handle, stream_handle(stream)), "fs_plan_check")
+
+    def close(self):
+        if self.handle:
+            self._lib.fs_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def fs_splice_gemm(plan: Plan, xq: Packed, wq: Packed, alpha: torch.Tensor, Y: torch.Tensor | None = None,
+                   stream=None):
+    lib = _lib.load()
+    M = xq.rows
+    if Y is None:
+        dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
+        Y = torch.empty(M, plan.N, dtype=dt, device=xq.q.device)
+    check(lib.fs_splice_gemm(plan.handle, M, xq.p, _ptr(xq.q), _ptr(xq.sf), _ptr(xq.side) if xq.p else None,
+                             _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, _ptr(alpha), _ptr(Y),
+                             Y.stride(0), stream_handle(stream)), "fs_splice_gemm")
+    return Y
+
+
+def fs_splice_gemm_grouped(plan: Plan, row_offsets: torch.Tensor, max_rows: int, xq: Packed, wq: Packed,
+                           alpha: torch.Tensor, Y: torch.Tensor | None = None, stream=None):
+    lib = _lib.load()
+    E = row_offsets.numel() - 1
+    if Y is None:
+        dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
+        Y = torch.empty(max_rows, plan.N, dtype=dt, device=xq.q.device)
+    check(lib.fs_splice_gemm_grouped(plan.handle, E, _ptr(row_offsets), max_rows, xq.p, _ptr(xq.q), _ptr(xq.sf),
+                                     _ptr(xq.side) if xq.p else None, _ptr(wq.q), _ptr(wq.sf),
+                                     _ptr(wq.side) if wq.p else None, _ptr(alpha), _ptr(Y), Y.stride(0),
+                                     stream_handle(stream)), "fs_splice_gemm_grouped")
+    return Y
+
+
+def fs_seq_filter(logp: torch.Tensor, log_tau: float, K1: int, K2: int, lengths=None, G: int = 0, rewards=None,
+                  adv=None, stream=None):
+    lib = _lib.load()
+    S, T = logp.shape
+    dev = logp.device
+    keep = torch.empty(max(S, 1), dtype=torch.uint8, device=dev)[:S]
+    cnt = torch.empty(max(S, 1), dtype=torch.int32, device=dev)[:S]
+    run = torch.empty(max(S, 1), dtype=torch.int32, device=dev)[:S]
+    if rewards is not None and adv is None:
+        adv = torch.empty(S, dtype=torch.float32, device=dev)
+    check(lib.fs_seq_filter(_ptr(logp), logp.stride(0), _ptr(lengths), S, T, float(log_tau), K1, K2, G,
+                            _ptr(rewards), _ptr(adv), _ptr(keep), _ptr(cnt), _ptr(run), stream_handle(stream)),
+          "fs_seq_filter")
+    return keep, cnt, run, adv

@@ -49,10 +49,13 @@ def test_variance_key_matches_population_variance():
 
 
 def test_range_flag():
-    x = np.zeros((2, 16), np.float32); x[1, 3] = 70000.0
-    assert stats.accumulate(stats.new_state(16), x)["flags"] == 1
+    x = np.zeros((2, 16), np.float32); x[1, 3] = 70000.0; x[0, 3] = 2.0
+    st = stats.accumulate(stats.new_state(16), x)
+    assert st["flags"] == 1 and st["s1"][3] == 2 * 65536 and st["amax"][3] == 2.0
     x[1, 3] = np.inf
     assert stats.accumulate(stats.new_state(16), x)["flags"] == 1
+    x[1, 3] = 65535.0
+    assert stats.accumulate(stats.new_state(16), x)["flags"] == 0
 
 
 def test_topk_order_and_ties():
