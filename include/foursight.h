@@ -72,7 +72,9 @@ enum {
                               "auxiliary residual" prior art FourSight contrasts with, §1, §7.1) */
   FS_KEY_M2 = 1u << 1,     /* select by second moment E[x^2] instead of variance (§9.3 Prop. 2) */
   FS_GAIN_EXACT = 1u << 2, /* encode gain fl32(2688/amax) instead of the power-of-two gain */
-  FS_OUT_BF16 = 1u << 3    /* fs_splice_gemm writes bf16 Y instead of fp32 */
+  FS_OUT_BF16 = 1u << 3,   /* fs_splice_gemm writes bf16 Y instead of fp32 */
+  FS_PATH_TENSOR = 1u << 4, /* plan option: always use the tcgen05 tensor-core kernel */
+  FS_PATH_DECODE = 1u << 5  /* plan option: always use the weight-streaming decode kernel (M <= 16) */
 };
 
 /* Readable name of a status code (static storage). */
@@ -200,9 +202,10 @@ fs_status fs_plan_check(fs_plan plan, void* stream);
 
 /* Packed operands as written above (activation rows M; weight rows N = the plan's N), p <= the
  * plan's p_max; alpha: device float.  Y [M][ldy] fp32 (bf16 with FS_OUT_BF16 in the plan's
- * opts), ldy >= N.  M <= 16 runs the weight-streaming decode kernel, larger M the tcgen05
- * tensor-core kernel.  Requirements: K % 256 == 0 or K % 64 == 0 with the decode path
- * (FS_ERR_UNSUPPORTED otherwise), N % 16 == 0, 256-byte aligned q/sf/side pointers. */
+ * opts), ldy >= N, 16-byte aligned rows.  M <= 16 runs the weight-streaming decode kernel, larger
+ * M the tcgen05 tensor-core kernel (FS_PATH_TENSOR / FS_PATH_DECODE in the plan's opts force one).
+ * Plan requirements: N % 16 == 0 and K % 256 == 0 (FS_ERR_UNSUPPORTED otherwise); the packed
+ * operands must be 16-byte aligned.  The output is not accumulated into: Y is overwritten. */
 fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, const uint8_t* sfx,
                          const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
                          const float* alpha, void* Y, int64_t ldy, void* stream);
@@ -210,7 +213,8 @@ fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, 
 /* Grouped SpliceGEMM over E experts (the mixture-of-experts projections).  Activations are the
  * padded-row outputs of fs_quantize_splice_grouped (row_offsets as given there); expert e's
  * weights are rows [e*N, (e+1)*N) of stacked wq [E*N][K/2], sfw (tiled over E*N rows) and
- * ws [E*N][Pp]; alpha [E].  Y [row_offsets[E]][ldy] in the original (unpadded) row order. */
+ * ws [E*N][Pp]; alpha [E].  Y [row_offsets[E]][ldy] in the original (unpadded) row order.
+ * Always runs the tensor-core kernel; needs N % 128 == 0 and E <= 256. */
 fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64_t* row_offsets, int64_t max_rows,
                                  int32_t p, const uint8_t* xq, const uint8_t* sfx, const uint16_t* xs,
                                  const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,

@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(HERE, "libfoursight.so")
 
 FS_OK, FS_ERR_INVALID_ARGUMENT, FS_ERR_UNSUPPORTED, FS_ERR_CUDA, FS_ERR_RANGE, FS_ERR_TIMEOUT = range(6)
 FS_DTYPE_BF16, FS_DTYPE_F32 = 0, 1
-FS_RESIDUAL, FS_KEY_M2, FS_GAIN_EXACT, FS_OUT_BF16 = 1, 2, 4, 8
+FS_RESIDUAL, FS_KEY_M2, FS_GAIN_EXACT, FS_OUT_BF16, FS_PATH_TENSOR, FS_PATH_DECODE = 1, 2, 4, 8, 16, 32
 
 P = C.c_void_p
 i32, i64, u32, f32 = C.c_int32, C.c_int64, C.c_uint32, C.c_float

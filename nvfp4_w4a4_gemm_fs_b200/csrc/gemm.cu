@@ -1,0 +1,132 @@
+// SpliceGEMM plans and entry points: argument checks and dispatch between the tensor-core path
+// (large M, FourSight §5.1 "High-throughput prefill path") and the weight-streaming decode path
+// (M <= 16, the small-M regime of §5.1 "Low-latency decode path").
+#include "common.cuh"
+#include "gemm.cuh"
+
+struct fs_plan_s {
+  int32_t N, K, p_max;
+  uint32_t opts;
+  uint32_t* err;      // device error word (bounded-wait timeouts)
+  int device;
+};
+
+using namespace fs;
+
+namespace {
+
+constexpr uint32_t kPathMask = FS_PATH_TENSOR | FS_PATH_DECODE;
+
+fs_status check_operands(const char* who, const fs_plan_s* pl, int32_t p, const uint8_t* xq, const uint8_t* sfx,
+                         const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
+                         const float* alpha, const void* Y, int64_t ldy) {
+  if (!pl) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null plan", who);
+  if (p < 0 || p > pl->p_max) return fail(FS_ERR_INVALID_ARGUMENT, "%s: p=%d outside [0, p_max=%d]", who, p, pl->p_max);
+  if (!xq || !sfx || !wq || !sfw || !alpha || !Y || (p > 0 && (!xs || !ws)))
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: null pointer", who);
+  if (!aligned(xq, 16) || !aligned(sfx, 16) || !aligned(wq, 16) || !aligned(sfw, 16) ||
+      (p > 0 && (!aligned(xs, 16) || !aligned(ws, 16))))
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: packed operands must be 16-byte aligned", who);
+  const bool bf16 = pl->opts & FS_OUT_BF16;
+  if (ldy < pl->N || !aligned(Y, 16) || (ldy % (bf16 ? 8 : 4)) != 0)
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: Y must be 16-byte aligned with ldy >= N and 16-byte rows", who);
+  return FS_OK;
+}
+
+}  // namespace
+
+extern "C" fs_status fs_plan_create(fs_plan* out, int32_t N, int32_t K, int32_t p_max, uint32_t opts) {
+  if (!out) return fail(FS_ERR_INVALID_ARGUMENT, "fs_plan_create: null out");
+  *out = nullptr;
+  if (N < 16 || N % 16 != 0) return fail(FS_ERR_INVALID_ARGUMENT, "fs_plan_create: need N >= 16 and N %% 16 == 0 (N=%d)", N);
+  if (K < 256 || K % 256 != 0 || K > 65536) return fail(FS_ERR_UNSUPPORTED, "fs_plan_create: need K %% 256 == 0, 256 <= K <= 65536 (K=%d)", K);
+  if (p_max < 0 || p_max > 256 || p_max > K) return fail(FS_ERR_INVALID_ARGUMENT, "fs_plan_create: need 0 <= p_max <= min(K, 256)");
+  if ((opts & kPathMask) == kPathMask) return fail(FS_ERR_INVALID_ARGUMENT, "fs_plan_create: FS_PATH_TENSOR and FS_PATH_DECODE are exclusive");
+  auto* pl = new fs_plan_s{N, K, p_max, opts, nullptr, 0};
+  cudaGetDevice(&pl->device);
+  cudaError_t e = cudaMalloc(&pl->err, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(pl->err, 0, sizeof(uint32_t));
+  if (e != cudaSuccess) {
+    if (pl->err) cudaFree(pl->err);
+    delete pl;
+    return cuda_status(e, "fs_plan_create");
+  }
+  *out = pl;
+  return FS_OK;
+}
+
+extern "C" fs_status fs_plan_destroy(fs_plan plan) {
+  if (!plan) return FS_OK;
+  cudaFree(plan->err);
+  delete plan;
+  return FS_OK;
+}
+
+extern "C" fs_status fs_plan_check(fs_plan plan, void* stream) {
+  if (!plan) return fail(FS_ERR_INVALID_ARGUMENT, "fs_plan_check: null plan");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t w = 0;
+  cudaError_t e = cudaMemcpyAsync(&w, plan->err, sizeof(w), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e, "fs_plan_check");
+  if (w) {
+    cudaMemsetAsync(plan->err, 0, sizeof(uint32_t), s);
+    cudaStreamSynchronize(s);
+    return fail(FS_ERR_TIMEOUT, "a SpliceGEMM kernel gave up a bounded wait (error word 0x%x)", w);
+  }
+  return FS_OK;
+}
+
+extern "C" fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, const uint8_t* sfx,
+                                    const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
+                                    const float* alpha, void* Y, int64_t ldy, void* stream) {
+  if (M < 0) return fail(FS_ERR_INVALID_ARGUMENT, "fs_splice_gemm: M < 0");
+  fs_status st = check_operands("fs_splice_gemm", plan, p, xq, sfx, xs, wq, sfw, ws, alpha, Y, ldy);
+  if (st != FS_OK) return st;
+  if (M == 0) return FS_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int pp = side_cols(p);
+  const bool decode = (plan->opts & FS_PATH_DECODE) || (!(plan->opts & FS_PATH_TENSOR) && M <= 16);
+  if (decode) {
+    if (M > 16) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm: the decode path takes M <= 16 (M=%lld)", (long long)M);
+    DecodeParams d{};
+    d.M = static_cast<int>(M); d.N = plan->N; d.K = plan->K; d.pp = pp;
+    d.kb4 = static_cast<int>(round_up(plan->K / 16, 4) / 4);
+    d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha;
+    d.Y = Y; d.ldy = ldy; d.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0;
+    return launch_splice_gemm_decode(d, s);
+  }
+  if (M > (int64_t{1} << 31) - 256) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm: M too large");
+  TcParams prm{};
+  prm.M = M; prm.N = plan->N; prm.K = plan->K; prm.KT = plan->K / 256; prm.ST = static_cast<int>(ceil_div(pp, 64));
+  prm.E = 1; prm.kb4 = plan->K / 64; prm.offsets = nullptr; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
+  prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
+  TcLaunch L{};
+  L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = M; L.b_rows = plan->N; L.pp = pp;
+  L.bn = (plan->N % 256 == 0) ? 256 : 128;
+  L.max_tiles = ceil_div(M, 128) * ceil_div(plan->N, L.bn);
+  return launch_splice_gemm_tc(L, prm, s);
+}
+
+extern "C" fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64_t* row_offsets, int64_t max_rows,
+                                            int32_t p, const uint8_t* xq, const uint8_t* sfx, const uint16_t* xs,
+                                            const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
+                                            const float* alpha, void* Y, int64_t ldy, void* stream) {
+  if (E <= 0 || !row_offsets || max_rows < 0) return fail(FS_ERR_INVALID_ARGUMENT, "fs_splice_gemm_grouped: need E > 0, row_offsets, max_rows >= 0");
+  fs_status st = check_operands("fs_splice_gemm_grouped", plan, p, xq, sfx, xs, wq, sfw, ws, alpha, Y, ldy);
+  if (st != FS_OK) return st;
+  if (plan->N % 128 != 0) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm_grouped: need N %% 128 == 0");
+  if (max_rows == 0) return FS_OK;
+  const int64_t a_rows = fs_grouped_rows(max_rows, E);
+  if (a_rows > (int64_t{1} << 31) - 256) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm_grouped: too many rows");
+  const int pp = side_cols(p);
+  TcParams prm{};
+  prm.M = 0; prm.N = plan->N; prm.K = plan->K; prm.KT = plan->K / 256; prm.ST = static_cast<int>(ceil_div(pp, 64));
+  prm.E = E; prm.kb4 = plan->K / 64; prm.offsets = row_offsets; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
+  prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
+  TcLaunch L{};
+  L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = a_rows; L.b_rows = static_cast<int64_t>(E) * plan->N; L.pp = pp;
+  L.bn = (plan->N % 256 == 0) ? 256 : 128;
+  L.max_tiles = ceil_div(a_rows, 128) * (plan->N / L.bn);
+  return launch_splice_gemm_tc(L, prm, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,52 @@
+// Internal launch interface shared by the SpliceGEMM kernels and the ABI layer.
+#pragma once
+#include "common.cuh"
+
+namespace fs {
+
+// Kernel parameters of the tensor-core path (plain: E = 1, offsets = null).
+struct TcParams {
+  int64_t M;
+  int N, K, KT, ST, BN, n_tiles, E, kb4;
+  const int64_t* offsets;
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* alpha;
+  void* Y;
+  int64_t ldy;
+  int out_bf16;
+  uint32_t* err;
+};
+
+// Host-side description of the operand buffers for tensor-map encoding.
+struct TcLaunch {
+  const void* xq;
+  const void* wq;
+  const void* xs;
+  const void* ws;
+  int64_t a_rows;     // rows of the activation buffers (padded rows for experts)
+  int64_t b_rows;     // rows of the weight buffers (E * N for experts)
+  int pp;
+  int bn;
+  int64_t max_tiles;
+};
+
+fs_status launch_splice_gemm_tc(const TcLaunch& L, const TcParams& prm, cudaStream_t s);
+
+struct DecodeParams {
+  int M, N, K, pp, kb4;
+  const uint8_t* xq;
+  const uint8_t* sfx;
+  const uint16_t* xs;
+  const uint8_t* wq;
+  const uint8_t* sfw;
+  const uint16_t* ws;
+  const float* alpha;
+  void* Y;
+  int64_t ldy;
+  int out_bf16;
+};
+
+fs_status launch_splice_gemm_decode(const DecodeParams& p, cudaStream_t s);
+
+}  // namespace fs

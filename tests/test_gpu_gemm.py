@@ -1,0 +1,128 @@
+"""GPU parity of fs_splice_gemm (both paths) against the oracle's Eq. 5 in float64.
+
+Tolerance (the stated bound): |Y - Y_ref| <= 1e-5 * sum_k |x_hat_k w_hat_k| per element, with the
+hats the oracle's dequantised operands; a bf16 output adds its own rounding, 2^-8 |Y_ref|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import nvfp4, splice, stats
+from tests._util import bf16_tensor, f32_tensor, mask_tensor
+
+pytestmark = pytest.mark.gpu
+
+F = pytest.importorskip("nvfp4_w4a4_gemm_fs_b200")
+
+REL = 1e-5
+
+
+def _problem(seed, M, N, K, p, dtype="bf16", residual=False, calib_rows=None):
+    bf = dtype == "bf16"
+    x, _ = synth.outlier_activations(seed, M, K, as_bf16=bf)
+    w = synth.gaussian_weights(seed + 1, N, K, as_bf16=bf)
+    X, W = splice.as_f32(x, bf), splice.as_f32(w, bf)
+    st = stats.accumulate(stats.new_state(K), X)
+    P = stats.select_topk(st, p)
+    gA = stats.next_gain(st, P, residual=residual)
+    Xt = bf16_tensor(x) if bf else f32_tensor(x)
+    Wt = bf16_tensor(w) if bf else f32_tensor(w)
+    return X, W, Xt, Wt, P, gA
+
+
+def _run_gpu(Xt, Wt, P, gA, p, N, K, opts=0, plan_opts=0):
+    mask = mask_tensor(stats.protect_mask(P, K))
+    g = torch.tensor([float(gA)], device="cuda")
+    wq, gW, alpha = F.fs_prepare_weights(Wt, mask, p, g, opts=opts)
+    xq = F.fs_quantize_splice(Xt, mask, p, g, opts=opts)
+    plan = F.Plan(N, K, max(p, 1), plan_opts)
+    Y = F.fs_splice_gemm(plan, xq, wq, alpha)
+    plan.check()
+    return Y, plan
+
+
+def _ref(X, W, P, gA, residual=False, rows=None):
+    mode = splice.RESIDUAL if residual else splice.SPLIT
+    xq = splice.quantize_splice(X if rows is None else X[rows], P, gA, mode)
+    wq = splice.prepare_weights(W, P, gA, mode)
+    return splice.splice_gemm(xq, wq, wq["alpha"])
+
+
+def _assert_close(Y, Yr, mag, bf16_out=False):
+    Yg = Y.float().cpu().numpy().astype(np.float64)
+    tol = REL * mag + (2.0 ** -8 * np.abs(Yr) if bf16_out else 0.0)
+    bad = np.abs(Yg - Yr) > tol
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} outside tolerance; worst excess "
+                           f"{np.max(np.abs(Yg - Yr) - tol):.3e} at {np.unravel_index(np.argmax(np.abs(Yg - Yr) - tol), Yr.shape)}")
+
+
+def test_single_projection_case_both_paths():
+    """X 8x512 fp32 with 8 outlier channels x50, W 256x512, P = top-64 variance channels."""
+    x, w, _ = synth.single_projection(0)
+    st = stats.accumulate(stats.new_state(512), x)
+    P = stats.select_topk(st, 64)
+    gA = stats.next_gain(st, P)
+    Yr, mag = _ref(x, w, P, gA)
+    for path in (F.FS_PATH_DECODE, F.FS_PATH_TENSOR):
+        Y, _ = _run_gpu(f32_tensor(x), f32_tensor(w), P, gA, 64, 256, 512, plan_opts=path)
+        _assert_close(Y, Yr, mag)
+
+
+@pytest.mark.parametrize("M,N,K,p", [(1, 1024, 4096, 64), (4, 4096, 4096, 64), (16, 1024, 4096, 64),
+                                     (16, 4096, 12288, 64), (7, 256, 512, 0), (16, 512, 1024, 256),
+                                     (3, 160, 768, 5)])
+def test_decode_path(M, N, K, p):
+    X, W, Xt, Wt, P, gA = _problem(40 + M + N, M, N, K, p)
+    Y, _ = _run_gpu(Xt, Wt, P, gA, p, N, K, plan_opts=F.FS_PATH_DECODE)
+    Yr, mag = _ref(X, W, P, gA)
+    _assert_close(Y, Yr, mag)
+
+
+@pytest.mark.parametrize("M,N,K,p", [(128, 256, 256, 0), (128, 256, 512, 64), (300, 1024, 4096, 64),
+                                     (17, 384, 1024, 64), (1000, 512, 2048, 256), (256, 128, 768, 16),
+                                     (200, 768, 4096, 5), (129, 256, 12288, 64)])
+def test_tensor_core_path(M, N, K, p):
+    X, W, Xt, Wt, P, gA = _problem(70 + M + N + K, M, N, K, p)
+    Y, _ = _run_gpu(Xt, Wt, P, gA, p, N, K, plan_opts=F.FS_PATH_TENSOR)
+    Yr, mag = _ref(X, W, P, gA)
+    _assert_close(Y, Yr, mag)
+
+
+@pytest.mark.parametrize("path", ["decode", "tensor"])
+def test_residual_form_and_bf16_output(path):
+    M = 8 if path == "decode" else 160
+    X, W, Xt, Wt, P, gA = _problem(90, M, 512, 1024, 64, residual=True)
+    popts = (F.FS_PATH_DECODE if path == "decode" else F.FS_PATH_TENSOR) | F.FS_OUT_BF16
+    Y, _ = _run_gpu(Xt, Wt, P, gA, 64, 512, 1024, opts=F.FS_RESIDUAL, plan_opts=popts)
+    assert Y.dtype == torch.bfloat16
+    Yr, mag = _ref(X, W, P, gA, residual=True)
+    _assert_close(Y, Yr, mag, bf16_out=True)
+
+
+def test_paths_agree_on_the_same_inputs():
+    X, W, Xt, Wt, P, gA = _problem(91, 16, 1024, 4096, 64)
+    Yd, _ = _run_gpu(Xt, Wt, P, gA, 64, 1024, 4096, plan_opts=F.FS_PATH_DECODE)
+    Yt, _ = _run_gpu(Xt, Wt, P, gA, 64, 1024, 4096, plan_opts=F.FS_PATH_TENSOR)
+    Yr, mag = _ref(X, W, P, gA)
+    _assert_close(Yd, Yr, mag)
+    _assert_close(Yt, Yr, mag)
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (1024, 4096), (12288, 4096), (4096, 12288)])
+def test_full_size_prefill_sampled_rows(N, K):
+    """M = 8192 tokens as timed; the oracle checks 48 sampled rows spread over all row tiles."""
+    M, p = 8192, 64
+    X, W, Xt, Wt, P, gA = _problem(7, M, N, K, p)
+    Y, _ = _run_gpu(Xt, Wt, P, gA, p, N, K)
+    rows = np.sort(np.random.default_rng(N + K).choice(M, 48, replace=False))
+    rows[0], rows[-1] = 0, M - 1
+    Yr, mag = _ref(X, W, P, gA, rows=rows)
+    _assert_close(Y[torch.from_numpy(rows).cuda()], Yr, mag)
+
+
+def test_repeatable_and_overwrites_output():
+    X, W, Xt, Wt, P, gA = _problem(92, 256, 512, 1024, 64)
+    Y1, _ = _run_gpu(Xt, Wt, P, gA, 64, 512, 1024)
+    Y2, _ = _run_gpu(Xt, Wt, P, gA, 64, 512, 1024)
+    assert torch.equal(Y1, Y2)
