@@ -1,0 +1,523 @@
+"""Benchmark of the SpliceGEMM hot path on B200.
+
+Default workload (one GPU): the Qwen3-8B-shaped prefill pass of FourSight's data-parallel hot
+path, M = 8192 tokens (8 x 1024) in bf16, P = 64 protected channels per projection.  One step is
+one pass of the per-step path over one layer:
+
+  fs_channel_stats   on the 4 input groups (qkv / o / gate-up / down inputs)
+  fs_select_topk     top-64 reselection (batched per K)
+  fs_prepare_weights pre-split of the 7 projections with the new protected set
+  fs_quantize_splice the 4 activation groups
+  fs_splice_gemm     q, k, v, o, gate, up, down
+
+`value` is the whole-step throughput in TFLOP/s, counting 2*M*N*K per projection (the same
+numerator for every P).  Inputs (activations and bf16 weights, about 0.85 GB) are larger than the
+126 MB L2 and are resident in HBM when timing starts.  Extra keys report the decode path (M in
+{1,4,16}, 36 distinct layers per CUDA-graph replay) in GB/s and the overhead against P = 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extras]
+
+Under torchrun each rank runs its own batch (weak scaling); the only exchange is an all-reduce of
+the integer channel statistics before reselection, so every rank selects the same channels.
+`--impl reference` times the CPU oracle, as it stands, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SpliceGEMM prefill TFLOPS & decode GB/s at P=64, % of roofline, overhead vs P=0"
+PROJ = (("q", 4096, 4096, 0), ("k", 1024, 4096, 0), ("v", 1024, 4096, 0), ("o", 4096, 4096, 1),
+        ("gate", 12288, 4096, 2), ("up", 12288, 4096, 2), ("down", 4096, 12288, 3))
+GROUP_K = (4096, 4096, 4096, 12288)          # input groups: qkv, o, gate/up, down
+M_PREFILL = 8192
+P_DEFAULT = 64
+DECODE_LAYERS = 36
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.lines = index, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# workload
+# ------------------------------------------------------------------------------------------
+def make_activations(M, K, seed, device):
+    """X ~ N(0,1) bf16 with 1% of channels (seeded) scaled by 30."""
+    import torch
+    g = torch.Generator(device=device).manual_seed(seed)
+    x = torch.randn(M, K, generator=g, device=device, dtype=torch.float32)
+    idx = torch.randperm(K, generator=g, device=device)[: math.ceil(0.01 * K)]
+    x[:, idx] *= 30.0
+    return x.to(torch.bfloat16)
+
+
+def make_weights(N, K, seed, device):
+    import torch
+    g = torch.Generator(device=device).manual_seed(seed)
+    return (torch.randn(N, K, generator=g, device=device, dtype=torch.float32) * 0.02).to(torch.bfloat16)
+
+
+class PrefillLayer:
+    """Buffers and launches of one per-step pass over a Qwen3-8B layer."""
+
+    def __init__(self, F, M, p, seed, device, out_bf16=False):
+        import torch
+        self.F, self.M, self.p = F, M, p
+        self.X = [make_activations(M, K, seed * 100 + i, device) for i, K in enumerate(GROUP_K)]
+        self.W = [make_weights(N, K, seed * 100 + 10 + j, device) for j, (_, N, K, _) in enumerate(PROJ)]
+        self.st4 = F.StatsState(3, 4096, device=device)
+        self.st12 = F.StatsState(1, 12288, device=device)
+        self.P4 = torch.empty(3, max(p, 1), dtype=torch.int32, device=device)[:, :p]
+        self.m4 = torch.empty(3, 128, dtype=torch.int32, device=device)
+        self.g4 = torch.empty(3, dtype=torch.float32, device=device)
+        self.P12 = torch.empty(1, max(p, 1), dtype=torch.int32, device=device)[:, :p]
+        self.m12 = torch.empty(1, 384, dtype=torch.int32, device=device)
+        self.g12 = torch.empty(1, dtype=torch.float32, device=device)
+        self.xq = [F.alloc_packed(M, K, p, device) for K in GROUP_K]
+        self.wq = [F.alloc_packed(N, K, p, device) for (_, N, K, _) in PROJ]
+        self.gW = torch.empty(len(PROJ), dtype=torch.float32, device=device)
+        self.alpha = torch.empty(len(PROJ), dtype=torch.float32, device=device)
+        popts = F.FS_OUT_BF16 if out_bf16 else 0
+        self.plans = [F.Plan(N, K, max(p, 1), popts) for (_, N, K, _) in PROJ]
+        dt = torch.bfloat16 if out_bf16 else torch.float32
+        self.Y = [torch.empty(M, N, dtype=dt, device=device) for (_, N, K, _) in PROJ]
+        self.flops = sum(2.0 * M * N * K for (_, N, K, _) in PROJ)
+        self.launches_per_step = 4 + 2 + 3 * len(PROJ) + 4 + len(PROJ)   # prepare = amax + gain + quantise
+
+    def mask_gain(self, gi):
+        if gi < 3:
+            return self.m4[gi], self.g4[gi:gi + 1]
+        return self.m12[0], self.g12[0:1]
+
+    def step(self, allreduce=None, events=None):
+        F = self.F
+        for gi in range(4):
+            st, gidx = (self.st4, gi) if gi < 3 else (self.st12, 0)
+            F.fs_channel_stats(self.X[gi], st, group=gidx)
+        if allreduce is not None:
+            allreduce(self.st4)
+            allreduce(self.st12)
+        F.fs_select_topk(self.st4, self.p, reset=True, P=self.P4, mask=self.m4, gA=self.g4)
+        F.fs_select_topk(self.st12, self.p, reset=True, P=self.P12, mask=self.m12, gA=self.g12)
+        for j, (_, N, K, gi) in enumerate(PROJ):
+            mask, g = self.mask_gain(gi)
+            F.fs_prepare_weights(self.W[j], mask, self.p, g, out=self.wq[j], gW=self.gW[j:j + 1],
+                                 alpha=self.alpha[j:j + 1])
+        for gi in range(4):
+            mask, g = self.mask_gain(gi)
+            F.fs_quantize_splice(self.X[gi], mask, self.p, g, out=self.xq[gi])
+        for j, (name, N, K, gi) in enumerate(PROJ):
+            if events is not None:
+                events[j][0].record()
+            F.fs_splice_gemm(self.plans[j], self.xq[gi], self.wq[j], self.alpha[j:j + 1], Y=self.Y[j])
+            if events is not None:
+                events[j][1].record()
+
+    def check(self):
+        for pl in self.plans:
+            pl.check()
+
+
+def stats_allreduce_fn(dist):
+    """The DP exchange: sum the integer moments and counts, max the per-channel maxima."""
+    import torch
+
+    def f(st):
+        dist.all_reduce(st.s1, op=dist.ReduceOp.SUM)
+        dist.all_reduce(st.s2, op=dist.ReduceOp.SUM)
+        dist.all_reduce(st.n, op=dist.ReduceOp.SUM)
+        dist.all_reduce(st.amax, op=dist.ReduceOp.MAX)      # non-negative float bits order as ints
+        dist.all_reduce(st.flags, op=dist.ReduceOp.MAX)
+    return f
+
+
+def timed(fn, steps, dist=None):
+    import torch
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+# ------------------------------------------------------------------------------------------
+# decode sweep (M <= 16), CUDA-graph replay over 36 distinct layers
+# ------------------------------------------------------------------------------------------
+def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20):
+    import torch
+    res = {}
+    packed = []          # per layer: list of (wq, alpha) per projection
+    st = F.StatsState(1, 4096, device=device)
+    calib = make_activations(4096, 4096, 999, device)
+    F.fs_channel_stats(calib, st)
+    _, m4, g4 = F.fs_select_topk(st, p)
+    st12 = F.StatsState(1, 12288, device=device)
+    F.fs_channel_stats(make_activations(4096, 12288, 998, device), st12)
+    _, m12, g12 = F.fs_select_topk(st12, p)
+    for layer in range(layers):
+        row = []
+        for j, (_, N, K, gi) in enumerate(PROJ):
+            W = make_weights(N, K, 5000 + layer * 10 + j, device)
+            mask, g = (m4[0], g4[0:1]) if K == 4096 else (m12[0], g12[0:1])
+            wq, gW, alpha = F.fs_prepare_weights(W, mask, p, g)
+            row.append((wq, alpha))
+            del W
+        packed.append(row)
+    torch.cuda.synchronize()
+    wbytes = sum(wq.q.numel() + N * (K // 16) + N * F.side_cols(p) * 2 for (wq, _), (_, N, K, _) in zip(packed[0], PROJ))
+    for M in Ms:
+        Xs = [make_activations(M, K, 77 + gi, device) for gi, K in enumerate(GROUP_K)]
+        xq = [F.alloc_packed(M, K, p, device) for K in GROUP_K]
+        plans = [F.Plan(N, K, max(p, 1)) for (_, N, K, _) in PROJ]
+        Ys = [torch.empty(M, N, dtype=torch.float32, device=device) for (_, N, K, _) in PROJ]
+
+        def run_layers(with_quant: bool):
+            for layer in range(layers):
+                if with_quant:
+                    for gi, K in enumerate(GROUP_K):
+                        mask, g = (m4[0], g4[0:1]) if K == 4096 else (m12[0], g12[0:1])
+                        F.fs_quantize_splice(Xs[gi], mask, p, g, out=xq[gi])
+                for j, (_, N, K, gi) in enumerate(PROJ):
+                    wq, alpha = packed[layer][j]
+                    F.fs_splice_gemm(plans[j], xq[gi], wq, alpha, Y=Ys[j])
+
+        out = {}
+        for tag, wq_flag in (("gemm", False), ("quant+gemm", True)):
+            run_layers(True)
+            torch.cuda.synchronize()
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s):
+                run_layers(wq_flag)          # warm (also sets kernel attributes before capture)
+                with torch.cuda.graph(graph, stream=s):
+                    run_layers(wq_flag)
+            torch.cuda.synchronize()
+            for _ in range(3):
+                graph.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            xbytes = sum(M * K * 2 + M * (K // 2 + K // 16 + F.side_cols(p) * 2) for K in GROUP_K) if wq_flag else 0
+            abytes = sum(M * (K // 2 + K // 16 + F.side_cols(p) * 2) + M * N * 4 for (_, N, K, _) in PROJ)
+            total = layers * (wbytes + abytes + xbytes)
+            out[tag] = {"us_per_layer": 1000.0 * ms / layers, "GBps": total / (ms * 1e-3) / 1e9,
+                        "bytes_per_layer": wbytes + abytes + xbytes}
+            del graph
+        for pl in plans:
+            pl.check()
+        res[f"M{M}"] = out
+    return res, wbytes
+
+
+# ------------------------------------------------------------------------------------------
+# reference arm / CPU baseline: the oracle as it stands on a bounded sample
+# ------------------------------------------------------------------------------------------
+def oracle_sample_step(rows=128, seed=0):
+    """One bounded sample of the step through the CPU oracle: the q projection (4096 <- 4096) of
+    `rows` tokens: statistics, top-64 selection, weight pre-split, activation quantisation and the
+    float64 SpliceGEMM.  Returns (seconds, flops counted as 2*rows*N*K)."""
+    import numpy as np
+
+    import synth
+    from oracle import splice, stats
+    x, _ = synth.outlier_activations(seed, rows, 4096)
+    w = synth.gaussian_weights(seed + 1, 4096, 4096)
+    X, W = splice.as_f32(x, True), splice.as_f32(w, True)
+    t0 = time.perf_counter()
+    st = stats.accumulate(stats.new_state(4096), X)
+    P = stats.select_topk(st, P_DEFAULT)
+    gA = stats.next_gain(st, P)
+    wq = splice.prepare_weights(W, P, gA)
+    xq = splice.quantize_splice(X, P, gA)
+    Y, _ = splice.splice_gemm(xq, wq, wq["alpha"])
+    dt = time.perf_counter() - t0
+    assert np.isfinite(Y).all()
+    return dt, 2.0 * rows * 4096 * 4096
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(rows=128):
+    dt, flops = oracle_sample_step(rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"q projection 4096x4096 of {rows} of the 8192 tokens, P=64: stats, select, "
+                      f"weight pre-split, quantise, float64 SpliceGEMM ({dt:.1f} s)",
+            "seconds": dt}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(max(0, args.warmup)):
+        oracle_sample_step(32)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample_step(128)
+        times.append(dt)
+        flops = fl
+    tot = sum(times)
+    value = flops * len(times) / tot / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "Qwen3-8B-shaped prefill, M=8192 bf16, P=64 (oracle sample: q projection, 128 rows)",
+                       "global_batch": M_PREFILL, "seq_len": 1024, "parallelism": "cpu"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": "q projection 4096x4096 of 128 tokens per step, P=64"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def kernel_case(F, args, device):
+    """fs_splice_gemm alone on the q projection (4096 <- 4096), for profiling one kernel."""
+    import torch
+    M = M_PREFILL if args.case == "gemm" else 16
+    X = make_activations(M, 4096, 3, device)
+    W = make_weights(4096, 4096, 4, device)
+    st = F.StatsState(1, 4096, device=device)
+    F.fs_channel_stats(X, st)
+    _, mask, g = F.fs_select_topk(st, args.p)
+    wq, _, alpha = F.fs_prepare_weights(W, mask[0], args.p, g)
+    xq = F.fs_quantize_splice(X, mask[0], args.p, g)
+    plan = F.Plan(4096, 4096, max(args.p, 1))
+    Y = torch.empty(M, 4096, dtype=torch.float32, device=device)
+    for _ in range(args.warmup):
+        F.fs_splice_gemm(plan, xq, wq, alpha, Y=Y)
+    ms = timed(lambda: F.fs_splice_gemm(plan, xq, wq, alpha, Y=Y), args.steps) / args.steps
+    plan.check()
+    print(json.dumps({"case": args.case, "M": M, "N": 4096, "K": 4096, "p": args.p, "us": ms * 1000.0,
+                      "tflops": 2.0 * M * 4096 * 4096 / (ms * 1e-3) / 1e12}))
+
+
+# ------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--p", type=int, default=P_DEFAULT)
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default="step", choices=["step", "gemm", "decode"],
+                    help="step: the full benchmark; gemm / decode: only fs_splice_gemm on the q projection "
+                         "(M=8192, or M=16) for profiling one kernel")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    use_dist = world > 1
+    if use_dist:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device(device))
+
+    import nvfp4_w4a4_gemm_fs_b200 as F
+    F.load()
+    peaks = _peaks()
+    p = args.p
+
+    if args.case != "step":
+        return kernel_case(F, args, device)
+
+    layer = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device)
+    allreduce = stats_allreduce_fn(dist) if use_dist else None
+    for _ in range(args.warmup):
+        layer.step(allreduce)
+    torch.cuda.synchronize()
+    layer.check()
+
+    # timed region: exactly `steps` steps, GEMM launches bracketed by events for the roofline
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in PROJ]
+          for _ in range(args.steps)]
+    it = iter(range(args.steps))
+    with Clocks(local) as clk:
+        ms = timed(lambda: layer.step(allreduce, events=ev[next(it)]), args.steps, dist if use_dist else None)
+    layer.check()
+    ms_step = ms / args.steps
+    value = world * layer.flops / (ms_step * 1e-3) / 1e12
+    gemm_ms = [[a.elapsed_time(b) for (a, b) in e] for e in ev]
+    gemm_total_ms = sum(sum(r) for r in gemm_ms) / args.steps
+    gemm_tflops = layer.flops / (gemm_total_ms * 1e-3) / 1e12
+    per_proj = {name: statistics.mean(r[j] for r in gemm_ms) * 1000.0 for j, (name, _, _, _) in enumerate(PROJ)}
+    fp4_peak = peaks["bf16_tflops"] * 4.0         # dense NVFP4 = 4x dense BF16 (nominal 9 vs 2.25 PFLOP/s)
+
+    # end to end: host (pinned) activations in, all projection outputs back to host, every step
+    host_x = [x.cpu().pin_memory() for x in layer.X]
+    host_y = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in layer.Y]
+    h2d = sum(x.numel() * x.element_size() for x in host_x)
+    d2h = sum(y.numel() * y.element_size() for y in host_y)
+
+    def e2e_step():
+        for dx, hx in zip(layer.X, host_x):
+            dx.copy_(hx, non_blocking=True)
+        layer.step(allreduce)
+        for hy, dy in zip(host_y, layer.Y):
+            hy.copy_(dy, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 5))
+    for _ in range(2):
+        e2e_step()
+    ms_e2e = timed(e2e_step, e2e_steps, dist if use_dist else None) / e2e_steps
+    e2e_value = world * layer.flops / (ms_e2e * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 e2m1/ue4m3 + bf16 side, fp32 accumulate and output",
+        "data": "synthetic (seeded N(0,1) activations with 1% channels x30, N(0,0.02) weights)",
+        "config": {"workload": "Qwen3-8B-shaped prefill layer: M=8192 bf16 tokens (8x1024), 7 projections, P=64; "
+                               "per step stats + top-64 reselect + weight pre-split + quantise + SpliceGEMM",
+                   "global_batch": world * M_PREFILL, "seq_len": 1024, "parallelism": f"dp{world}",
+                   "p": p, "l2": "inputs larger than L2 (0.85 GB of bf16 activations and weights per step)"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / fp4_peak, "traffic": None,
+                     "kernel": "splice_gemm_tc_kernel (all 7 projections; 2MNK per launch / CUDA-event time)",
+                     "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16 ratio)"},
+        "gemm_us": per_proj,
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": ms_e2e},
+        "gpu_launches": layer.launches_per_step * args.steps,
+    }
+
+    if not args.no_extras and rank == 0:
+        # overhead against P = 0: the same step and the GEMMs alone
+        del host_x, host_y
+        torch.cuda.empty_cache()
+        l0 = PrefillLayer(F, M_PREFILL, 0, seed=2 + rank, device=device)
+        for _ in range(3):
+            l0.step()
+        ev0 = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in PROJ]
+               for _ in range(args.steps)]
+        it0 = iter(range(args.steps))
+        ms0 = timed(lambda: l0.step(events=ev0[next(it0)]), args.steps) / args.steps
+        l0.check()
+        g0 = sum(sum(a.elapsed_time(b) for a, b in e) for e in ev0) / args.steps
+        line["overhead_vs_p0"] = {"step_ms_p0": ms0, "step_ms_p": ms_step, "step_overhead": ms_step / ms0 - 1.0,
+                                  "gemm_ms_p0": g0, "gemm_ms_p": gemm_total_ms, "gemm_overhead": gemm_total_ms / g0 - 1.0,
+                                  "gemm_tflops_p0": l0.flops / (g0 * 1e-3) / 1e12}
+        del l0
+        torch.cuda.empty_cache()
+        dec, wbytes = decode_sweep(F, p, device)
+        dec0, wbytes0 = decode_sweep(F, 0, device, Ms=(16,))
+        hbm = peaks["hbm_gbs"]
+        line["decode"] = {k: {**v["gemm"], "frac_hbm": v["gemm"]["GBps"] / hbm,
+                              "with_quantise": {**v["quant+gemm"], "frac_hbm": v["quant+gemm"]["GBps"] / hbm}}
+                          for k, v in dec.items()}
+        line["decode"]["layers"] = DECODE_LAYERS
+        line["decode"]["weight_bytes_per_layer"] = wbytes
+        line["decode"]["overhead_vs_p0_M16"] = dec["M16"]["gemm"]["us_per_layer"] / dec0["M16"]["gemm"]["us_per_layer"] - 1.0
+        line["decode"]["hbm_peak_gbs"] = hbm
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line))
+    if use_dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -15,7 +15,7 @@
 #include <string>
 #include <algorithm>
 
-#include "../../include/foursight.h"
+#include "foursight.h"
 
 namespace fs {
 
