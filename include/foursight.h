@@ -220,6 +220,30 @@ fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64_t* row_off
                                  const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
                                  const float* alpha, void* Y, int64_t ldy, void* stream);
 
+/* SpliceGEMM for callers that cannot allocate device memory.  The paper has no counterpart to
+ * this call; it exists for integration.  fs_splice_gemm needs a plan, and fs_plan_create calls
+ * cudaMalloc for the tensor-core kernel's error word.  Code that must not allocate at call time
+ * (an allocator or memory-pool callback, a runtime that serves every device byte from an arena
+ * reserved at start-up, a plugin whose host forbids allocations) calls this instead: same
+ * operands, same results, no plan.  Its only scratch is one 32-bit error word in a file-scope
+ * __device__ array of the library (1 word, 256-byte aligned); every GPU that loads the library
+ * holds it until the process exits.  No problem size needs more scratch than that; shapes beyond
+ * the kernels' limits (N % 16, K % 256 or 256 <= K <= 65536, M < 2^31 - 256, p <= min(K, 256)) are
+ * rejected with FS_ERR_INVALID_ARGUMENT / FS_ERR_UNSUPPORTED.
+ *   N, K, opts  as for fs_plan_create (FS_OUT_BF16, FS_PATH_TENSOR, FS_PATH_DECODE apply);
+ *   M .. ldy    as for fs_splice_gemm;
+ *   check != 0  synchronise `stream` after the launch and return FS_ERR_TIMEOUT if the kernel gave
+ *               up a bounded wait (check == 0: fully asynchronous, no device-to-host read).
+ * The call never calls cudaMalloc, cudaFree or any allocating routine.  Its first call on a device
+ * looks up the device address of the scratch array (cudaGetSymbolAddress, with that device
+ * current); make that first call before any stream capture.  Every call clears the word on
+ * `stream` before its kernel; calls that overlap on the GPU (unordered streams) share the word and
+ * race on it. */
+fs_status fs_splice_gemm_noalloc(int32_t N, int32_t K, uint32_t opts, int64_t M, int32_t p, const uint8_t* xq,
+                                 const uint8_t* sfx, const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw,
+                                 const uint16_t* ws, const float* alpha, void* Y, int64_t ldy, int32_t check,
+                                 void* stream);
+
 /* ------------------------------------------------------------------------------------------
  * TIM-aware sequence filter — FourSight §4.1 "The dual-gate mechanism" and Eq. 3-4; §2.1 for the
  * group advantage; §6.1 for tau = 1e-4, K1 = 0.01 x output_len, K2 = 5.
