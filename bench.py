@@ -153,33 +153,69 @@ class PrefillLayer:
             return self.m4[gi], self.g4[gi:gi + 1]
         return self.m12[0], self.g12[0:1]
 
-    def step(self, allreduce=None, events=None):
+    PHASES = ("stats", "select", "prepare_weights", "quantize", "gemm")
+
+    def step(self, allreduce=None):
+        for fn in self.phase_fns(allreduce):
+            fn()
+
+    def phase_fns(self, allreduce=None):
+        """The step split into its phases (same order and launches as step())."""
         F = self.F
-        for gi in range(4):
-            st, gidx = (self.st4, gi) if gi < 3 else (self.st12, 0)
-            F.fs_channel_stats(self.X[gi], st, group=gidx)
-        if allreduce is not None:
-            allreduce(self.st4)
-            allreduce(self.st12)
-        F.fs_select_topk(self.st4, self.p, reset=True, P=self.P4, mask=self.m4, gA=self.g4)
-        F.fs_select_topk(self.st12, self.p, reset=True, P=self.P12, mask=self.m12, gA=self.g12)
-        for j, (_, N, K, gi) in enumerate(PROJ):
-            mask, g = self.mask_gain(gi)
-            F.fs_prepare_weights(self.W[j], mask, self.p, g, out=self.wq[j], gW=self.gW[j:j + 1],
-                                 alpha=self.alpha[j:j + 1])
-        for gi in range(4):
-            mask, g = self.mask_gain(gi)
-            F.fs_quantize_splice(self.X[gi], mask, self.p, g, out=self.xq[gi])
-        for j, (name, N, K, gi) in enumerate(PROJ):
-            if events is not None:
-                events[j][0].record()
-            F.fs_splice_gemm(self.plans[j], self.xq[gi], self.wq[j], self.alpha[j:j + 1], Y=self.Y[j])
-            if events is not None:
-                events[j][1].record()
+
+        def stats():
+            for gi in range(4):
+                st, gidx = (self.st4, gi) if gi < 3 else (self.st12, 0)
+                F.fs_channel_stats(self.X[gi], st, group=gidx)
+            if allreduce is not None:
+                allreduce(self.st4)
+                allreduce(self.st12)
+
+        def select():
+            F.fs_select_topk(self.st4, self.p, reset=True, P=self.P4, mask=self.m4, gA=self.g4)
+            F.fs_select_topk(self.st12, self.p, reset=True, P=self.P12, mask=self.m12, gA=self.g12)
+
+        def prepare():
+            for j, (_, N, K, gi) in enumerate(PROJ):
+                mask, g = self.mask_gain(gi)
+                F.fs_prepare_weights(self.W[j], mask, self.p, g, out=self.wq[j], gW=self.gW[j:j + 1],
+                                     alpha=self.alpha[j:j + 1])
+
+        def quantize():
+            for gi in range(4):
+                mask, g = self.mask_gain(gi)
+                F.fs_quantize_splice(self.X[gi], mask, self.p, g, out=self.xq[gi])
+
+        def gemm():
+            for fn in self.gemm_fns():
+                fn()
+        return [stats, select, prepare, quantize, gemm]
+
+    def gemm_fns(self):
+        F = self.F
+
+        def make(j, gi):
+            return lambda: F.fs_splice_gemm(self.plans[j], self.xq[gi], self.wq[j], self.alpha[j:j + 1], Y=self.Y[j])
+        return [make(j, gi) for j, (_, N, K, gi) in enumerate(PROJ)]
 
     def check(self):
         for pl in self.plans:
             pl.check()
+
+
+def capture(fn):
+    """Capture fn's launches (on a side stream) into a CUDA graph."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        fn()                                   # warm: sets kernel attributes before capture
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
 
 
 def stats_allreduce_fn(dist):
@@ -359,9 +395,36 @@ def run_reference(args):
     print(json.dumps(line))
 
 
+def prep_case(F, args, device):
+    """The preparation kernels alone on the q-projection input (8192 x 4096) and weights, for profiling."""
+    import torch
+    X = make_activations(M_PREFILL, 4096, 3, device)
+    W = make_weights(4096, 4096, 4, device)
+    st = F.StatsState(1, 4096, device=device)
+    xq = F.alloc_packed(M_PREFILL, 4096, args.p, device)
+    wq = F.alloc_packed(4096, 4096, args.p, device)
+    P = torch.empty(1, args.p, dtype=torch.int32, device=device)
+    mask = torch.empty(1, 128, dtype=torch.int32, device=device)
+    g = torch.empty(1, dtype=torch.float32, device=device)
+    gW = torch.empty(1, dtype=torch.float32, device=device)
+    alpha = torch.empty(1, dtype=torch.float32, device=device)
+
+    def run():
+        F.fs_channel_stats(X, st)
+        F.fs_select_topk(st, args.p, reset=True, P=P, mask=mask, gA=g)
+        F.fs_prepare_weights(W, mask[0], args.p, g, out=wq, gW=gW, alpha=alpha)
+        F.fs_quantize_splice(X, mask[0], args.p, g, out=xq)
+    for _ in range(args.warmup):
+        run()
+    ms = timed(run, args.steps) / args.steps
+    print(json.dumps({"case": "prep", "us_per_pass": ms * 1000.0}))
+
+
 def kernel_case(F, args, device):
     """fs_splice_gemm alone on the q projection (4096 <- 4096), for profiling one kernel."""
     import torch
+    if args.case == "prep":
+        return prep_case(F, args, device)
     M = M_PREFILL if args.case == "gemm" else 16
     X = make_activations(M, 4096, 3, device)
     W = make_weights(4096, 4096, 4, device)
@@ -390,7 +453,7 @@ def main():
     ap.add_argument("--p", type=int, default=P_DEFAULT)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", default="step", choices=["step", "gemm", "decode"],
+    ap.add_argument("--case", default="step", choices=["step", "gemm", "decode", "prep"],
                     help="step: the full benchmark; gemm / decode: only fs_splice_gemm on the q projection "
                          "(M=8192, or M=16) for profiling one kernel")
     args = ap.parse_args()
@@ -428,20 +491,45 @@ def main():
     torch.cuda.synchronize()
     layer.check()
 
-    # timed region: exactly `steps` steps, GEMM launches bracketed by events for the roofline
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in PROJ]
-          for _ in range(args.steps)]
-    it = iter(range(args.steps))
+    # The step is captured once into a CUDA graph and replayed: host launch latency of the 38
+    # small library calls would otherwise show up as GPU idle time.  Each phase (and each GEMM)
+    # is also captured on its own, replayed back to back with events in between, to attribute
+    # time per kernel on the device.
+    step_graph = capture(lambda: layer.step(allreduce))
+    for _ in range(args.warmup):
+        step_graph.replay()
+    torch.cuda.synchronize()
     with Clocks(local) as clk:
-        ms = timed(lambda: layer.step(allreduce, events=ev[next(it)]), args.steps, dist if use_dist else None)
+        ms = timed(step_graph.replay, args.steps, dist if use_dist else None)
     layer.check()
     ms_step = ms / args.steps
     value = world * layer.flops / (ms_step * 1e-3) / 1e12
-    gemm_ms = [[a.elapsed_time(b) for (a, b) in e] for e in ev]
+
+    phase_graphs = [capture(fn) for fn in layer.phase_fns(allreduce)]
+    gemm_graphs = [capture(fn) for fn in layer.gemm_fns()]
+    phase_us = {name: 0.0 for name in PrefillLayer.PHASES}
+    gemm_ms = [[0.0] * len(PROJ) for _ in range(args.steps)]
+    for it_ in range(args.steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(phase_graphs) + len(gemm_graphs) + 1)]
+        evs[0].record()
+        k = 1
+        for g_ in phase_graphs[:-1]:
+            g_.replay(); evs[k].record(); k += 1
+        for g_ in gemm_graphs:
+            g_.replay(); evs[k].record(); k += 1
+        torch.cuda.synchronize()
+        for i, name in enumerate(PrefillLayer.PHASES[:-1]):
+            phase_us[name] += evs[i].elapsed_time(evs[i + 1]) * 1000.0 / args.steps
+        base = len(phase_graphs) - 1
+        for j in range(len(PROJ)):
+            gemm_ms[it_][j] = evs[base + j].elapsed_time(evs[base + j + 1])
+    layer.check()
     gemm_total_ms = sum(sum(r) for r in gemm_ms) / args.steps
+    phase_us["gemm"] = gemm_total_ms * 1000.0
     gemm_tflops = layer.flops / (gemm_total_ms * 1e-3) / 1e12
     per_proj = {name: statistics.mean(r[j] for r in gemm_ms) * 1000.0 for j, (name, _, _, _) in enumerate(PROJ)}
     fp4_peak = peaks["bf16_tflops"] * 4.0         # dense NVFP4 = 4x dense BF16 (nominal 9 vs 2.25 PFLOP/s)
+    del phase_graphs, gemm_graphs
 
     # end to end: host (pinned) activations in, all projection outputs back to host, every step
     host_x = [x.cpu().pin_memory() for x in layer.X]
@@ -476,10 +564,12 @@ def main():
                      "kernel": "splice_gemm_tc_kernel (all 7 projections; 2MNK per launch / CUDA-event time)",
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16 ratio)"},
         "gemm_us": per_proj,
+        "phase_us": phase_us,
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": ms_e2e},
         "gpu_launches": layer.launches_per_step * args.steps,
+        "graph": "each timed step is one CUDA-graph replay of the step's 38 launches",
     }
 
     if not args.no_extras and rank == 0:
@@ -489,15 +579,24 @@ def main():
         l0 = PrefillLayer(F, M_PREFILL, 0, seed=2 + rank, device=device)
         for _ in range(3):
             l0.step()
-        ev0 = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in PROJ]
-               for _ in range(args.steps)]
-        it0 = iter(range(args.steps))
-        ms0 = timed(lambda: l0.step(events=ev0[next(it0)]), args.steps) / args.steps
+        g0s = capture(l0.step)
+        for _ in range(3):
+            g0s.replay()
+        ms0 = timed(g0s.replay, args.steps) / args.steps
+        gg0 = [capture(fn) for fn in l0.gemm_fns()]
+        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev0[0].record()
+        for _ in range(args.steps):
+            for g_ in gg0:
+                g_.replay()
+        ev0[1].record()
+        torch.cuda.synchronize()
+        g0 = ev0[0].elapsed_time(ev0[1]) / args.steps
         l0.check()
-        g0 = sum(sum(a.elapsed_time(b) for a, b in e) for e in ev0) / args.steps
         line["overhead_vs_p0"] = {"step_ms_p0": ms0, "step_ms_p": ms_step, "step_overhead": ms_step / ms0 - 1.0,
                                   "gemm_ms_p0": g0, "gemm_ms_p": gemm_total_ms, "gemm_overhead": gemm_total_ms / g0 - 1.0,
                                   "gemm_tflops_p0": l0.flops / (g0 * 1e-3) / 1e12}
+        del g0s, gg0
         del l0
         torch.cuda.empty_cache()
         dec, wbytes = decode_sweep(F, p, device)

@@ -99,10 +99,11 @@ int64_t fs_sf_bytes(int64_t R, int32_t K);
  *   s1    [K] int64   += sum rint(x * 2^16)          (exact integer fixed point)
  *   s2    [K] int64   += sum rint(x^2 * 2^14)        (x^2 formed exactly)
  *   amax  [K] uint32  = bits of max(|x|) as float32
- *   flags [1] uint32  |= 1 if some |x| >= 2^16 or x is not finite (read by fs_stats_check)
+ *   flags [1] uint32  |= 1 if some |x| >= 2^15 or x is not finite (read by fs_stats_check);
+ *                      such an element adds nothing to the sums or the maximum
  * Integer sums make the state independent of the reduction order.  The state must be
  * zeroed before the first call (e.g. cudaMemsetAsync or fs_select_topk with reset=1).
- * Requirements: K % 8 == 0, M >= 0, row_stride >= 1; the state must hold fewer than 2^17
+ * Requirements: K % 8 == 0, M >= 0, row_stride >= 1; the state must hold fewer than 2^19
  * rows of values near the range limit for s2 not to overflow.
  * ---------------------------------------------------------------------------------------- */
 fs_status fs_channel_stats(const void* X, int32_t dtype, int64_t M, int32_t K, int64_t ldx,
@@ -174,7 +175,7 @@ fs_status fs_quantize_splice(const void* X, int32_t dtype, int64_t M, int32_t K,
 /* Grouped (mixture-of-experts) form: E experts, expert e owning rows
  * [row_offsets[e], row_offsets[e+1]) of X (row_offsets: device int64 [E+1], row_offsets[0] == 0,
  * non-decreasing, row_offsets[E] <= max_rows).  Each expert has its own mask [E][ceil(K/32)] and
- * gain gA [E]; all share p.  Expert e's packed rows start at the padded offset
+ * gain gA [E]; all share p; E <= 256.  Expert e's packed rows start at the padded offset
  * pad_e = sum_{e'<e} roundup(rows_e', 128) in xq [.][K/2], sfx and xs [.][Pp]; size the buffers
  * with fs_grouped_rows(max_rows, E) rows.  Rows of the padding are zero. */
 fs_status fs_quantize_splice_grouped(const void* X, int32_t dtype, int32_t E, const int64_t* row_offsets,

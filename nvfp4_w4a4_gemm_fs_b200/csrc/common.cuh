@@ -79,11 +79,29 @@ __device__ __forceinline__ float ue4m3_value(uint32_t c) {
 // midpoint (y has 24 significant bits, so y - M*d, for an fp32 midpoint M with 25 bits, is a
 // non-zero multiple of M's last unit unless y/d == M, which would need y to span more than
 // 24 bits).  The fp64 error therefore never moves the result across a rounding boundary.
-// Both block-scale steps divide by such a d: 6 = 3*2 and any UE4M3 value.
+// Used for the per-block step t = fl32(a_b*g)/6 (6 = 3*2).
 __device__ __forceinline__ float div_small_divisor(float y, double inv_d) {
   return __double2float_rn(__dmul_rn(static_cast<double>(y), inv_d));
 }
 constexpr double kInvSix = 1.0 / 6.0;   // RN64(1/6): compile-time IEEE division
+
+// Correctly rounded y / d in fp32 by Markstein's correction (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990):
+// with r = RN(1/d), a quotient q within one ulp of y/d and the remainder e = y - d*q (exact when
+// formed by one fused multiply-add), RN(q + e*r) is the correctly rounded quotient.  The first
+// correction brings q0 = RN(y*r) within one ulp; the second rounds correctly.  Used per element
+// (v = fl32(x*g) / sf), where it replaces an IEEE division by five fp32 operations.  Requires
+// finite y and d > 0 (d = 1, r = 0 yields +-0 with the sign of y, the zero-scale rule).  The
+// quotient takes the sign of y explicitly: for y = -0 the remainder y - d*q0 = (-0) + (+0) is +0, and the
+// corrections would otherwise return +0.
+__device__ __forceinline__ float div_markstein(float y, float d, float r) {
+  const float q0 = __fmul_rn(y, r);
+  const float e0 = __fmaf_rn(-q0, d, y);
+  const float q1 = __fmaf_rn(e0, r, q0);
+  const float e1 = __fmaf_rn(-q1, d, y);
+  const float q2 = __fmaf_rn(e1, r, q1);
+  return __uint_as_float((__float_as_uint(q2) & 0x7FFFFFFFu) | (__float_as_uint(y) & 0x80000000u));
+}
 
 // Packs two fp32 values into one byte of E2M1 codes (round to nearest even, saturating at 6),
 // `lo` into the low nibble.  The PTX conversion places its first source in the high nibble.
@@ -91,6 +109,20 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
   uint32_t r;
   asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
       : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Packs eight fp32 values into one 32-bit word of E2M1 codes (element 0 in the low nibble).
+__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
+                                           float v7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r) : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
   return r;
 }
 

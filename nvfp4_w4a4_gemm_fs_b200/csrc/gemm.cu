@@ -102,7 +102,7 @@ extern "C" fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const ui
   prm.E = 1; prm.kb4 = plan->K / 64; prm.offsets = nullptr; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
   prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
   TcLaunch L{};
-  L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = M; L.b_rows = plan->N; L.pp = pp;
+  L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = M; L.b_rows = plan->N; L.y_rows = M; L.pp = pp;
   L.bn = (plan->N % 256 == 0) ? 256 : 128;
   L.max_tiles = ceil_div(M, 128) * ceil_div(plan->N, L.bn);
   return launch_splice_gemm_tc(L, prm, s);
@@ -125,7 +125,7 @@ extern "C" fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64
   prm.E = E; prm.kb4 = plan->K / 64; prm.offsets = row_offsets; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
   prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
   TcLaunch L{};
-  L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = a_rows; L.b_rows = static_cast<int64_t>(E) * plan->N; L.pp = pp;
+  L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = a_rows; L.b_rows = static_cast<int64_t>(E) * plan->N; L.y_rows = max_rows; L.pp = pp;
   L.bn = (plan->N % 256 == 0) ? 256 : 128;
   L.max_tiles = ceil_div(a_rows, 128) * (plan->N / L.bn);
   return launch_splice_gemm_tc(L, prm, static_cast<cudaStream_t>(stream));

@@ -26,6 +26,7 @@ struct TcLaunch {
   const void* ws;
   int64_t a_rows;     // rows of the activation buffers (padded rows for experts)
   int64_t b_rows;     // rows of the weight buffers (E * N for experts)
+  int64_t y_rows;     // rows of Y
   int pp;
   int bn;
   int64_t max_tiles;

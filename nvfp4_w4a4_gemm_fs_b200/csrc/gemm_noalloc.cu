@@ -98,7 +98,7 @@ extern "C" fs_status fs_splice_gemm_noalloc(int32_t N, int32_t K, uint32_t opts,
     prm.E = 1; prm.kb4 = K / 64; prm.offsets = nullptr; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
     prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = bf16 ? 1 : 0; prm.err = scratch;
     TcLaunch L{};
-    L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = M; L.b_rows = N; L.pp = pp;
+    L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = M; L.b_rows = N; L.y_rows = M; L.pp = pp;
     L.bn = (N % 256 == 0) ? 256 : 128;
     L.max_tiles = ceil_div(M, 128) * ceil_div(N, L.bn);
     st = launch_splice_gemm_tc(L, prm, s);

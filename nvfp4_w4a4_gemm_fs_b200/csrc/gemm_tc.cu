@@ -36,14 +36,18 @@ struct Cfg {
   static constexpr int SFA_BYTES = kBM * 16;           // 16 scales per row per k-tile
   static constexpr int SFB_BYTES = BN * 16;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = BN == 256 ? 3 : 5;
   static constexpr int NUM_ACC = BN == 256 ? 1 : 2;    // TMEM accumulator buffers
   static constexpr int ACC_COLS = BN * NUM_ACC;
-  static constexpr int SFA_COL = ACC_COLS;             // 4 MMAs x 4 columns
-  static constexpr int SFB_COL = ACC_COLS + 16;        // 4 MMAs x BN/32 columns
+  // Scale factors in TMEM, double-buffered by k-tile parity so that the copy for k-tile kt+1
+  // does not overwrite columns the MMAs of k-tile kt may still read.
+  static constexpr int SF_COLS = 16 + 4 * (BN / 32);   // SFA: 4 MMAs x 4 columns; SFB: 4 MMAs x BN/32
+  static constexpr int SFA_COL = ACC_COLS;
+  static constexpr int SFB_COL = ACC_COLS + 16;
   static constexpr int TMEM_COLS = 512;
-  static_assert(SFB_COL + 4 * (BN / 32) <= TMEM_COLS, "TMEM budget");
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 1024 + 4 * (kMaxExperts + 1);
+  static_assert(ACC_COLS + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static constexpr int STAGING_BYTES = 4 * 2 * 4096;  // 4 epilogue warps x 2 buffers x (32 rows x 128 B)
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 1024 + 4 * (kMaxExperts + 1);
 };
 
 __device__ __forceinline__ uint64_t now_ns() {
@@ -110,12 +114,13 @@ template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                      const TcParams p) {
+                      const __grid_constant__ CUtensorMap tmY, const TcParams p) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;           // 1024-byte aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::STAGING_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + C::NUM_ACC;
@@ -143,7 +148,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     for (int s = 0; s < C::STAGES; ++s) { ptx::mbar_init(full + s, 1); ptx::mbar_init(empty + s, 1); }
     for (int a = 0; a < C::NUM_ACC; ++a) { ptx::mbar_init(acc_full + a, 1); ptx::mbar_init(acc_empty + a, 128); }
     ptx::fence_mbar_init();
-    ptx::prefetch_tensormap(&tmA); ptx::prefetch_tensormap(&tmB);
+    ptx::prefetch_tensormap(&tmA); ptx::prefetch_tensormap(&tmB); ptx::prefetch_tensormap(&tmY);
     if (p.ST > 0) { ptx::prefetch_tensormap(&tmSA); ptx::prefetch_tensormap(&tmSB); }
   }
   if (warp == 1) {
@@ -205,18 +210,19 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           if (kt < p.KT) {
             const uint32_t sfa = ptx::smem_u32(SFA_at(stage));
             const uint32_t sfb = ptx::smem_u32(SFB_at(stage));
+            const uint32_t sf_off = (kt & 1) * C::SF_COLS;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              ptx::tc_cp_32x128b_warpx4(tmem + C::SFA_COL + 4 * j, ptx::desc_sf_block(sfa + 512 * j));
+              ptx::tc_cp_32x128b_warpx4(tmem + C::SFA_COL + sf_off + 4 * j, ptx::desc_sf_block(sfa + 512 * j));
 #pragma unroll
               for (int rg = 0; rg < BN / 128; ++rg)
-                ptx::tc_cp_32x128b_warpx4(tmem + C::SFB_COL + (BN / 32) * j + 4 * rg,
+                ptx::tc_cp_32x128b_warpx4(tmem + C::SFB_COL + sf_off + (BN / 32) * j + 4 * rg,
                                           ptx::desc_sf_block(sfb + 2048 * rg + 512 * j));
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              ptx::tc_mma_nvf4(d, adesc + 2 * j, bdesc + 2 * j, idesc_f4, tmem + C::SFA_COL + 4 * j,
-                               tmem + C::SFB_COL + (BN / 32) * j, (kt | j) != 0);
+              ptx::tc_mma_nvf4(d, adesc + 2 * j, bdesc + 2 * j, idesc_f4, tmem + C::SFA_COL + sf_off + 4 * j,
+                               tmem + C::SFB_COL + sf_off + (BN / 32) * j, (kt | j) != 0);
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) ptx::tc_mma_bf16(d, adesc + 2 * j, bdesc + 2 * j, idesc_bf, 1u);
@@ -231,15 +237,22 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     }
   } else {
     // ------------------------------------------------------------------ epilogue
+    // TMEM -> registers (x alpha) -> swizzled staging in shared memory -> TMA store of a
+    // 32-row x 32-column box per warp; the accumulator is released right after the last TMEM
+    // load, so the next tile's MMAs overlap the stores.  Partial tiles of an expert (rows that
+    // end inside the output) use direct stores instead, since a box would cross into the next
+    // expert's rows.
     const int quad = warp & 3;                  // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;           // row of the tile held by this thread
-    int acc = 0;
+    uint8_t* stage_buf = staging + quad * 2 * 4096;
+    int acc = 0, nbuf = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       const TileMap m = map_tile(t, p, cum_m);
       if (!wait_bar(acc_full + acc, acc_phase, abort_flag, p.err)) break;
       ptx::tc_fence_after();
       const float alpha = __ldg(p.alpha + m.e);
+      const bool use_tma = !(p.offsets && m.rows < kBM);
       const bool row_ok = row < m.rows;
       const int64_t yrow = m.yrow + row;
 #pragma unroll 1
@@ -247,47 +260,60 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         uint32_t r[32];
         ptx::tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + c * 32, r);
         ptx::tmem_ld_wait();
+        if (c == BN / 32 - 1) {
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(acc_empty + acc);
+        }
         const int col0 = m.n0 + c * 32;
-        if (row_ok && col0 < p.N) {
+        if (col0 >= p.N) continue;
+        if (use_tma) {
+          if (quad * 32 >= m.rows) continue;            // this warp's rows are all past the end
+          uint8_t* buf = stage_buf + (nbuf & 1) * 4096;
+          if (lane == 0) ptx::bulk_wait_read<1>();       // the store issued two chunks ago has read `buf`
+          __syncwarp();
           if (p.out_bf16) {
-            uint16_t* y = static_cast<uint16_t*>(p.Y) + yrow * p.ldy + col0;
-            if (col0 + 32 <= p.N) {
+            // 32 rows x 64 bytes, 64-byte swizzle: 16-byte chunk j of row r sits at j ^ ((r >> 1) & 3)
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                uint32_t w[4];
+            for (int j = 0; j < 4; ++j) {
+              uint32_t w[4];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  const float a0 = __uint_as_float(r[8 * v + 2 * h]) * alpha;
-                  const float a1 = __uint_as_float(r[8 * v + 2 * h + 1]) * alpha;
-                  w[h] = static_cast<uint32_t>(f32_to_bf16_bits(a0)) | (static_cast<uint32_t>(f32_to_bf16_bits(a1)) << 16);
-                }
-                *reinterpret_cast<uint4*>(y + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (col0 + i < p.N) y[i] = f32_to_bf16_bits(__uint_as_float(r[i]) * alpha);
+              for (int h = 0; h < 4; ++h)
+                w[h] = static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[8 * j + 2 * h]) * alpha)) |
+                       (static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[8 * j + 2 * h + 1]) * alpha)) << 16);
+              *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
             }
           } else {
+            // 32 rows x 128 bytes, 128-byte swizzle: 16-byte chunk j of row r sits at j ^ (r & 7)
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_float4(__uint_as_float(r[4 * j]) * alpha, __uint_as_float(r[4 * j + 1]) * alpha,
+                              __uint_as_float(r[4 * j + 2]) * alpha, __uint_as_float(r[4 * j + 3]) * alpha);
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_store_2d(&tmY, col0, static_cast<int32_t>(m.yrow + quad * 32), buf);
+            ptx::bulk_commit();
+          }
+          ++nbuf;
+        } else if (row_ok) {
+          if (p.out_bf16) {
+            uint16_t* y = static_cast<uint16_t*>(p.Y) + yrow * p.ldy + col0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col0 + i < p.N) y[i] = f32_to_bf16_bits(__uint_as_float(r[i]) * alpha);
+          } else {
             float* y = static_cast<float*>(p.Y) + yrow * p.ldy + col0;
-            if (col0 + 32 <= p.N) {
 #pragma unroll
-              for (int v = 0; v < 8; ++v)
-                *reinterpret_cast<float4*>(y + 4 * v) =
-                    make_float4(__uint_as_float(r[4 * v]) * alpha, __uint_as_float(r[4 * v + 1]) * alpha,
-                                __uint_as_float(r[4 * v + 2]) * alpha, __uint_as_float(r[4 * v + 3]) * alpha);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (col0 + i < p.N) y[i] = __uint_as_float(r[i]) * alpha;
-            }
+            for (int i = 0; i < 32; ++i)
+              if (col0 + i < p.N) y[i] = __uint_as_float(r[i]) * alpha;
           }
         }
       }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(acc_empty + acc);
       if (++acc == C::NUM_ACC) { acc = 0; acc_phase ^= 1; }
     }
+    if (lane == 0) ptx::bulk_wait_all();
   }
 
   ptx::tc_fence_before();
@@ -364,8 +390,22 @@ fs_status launch_bn(const TcLaunch& L, TcParams prm, cudaStream_t s) {
     tmSA = tmA;
     tmSB = tmB;
   }
+  CUtensorMap tmY;
+  {
+    auto fn = encode_fn();
+    const int esz = prm.out_bf16 ? 2 : 4;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(prm.N), static_cast<cuuint64_t>(L.y_rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(prm.ldy) * esz};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&tmY, prm.out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, prm.Y,
+                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    prm.out_bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FS_ERR_CUDA, "cuTensorMapEncodeTiled (Y) failed (%d)", static_cast<int>(r));
+  }
   const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(L.max_tiles, 1), sm_count()));
-  splice_gemm_tc_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, s>>>(tmA, tmB, tmSA, tmSB, prm);
+  splice_gemm_tc_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, s>>>(tmA, tmB, tmSA, tmSB, tmY, prm);
   FS_CHECK_LAUNCH("fs_splice_gemm (tensor-core path)");
   return FS_OK;
 }

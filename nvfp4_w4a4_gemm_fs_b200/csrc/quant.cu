@@ -57,146 +57,222 @@ __device__ __forceinline__ void load_block(const T* src, float (&x)[16]) {
   }
 }
 
-// One CTA covers `rows_per_cta` consecutive packed rows, all inside one expert's padded region.
+// Raw 16-element block as loaded: bf16 pairs packed in 8 words (widened on use) or 16 floats.
+template <typename T>
+struct RawBlock {
+  static constexpr int kWords = sizeof(T) == 2 ? 8 : 16;
+  uint32_t w[kWords];
+  __device__ __forceinline__ float get(int j) const {
+    if constexpr (sizeof(T) == 2) return (j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]);
+    else return __uint_as_float(w[j]);
+  }
+  // The block with the lanes whose bit is set in `mbits` replaced by +0.
+  __device__ __forceinline__ RawBlock masked(uint32_t mbits) const {
+    RawBlock m;
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t two = (mbits >> (2 * j)) & 3u;                        // lanes 2j, 2j+1
+        const uint32_t kill = ((two & 1u) | ((two & 2u) << 15)) * 0xFFFFu;   // 16-bit fields to clear
+        m.w[j] = w[j] & ~kill;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) m.w[j] = ((mbits >> j) & 1u) ? 0u : w[j];
+    }
+    return m;
+  }
+};
+
+template <typename T>
+__device__ __forceinline__ void load_raw(const T* src, RawBlock<T>& x) {
+  const uint4* p = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int v = 0; v < RawBlock<T>::kWords / 4; ++v) {
+    const uint4 q = __ldg(p + v);
+    x.w[4 * v] = q.x; x.w[4 * v + 1] = q.y; x.w[4 * v + 2] = q.z; x.w[4 * v + 3] = q.w;
+  }
+}
+
+constexpr int kMaxGroupedExperts = 256;
+
+// Where a chunk of `rows_per_cta` packed rows lives: its expert, first source row and how many
+// of its rows carry data (the rest are padding of the expert's 128-row-aligned region).
+struct ChunkLoc {
+  int e;              // -1: past the last expert (or past the padded rows)
+  int64_t prow0;      // first packed row
+  int64_t src_row0;   // first source row of X
+  int64_t valid;      // rows of the chunk with data (may be <= 0)
+};
+
+// Persistent CTAs loop over chunks of `rows_per_cta` packed rows; a chunk never straddles an
+// expert's padded region (rows_per_cta divides 128).  Each thread owns one 16-element block per
+// pass; the load of the next pass (or of the next chunk) is issued before the current block is
+// computed, so every thread keeps a load in flight.  Divisions by the UE4M3 scale use per-code
+// tables of the scale value and its reciprocal in shared memory.
 template <typename T, Side kSide, bool kGrouped>
-__global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a) {
-  __shared__ int sh_prefix[16384 / 32 + 1];       // protected channels before each mask word
-  __shared__ int sh_expert;
-  __shared__ int64_t sh_src_row0, sh_valid;        // source row of the CTA's first row, valid rows
+__global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_t nchunks) {
+  __shared__ int sh_prefix[16384 / 32 + 1];             // protected channels before each mask word
+  __shared__ float sh_val[128], sh_rcp[128];            // UE4M3 value and RN(1/value) per code
+  __shared__ int64_t sh_pad[kGrouped ? kMaxGroupedExperts + 1 : 1];   // padded start of each expert
+  __shared__ int64_t sh_off[kGrouped ? kMaxGroupedExperts + 1 : 1];   // row offsets of the experts
 
   const int tid = threadIdx.x;
-  const int64_t prow0 = static_cast<int64_t>(blockIdx.x) * a.rows_per_cta;   // first packed row
-
-  // ---- locate the expert and the source rows -------------------------------------------
+  if (tid < 128) {
+    // code 0 (zero scale) and the unused NaN code: d = 1, r = 0 gives +-0 with the sign of x
+    const bool real = tid > 0 && tid < 127;
+    const float d = real ? ue4m3_value(tid) : 1.0f;
+    sh_val[tid] = d;
+    sh_rcp[tid] = real ? __frcp_rn(d) : 0.0f;
+  }
   if constexpr (kGrouped) {
     if (tid == 0) {
-      int64_t pad = 0;
-      int e = -1;
-      int64_t src0 = 0, valid = 0;
+      sh_pad[0] = 0;
       for (int i = 0; i < a.E; ++i) {
-        const int64_t r0 = a.offsets[i], r1 = a.offsets[i + 1];
-        const int64_t span = ((r1 - r0) + 127) / 128 * 128;
-        if (prow0 < pad + span) {
-          e = i;
-          const int64_t local = prow0 - pad;
-          src0 = r0 + local;
-          valid = (r1 - r0) - local;
-          break;
-        }
-        pad += span;
+        sh_off[i] = a.offsets[i];
+        sh_pad[i + 1] = sh_pad[i] + (a.offsets[i + 1] - a.offsets[i] + 127) / 128 * 128;
       }
-      sh_expert = e;
-      sh_src_row0 = src0;
-      sh_valid = valid;
+      sh_off[a.E] = a.offsets[a.E];
     }
-    __syncthreads();
-    if (sh_expert < 0) return;                 // beyond the last expert's padded region
-  } else {
-    if (tid == 0) {
-      sh_expert = 0;
-      sh_src_row0 = prow0;
-      sh_valid = a.rows - prow0;
-    }
-    __syncthreads();
   }
-  const int e = sh_expert;
-  const int64_t src_row0 = sh_src_row0;
-  const int64_t valid = sh_valid;               // rows of this CTA with data (may be <= 0)
+  __syncthreads();
+  auto locate = [&](int64_t chunk) {
+    ChunkLoc L;
+    L.prow0 = chunk * a.rows_per_cta;
+    if (chunk >= nchunks) { L.e = -1; L.src_row0 = 0; L.valid = 0; return L; }
+    if constexpr (kGrouped) {
+      if (L.prow0 >= sh_pad[a.E]) { L.e = -1; L.src_row0 = 0; L.valid = 0; return L; }
+      int lo = 0, hi = a.E - 1;                   // expert with pad[e] <= prow0 < pad[e+1]
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sh_pad[mid] <= L.prow0) lo = mid; else hi = mid - 1;
+      }
+      L.e = lo;
+      const int64_t local = L.prow0 - sh_pad[lo];
+      L.src_row0 = sh_off[lo] + local;
+      L.valid = (sh_off[lo + 1] - sh_off[lo]) - local;
+    } else {
+      L.e = 0;
+      L.src_row0 = L.prow0;
+      L.valid = a.rows - L.prow0;
+    }
+    return L;
+  };
+
   const int words = a.K / 32;
-  const uint32_t* mask = (a.p > 0) ? a.masks + static_cast<int64_t>(e) * words : nullptr;
-
-  // ---- protected-channel prefix counts per mask word (for the X_S column of a lane) -----
-  if (a.p > 0) {
-    if (tid < 32) {
-      int carry = 0;
-      for (int w0 = 0; w0 < words; w0 += 32) {
-        const int w = w0 + tid;
-        const int c = (w < words) ? __popc(__ldg(mask + w)) : 0;
-        int incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (tid >= o) incl += y;
-        }
-        if (w < words) sh_prefix[w] = carry + incl - c;
-        carry += __shfl_sync(0xffffffffu, incl, 31);
-      }
-    }
-    __syncthreads();
-  }
-
-  const float g = __ldg(a.gains + e);
-  float alpha_v = 0.0f;
-  if constexpr (kSide == Side::Weight) alpha_v = __ldg(a.alpha);
   const bool residual = a.opts & FS_RESIDUAL;
   const T* X = static_cast<const T*>(a.X);
-  const int total = a.rows_per_cta * a.nb;
+  const int total = a.rows_per_cta * a.nb;            // blocks per chunk
+  float alpha_v = 0.0f;
+  if constexpr (kSide == Side::Weight) alpha_v = __ldg(a.alpha);
+  const float inv6 = __frcp_rn(6.0f);
 
-  for (int i0 = 0; i0 < total; i0 += kQThreads) {
+  const bool one_row = a.rows_per_cta == 1;
+  auto load_one = [&](const ChunkLoc& L, int i0, RawBlock<T>& x) {
     const int i = i0 + tid;
-    const bool in_range = i < total;
-    const int r = in_range ? i / a.nb : 0;
-    const int b = in_range ? i % a.nb : 0;
-    const int64_t prow = prow0 + r;
-    const bool has_data = in_range && r < valid;
-    uint32_t sfc = 0;
-    if (has_data) {
-      const int64_t srow = src_row0 + r;
-      float x[16];
-      load_block<T>(X + srow * a.ldx + static_cast<int64_t>(b) * 16, x);
-      const uint32_t mbits = mask ? ((__ldg(mask + (b >> 1)) >> ((b & 1) * 16)) & 0xFFFFu) : 0u;
-      float amax = 0.0f;
+    const int r = one_row ? 0 : i / a.nb;
+    if (L.e >= 0 && i < total && r < L.valid) {
+      const int b = one_row ? i : i % a.nb;
+      load_raw<T>(X + (L.src_row0 + r) * a.ldx + static_cast<int64_t>(b) * 16, x);
+    }
+  };
+
+  ChunkLoc L = locate(blockIdx.x);
+  RawBlock<T> xc;
+  load_one(L, 0, xc);
+  int cur_e = -1;
+  const uint32_t* mask = nullptr;
+  float g = 1.0f;
+
+  for (int64_t chunk = blockIdx.x; chunk < nchunks && L.e >= 0; chunk += gridDim.x) {
+    if (L.e != cur_e) {                            // uniform across the CTA
+      cur_e = L.e;
+      mask = (a.p > 0) ? a.masks + static_cast<int64_t>(cur_e) * words : nullptr;
+      g = __ldg(a.gains + cur_e);
+      if (a.p > 0) {
+        __syncthreads();                           // previous expert's prefix no longer read
+        if (tid < 32) {
+          int carry = 0;
+          for (int w0 = 0; w0 < words; w0 += 32) {
+            const int w = w0 + tid;
+            const int c = (w < words) ? __popc(__ldg(mask + w)) : 0;
+            int incl = c;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const bool prot = (mbits >> j) & 1u;
-        if (residual || !prot) amax = fmaxf(amax, fabsf(x[j]));
-      }
-      const float t = div_small_divisor(__fmul_rn(amax, g), kInvSix);
-      sfc = ue4m3_rne(t);
-      const double inv = sfc ? __drcp_rn(static_cast<double>(ue4m3_value(sfc))) : 0.0;
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int j = 0; j < 16; j += 2) {
-        const float x0 = ((mbits >> j) & 1u) ? 0.0f : x[j];
-        const float x1 = ((mbits >> (j + 1)) & 1u) ? 0.0f : x[j + 1];
-        const float v0 = div_small_divisor(__fmul_rn(x0, g), inv);
-        const float v1 = div_small_divisor(__fmul_rn(x1, g), inv);
-        const uint32_t byte = e2m1x2(v0, v1);
-        if (j < 8) lo |= byte << (j * 4); else hi |= byte << ((j - 8) * 4);
-      }
-      *reinterpret_cast<uint2*>(a.q + prow * (a.K / 2) + static_cast<int64_t>(b) * 8) = make_uint2(lo, hi);
-      // Extract the protected lanes into the side buffer.
-      if (mbits) {
-        int col = sh_prefix[b >> 1] + ((b & 1) ? __popc(__ldg(mask + (b >> 1)) & 0xFFFFu) : 0);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          if ((mbits >> j) & 1u) {
-            uint16_t h;
-            if constexpr (kSide == Side::Activation) {
-              h = f32_to_bf16_bits(x[j]);
-            } else {
-              const float wb = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_bits(x[j])) << 16);
-              h = f32_to_bf16_bits(__fdiv_rn(wb, alpha_v));
+            for (int o = 1; o < 32; o <<= 1) {
+              const int y = __shfl_up_sync(0xffffffffu, incl, o);
+              if (tid >= o) incl += y;
             }
-            a.side[prow * a.pp + col] = h;
-            ++col;
+            if (w < words) sh_prefix[w] = carry + incl - c;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
           }
         }
+        __syncthreads();
       }
-      if (b == 0)
-        for (int c = a.p; c < a.pp; ++c) a.side[prow * a.pp + c] = 0;
-    } else if (in_range && kGrouped) {
-      // padding rows of a grouped buffer: zero codes and side columns
-      *reinterpret_cast<uint2*>(a.q + prow * (a.K / 2) + static_cast<int64_t>(b) * 8) = make_uint2(0, 0);
-      if (b == 0)
-        for (int c = 0; c < a.pp; ++c) a.side[prow * a.pp + c] = 0;
     }
-    // Gather the 4 scales of blocks b..b+3 (same row since K/16 % 4 == 0) into one word.
-    const uint32_t s1 = __shfl_down_sync(0xffffffffu, sfc, 1);
-    const uint32_t s2 = __shfl_down_sync(0xffffffffu, sfc, 2);
-    const uint32_t s3 = __shfl_down_sync(0xffffffffu, sfc, 3);
-    if (in_range && (b & 3) == 0)
-      *reinterpret_cast<uint32_t*>(a.sf + sf_offset(prow, b, a.kb4)) = sfc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    const ChunkLoc Ln = locate(chunk + gridDim.x);
+    for (int i0 = 0; i0 < total; i0 += kQThreads) {
+      RawBlock<T> xn;
+      if (i0 + kQThreads < total) load_one(L, i0 + kQThreads, xn);   // prefetch the next pass
+      else load_one(Ln, 0, xn);                                       // or the next chunk's first
+      const RawBlock<T>& x = xc;
+      const int i = i0 + tid;
+      const bool in_range = i < total;
+      const int r = (!in_range || one_row) ? 0 : i / a.nb;
+      const int b = !in_range ? 0 : (one_row ? i : i % a.nb);
+      const int64_t prow = L.prow0 + r;
+      const bool has_data = in_range && r < L.valid;
+      uint32_t sfc = 0;
+      if (has_data) {
+        const uint32_t mbits = mask ? ((__ldg(mask + (b >> 1)) >> ((b & 1) * 16)) & 0xFFFFu) : 0u;
+        const RawBlock<T> xm = mbits ? x.masked(mbits) : x;
+        const RawBlock<T>& xs = residual ? x : xm;    // lanes that set the block scale
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xs.get(j)));
+        const float t = div_markstein(__fmul_rn(amax, g), 6.0f, inv6);
+        sfc = ue4m3_rne(t);
+        const float sd = sh_val[sfc], sr = sh_rcp[sfc];
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = div_markstein(__fmul_rn(xm.get(j), g), sd, sr);
+        const uint32_t lo = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+        const uint32_t hi = e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+        *reinterpret_cast<uint2*>(a.q + prow * (a.K / 2) + static_cast<int64_t>(b) * 8) = make_uint2(lo, hi);
+        // Extract the protected lanes into the side buffer.
+        if (mbits) {
+          int col = sh_prefix[b >> 1] + ((b & 1) ? __popc(__ldg(mask + (b >> 1)) & 0xFFFFu) : 0);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if ((mbits >> j) & 1u) {
+              uint16_t hv;
+              if constexpr (kSide == Side::Activation) {
+                hv = f32_to_bf16_bits(x.get(j));
+              } else {
+                const float wb = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_bits(x.get(j))) << 16);
+                hv = f32_to_bf16_bits(__fdiv_rn(wb, alpha_v));
+              }
+              a.side[prow * a.pp + col] = hv;
+              ++col;
+            }
+          }
+        }
+        if (b == 0)
+          for (int c = a.p; c < a.pp; ++c) a.side[prow * a.pp + c] = 0;
+      } else if (in_range && kGrouped) {
+        // padding rows of a grouped buffer: zero codes and side columns
+        *reinterpret_cast<uint2*>(a.q + prow * (a.K / 2) + static_cast<int64_t>(b) * 8) = make_uint2(0, 0);
+        if (b == 0)
+          for (int c = 0; c < a.pp; ++c) a.side[prow * a.pp + c] = 0;
+      }
+      // Gather the 4 scales of blocks b..b+3 (same row since K/16 % 4 == 0) into one word.
+      const uint32_t s1 = __shfl_down_sync(0xffffffffu, sfc, 1);
+      const uint32_t s2 = __shfl_down_sync(0xffffffffu, sfc, 2);
+      const uint32_t s3 = __shfl_down_sync(0xffffffffu, sfc, 3);
+      if (in_range && (b & 3) == 0)
+        *reinterpret_cast<uint32_t*>(a.sf + sf_offset(prow, b, a.kb4)) = sfc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      xc = xn;
+    }
+    L = Ln;
   }
 }
 
@@ -233,19 +309,30 @@ __global__ void weight_gain_kernel(float* gW, float* alpha, const float* gA, uin
   *alpha = __fdiv_rn(1.0f, __fmul_rn(*gA, g));
 }
 
+int quant_sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 template <Side kSide, bool kGrouped>
 fs_status launch_quantize(int dtype, QuantArgs& a, int64_t padded_rows, cudaStream_t s) {
-  // rows per CTA: a power of two dividing 128, so a CTA never straddles a 128-row tile
+  // rows per chunk: a power of two dividing 128, so a chunk never straddles a 128-row tile
   int rpc = 1;
   while (rpc < 128 && rpc * a.nb < kQThreads) rpc *= 2;
   a.rows_per_cta = rpc;
-  const int64_t ctas = ceil_div(padded_rows, rpc);
-  if (ctas == 0) return FS_OK;
-  if (ctas > 0x7FFFFFFF) return fail(FS_ERR_UNSUPPORTED, "too many rows");
-  if (dtype == FS_DTYPE_BF16)
-    quantize_kernel<uint16_t, kSide, kGrouped><<<static_cast<unsigned>(ctas), kQThreads, 0, s>>>(a);
-  else
-    quantize_kernel<float, kSide, kGrouped><<<static_cast<unsigned>(ctas), kQThreads, 0, s>>>(a);
+  const int64_t chunks = ceil_div(padded_rows, rpc);
+  if (chunks == 0) return FS_OK;
+  auto kernel = dtype == FS_DTYPE_BF16 ? quantize_kernel<uint16_t, kSide, kGrouped> : quantize_kernel<float, kSide, kGrouped>;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQThreads, 0) != cudaSuccess || per_sm < 1) per_sm = 2;
+  const int64_t grid = std::min<int64_t>(chunks, static_cast<int64_t>(quant_sm_count()) * per_sm);
+  kernel<<<static_cast<unsigned>(grid), kQThreads, 0, s>>>(a, chunks);
   FS_CHECK_LAUNCH("quantize kernel");
   return FS_OK;
 }
@@ -287,7 +374,8 @@ extern "C" fs_status fs_quantize_splice_grouped(const void* X, int32_t dtype, in
                                                 int64_t max_rows, int32_t K, int64_t ldx, const uint32_t* masks,
                                                 int32_t p, const float* gA, uint32_t opts, uint8_t* xq,
                                                 uint8_t* sfx, uint16_t* xs, void* stream) {
-  if (E <= 0 || E > 1024 || max_rows < 0 || !row_offsets) return fail(FS_ERR_INVALID_ARGUMENT, "fs_quantize_splice_grouped: need 0 < E <= 1024, max_rows >= 0, row_offsets");
+  if (E <= 0 || E > kMaxGroupedExperts || max_rows < 0 || !row_offsets)
+    return fail(FS_ERR_INVALID_ARGUMENT, "fs_quantize_splice_grouped: need 0 < E <= %d, max_rows >= 0, row_offsets", kMaxGroupedExperts);
   if (max_rows == 0) return FS_OK;
   fs_status st = check_common("fs_quantize_splice_grouped", dtype, K, ldx, X, p, masks, gA, xq, sfx, xs);
   if (st != FS_OK) return st;

@@ -15,94 +15,150 @@ namespace {
 constexpr int kStatsWarps = 8;
 constexpr double kS1Scale = 65536.0;
 constexpr double kS2Scale = 16384.0;
-constexpr float kRangeLimit = 65536.0f;
+constexpr float kRangeLimit = 32768.0f;
 
-struct ChanAcc {
-  long long s1, s2;
+// Exact integer moments without 64-bit conversions, branch-free, for |x| < 2^15.
+//
+// Magic rounding: for |t| < 2^22, fl32(t + 1.5*2^23) lies in [2^23, 2^24) where the float spacing
+// is 1, so the addition rounds t to the nearest integer (ties to even) and the integer is the
+// bit pattern minus that of 1.5*2^23; with 1.5*2^31 the spacing is 2^8 and the addition rounds to
+// a multiple of 2^8 for |t| < 2^30.
+//   s1 term rint(x*2^16) = rint(x)*2^16 + rint((x - rint(x))*2^16)   (rint(x)*2^16 is even, so
+//     the split keeps ties-to-even; |x - rint(x)| <= 1/2 and both parts are exact in fp32);
+//   s2 term rint(y*2^14), y = x^2 (exact for bf16 x, y < 2^30) = yh*2^14 + rint(yl*2^14) with
+//     yh the multiple of 2^8 nearest y and yl = y - yh, |yl| <= 2^7 (yh*2^14 is a multiple of
+//     2^22, so again the split keeps ties-to-even).
+// The raw bit patterns are summed in wrapping 32-bit registers for a few rows; subtracting
+// count * magic-bits recovers the exact small sums, which are then added to 64-bit totals.
+constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23
+constexpr float kMagic8 = 3221225472.0f;       // 1.5 * 2^31 (rounds to multiples of 2^8)
+constexpr uint32_t kMagicBits = 0x4B400000u;
+constexpr uint32_t kMagic8Bits = 0x4F400000u;
+
+struct SmallSums {
+  uint32_t a1, b1, c2, d2;   // raw-bit sums: rint(x), rint(frac*2^16), yh/2^8, rint(yl*2^14)
   float amax;
-  bool bad;
 };
 
-__device__ __forceinline__ void add_value(ChanAcc& a, float x, bool f32_input) {
+__device__ __forceinline__ void add_bf16(SmallSums& a, float x, bool& bad) {
   const float ax = fabsf(x);
-  if (!(ax < kRangeLimit)) {     // also catches NaN
-    a.bad = true;
-    return;
-  }
-  a.amax = fmaxf(a.amax, ax);
-  a.s1 += __float2ll_rn(x * 65536.0f);               // exact scaling, round half even
-  if (f32_input) {
-    const double xd = static_cast<double>(x);
-    a.s2 += __double2ll_rn(__dmul_rn(__dmul_rn(xd, xd), kS2Scale));
-  } else {
-    a.s2 += __float2ll_rn(__fmul_rn(x, x) * 16384.0f);   // bf16 x: x^2 exact in fp32
-  }
+  const bool ok = ax < kRangeLimit;              // false for NaN too
+  bad |= !ok;
+  x = ok ? x : 0.0f;
+  a.amax = fmaxf(a.amax, ok ? ax : 0.0f);
+  const float t1 = __fadd_rn(x, kMagic);
+  a.a1 += __float_as_uint(t1);
+  const float frac = __fsub_rn(x, __fsub_rn(t1, kMagic));
+  a.b1 += __float_as_uint(__fmaf_rn(frac, 65536.0f, kMagic));
+  const float y = __fmul_rn(x, x);
+  const float u = __fadd_rn(y, kMagic8);
+  a.c2 += __float_as_uint(u);
+  const float yl = __fsub_rn(y, __fsub_rn(u, kMagic8));
+  a.d2 += __float_as_uint(__fmaf_rn(yl, 16384.0f, kMagic));
 }
 
-// Grid: x = channel chunks (a warp-width of channels each), y = row groups.
-// Block: kStatsWarps warps; warp w takes rows (blockIdx.y*W + w) * stride + i*gridDim.y*W*stride.
-// Lane l holds VEC consecutive channels.  Per-CTA partial sums are reduced across warps in
-// shared memory and added to the global state with integer atomics.
+// fp32 inputs (small problems): convert directly.
+__device__ __forceinline__ void add_f32(long long& s1, long long& s2, float& amax, float x, bool& bad) {
+  const float ax = fabsf(x);
+  if (!(ax < kRangeLimit)) {
+    bad = true;
+    return;
+  }
+  amax = fmaxf(amax, ax);
+  s1 += __float2ll_rn(x * 65536.0f);
+  const double xd = static_cast<double>(x);
+  s2 += __double2ll_rn(__dmul_rn(__dmul_rn(xd, xd), kS2Scale));
+}
+
+// Grid: x = channel chunks (32*VEC channels), y = row groups.  Block: kStatsWarps warps; warp w
+// takes rows (blockIdx.y*W + w) + i*gridDim.y*W of the subsampled rows, kUnroll rows per pass
+// with all loads issued first.  Lane l holds VEC consecutive channels.  Each thread keeps its
+// 64-bit totals in its own shared-memory slots ([warp][v][lane], conflict-free); the CTA reduces
+// them over warps and adds to the global state with integer atomics.
 template <typename T, int VEC>
 __global__ void __launch_bounds__(kStatsWarps * 32)
 channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int row_stride,
                      unsigned long long* n, unsigned long long* s1, unsigned long long* s2,
                      uint32_t* amax, uint32_t* flags) {
   constexpr bool kF32 = sizeof(T) == 4;
-  __shared__ long long sh_s1[kStatsWarps][32 * VEC];
-  __shared__ long long sh_s2[kStatsWarps][32 * VEC];
-  __shared__ float sh_am[kStatsWarps][32 * VEC];
+  constexpr int kUnroll = 4;
+  __shared__ long long sh_s1[kStatsWarps][VEC][32];
+  __shared__ long long sh_s2[kStatsWarps][VEC][32];
+  __shared__ float sh_am[kStatsWarps][VEC][32];
   __shared__ int sh_bad;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c0 = blockIdx.x * 32 * VEC + lane * VEC;
   const bool active = c0 < K;
   if (threadIdx.x == 0) sh_bad = 0;
-
-  ChanAcc acc[VEC];
 #pragma unroll
-  for (int v = 0; v < VEC; ++v) acc[v] = ChanAcc{0, 0, 0.0f, false};
+  for (int v = 0; v < VEC; ++v) { sh_s1[warp][v][lane] = 0; sh_s2[warp][v][lane] = 0; }
+  bool bad = false;
+  float am[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) am[v] = 0.0f;
 
   const int64_t taken = (M + row_stride - 1) / row_stride;     // rows 0, s, 2s, ...
   const int64_t step = static_cast<int64_t>(gridDim.y) * kStatsWarps;
   if (active) {
-    for (int64_t i = static_cast<int64_t>(blockIdx.y) * kStatsWarps + warp; i < taken; i += step) {
-      const T* row = X + i * row_stride * ldx + c0;
-      if constexpr (kF32) {
-        const float4 q = __ldg(reinterpret_cast<const float4*>(row));
-        add_value(acc[0], q.x, true); add_value(acc[1], q.y, true);
-        add_value(acc[2], q.z, true); add_value(acc[3], q.w, true);
-      } else {
-        const uint4 q = __ldg(reinterpret_cast<const uint4*>(row));
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    for (int64_t i = static_cast<int64_t>(blockIdx.y) * kStatsWarps + warp; i < taken; i += kUnroll * step) {
+      uint4 q[kUnroll];
+      int rows = 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          add_value(acc[2 * j], bf16_lo(w[j]), false);
-          add_value(acc[2 * j + 1], bf16_hi(w[j]), false);
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t idx = i + u * step;
+        if (idx < taken) {
+          q[u] = __ldg(reinterpret_cast<const uint4*>(X + idx * row_stride * ldx + c0));
+          ++rows;
+        } else {
+          q[u] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if constexpr (kF32) {
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          if (u >= rows) break;
+          const float xs[4] = {__uint_as_float(q[u].x), __uint_as_float(q[u].y), __uint_as_float(q[u].z), __uint_as_float(q[u].w)};
+#pragma unroll
+          for (int v = 0; v < 4; ++v) add_f32(sh_s1[warp][v][lane], sh_s2[warp][v][lane], am[v], xs[v], bad);
+        }
+      } else {
+        // zero rows past the end contribute rint(0) = 0 (their raw bits are the magic patterns,
+        // removed below with the count of kUnroll rows)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          SmallSums a{0u, 0u, 0u, 0u, am[v]};
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) {
+            const uint32_t w = (&q[u].x)[v >> 1];
+            add_bf16(a, (v & 1) ? bf16_hi(w) : bf16_lo(w), bad);
+          }
+          am[v] = a.amax;
+          const int A1 = static_cast<int>(a.a1 - kUnroll * kMagicBits);
+          const int B1 = static_cast<int>(a.b1 - kUnroll * kMagicBits);
+          const int C2 = static_cast<int>(a.c2 - kUnroll * kMagic8Bits);
+          const int D2 = static_cast<int>(a.d2 - kUnroll * kMagicBits);
+          sh_s1[warp][v][lane] += static_cast<long long>(A1) * 65536 + B1;
+          sh_s2[warp][v][lane] += static_cast<long long>(C2) * 4194304 + D2;   // yh*2^14 = (yh/2^8)*2^22
         }
       }
     }
   }
-  bool bad = false;
 #pragma unroll
-  for (int v = 0; v < VEC; ++v) {
-    sh_s1[warp][lane * VEC + v] = acc[v].s1;
-    sh_s2[warp][lane * VEC + v] = acc[v].s2;
-    sh_am[warp][lane * VEC + v] = acc[v].amax;
-    bad |= acc[v].bad;
-  }
+  for (int v = 0; v < VEC; ++v) sh_am[warp][v][lane] = am[v];
   if (bad) atomicOr(&sh_bad, 1);
   __syncthreads();
   for (int c = threadIdx.x; c < 32 * VEC; c += blockDim.x) {
     const int ch = blockIdx.x * 32 * VEC + c;
     if (ch >= K) continue;
+    const int v = c % VEC, l = c / VEC;
     long long a = 0, b = 0;
     float m = 0.0f;
 #pragma unroll
     for (int w = 0; w < kStatsWarps; ++w) {
-      a += sh_s1[w][c];
-      b += sh_s2[w][c];
-      m = fmaxf(m, sh_am[w][c]);
+      a += sh_s1[w][v][l];
+      b += sh_s2[w][v][l];
+      m = fmaxf(m, sh_am[w][v][l]);
     }
     if (a) atomicAdd(s1 + ch, static_cast<unsigned long long>(a));    // two's complement wraps
     if (b) atomicAdd(s2 + ch, static_cast<unsigned long long>(b));
@@ -162,28 +218,48 @@ select_topk_kernel(int K, long long* n_all, long long* s1_all, long long* s2_all
   if (tid == 0) { sh_prefix = 0; sh_need = p; }
   __syncthreads();
 
-  // Radix select of the p-th largest ordered key, 8 bits at a time from the top.
+  // Radix select of the p-th largest ordered key, 8 bits at a time from the top.  Histogram
+  // updates are aggregated per warp (lanes with the same digit add once), and warp 0 finds the
+  // threshold digit with a suffix scan over 8 bins per lane.
   unsigned long long prefix = 0;
   int need = p;
+  const int lane = tid & 31, warp_id = tid >> 5;
   if (p > 0) {
     for (int shift = 56; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
       __syncthreads();
       const unsigned long long hi_mask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
-      for (int j = tid; j < K; j += blockDim.x) {
-        const unsigned long long k = sh_keys[j];
-        if ((k & hi_mask) == prefix) atomicAdd(&hist[(k >> shift) & 0xFF], 1u);
+      for (int j0 = 0; j0 < K; j0 += blockDim.x) {
+        const int j = j0 + tid;
+        int bin = -1;
+        if (j < K) {
+          const unsigned long long k = sh_keys[j];
+          if ((k & hi_mask) == prefix) bin = static_cast<int>((k >> shift) & 0xFF);
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<unsigned>(__popc(peers)));
       }
       __syncthreads();
-      if (tid == 0) {
-        int rem = need;
-        int d = 255;
-        for (; d > 0; --d) {
-          if (static_cast<int>(hist[d]) >= rem) break;
-          rem -= hist[d];
+      if (warp_id == 0) {
+        int c[8], local = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { c[i] = static_cast<int>(hist[8 * lane + i]); local += c[i]; }
+        int incl = local;                                  // sum over lanes >= this lane
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_down_sync(0xffffffffu, incl, o);
+          if (lane + o < 32) incl += y;
         }
-        sh_prefix = prefix | (static_cast<unsigned long long>(d) << shift);
-        sh_need = rem;
+        const int above = incl - local;
+        if (above < need && need <= incl) {
+          int r = need - above, d = 8 * lane;
+          for (int i = 7; i >= 0; --i) {
+            if (c[i] >= r) { d = 8 * lane + i; break; }
+            r -= c[i];
+          }
+          sh_prefix = prefix | (static_cast<unsigned long long>(d) << shift);
+          sh_need = r;
+        }
       }
       __syncthreads();
       prefix = sh_prefix;
@@ -305,7 +381,7 @@ extern "C" fs_status fs_channel_stats(const void* X, int32_t dtype, int64_t M, i
   const int64_t taken = ceil_div(M, row_stride);
   // Enough CTAs for ~4 per SM, each reading at least 64 rows.
   int64_t gy = ceil_div(148 * 4, chunks);
-  gy = std::min<int64_t>(gy, std::max<int64_t>(1, ceil_div(taken, 64)));
+  gy = std::min<int64_t>(gy, std::max<int64_t>(1, ceil_div(taken, 128)));
   gy = std::min<int64_t>(gy, 65535);
   dim3 grid(chunks, static_cast<unsigned>(gy));
   auto* un = reinterpret_cast<unsigned long long*>(n);

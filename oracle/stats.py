@@ -15,7 +15,8 @@ Readings taken (the paper gives no formula):
   the same for every reduction order; n counts the accumulated rows, taken at
   row indices r = 0, stride, 2*stride, ... of each call;
 * amax is the float32 absolute maximum per channel (kept as its bit pattern);
-* a range flag is raised for |x| >= 2^16 or a non-finite x;
+* a range flag is raised for |x| >= 2^15 or a non-finite x, and such an element
+  contributes nothing to the sums or the maximum;
 * key_j = m2 - m1*m1 with m1 = s1/65536/n, m2 = s2/16384/n in float64, in that
   order (second-moment key: m2); n = 0 gives key 0;
 * top-p by (key descending, index ascending), reported in ascending index order;
@@ -30,7 +31,7 @@ from . import nvfp4
 
 S1_SCALE = 2.0 ** 16
 S2_SCALE = 2.0 ** 14
-RANGE_LIMIT = 2.0 ** 16
+RANGE_LIMIT = 2.0 ** 15
 
 
 def new_state(K: int) -> dict:
@@ -39,22 +40,25 @@ def new_state(K: int) -> dict:
 
 
 def accumulate(state: dict, X, row_stride: int = 1) -> dict:
-    """Add the rows 0, stride, 2*stride, ... of X (float32 [M,K]) to the running moments."""
+    """Add the rows 0, stride, 2*stride, ... of X (float32 [M,K]) to the running moments.
+
+    An element with |x| >= 2^15 or a non-finite one raises the range flag and adds nothing.
+    """
     X = np.asarray(X, dtype=np.float32)
-    rows = X[:: int(row_stride)].astype(np.float64)
-    if rows.size and (not np.all(np.isfinite(rows)) or np.abs(rows).max() >= RANGE_LIMIT):
-        state["flags"] |= 1
+    rows32 = X[:: int(row_stride)]
     with np.errstate(invalid="ignore"):
-        t1 = np.rint(rows * S1_SCALE)
-        t2 = np.rint(rows * rows * S2_SCALE)
-    t1 = np.nan_to_num(t1, nan=0.0, posinf=0.0, neginf=0.0)
-    t2 = np.nan_to_num(t2, nan=0.0, posinf=0.0, neginf=0.0)
-    state["s1"] = state["s1"] + t1.astype(np.int64).sum(axis=0)
-    state["s2"] = state["s2"] + t2.astype(np.int64).sum(axis=0)
+        ok = np.isfinite(rows32) & (np.abs(rows32) < np.float32(RANGE_LIMIT))
+    if not np.all(ok):
+        state["flags"] |= 1
+    rows = np.where(ok, rows32, np.float32(0)).astype(np.float64)
+    t1 = np.rint(rows * S1_SCALE).astype(np.int64)
+    t2 = np.rint(rows * rows * S2_SCALE).astype(np.int64)
+    state["s1"] = state["s1"] + t1.sum(axis=0)
+    state["s2"] = state["s2"] + t2.sum(axis=0)
     state["n"] += rows.shape[0]
     if rows.size:
-        am = np.abs(X[:: int(row_stride)]).max(axis=0)
-        state["amax"] = np.maximum(state["amax"], np.nan_to_num(am, nan=0.0)).astype(np.float32)
+        am = np.abs(rows).max(axis=0).astype(np.float32)
+        state["amax"] = np.maximum(state["amax"], am).astype(np.float32)
     return state
 
 

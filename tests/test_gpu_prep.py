@@ -46,7 +46,7 @@ def test_channel_stats_bit_exact(dtype, M, K, stride):
 
 
 def test_channel_stats_range_flag():
-    x = np.zeros((4, 64), np.float32); x[2, 7] = 70000.0; x[1, 9] = np.nan; x[0, 7] = 3.0
+    x = np.zeros((4, 64), np.float32); x[2, 7] = 40000.0; x[1, 9] = np.nan; x[0, 7] = 3.0; x[3, 11] = 32767.0
     st = F.StatsState(1, 64)
     F.fs_channel_stats(f32_tensor(x), st)
     ref = stats.accumulate(stats.new_state(64), x)
@@ -121,7 +121,12 @@ def test_quantize_splice_bit_exact(dtype, M, K, p, residual):
 def test_quantize_every_scale_code_and_rounding_boundary():
     """Blocks built so that every normal UE4M3 scale is hit and elements sit on E2M1 midpoints +-1 ulp."""
     mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.0, 6.5, 0.1, 0.0], np.float32)
-    probes = np.concatenate([mids, np.nextafter(mids, np.float32(np.inf)), np.nextafter(mids, np.float32(0))])
+    probes = [mids]
+    up, down = mids.copy(), mids.copy()
+    for _ in range(4):                                  # +-1..4 ulps around every midpoint
+        up, down = np.nextafter(up, np.float32(np.inf)), np.nextafter(down, np.float32(0))
+        probes += [up, down]
+    probes = np.concatenate(probes)
     probes = np.concatenate([probes, -probes, np.float32([-0.0])])
     rows = []
     for code in range(1, 126):

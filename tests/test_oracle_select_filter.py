@@ -54,8 +54,10 @@ def test_range_flag():
     assert st["flags"] == 1 and st["s1"][3] == 2 * 65536 and st["amax"][3] == 2.0
     x[1, 3] = np.inf
     assert stats.accumulate(stats.new_state(16), x)["flags"] == 1
-    x[1, 3] = 65535.0
+    x[1, 3] = 32767.0
     assert stats.accumulate(stats.new_state(16), x)["flags"] == 0
+    x[1, 3] = 32768.0
+    assert stats.accumulate(stats.new_state(16), x)["flags"] == 1
 
 
 def test_topk_order_and_ties():
