@@ -11,15 +11,14 @@
 //     significant bits and lies in [2^-10, 2688]), so the f16 MMA with FP32 accumulation sums the
 //     same dequantised values as the tensor-core path;
 //   * the protected slice X_S W'_S^T runs as BF16 MMAs into the same FP32 accumulators;
-//   * the warps of a CTA split K and are reduced in shared memory; the result is scaled once by
-//     alpha and stored.
+//   * the warps of a CTA split K, each with its next chunk's loads in flight; the partial sums
+//     are reduced in shared memory, scaled once by alpha and stored.
 #include "common.cuh"
 #include "gemm.cuh"
 
 namespace fs {
 namespace {
 
-constexpr int kDecWarps = 8;
 
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   uint32_t r;
@@ -86,13 +85,57 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t sf4, int b) {
   return e4m3x2_to_f16x2(byte | (byte << 8));
 }
 
-template <int NT>   // n-tiles of 8 tokens: 1 (M <= 8) or 2 (M <= 16)
-__global__ void __launch_bounds__(kDecWarps * 32)
+constexpr int kRowsPerWarp = 16;
+
+struct ChunkData {
+  Span wa, wb, x0, x1;
+};
+
+template <int NT>
+__device__ __forceinline__ ChunkData load_chunk(const DecodeParams& p, const uint8_t* wA, const uint8_t* wB,
+                                                int64_t rowA, int64_t rowB, int tok0, int tok1, bool t0ok,
+                                                bool t1ok, int k0) {
+  ChunkData d;
+  const int64_t kbytes = p.K / 2;
+  d.wa = load_span(wA, p.sfw, rowA, k0, p.kb4);
+  d.wb = load_span(wB, p.sfw, rowB, k0, p.kb4);
+  d.x0.lo = d.x0.hi = make_uint4(0, 0, 0, 0);
+  d.x0.sf = 0;
+  d.x1 = d.x0;
+  if (t0ok) d.x0 = load_span(p.xq + tok0 * kbytes, p.sfx, tok0, k0, p.kb4);
+  if (NT == 2 && t1ok) d.x1 = load_span(p.xq + tok1 * kbytes, p.sfx, tok1, k0, p.kb4);
+  return d;
+}
+
+template <int NT>
+__device__ __forceinline__ void mma_chunk(const ChunkData& d, float (&acc)[NT][4]) {
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {                 // the span's 4 blocks, 4 k-steps each
+    const uint32_t ssa = scale_pair(d.wa.sf, b), ssb = scale_pair(d.wb.sf, b);
+    const uint32_t sx0 = scale_pair(d.x0.sf, b);
+    const uint32_t sx1 = NT == 2 ? scale_pair(d.x1.sf, b) : 0u;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = 4 * b + jj;
+      const uint32_t a0 = span_pair(d.wa, j, 0, ssa), a2 = span_pair(d.wa, j, 1, ssa);
+      const uint32_t a1 = span_pair(d.wb, j, 0, ssb), a3 = span_pair(d.wb, j, 1, ssb);
+      mma_f16(acc[0], a0, a1, a2, a3, span_pair(d.x0, j, 0, sx0), span_pair(d.x0, j, 1, sx0));
+      if (NT == 2) mma_f16(acc[NT - 1], a0, a1, a2, a3, span_pair(d.x1, j, 0, sx1), span_pair(d.x1, j, 1, sx1));
+    }
+  }
+}
+
+// Grid: one CTA per 16 output features.  The WARPS warps of a CTA split K in 256-element chunks
+// (warp w takes chunks w, w+WARPS, ...), each keeping its next chunk's loads in flight; the
+// partial sums are reduced in shared memory, the protected BF16 slice is added by the warps
+// (one 16-wide k-step each), and warp 0 scales by alpha and stores Y.
+template <int NT, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32)
 splice_gemm_decode_kernel(const DecodeParams p) {
-  __shared__ float red[kDecWarps][32][4 * NT];
+  __shared__ float red[WARPS][32][4 * NT];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 16;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kRowsPerWarp;
   const int64_t rowA = n0 + g, rowB = n0 + g + 8;
   const int64_t kbytes = p.K / 2;
   const uint8_t* wA = p.wq + rowA * kbytes;
@@ -104,35 +147,21 @@ splice_gemm_decode_kernel(const DecodeParams p) {
   for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
 
   const int chunks = p.K / 256;
-  for (int ch = warp; ch < chunks; ch += kDecWarps) {
-    const int k0 = ch * 256 + c * 64;             // this thread's 64-element span
-    const Span sa = load_span(wA, p.sfw, rowA, k0, p.kb4);
-    const Span sb = load_span(wB, p.sfw, rowB, k0, p.kb4);
-    Span x0, x1;
-    x0.lo = x0.hi = make_uint4(0, 0, 0, 0); x0.sf = 0;
-    x1 = x0;
-    if (t0ok) x0 = load_span(p.xq + tok0 * kbytes, p.sfx, tok0, k0, p.kb4);
-    if (NT == 2 && t1ok) x1 = load_span(p.xq + tok1 * kbytes, p.sfx, tok1, k0, p.kb4);
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {                 // the span's 4 blocks, 4 k-steps each
-      const uint32_t ssa = scale_pair(sa.sf, b), ssb = scale_pair(sb.sf, b);
-      const uint32_t sx0 = scale_pair(x0.sf, b);
-      const uint32_t sx1 = NT == 2 ? scale_pair(x1.sf, b) : 0u;
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int j = 4 * b + jj;
-        const uint32_t a0 = span_pair(sa, j, 0, ssa), a2 = span_pair(sa, j, 1, ssa);
-        const uint32_t a1 = span_pair(sb, j, 0, ssb), a3 = span_pair(sb, j, 1, ssb);
-        mma_f16(acc[0], a0, a1, a2, a3, span_pair(x0, j, 0, sx0), span_pair(x0, j, 1, sx0));
-        if (NT == 2) mma_f16(acc[NT - 1], a0, a1, a2, a3, span_pair(x1, j, 0, sx1), span_pair(x1, j, 1, sx1));
-      }
+  if (warp < chunks) {
+    ChunkData cur = load_chunk<NT>(p, wA, wB, rowA, rowB, tok0, tok1, t0ok, t1ok, warp * 256 + c * 64);
+    for (int ch = warp; ch < chunks; ch += WARPS) {
+      ChunkData nxt;
+      const bool more = ch + WARPS < chunks;
+      if (more) nxt = load_chunk<NT>(p, wA, wB, rowA, rowB, tok0, tok1, t0ok, t1ok, (ch + WARPS) * 256 + c * 64);
+      mma_chunk<NT>(cur, acc);
+      if (more) cur = nxt;
     }
   }
-  // protected slice in BF16 (natural K order), spread over the warps by k-step
+  // protected slice in BF16 (natural K order), one 16-wide k-step per warp
   if (p.pp > 0) {
     const uint32_t* wsA = reinterpret_cast<const uint32_t*>(p.ws + rowA * p.pp);
     const uint32_t* wsB = reinterpret_cast<const uint32_t*>(p.ws + rowB * p.pp);
-    for (int ks = warp; ks < p.pp / 16; ks += kDecWarps) {
+    for (int ks = warp; ks < p.pp / 16; ks += WARPS) {
       const int e0 = ks * 8 + c;                   // 32-bit word index of elements 16ks + 2c
       const uint32_t a0 = __ldg(wsA + e0), a2 = __ldg(wsA + e0 + 4);
       const uint32_t a1 = __ldg(wsB + e0), a3 = __ldg(wsB + e0 + 4);
@@ -158,26 +187,19 @@ splice_gemm_decode_kernel(const DecodeParams p) {
     for (int i = 0; i < 4; ++i) red[warp][lane][4 * t + i] = acc[t][i];
   __syncthreads();
   if (warp == 0) {
-    float sum[NT][4];
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float s = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) s += red[w][lane][4 * t + i];
-        sum[t][i] = s;
-      }
     const float alpha = __ldg(p.alpha);
-    // D fragment: c0,c1 -> (feature g, tokens 2c, 2c+1); c2,c3 -> (feature g+8, same tokens)
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
+        float v = 0.0f;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) v += red[w][lane][4 * t + i];
+        // D fragment: c0,c1 -> (feature g, tokens 2c, 2c+1); c2,c3 -> (feature g+8, same tokens)
         const int tok = 8 * t + 2 * c + (i & 1);
         const int64_t feat = n0 + g + (i >> 1) * 8;
         if (tok < p.M && feat < p.N) {
-          const float v = sum[t][i] * alpha;
+          v *= alpha;
           if (p.out_bf16) static_cast<uint16_t*>(p.Y)[tok * p.ldy + feat] = f32_to_bf16_bits(v);
           else static_cast<float*>(p.Y)[tok * p.ldy + feat] = v;
         }
@@ -188,9 +210,10 @@ splice_gemm_decode_kernel(const DecodeParams p) {
 }  // namespace
 
 fs_status launch_splice_gemm_decode(const DecodeParams& p, cudaStream_t s) {
-  const unsigned grid = static_cast<unsigned>(ceil_div(p.N, 16));
-  if (p.M <= 8) splice_gemm_decode_kernel<1><<<grid, kDecWarps * 32, 0, s>>>(p);
-  else splice_gemm_decode_kernel<2><<<grid, kDecWarps * 32, 0, s>>>(p);
+  constexpr int kWarps = 8;
+  const unsigned grid = static_cast<unsigned>(ceil_div(p.N, kRowsPerWarp));
+  if (p.M <= 8) splice_gemm_decode_kernel<1, kWarps><<<grid, kWarps * 32, 0, s>>>(p);
+  else splice_gemm_decode_kernel<2, kWarps><<<grid, kWarps * 32, 0, s>>>(p);
   FS_CHECK_LAUNCH("fs_splice_gemm (decode path)");
   return FS_OK;
 }
