@@ -25,7 +25,7 @@ namespace fs {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;                  // producer, MMA, 4 epilogue and 4 scale warps
 constexpr int kMaxExperts = 256;
 constexpr uint64_t kWaitNs = 4000000000ull;     // 4 s bound on any single wait
 
@@ -124,7 +124,9 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + C::NUM_ACC;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + C::NUM_ACC);
+  uint64_t* sf_full = acc_empty + C::NUM_ACC;      // [2]: scales of a k-tile are in TMEM
+  uint64_t* sf_empty = sf_full + 2;                // [2]: the MMAs reading a scale buffer are done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* cum_m = reinterpret_cast<int*>(tmem_slot + 2);
 
@@ -147,6 +149,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     }
     for (int s = 0; s < C::STAGES; ++s) { ptx::mbar_init(full + s, 1); ptx::mbar_init(empty + s, 1); }
     for (int a = 0; a < C::NUM_ACC; ++a) { ptx::mbar_init(acc_full + a, 1); ptx::mbar_init(acc_empty + a, 128); }
+    for (int b = 0; b < 2; ++b) { ptx::mbar_init(sf_full + b, 4); ptx::mbar_init(sf_empty + b, 1); }
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tmA); ptx::prefetch_tensormap(&tmB); ptx::prefetch_tensormap(&tmY);
     if (p.ST > 0) { ptx::prefetch_tensormap(&tmSA); ptx::prefetch_tensormap(&tmSB); }
@@ -195,7 +198,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     if (lane == 0) {
       constexpr uint32_t idesc_f4 = ptx::idesc_nvf4(kBM, BN);
       constexpr uint32_t idesc_bf = ptx::idesc_bf16(kBM, BN);
-      int stage = 0, acc = 0;
+      int stage = 0, acc = 0, sf_count = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
@@ -208,21 +211,16 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           const uint64_t adesc = ptx::desc_kmajor_sw128(ptx::smem_u32(A_at(stage)));
           const uint64_t bdesc = ptx::desc_kmajor_sw128(ptx::smem_u32(B_at(stage)));
           if (kt < p.KT) {
-            const uint32_t sfa = ptx::smem_u32(SFA_at(stage));
-            const uint32_t sfb = ptx::smem_u32(SFB_at(stage));
-            const uint32_t sf_off = (kt & 1) * C::SF_COLS;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              ptx::tc_cp_32x128b_warpx4(tmem + C::SFA_COL + sf_off + 4 * j, ptx::desc_sf_block(sfa + 512 * j));
-#pragma unroll
-              for (int rg = 0; rg < BN / 128; ++rg)
-                ptx::tc_cp_32x128b_warpx4(tmem + C::SFB_COL + sf_off + (BN / 32) * j + 4 * rg,
-                                          ptx::desc_sf_block(sfb + 2048 * rg + 512 * j));
-            }
+            const int buf = sf_count & 1;
+            if (!wait_bar(sf_full + buf, (sf_count >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const uint32_t sf_off = buf * C::SF_COLS;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               ptx::tc_mma_nvf4(d, adesc + 2 * j, bdesc + 2 * j, idesc_f4, tmem + C::SFA_COL + sf_off + 4 * j,
                                tmem + C::SFB_COL + sf_off + (BN / 32) * j, (kt | j) != 0);
+            ptx::tc_commit(sf_empty + buf);
+            ++sf_count;
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) ptx::tc_mma_bf16(d, adesc + 2 * j, bdesc + 2 * j, idesc_bf, 1u);
@@ -233,6 +231,48 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         if (!ok) break;
         ptx::tc_commit(acc_full + acc);
         if (++acc == C::NUM_ACC) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------------ scale warps
+    // Each warp owns one TMEM lane quadrant and writes, for every FP4 k-tile, the block scales
+    // of its 32 lanes exactly as tcgen05.cp.32x128b.warpx4 would lay them out: lane l, columns
+    // 4c..4c+3 of an atom's slot hold the atom's 16-byte row l (SFA: one atom per MMA; SFB: the
+    // BN/128 row-group atoms side by side).  Scales are double-buffered in TMEM by k-tile parity.
+    const int quad = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    int stage = 0, sf_count = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      for (int kt = 0; kt < ktiles; ++kt) {
+        if (kt < p.KT) {
+          const int buf = sf_count & 1;
+          if (!wait_bar(sf_empty + buf, ((sf_count >> 1) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
+          if (!wait_bar(full + stage, phase, abort_flag, p.err)) { ok = false; break; }
+          const uint8_t* sfa = SFA_at(stage);
+          const uint8_t* sfb = SFB_at(stage);
+          const uint32_t col = tmem + lane_base + buf * C::SF_COLS;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j + lane * 16);
+            ptx::tmem_st_32x32b_x4(col + C::SFA_COL + 4 * j, a.x, a.y, a.z, a.w);
+            if constexpr (BN == 256) {
+              const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j + lane * 16);
+              const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + 512 * j + lane * 16);
+              ptx::tmem_st_32x32b_x8(col + C::SFB_COL + 8 * j, b0, b1);
+            } else {
+              const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j + lane * 16);
+              ptx::tmem_st_32x32b_x4(col + C::SFB_COL + 4 * j, b0.x, b0.y, b0.z, b0.w);
+            }
+          }
+          ptx::tmem_st_wait();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(sf_full + buf);
+          ++sf_count;
+        }
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
   } else {
