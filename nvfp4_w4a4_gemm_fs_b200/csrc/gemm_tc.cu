@@ -36,7 +36,7 @@ struct Cfg {
   static constexpr int SFA_BYTES = kBM * 16;           // 16 scales per row per k-tile
   static constexpr int SFB_BYTES = BN * 16;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = BN == 256 ? 3 : 5;
+  static constexpr int STAGES = BN == 256 ? 3 : 4;
   static constexpr int NUM_ACC = BN == 256 ? 1 : 2;    // TMEM accumulator buffers
   static constexpr int ACC_COLS = BN * NUM_ACC;
   // Scale factors in TMEM, double-buffered by k-tile parity so that the copy for k-tile kt+1
@@ -46,8 +46,10 @@ struct Cfg {
   static constexpr int SFB_COL = ACC_COLS + 16;
   static constexpr int TMEM_COLS = 512;
   static_assert(ACC_COLS + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
-  static constexpr int STAGING_BYTES = 4 * 2 * 4096;  // 4 epilogue warps x 2 buffers x (32 rows x 128 B)
+  static constexpr int STAGING_BUFS = 3;                // per epilogue warp
+  static constexpr int STAGING_BYTES = 4 * STAGING_BUFS * 4096;  // 4 warps x buffers x (32 rows x 128 B)
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 1024 + 4 * (kMaxExperts + 1);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 };
 
 __device__ __forceinline__ uint64_t now_ns() {
@@ -284,7 +286,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     // expert's rows.
     const int quad = warp & 3;                  // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;           // row of the tile held by this thread
-    uint8_t* stage_buf = staging + quad * 2 * 4096;
+    uint8_t* stage_buf = staging + quad * C::STAGING_BUFS * 4096;
     int acc = 0, nbuf = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
@@ -308,8 +310,8 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         if (col0 >= p.N) continue;
         if (use_tma) {
           if (quad * 32 >= m.rows) continue;            // this warp's rows are all past the end
-          uint8_t* buf = stage_buf + (nbuf & 1) * 4096;
-          if (lane == 0) ptx::bulk_wait_read<1>();       // the store issued two chunks ago has read `buf`
+          uint8_t* buf = stage_buf + (nbuf % C::STAGING_BUFS) * 4096;
+          if (lane == 0) ptx::bulk_wait_read<C::STAGING_BUFS - 1>();   // the store that last used `buf` has read it
           __syncwarp();
           if (p.out_bf16) {
             // 32 rows x 64 bytes, 64-byte swizzle: 16-byte chunk j of row r sits at j ^ ((r >> 1) & 3)
