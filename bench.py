@@ -146,7 +146,19 @@ class PrefillLayer:
         dt = torch.bfloat16 if out_bf16 else torch.float32
         self.Y = [torch.empty(M, N, dtype=dt, device=device) for (_, N, K, _) in PROJ]
         self.flops = sum(2.0 * M * N * K for (_, N, K, _) in PROJ)
-        self.launches_per_step = 4 + 2 + 3 * len(PROJ) + 4 + len(PROJ)   # prepare = amax + gain + quantise
+        # per-group views for the multi-stream step (one selection problem per group)
+        self.gstate = []
+        for gi in range(4):
+            st, gidx = (self.st4, gi) if gi < 3 else (self.st12, 0)
+            v = F.StatsState.__new__(F.StatsState)
+            v.nprob, v.K = 1, st.K
+            v.n, v.s1, v.s2 = st.n[gidx:gidx + 1], st.s1[gidx:gidx + 1], st.s2[gidx:gidx + 1]
+            v.amax, v.flags = st.amax[gidx:gidx + 1], st.flags[gidx:gidx + 1]
+            self.gstate.append(v)
+        self.gP = [self.P4[i:i + 1] for i in range(3)] + [self.P12]
+        self.gm = [self.m4[i:i + 1] for i in range(3)] + [self.m12]
+        self.gg = [self.g4[i:i + 1] for i in range(3)] + [self.g12]
+        self.launches_per_step = 4 + 4 + 3 * len(PROJ) + 4 + len(PROJ)   # select per group; prepare = amax + gain + quantise
 
     def mask_gain(self, gi):
         if gi < 3:
@@ -158,6 +170,38 @@ class PrefillLayer:
     def step(self, allreduce=None):
         for fn in self.phase_fns(allreduce):
             fn()
+
+    def group_chain(self, gi, allreduce=None):
+        """Everything of input group gi, in dependency order: statistics, reselection, weight
+        pre-split of its projections, activation quantise, its GEMMs."""
+        F = self.F
+        st, gidx = (self.st4, gi) if gi < 3 else (self.st12, 0)
+        F.fs_channel_stats(self.X[gi], st, group=gidx)
+        if allreduce is not None:
+            allreduce(self.gstate[gi])
+        g = self.gstate[gi]
+        F.fs_select_topk(g, self.p, reset=True, P=self.gP[gi], mask=self.gm[gi], gA=self.gg[gi])
+        mask, gA = self.gm[gi][0], self.gg[gi][0:1]
+        for j, (_, N, K, pg) in enumerate(PROJ):
+            if pg == gi:
+                F.fs_prepare_weights(self.W[j], mask, self.p, gA, out=self.wq[j], gW=self.gW[j:j + 1],
+                                     alpha=self.alpha[j:j + 1])
+        F.fs_quantize_splice(self.X[gi], mask, self.p, gA, out=self.xq[gi])
+        for j, (_, N, K, pg) in enumerate(PROJ):
+            if pg == gi:
+                F.fs_splice_gemm(self.plans[j], self.xq[gi], self.wq[j], self.alpha[j:j + 1], Y=self.Y[j])
+
+    def step_streams(self, streams, allreduce=None):
+        """The same work as step(), with the four independent input-group chains on four streams."""
+        import torch
+        main = torch.cuda.current_stream()
+        for s_ in streams:
+            s_.wait_stream(main)
+        for gi, s_ in enumerate(streams):
+            with torch.cuda.stream(s_):
+                self.group_chain(gi, allreduce)
+        for s_ in streams:
+            main.wait_stream(s_)
 
     def phase_fns(self, allreduce=None):
         """The step split into its phases (same order and launches as step())."""
@@ -453,6 +497,7 @@ def main():
     ap.add_argument("--p", type=int, default=P_DEFAULT)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--serial", action="store_true", help="one stream for the whole step (no group concurrency)")
     ap.add_argument("--case", default="step", choices=["step", "gemm", "decode", "prep"],
                     help="step: the full benchmark; gemm / decode: only fs_splice_gemm on the q projection "
                          "(M=8192, or M=16) for profiling one kernel")
@@ -495,7 +540,13 @@ def main():
     # small library calls would otherwise show up as GPU idle time.  Each phase (and each GEMM)
     # is also captured on its own, replayed back to back with events in between, to attribute
     # time per kernel on the device.
-    step_graph = capture(lambda: layer.step(allreduce))
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    if use_dist:
+        args.serial = True          # collectives on concurrent streams could be ordered differently per rank
+    if args.serial:
+        step_graph = capture(lambda: layer.step(allreduce))
+    else:
+        step_graph = capture(lambda: layer.step_streams(streams, allreduce))
     for _ in range(args.warmup):
         step_graph.replay()
     torch.cuda.synchronize()
@@ -568,8 +619,9 @@ def main():
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": ms_e2e},
-        "gpu_launches": layer.launches_per_step * args.steps,
-        "graph": "each timed step is one CUDA-graph replay of the step's 38 launches",
+        "gpu_launches": (38 if args.serial else layer.launches_per_step) * args.steps,
+        "graph": "each timed step is one CUDA-graph replay of the step's launches" +
+                 ("" if args.serial else "; the 4 independent input-group chains run on 4 streams"),
     }
 
     if not args.no_extras and rank == 0:

@@ -112,7 +112,9 @@ struct ChunkLoc {
 // tables of the scale value and its reciprocal in shared memory.
 template <typename T, Side kSide, bool kGrouped>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_t nchunks) {
-  __shared__ int sh_prefix[16384 / 32 + 1];             // protected channels before each mask word
+  __shared__ uint16_t sh_mbits[16384 / 16];             // protected lanes of each 16-element block
+  __shared__ uint4 sh_kill[sizeof(T) == 2 ? 2 * 16384 / 16 : 1];   // bf16: per block, 8 words of lanes to clear
+  __shared__ uint16_t sh_col[16384 / 16];               // side-buffer column of each block's first protected lane
   __shared__ float sh_val[128], sh_rcp[128];            // UE4M3 value and RN(1/value) per code
   __shared__ int64_t sh_pad[kGrouped ? kMaxGroupedExperts + 1 : 1];   // padded start of each expert
   __shared__ int64_t sh_off[kGrouped ? kMaxGroupedExperts + 1 : 1];   // row offsets of the experts
@@ -190,20 +192,40 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
       mask = (a.p > 0) ? a.masks + static_cast<int64_t>(cur_e) * words : nullptr;
       g = __ldg(a.gains + cur_e);
       if (a.p > 0) {
-        __syncthreads();                           // previous expert's prefix no longer read
-        if (tid < 32) {
-          int carry = 0;
-          for (int w0 = 0; w0 < words; w0 += 32) {
-            const int w = w0 + tid;
-            const int c = (w < words) ? __popc(__ldg(mask + w)) : 0;
-            int incl = c;
+        __syncthreads();                           // previous expert's tables no longer read
+        // per block: its 16 mask bits and the side column of its first protected lane
+        // (protected channels before it), by a block-wide scan in 32-block steps
+        const int nb = a.nb;
+        int carry = 0;
+        for (int b0 = 0; b0 < nb; b0 += 32) {
+          if (tid < 32) {
+            const int b = b0 + tid;
+            const uint32_t mb = (b < nb) ? ((__ldg(mask + (b >> 1)) >> ((b & 1) * 16)) & 0xFFFFu) : 0u;
+            const int cnt = __popc(mb);
+            int incl = cnt;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
               const int y = __shfl_up_sync(0xffffffffu, incl, o);
               if (tid >= o) incl += y;
             }
-            if (w < words) sh_prefix[w] = carry + incl - c;
+            if (b < nb) {
+              sh_mbits[b] = static_cast<uint16_t>(mb);
+              sh_col[b] = static_cast<uint16_t>(carry + incl - cnt);
+            }
             carry += __shfl_sync(0xffffffffu, incl, 31);
+          }
+        }
+        if constexpr (sizeof(T) == 2) {
+          for (int b = tid; b < nb; b += kQThreads) {
+            const uint32_t mb = (__ldg(mask + (b >> 1)) >> ((b & 1) * 16)) & 0xFFFFu;
+            uint32_t k[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint32_t two = (mb >> (2 * j)) & 3u;
+              k[j] = ((two & 1u) | ((two & 2u) << 15)) * 0xFFFFu;
+            }
+            sh_kill[2 * b] = make_uint4(k[0], k[1], k[2], k[3]);
+            sh_kill[2 * b + 1] = make_uint4(k[4], k[5], k[6], k[7]);
           }
         }
         __syncthreads();
@@ -223,8 +245,19 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
       const bool has_data = in_range && r < L.valid;
       uint32_t sfc = 0;
       if (has_data) {
-        const uint32_t mbits = mask ? ((__ldg(mask + (b >> 1)) >> ((b & 1) * 16)) & 0xFFFFu) : 0u;
-        const RawBlock<T> xm = mbits ? x.masked(mbits) : x;
+        const uint32_t mbits = mask ? sh_mbits[b] : 0u;
+        RawBlock<T> xm;
+        if constexpr (sizeof(T) == 2) {
+          if (mask) {                                // uniform: clear protected lanes, no branch per block
+            const uint4 k0 = sh_kill[2 * b], k1 = sh_kill[2 * b + 1];
+            xm.w[0] = x.w[0] & ~k0.x; xm.w[1] = x.w[1] & ~k0.y; xm.w[2] = x.w[2] & ~k0.z; xm.w[3] = x.w[3] & ~k0.w;
+            xm.w[4] = x.w[4] & ~k1.x; xm.w[5] = x.w[5] & ~k1.y; xm.w[6] = x.w[6] & ~k1.z; xm.w[7] = x.w[7] & ~k1.w;
+          } else {
+            xm = x;
+          }
+        } else {
+          xm = mbits ? x.masked(mbits) : x;
+        }
         const RawBlock<T>& xs = residual ? x : xm;    // lanes that set the block scale
         float amax = 0.0f;
 #pragma unroll
@@ -240,7 +273,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
         *reinterpret_cast<uint2*>(a.q + prow * (a.K / 2) + static_cast<int64_t>(b) * 8) = make_uint2(lo, hi);
         // Extract the protected lanes into the side buffer.
         if (mbits) {
-          int col = sh_prefix[b >> 1] + ((b & 1) ? __popc(__ldg(mask + (b >> 1)) & 0xFFFFu) : 0);
+          int col = sh_col[b];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if ((mbits >> j) & 1u) {
