@@ -138,6 +138,22 @@ splice_gemm_decode_kernel(const DecodeParams p) {
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kRowsPerWarp;
   const int64_t rowA = n0 + g, rowB = n0 + g + 8;
   const int64_t kbytes = p.K / 2;
+  // Programmatic dependent launch: let the next kernel in the stream start its own prologue now,
+  // and pull this CTA's weight rows (and their BF16 protected columns) into L2 while the previous
+  // kernel may still be running.  An L2 prefetch is safe whatever that kernel writes (L2 is
+  // coherent); every real load and store below comes after griddepcontrol.wait.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (warp == 0 && lane < kRowsPerWarp && n0 + lane < p.N) {
+    const uint8_t* row = p.wq + (n0 + lane) * kbytes;
+    for (int64_t off = 0; off < kbytes; off += 16384) {
+      const uint32_t bytes = static_cast<uint32_t>(kbytes - off < 16384 ? kbytes - off : 16384);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(row + off), "r"(bytes) : "memory");
+    }
+    if (p.pp > 0)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.ws + (n0 + lane) * p.pp),
+                   "r"(static_cast<uint32_t>(p.pp * 2)) : "memory");
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint8_t* wA = p.wq + rowA * kbytes;
   const uint8_t* wB = p.wq + rowB * kbytes;
   const int tok0 = g, tok1 = g + 8;
@@ -211,9 +227,19 @@ splice_gemm_decode_kernel(const DecodeParams p) {
 
 fs_status launch_splice_gemm_decode(const DecodeParams& p, cudaStream_t s) {
   constexpr int kWarps = 8;
-  const unsigned grid = static_cast<unsigned>(ceil_div(p.N, kRowsPerWarp));
-  if (p.M <= 8) splice_gemm_decode_kernel<1, kWarps><<<grid, kWarps * 32, 0, s>>>(p);
-  else splice_gemm_decode_kernel<2, kWarps><<<grid, kWarps * 32, 0, s>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(p.N, kRowsPerWarp)), 1, 1);
+  cfg.blockDim = dim3(kWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = (p.M <= 8) ? cudaLaunchKernelEx(&cfg, splice_gemm_decode_kernel<1, kWarps>, p)
+                             : cudaLaunchKernelEx(&cfg, splice_gemm_decode_kernel<2, kWarps>, p);
+  if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm (decode path)");
   FS_CHECK_LAUNCH("fs_splice_gemm (decode path)");
   return FS_OK;
 }
