@@ -5,16 +5,27 @@
 // SAME shared-memory stage buffers and their BF16 MMAs accumulate into the SAME FP32 TMEM
 // accumulator; the epilogue moves TMEM to registers, multiplies by alpha once and stores Y.
 //
-// Per CTA (persistent, one per SM): a 128 x BN output tile at a time.
-//   warp 0      TMA producer: per k-tile one 128x128-byte box of A and a BNx128-byte box of B
-//               (128-byte swizzle) plus the tile's UE4M3 scale atoms (plain bulk copies); the
-//               BF16 side tiles use the same boxes, 64 bf16 wide.
-//   warp 1      allocates TMEM; one thread issues tcgen05.cp (scales SMEM->TMEM) and
-//               tcgen05.mma: kind::mxf4nvf4 (K = 64 per instruction) over all of K, then
-//               kind::f16 (K = 16) over the protected slice, then commits to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, x alpha, store.
-// Every mbarrier wait is bounded; on expiry the kernel records a timeout in the plan's error
-// word, all roles stop issuing work, and TMEM is still released.
+// Persistent kernel, one CTA per SM.  Output tiles are 128 x BN per CTA.  With CG = 2 two CTAs of
+// a cluster form a pair that computes a 256 x 256 tile with cta_group::2 MMAs: each CTA loads
+// its own 128 rows of A and half (128 rows) of the B tile, the leader CTA issues the MMAs for
+// both, and each CTA's TMEM receives its 128 output rows.  Halving B per CTA cuts the operand
+// bytes per k-tile from 48 KB to 32 KB, which buys pipeline depth and L2->SM bandwidth.
+//   warp 0      TMA producer: per k-tile one 128x128-byte box of A and a (BN/CG)x128-byte box of
+//               B (128-byte swizzle), plus the tile's UE4M3 scale atoms (plain bulk copies of
+//               this CTA's A rows and all BN columns of B); the BF16 side tiles use the same
+//               boxes, 64 bf16 wide.
+//   warp 1      allocates TMEM; one thread of the leader issues tcgen05.mma: kind::mxf4nvf4
+//               (K = 64 per instruction) over all of K, then kind::f16 (K = 16) over the
+//               protected slice, and commits the stage / scale / accumulator barriers.
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, x alpha, staged in shared memory
+//               and written with TMA stores.
+//   warps 6..9  scale warps: tcgen05.st of each k-tile's block scales into TMEM.
+// Accumulators (BN = 256) overlap in TMEM: tile i uses columns [128*(i&1), 128*(i&1) + 256), so
+// consecutive tiles share columns [128, 256).  The epilogue loads that shared half into
+// registers first and releases it at once; the next tile's MMAs then run while the epilogue
+// drains the other half and the stores, so output traffic overlaps the main loop.
+// Every mbarrier wait is bounded; on expiry the kernel records a timeout in the error word,
+// stops issuing work, waits (bounded) for its own copies in flight and still releases TMEM.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -28,27 +39,53 @@ constexpr int kBM = 128;
 constexpr int kThreads = 320;                  // producer, MMA, 4 epilogue and 4 scale warps
 constexpr int kMaxExperts = 256;
 constexpr uint64_t kWaitNs = 4000000000ull;     // 4 s bound on any single wait
+constexpr uint64_t kDrainNs = 50000000ull;      // 50 ms bound on each wait of the abort path
 
-template <int BN>
+#ifndef FS_TC_PAIR_STAGES
+#define FS_TC_PAIR_STAGES 5
+#endif
+#ifndef FS_TC_PAIR_STAGING
+#define FS_TC_PAIR_STAGING 2
+#endif
+#ifndef FS_TC_SF_BUFS
+#define FS_TC_SF_BUFS 2
+#endif
+#ifndef FS_TC_OVERLAP_ACC
+#define FS_TC_OVERLAP_ACC 1
+#endif
+
+template <int BN, int CG>
 struct Cfg {
+  static_assert(CG == 1 || (CG == 2 && BN == 256), "CTA pairs use 256 x 256 tiles");
+  static constexpr int B_ROWS = BN / CG;               // rows of the B tile this CTA loads
   static constexpr int A_BYTES = kBM * 128;            // 128 rows x 128 bytes (256 fp4 or 64 bf16)
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_BYTES = B_ROWS * 128;
   static constexpr int SFA_BYTES = kBM * 16;           // 16 scales per row per k-tile
-  static constexpr int SFB_BYTES = BN * 16;
+  static constexpr int SFB_BYTES = BN * 16;            // every CTA holds the scales of all BN columns
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = BN == 256 ? 3 : 4;
-  static constexpr int NUM_ACC = BN == 256 ? 1 : 2;    // TMEM accumulator buffers
-  static constexpr int ACC_COLS = BN * NUM_ACC;
-  // Scale factors in TMEM, double-buffered by k-tile parity so that the copy for k-tile kt+1
-  // does not overwrite columns the MMAs of k-tile kt may still read.
+  static constexpr int TX_BYTES = CG * (A_BYTES + B_BYTES);   // A/B bytes landing per stage in the pair
+  static constexpr int STAGES = CG == 2 ? FS_TC_PAIR_STAGES : (BN == 256 ? 3 : 4);
+  static constexpr int STAGING_BUFS = CG == 2 ? FS_TC_PAIR_STAGING : 3;   // per epilogue warp
+  // Accumulators: BN = 256 overlaps two 256-column buffers in 384 columns (OVERLAP; otherwise
+  // one 256-column buffer); BN = 128 keeps two disjoint 128-column buffers.  With two buffers
+  // tile i starts at column 128 * (i & 1).
+  static constexpr bool OVERLAP = BN == 128 || FS_TC_OVERLAP_ACC;
+  static constexpr int ACC_SLOTS = BN == 256 ? 1 : 2;  // accumulator barrier pairs
+  static constexpr int ACC_SPAN = BN == 256 ? (OVERLAP ? 384 : 256) : 256;
+  // Scale factors in TMEM: a ring of SF_BUFS k-tile buffers, so that the scales of later k-tiles
+  // do not overwrite columns the MMAs of earlier k-tiles may still read.
+  static constexpr int SF_BUFS = FS_TC_SF_BUFS;
   static constexpr int SF_COLS = 16 + 4 * (BN / 32);   // SFA: 4 MMAs x 4 columns; SFB: 4 MMAs x BN/32
-  static constexpr int SFA_COL = ACC_COLS;
-  static constexpr int SFB_COL = ACC_COLS + 16;
+  static constexpr int SFA_COL = ACC_SPAN;
+  static constexpr int SFB_COL = ACC_SPAN + 16;
   static constexpr int TMEM_COLS = 512;
-  static_assert(ACC_COLS + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
-  static constexpr int STAGING_BUFS = 3;                // per epilogue warp
+  static_assert(ACC_SPAN + SF_BUFS * SF_COLS <= TMEM_COLS, "TMEM budget");
   static constexpr int STAGING_BYTES = 4 * STAGING_BUFS * 4096;  // 4 warps x buffers x (32 rows x 128 B)
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 1024 + 4 * (kMaxExperts + 1);
+  // full, sf_loaded, empty per stage; acc_full, acc_empty per slot; sf_full, sf_empty per scale
+  // buffer; drain
+  static constexpr int NUM_BARS = 3 * STAGES + 2 * ACC_SLOTS + 2 * SF_BUFS + 1;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 8 * NUM_BARS + 16 +
+                                    4 * (kMaxExperts + 1);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 };
 
@@ -75,16 +112,26 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   }
 }
 
+// Abort path: wait up to `limit_ns` for one phase of a barrier, ignoring the abort flag.
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = now_ns();
+  while (!ptx::mbar_try_wait(bar, parity))
+    if (now_ns() - t0 > limit_ns) return;
+}
+
 struct TileMap {
   int e;           // expert
-  int64_t arow;    // first row in the packed activation buffers (padded for experts)
-  int64_t yrow;    // first output row
-  int rows;        // valid rows in this tile
-  int64_t brow;    // first row in the (stacked) weight buffers
+  int64_t arow;    // first row of this CTA's A rows in the packed activation buffers
+  int64_t yrow;    // first output row of this CTA
+  int rows;        // valid rows of this CTA (may be <= 0 for the second CTA of a pair)
+  int64_t brow;    // first row of the tile in the (stacked) weight buffers
   int n0;          // first output column
 };
 
-__device__ __forceinline__ TileMap map_tile(int t, const TcParams& p, const int* cum_m) {
+// Tile t -> rows / columns.  cum_m[e] counts the (kBM * CG)-row M-tiles before expert e; M-tiles
+// vary fastest so that the CTAs of one wave share B tiles in L2.
+template <int CG>
+__device__ __forceinline__ TileMap map_tile(int t, const TcParams& p, const int* cum_m, int rank) {
   TileMap m;
   const int total_m = cum_m[p.E];
   const int mt = t % total_m;
@@ -96,7 +143,7 @@ __device__ __forceinline__ TileMap map_tile(int t, const TcParams& p, const int*
   }
   m.e = lo;
   const int local = mt - cum_m[lo];
-  m.arow = static_cast<int64_t>(mt) * kBM;    // experts start at 128-row boundaries
+  m.arow = static_cast<int64_t>(mt) * (kBM * CG) + rank * kBM;   // experts start at 128-row boundaries
   if (p.offsets) {
     const int64_t r0 = p.offsets[lo], r1 = p.offsets[lo + 1];
     m.yrow = r0 + static_cast<int64_t>(local) * kBM;
@@ -105,38 +152,46 @@ __device__ __forceinline__ TileMap map_tile(int t, const TcParams& p, const int*
   } else {
     m.yrow = m.arow;
     const int64_t left = p.M - m.arow;
-    m.rows = static_cast<int>(left < kBM ? left : kBM);
+    m.rows = static_cast<int>(left < kBM ? (left < 0 ? 0 : left) : kBM);
   }
   m.n0 = nt * p.BN;
   m.brow = static_cast<int64_t>(lo) * p.N + m.n0;
   return m;
 }
 
-template <int BN>
+template <int BN, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
 splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                       const __grid_constant__ CUtensorMap tmY, const TcParams p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, CG>;
   extern __shared__ uint8_t smem_raw[];
+  // The same offset in both CTAs of a pair: the dynamic shared memory base is identical.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
   uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;           // 1024-byte aligned
-  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::STAGING_BYTES);
-  uint64_t* empty = full + C::STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::STAGING_BYTES);   // A/B landed (leader's counts both CTAs)
+  uint64_t* sfl = full + C::STAGES;                // this CTA's scale atoms landed
+  uint64_t* empty = sfl + C::STAGES;               // the MMAs reading a stage are done
   uint64_t* acc_full = empty + C::STAGES;
-  uint64_t* acc_empty = acc_full + C::NUM_ACC;
-  uint64_t* sf_full = acc_empty + C::NUM_ACC;      // [2]: scales of a k-tile are in TMEM
-  uint64_t* sf_empty = sf_full + 2;                // [2]: the MMAs reading a scale buffer are done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + 2);
+  uint64_t* acc_empty = acc_full + C::ACC_SLOTS;   // leader: released by the epilogues of both CTAs
+  uint64_t* sf_full = acc_empty + C::ACC_SLOTS;    // leader: scales of a k-tile are in TMEM (both CTAs)
+  uint64_t* sf_empty = sf_full + C::SF_BUFS;       // the MMAs reading a scale buffer are done
+  uint64_t* drain = sf_empty + C::SF_BUFS;         // leader: all MMAs issued so far are done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* cum_m = reinterpret_cast<int*>(tmem_slot + 2);
+  int* cum_m = reinterpret_cast<int*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = CG == 2 ? static_cast<int>(ptx::cluster_ctarank()) : 0;
+  const int unit = CG == 2 ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);   // CTA or pair
+  const int nunits = CG == 2 ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
   auto A_at = [&](int s) { return stages + s * C::STAGE_BYTES; };
   auto B_at = [&](int s) { return stages + s * C::STAGE_BYTES + C::A_BYTES; };
   auto SFA_at = [&](int s) { return stages + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES; };
   auto SFB_at = [&](int s) { return stages + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES + C::SFA_BYTES; };
+  // Leader-CTA barriers as shared::cluster addresses (the CTA's own address when CG = 1).
+  auto leader = [&](uint64_t* bar) { return CG == 2 ? ptx::mapa_shared(ptx::smem_u32(bar), 0) : ptx::smem_u32(bar); };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -147,111 +202,151 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         cum_m[e + 1] = cum_m[e] + static_cast<int>((rows + kBM - 1) / kBM);
       }
     } else {
-      cum_m[1] = static_cast<int>((p.M + kBM - 1) / kBM);
+      cum_m[1] = static_cast<int>((p.M + kBM * CG - 1) / (kBM * CG));
     }
-    for (int s = 0; s < C::STAGES; ++s) { ptx::mbar_init(full + s, 1); ptx::mbar_init(empty + s, 1); }
-    for (int a = 0; a < C::NUM_ACC; ++a) { ptx::mbar_init(acc_full + a, 1); ptx::mbar_init(acc_empty + a, 128); }
-    for (int b = 0; b < 2; ++b) { ptx::mbar_init(sf_full + b, 4); ptx::mbar_init(sf_empty + b, 1); }
+    for (int s = 0; s < C::STAGES; ++s) {
+      ptx::mbar_init(full + s, 1);
+      ptx::mbar_init(sfl + s, 1);
+      ptx::mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < C::ACC_SLOTS; ++a) { ptx::mbar_init(acc_full + a, 1); ptx::mbar_init(acc_empty + a, 4 * CG); }
+    for (int b = 0; b < C::SF_BUFS; ++b) { ptx::mbar_init(sf_full + b, 4 * CG); ptx::mbar_init(sf_empty + b, 1); }
+    ptx::mbar_init(drain, 1);
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tmA); ptx::prefetch_tensormap(&tmB); ptx::prefetch_tensormap(&tmY);
     if (p.ST > 0) { ptx::prefetch_tensormap(&tmSA); ptx::prefetch_tensormap(&tmSB); }
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc<CG>(tmem_slot, C::TMEM_COLS);
+    ptx::tmem_relinquish<CG>();
   }
   ptx::tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) ptx::cluster_sync();     // the peer's barriers exist before anyone signals them
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int total_tiles = cum_m[p.E] * p.n_tiles;
   const int ktiles = p.KT + p.ST;
+  const int m_groups = static_cast<int>((p.M + kBM - 1) / kBM);   // 128-row scale groups (dense)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int stage = 0;
+      int stage = 0, issued = 0;
       uint32_t phase = 0;
+      uint32_t sfl_bits = 0, last_fp4 = 0;   // per stage: parity of its next FP4 use; last use was FP4
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const TileMap m = map_tile(t, p, cum_m);
+      for (int t = unit; t < total_tiles && ok; t += nunits) {
+        const TileMap m = map_tile<CG>(t, p, cum_m, rank);
+        // Scale atoms of rows past the end of a dense problem are not in the buffer: skip them
+        // (those output rows are discarded).
+        const bool sfa_ok = p.offsets || (m.arow / kBM) < m_groups;
+        const int64_t brow = m.brow + rank * C::B_ROWS;
         for (int kt = 0; kt < ktiles; ++kt) {
           if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err)) { ok = false; break; }
-          if (kt < p.KT) {
-            ptx::mbar_arrive_expect_tx(full + stage, C::STAGE_BYTES);
-            ptx::tma_load_2d(A_at(stage), &tmA, kt * 128, static_cast<int32_t>(m.arow), full + stage);
-            ptx::tma_load_2d(B_at(stage), &tmB, kt * 128, static_cast<int32_t>(m.brow), full + stage);
-            ptx::bulk_load(SFA_at(stage), p.sfa + ((m.arow / kBM) * p.kb4 + kt * 4) * 512, C::SFA_BYTES, full + stage);
+          const bool fp4 = kt < p.KT;
+          last_fp4 = (last_fp4 & ~(1u << stage)) | (static_cast<uint32_t>(fp4) << stage);
+          if (fp4) {
+            sfl_bits ^= 1u << stage;
+            ptx::mbar_arrive_expect_tx(sfl + stage, (sfa_ok ? C::SFA_BYTES : 0) + C::SFB_BYTES);
+            if (sfa_ok)
+              ptx::bulk_load(SFA_at(stage), p.sfa + ((m.arow / kBM) * p.kb4 + kt * 4) * 512, C::SFA_BYTES, sfl + stage);
 #pragma unroll
             for (int rg = 0; rg < BN / 128; ++rg)
               ptx::bulk_load(SFB_at(stage) + rg * 2048, p.sfb + ((m.brow / kBM + rg) * p.kb4 + kt * 4) * 512, 2048,
-                             full + stage);
-          } else {
-            ptx::mbar_arrive_expect_tx(full + stage, C::A_BYTES + C::B_BYTES);
-            ptx::tma_load_2d(A_at(stage), &tmSA, (kt - p.KT) * 64, static_cast<int32_t>(m.arow), full + stage);
-            ptx::tma_load_2d(B_at(stage), &tmSB, (kt - p.KT) * 64, static_cast<int32_t>(m.brow), full + stage);
+                             sfl + stage);
           }
+          if (rank == 0) ptx::mbar_arrive_expect_tx(full + stage, C::TX_BYTES);
+          const CUtensorMap* ma = fp4 ? &tmA : &tmSA;
+          const CUtensorMap* mb = fp4 ? &tmB : &tmSB;
+          const int32_t kx = fp4 ? kt * 128 : (kt - p.KT) * 64;
+          if constexpr (CG == 1) {
+            ptx::tma_load_2d(A_at(stage), ma, kx, static_cast<int32_t>(m.arow), full + stage);
+            ptx::tma_load_2d(B_at(stage), mb, kx, static_cast<int32_t>(brow), full + stage);
+          } else {
+            const uint32_t bar = leader(full + stage);
+            ptx::tma_load_2d_pair(A_at(stage), ma, kx, static_cast<int32_t>(m.arow), bar);
+            ptx::tma_load_2d_pair(B_at(stage), mb, kx, static_cast<int32_t>(brow), bar);
+          }
+          ++issued;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        // Copies issued but possibly not landed: the last min(issued, STAGES) stages.  The leader
+        // can observe both CTAs' A/B bytes; every CTA observes its own scale atoms.
+        int s = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < C::STAGES && i < issued; ++i) {
+          if (--s < 0) { s = C::STAGES - 1; ph ^= 1; }
+          if (rank == 0) drain_bar(full + s, ph, kDrainNs);
+          if ((last_fp4 >> s) & 1) drain_bar(sfl + s, ((sfl_bits >> s) & 1) ^ 1, kDrainNs);
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_f4 = ptx::idesc_nvf4(kBM, BN);
-      constexpr uint32_t idesc_bf = ptx::idesc_bf16(kBM, BN);
-      int stage = 0, acc = 0, sf_count = 0;
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc_f4 = ptx::idesc_nvf4(kBM * CG, BN);
+      constexpr uint32_t idesc_bf = ptx::idesc_bf16(kBM * CG, BN);
+      int stage = 0, acc = 0, sf_count = 0, i = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      for (int t = unit; t < total_tiles && ok; t += nunits, ++i) {
         if (!wait_bar(acc_empty + acc, acc_phase ^ 1, abort_flag, p.err)) break;
         ptx::tc_fence_after();
-        const uint32_t d = tmem + acc * BN;
+        const uint32_t d = tmem + static_cast<uint32_t>(C::OVERLAP ? (i & 1) * 128 : 0);
         for (int kt = 0; kt < ktiles; ++kt) {
           if (!wait_bar(full + stage, phase, abort_flag, p.err)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint64_t adesc = ptx::desc_kmajor_sw128(ptx::smem_u32(A_at(stage)));
           const uint64_t bdesc = ptx::desc_kmajor_sw128(ptx::smem_u32(B_at(stage)));
           if (kt < p.KT) {
-            const int buf = sf_count & 1;
-            if (!wait_bar(sf_full + buf, (sf_count >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+            const int buf = sf_count % C::SF_BUFS;
+            if (!wait_bar(sf_full + buf, (sf_count / C::SF_BUFS) & 1, abort_flag, p.err)) { ok = false; break; }
             ptx::tc_fence_after();
             const uint32_t sf_off = buf * C::SF_COLS;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              ptx::tc_mma_nvf4(d, adesc + 2 * j, bdesc + 2 * j, idesc_f4, tmem + C::SFA_COL + sf_off + 4 * j,
-                               tmem + C::SFB_COL + sf_off + (BN / 32) * j, (kt | j) != 0);
-            ptx::tc_commit(sf_empty + buf);
+              ptx::tc_mma_nvf4<CG>(d, adesc + 2 * j, bdesc + 2 * j, idesc_f4, tmem + C::SFA_COL + sf_off + 4 * j,
+                                   tmem + C::SFB_COL + sf_off + (BN / 32) * j, (kt | j) != 0);
+            ptx::tc_commit<CG>(sf_empty + buf);
             ++sf_count;
           } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) ptx::tc_mma_bf16(d, adesc + 2 * j, bdesc + 2 * j, idesc_bf, 1u);
+            for (int j = 0; j < 4; ++j) ptx::tc_mma_bf16<CG>(d, adesc + 2 * j, bdesc + 2 * j, idesc_bf, 1u);
           }
-          ptx::tc_commit(empty + stage);
+          ptx::tc_commit<CG>(empty + stage);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        ptx::tc_commit(acc_full + acc);
-        if (++acc == C::NUM_ACC) { acc = 0; acc_phase ^= 1; }
+        ptx::tc_commit<CG>(acc_full + acc);
+        if (++acc == C::ACC_SLOTS) { acc = 0; acc_phase ^= 1; }
       }
+      // Every MMA issued above has completed before TMEM can be released.
+      ptx::tc_commit<CG>(drain);
+      drain_bar(drain, 0, kWaitNs);
     }
   } else if (warp >= 6) {
     // ------------------------------------------------------------------ scale warps
     // Each warp owns one TMEM lane quadrant and writes, for every FP4 k-tile, the block scales
     // of its 32 lanes exactly as tcgen05.cp.32x128b.warpx4 would lay them out: lane l, columns
     // 4c..4c+3 of an atom's slot hold the atom's 16-byte row l (SFA: one atom per MMA; SFB: the
-    // BN/128 row-group atoms side by side).  Scales are double-buffered in TMEM by k-tile parity.
+    // BN/128 row-group atoms side by side).  The k-tiles' scales rotate over SF_BUFS buffers.
+    // The scale-atom barrier of a stage completes one phase per FP4 use of that stage only, so
+    // its parity is tracked per stage (the producer keeps the same bits).
     const int quad = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     int stage = 0, sf_count = 0;
-    uint32_t phase = 0;
+    uint32_t sfl_bits = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+    for (int t = unit; t < total_tiles && ok; t += nunits) {
       for (int kt = 0; kt < ktiles; ++kt) {
         if (kt < p.KT) {
-          const int buf = sf_count & 1;
-          if (!wait_bar(sf_empty + buf, ((sf_count >> 1) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
-          if (!wait_bar(full + stage, phase, abort_flag, p.err)) { ok = false; break; }
+          const int buf = sf_count % C::SF_BUFS;
+          if (!wait_bar(sf_empty + buf, ((sf_count / C::SF_BUFS) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
+          if (!wait_bar(sfl + stage, (sfl_bits >> stage) & 1, abort_flag, p.err)) { ok = false; break; }
+          sfl_bits ^= 1u << stage;
           const uint8_t* sfa = SFA_at(stage);
           const uint8_t* sfb = SFB_at(stage);
           const uint32_t col = tmem + lane_base + buf * C::SF_COLS;
@@ -271,45 +366,48 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           ptx::tmem_st_wait();
           ptx::tc_fence_before();
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(sf_full + buf);
+          if (lane == 0) {
+            if constexpr (CG == 1) ptx::mbar_arrive(sf_full + buf);
+            else ptx::mbar_arrive_remote(leader(sf_full + buf));
+          }
           ++sf_count;
         }
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        if (++stage == C::STAGES) stage = 0;
       }
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    // TMEM -> registers (x alpha) -> swizzled staging in shared memory -> TMA store of a
-    // 32-row x 32-column box per warp; the accumulator is released right after the last TMEM
-    // load, so the next tile's MMAs overlap the stores.  Partial tiles of an expert (rows that
-    // end inside the output) use direct stores instead, since a box would cross into the next
-    // expert's rows.
+    // Part 1: the 128 accumulator columns the next tile will overwrite are loaded into registers
+    // and released at once (BN = 128: the whole tile).  Part 2 (BN = 256): the other 128 columns,
+    // 32 at a time, while the next tile's MMAs run.  Each 32 x 32 chunk is scaled by alpha,
+    // staged in shared memory with the TMA swizzle and written by a TMA store.  Partial tiles of
+    // an expert (rows that end inside the output) use direct stores instead, since a box would
+    // cross into the next expert's rows.
     const int quad = warp & 3;                  // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;           // row of the tile held by this thread
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     uint8_t* stage_buf = staging + quad * C::STAGING_BUFS * 4096;
-    int acc = 0, nbuf = 0;
+    int acc = 0, nbuf = 0, i = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-      const TileMap m = map_tile(t, p, cum_m);
+    for (int t = unit; t < total_tiles; t += nunits, ++i) {
+      const TileMap m = map_tile<CG>(t, p, cum_m, rank);
       if (!wait_bar(acc_full + acc, acc_phase, abort_flag, p.err)) break;
       ptx::tc_fence_after();
       const float alpha = __ldg(p.alpha + m.e);
       const bool use_tma = !(p.offsets && m.rows < kBM);
       const bool row_ok = row < m.rows;
       const int64_t yrow = m.yrow + row;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN + c * 32, r);
-        ptx::tmem_ld_wait();
-        if (c == BN / 32 - 1) {
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(acc_empty + acc);
-        }
-        const int col0 = m.n0 + c * 32;
-        if (col0 >= p.N) continue;
+      const int base = C::OVERLAP ? (i & 1) * 128 : 0;
+      // TMEM column and output column of each part.
+      const int p1_tcol = BN == 256 ? 128 : base;
+      const int p1_ocol = BN == 256 ? 128 - base : 0;
+      const int p2_tcol = base == 0 ? 0 : 256;
+      const int p2_ocol = base == 0 ? 0 : 128;
+
+      auto emit = [&](const uint32_t (&r)[32], int col0) {
+        if (col0 >= p.N) return;
         if (use_tma) {
-          if (quad * 32 >= m.rows) continue;            // this warp's rows are all past the end
+          if (quad * 32 >= m.rows) return;              // this warp's rows are all past the end
           uint8_t* buf = stage_buf + (nbuf % C::STAGING_BUFS) * 4096;
           if (lane == 0) ptx::bulk_wait_read<C::STAGING_BUFS - 1>();   // the store that last used `buf` has read it
           __syncwarp();
@@ -343,26 +441,65 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           if (p.out_bf16) {
             uint16_t* y = static_cast<uint16_t*>(p.Y) + yrow * p.ldy + col0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (col0 + i < p.N) y[i] = f32_to_bf16_bits(__uint_as_float(r[i]) * alpha);
+            for (int c = 0; c < 32; ++c)
+              if (col0 + c < p.N) y[c] = f32_to_bf16_bits(__uint_as_float(r[c]) * alpha);
           } else {
             float* y = static_cast<float*>(p.Y) + yrow * p.ldy + col0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (col0 + i < p.N) y[i] = __uint_as_float(r[i]) * alpha;
+            for (int c = 0; c < 32; ++c)
+              if (col0 + c < p.N) y[c] = __uint_as_float(r[c]) * alpha;
           }
         }
+      };
+
+      // The accumulator columns the next tile writes have been read: hand them back.
+      auto release = [&]() {
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (CG == 1) ptx::mbar_arrive(acc_empty + acc);
+          else ptx::mbar_arrive_remote(leader(acc_empty + acc));
+        }
+      };
+      {
+        uint32_t r[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_ld_32x32b_x32(lane_addr + p1_tcol + c * 32, r[c]);
+        ptx::tmem_ld_wait();
+        if constexpr (C::OVERLAP) release();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) emit(r[c], m.n0 + p1_ocol + c * 32);
       }
-      if (++acc == C::NUM_ACC) { acc = 0; acc_phase ^= 1; }
+      if constexpr (BN == 256) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld_32x32b_x32(lane_addr + p2_tcol + c * 32, r);
+          ptx::tmem_ld_wait();
+          if (!C::OVERLAP && c == 3) release();
+          emit(r, m.n0 + p2_ocol + c * 32);
+        }
+      }
+      if (++acc == C::ACC_SLOTS) { acc = 0; acc_phase ^= 1; }
     }
     if (lane == 0) ptx::bulk_wait_all();
   }
 
   ptx::tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) {
+    // Neither CTA leaves (or frees TMEM) while the other may still signal its barriers or, for
+    // the leader's MMAs, write its TMEM.
+    ptx::cluster_sync();
+  }
+  if (*abort_flag) {
+    // Copies of the peer that this CTA could not observe: give them time to land.
+    const uint64_t t0 = now_ns();
+    while (now_ns() - t0 < 100000ull) {}
+  }
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+    ptx::tmem_dealloc<CG>(tmem, C::TMEM_COLS);
   }
 }
 
@@ -407,26 +544,59 @@ int sm_count() {
   return n;
 }
 
-template <int BN>
-fs_status launch_bn(const TcLaunch& L, TcParams prm, cudaStream_t s) {
-  using C = Cfg<BN>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(splice_gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+template <int BN, int CG>
+fs_status set_smem_attr() {
+  static bool done = false;
+  if (!done) {
+    cudaError_t e = cudaFuncSetAttribute(splice_gemm_tc_kernel<BN, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<BN, CG>::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm: smem attribute");
-    attr = true;
+    done = true;
   }
+  return FS_OK;
+}
+
+// Number of CTA pairs that can be resident at once (clusters must fit inside a GPC, so this can
+// be below half the SM count); 0 when the query fails.
+int pair_slots() {
+  static int n = -1;
+  if (n < 0) {
+    n = 0;
+    if (set_smem_attr<256, 2>() != FS_OK) return n;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(sm_count() & ~1));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Cfg<256, 2>::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, splice_gemm_tc_kernel<256, 2>, &cfg) == cudaSuccess && c > 0) n = c;
+    else cudaGetLastError();
+  }
+  return n;
+}
+
+template <int BN, int CG>
+fs_status launch_cfg(const TcLaunch& L, TcParams prm, int units, cudaStream_t s) {
+  using C = Cfg<BN, CG>;
+  fs_status st = set_smem_attr<BN, CG>();
+  if (st != FS_OK) return st;
   prm.BN = BN;
   prm.n_tiles = static_cast<int>(ceil_div(prm.N, BN));
   CUtensorMap tmA, tmB, tmSA, tmSB;
   const uint64_t kbytes = static_cast<uint64_t>(prm.K) / 2;
-  fs_status st = make_map(&tmA, L.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, L.a_rows, kbytes, 128, kBM);
-  if (st == FS_OK) st = make_map(&tmB, L.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, L.b_rows, kbytes, 128, BN);
+  st = make_map(&tmA, L.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, L.a_rows, kbytes, 128, kBM);
+  if (st == FS_OK) st = make_map(&tmB, L.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, L.b_rows, kbytes, 128, C::B_ROWS);
   if (st != FS_OK) return st;
   if (prm.ST > 0) {
     const uint64_t pp = static_cast<uint64_t>(L.pp);
     st = make_map(&tmSA, L.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, L.a_rows, pp * 2, 64, kBM);
-    if (st == FS_OK) st = make_map(&tmSB, L.ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, L.b_rows, pp * 2, 64, BN);
+    if (st == FS_OK) st = make_map(&tmSB, L.ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, L.b_rows, pp * 2, 64, C::B_ROWS);
     if (st != FS_OK) return st;
   } else {
     tmSA = tmA;
@@ -446,8 +616,24 @@ fs_status launch_bn(const TcLaunch& L, TcParams prm, cudaStream_t s) {
                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(FS_ERR_CUDA, "cuTensorMapEncodeTiled (Y) failed (%d)", static_cast<int>(r));
   }
-  const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(L.max_tiles, 1), sm_count()));
-  splice_gemm_tc_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, s>>>(tmA, tmB, tmSA, tmSB, tmY, prm);
+  if constexpr (CG == 1) {
+    splice_gemm_tc_kernel<BN, 1><<<units, kThreads, C::SMEM_BYTES, s>>>(tmA, tmB, tmSA, tmSB, tmY, prm);
+  } else {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * units));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, splice_gemm_tc_kernel<256, 2>, tmA, tmB, tmSA, tmSB, tmY, prm);
+    if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm (tensor-core path, CTA pairs)");
+  }
   FS_CHECK_LAUNCH("fs_splice_gemm (tensor-core path)");
   return FS_OK;
 }
@@ -456,8 +642,19 @@ fs_status launch_bn(const TcLaunch& L, TcParams prm, cudaStream_t s) {
 
 fs_status launch_splice_gemm_tc(const TcLaunch& L, const TcParams& prm, cudaStream_t s) {
   if (prm.E > kMaxExperts) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm: at most %d experts", kMaxExperts);
-  if (L.bn == 256) return launch_bn<256>(L, prm, s);
-  return launch_bn<128>(L, prm, s);
+  const int64_t m_tiles = ceil_div(L.a_rows, kBM);
+  // Dense problems with N % 256 == 0 and at least two 128-row tiles run on CTA pairs.
+  if (L.bn == 256 && !prm.offsets && m_tiles >= 2) {
+    const int slots = pair_slots();
+    if (slots > 0) {
+      const int64_t tiles = ceil_div(L.a_rows, 2 * kBM) * (prm.N / 256);
+      const int units = static_cast<int>(std::min<int64_t>(tiles, slots));
+      return launch_cfg<256, 2>(L, prm, units, s);
+    }
+  }
+  const int units = static_cast<int>(std::min<int64_t>(std::max<int64_t>(L.max_tiles, 1), sm_count()));
+  if (L.bn == 256) return launch_cfg<256, 1>(L, prm, units, s);
+  return launch_cfg<128, 1>(L, prm, units, s);
 }
 
 }  // namespace fs

@@ -121,6 +121,20 @@ def test_full_size_prefill_sampled_rows(N, K):
     _assert_close(Y[torch.from_numpy(rows).cuda()], Yr, mag)
 
 
+@pytest.mark.parametrize("M,N,K,p", [(4096, 2048, 1024, 256), (2000, 1536, 2048, 130)])
+def test_tensor_core_pairs_several_tiles_sampled_rows(M, N, K, p):
+    """More 256 x 256 tiles than CTA pairs, so pairs run several tiles (both accumulator
+    positions); p = 256 puts four BF16 k-tiles after every four FP4 k-tiles.  Sampled rows
+    include both sides of every 128-row boundary of the first tiles and the ragged end."""
+    X, W, Xt, Wt, P, gA = _problem(93 + M, M, N, K, p)
+    Y, _ = _run_gpu(Xt, Wt, P, gA, p, N, K, plan_opts=F.FS_PATH_TENSOR)
+    rng = np.random.default_rng(M + N)
+    rows = np.unique(np.concatenate([[0, 127, 128, 255, 256, 383, 384, M - 1],
+                                     rng.choice(M, 40, replace=False)]))
+    Yr, mag = _ref(X, W, P, gA, rows=rows)
+    _assert_close(Y[torch.from_numpy(rows).cuda()], Yr, mag)
+
+
 def test_repeatable_and_overwrites_output():
     X, W, Xt, Wt, P, gA = _problem(92, 256, 512, 1024, 64)
     Y1, _ = _run_gpu(Xt, Wt, P, gA, 64, 512, 1024)

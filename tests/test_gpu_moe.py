@@ -116,3 +116,14 @@ def test_grouped_moe_config_sampled():
             wq = splice.prepare_weights(nvfp4.bf16_value(Ws[e]), Ps[e], gAs[e])
             Yr, mag = splice.splice_gemm(xq, wq, wq["alpha"])
             assert np.all(np.abs(Yc[r0 + sel] - Yr) <= 1e-5 * mag), f"expert {e} (N={N}, K={K})"
+
+
+@pytest.mark.parametrize("N", [512, 384])
+def test_grouped_more_tiles_than_sms_side_heavy(N):
+    """Enough tiles (> 148) that every CTA runs several, with p = 256 so that four BF16 k-tiles
+    follow two FP4 k-tiles; N = 512 takes 256-column tiles, N = 384 128-column tiles."""
+    counts = [300, 200, 129] * 20
+    K, p = 512, 256
+    E, offs, Xs, Ws, Ps, gAs = _build(counts, N, K, p, seed=3)
+    _, Y = _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p)
+    _check_expert_outputs(offs, Xs, Ws, Ps, gAs, Y, rows_per_expert=6)
