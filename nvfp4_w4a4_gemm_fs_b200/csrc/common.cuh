@@ -103,6 +103,27 @@ __device__ __forceinline__ float div_markstein(float y, float d, float r) {
   return __uint_as_float((__float_as_uint(q2) & 0x7FFFFFFFu) | (__float_as_uint(y) & 0x80000000u));
 }
 
+// Fast path of v = fl32(fl32(x*g)/sf) for the E2M1 decision, valid for bf16 x (at most 8
+// significant bits), a power-of-two g in [2^-100, 2^100] and a UE4M3 scale sf (at most 4
+// significant bits; sf_rcp = RN(1/sf), or 0 for the zero scale).
+//
+// The E2M1 code depends only on where q = x*g/sf lies relative to the rounding midpoints
+// mu/4, mu in {1,3,5,7,10,14,20}.  x*g - (mu/4)*sf is a difference of an 8-bit and a 7-bit
+// integer multiple of powers of two, so unless it is zero, |q - mu/4| >= 2^-8.3 * mu/4.
+// q' = RN(x * RN(g*sf_rcp)) is within 2^-22.9 of q, relatively, and rounding q' to 12
+// significant bits returns mu/4 exactly when q == mu/4 (a tie, which the E2M1 conversion then
+// breaks to even) and moves no other value across a midpoint.  The fp32 rounding of q in the
+// exact formula cannot create a tie either (q is at least 2^-8.3 away), so both give the same
+// code, the sign of zero included (the rounding keeps the sign bit).
+__device__ __forceinline__ float snap12(float v) {
+  return __uint_as_float((__float_as_uint(v) + 0x800u) & 0xFFFFF000u);
+}
+__device__ __forceinline__ bool pow2_gain_in_fast_range(float g) {
+  const uint32_t b = __float_as_uint(g);
+  const uint32_t e = b >> 23;                   // g > 0 here, sign bit clear
+  return (b & 0x7FFFFFu) == 0 && e >= 127u - 100u && e <= 127u + 100u;
+}
+
 // Packs two fp32 values into one byte of E2M1 codes (round to nearest even, saturating at 6),
 // `lo` into the low nibble.  The PTX conversion places its first source in the high nibble.
 __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {

@@ -109,12 +109,15 @@ struct ChunkLoc {
 // expert's padded region (rows_per_cta divides 128).  Each thread owns one 16-element block per
 // pass; the load of the next pass (or of the next chunk) is issued before the current block is
 // computed, so every thread keeps a load in flight.  Divisions by the UE4M3 scale use per-code
-// tables of the scale value and its reciprocal in shared memory.
-template <typename T, Side kSide, bool kGrouped>
+// tables of the scale value and its reciprocal in shared memory; for bf16 input under a
+// power-of-two gain the division is replaced by one multiply and a 12-bit snap (snap12), which
+// yields the same codes.
+template <typename T, Side kSide, bool kGrouped, bool kOneRow>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_t nchunks) {
   __shared__ uint16_t sh_mbits[16384 / 16];             // protected lanes of each 16-element block
   __shared__ uint4 sh_kill[sizeof(T) == 2 ? 2 * 16384 / 16 : 1];   // bf16: per block, 8 words of lanes to clear
   __shared__ uint16_t sh_col[16384 / 16];               // side-buffer column of each block's first protected lane
+  __shared__ uint16_t sh_pidx[256];                     // channel of each side-buffer column (p <= 256)
   __shared__ float sh_val[128], sh_rcp[128];            // UE4M3 value and RN(1/value) per code
   __shared__ int64_t sh_pad[kGrouped ? kMaxGroupedExperts + 1 : 1];   // padded start of each expert
   __shared__ int64_t sh_off[kGrouped ? kMaxGroupedExperts + 1 : 1];   // row offsets of the experts
@@ -169,7 +172,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
   if constexpr (kSide == Side::Weight) alpha_v = __ldg(a.alpha);
   const float inv6 = __frcp_rn(6.0f);
 
-  const bool one_row = a.rows_per_cta == 1;
+  constexpr bool one_row = kOneRow;                   // rows_per_cta == 1: chunk = one row
   auto load_one = [&](const ChunkLoc& L, int i0, RawBlock<T>& x) {
     const int i = i0 + tid;
     const int r = one_row ? 0 : i / a.nb;
@@ -185,12 +188,14 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
   int cur_e = -1;
   const uint32_t* mask = nullptr;
   float g = 1.0f;
+  bool fast = false;                               // snap12 path (bf16 input, power-of-two gain)
 
   for (int64_t chunk = blockIdx.x; chunk < nchunks && L.e >= 0; chunk += gridDim.x) {
     if (L.e != cur_e) {                            // uniform across the CTA
       cur_e = L.e;
       mask = (a.p > 0) ? a.masks + static_cast<int64_t>(cur_e) * words : nullptr;
       g = __ldg(a.gains + cur_e);
+      fast = sizeof(T) == 2 && pow2_gain_in_fast_range(g);
       if (a.p > 0) {
         __syncthreads();                           // previous expert's tables no longer read
         // per block: its 16 mask bits and the side column of its first protected lane
@@ -213,6 +218,17 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
               sh_col[b] = static_cast<uint16_t>(carry + incl - cnt);
             }
             carry += __shfl_sync(0xffffffffu, incl, 31);
+          }
+        }
+        __syncthreads();
+        // channel of every side column: the protected channels in ascending order
+        for (int b = tid; b < nb; b += kQThreads) {
+          uint32_t mb = sh_mbits[b];
+          int col = sh_col[b];
+          while (mb) {
+            const int j = __ffs(mb) - 1;
+            mb &= mb - 1;
+            sh_pidx[col++] = static_cast<uint16_t>(b * 16 + j);
           }
         }
         if constexpr (sizeof(T) == 2) {
@@ -266,36 +282,20 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
         sfc = ue4m3_rne(t);
         const float sd = sh_val[sfc], sr = sh_rcp[sfc];
         float v[16];
+        if (fast) {
+          const float R = __fmul_rn(g, sr);        // exact: g is a power of two in range
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = div_markstein(__fmul_rn(xm.get(j), g), sd, sr);
+          for (int j = 0; j < 16; ++j) v[j] = snap12(__fmul_rn(xm.get(j), R));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = div_markstein(__fmul_rn(xm.get(j), g), sd, sr);
+        }
         const uint32_t lo = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
         const uint32_t hi = e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
         *reinterpret_cast<uint2*>(a.q + prow * (a.K / 2) + static_cast<int64_t>(b) * 8) = make_uint2(lo, hi);
-        // Extract the protected lanes into the side buffer.
-        if (mbits) {
-          int col = sh_col[b];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if ((mbits >> j) & 1u) {
-              uint16_t hv;
-              if constexpr (kSide == Side::Activation) {
-                hv = f32_to_bf16_bits(x.get(j));
-              } else {
-                const float wb = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_bits(x.get(j))) << 16);
-                hv = f32_to_bf16_bits(__fdiv_rn(wb, alpha_v));
-              }
-              a.side[prow * a.pp + col] = hv;
-              ++col;
-            }
-          }
-        }
-        if (b == 0)
-          for (int c = a.p; c < a.pp; ++c) a.side[prow * a.pp + c] = 0;
       } else if (in_range && kGrouped) {
-        // padding rows of a grouped buffer: zero codes and side columns
+        // padding rows of a grouped buffer: zero codes (their side columns are zeroed below)
         *reinterpret_cast<uint2*>(a.q + prow * (a.K / 2) + static_cast<int64_t>(b) * 8) = make_uint2(0, 0);
-        if (b == 0)
-          for (int c = 0; c < a.pp; ++c) a.side[prow * a.pp + c] = 0;
       }
       // Gather the 4 scales of blocks b..b+3 (same row since K/16 % 4 == 0) into one word.
       const uint32_t s1 = __shfl_down_sync(0xffffffffu, sfc, 1);
@@ -305,15 +305,39 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
         *reinterpret_cast<uint32_t*>(a.sf + sf_offset(prow, b, a.kb4)) = sfc | (s1 << 8) | (s2 << 16) | (s3 << 24);
       xc = xn;
     }
+    // Extract X_S: side column c of each row is channel sh_pidx[c] (the block data is still in
+    // L1/L2), zero in the padding columns p..pp-1 and in the padding rows of a grouped buffer.
+    if (a.pp > 0) {
+      for (int idx = tid; idx < a.rows_per_cta * a.pp; idx += kQThreads) {
+        const int r = idx / a.pp;
+        const int c = idx - r * a.pp;
+        const bool data = r < L.valid;
+        if (!data && !kGrouped) continue;
+        uint16_t hv = 0;
+        if (data && c < a.p) {
+          const T* src = X + (L.src_row0 + r) * a.ldx + sh_pidx[c];
+          float xv;
+          if constexpr (sizeof(T) == 2) xv = __uint_as_float(static_cast<uint32_t>(__ldg(src)) << 16);
+          else xv = __ldg(src);
+          if constexpr (kSide == Side::Activation) {
+            hv = f32_to_bf16_bits(xv);
+          } else {
+            const float wb = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_bits(xv)) << 16);
+            hv = f32_to_bf16_bits(__fdiv_rn(wb, alpha_v));
+          }
+        }
+        a.side[(L.prow0 + r) * a.pp + c] = hv;
+      }
+    }
     L = Ln;
   }
 }
 
 // Max |W| over the unprotected columns (all columns in the residual form) as float bits.
-template <typename T>
-__global__ void __launch_bounds__(256) weight_amax_kernel(const T* __restrict__ W, int64_t N, int K, int64_t ldw,
-                                                          const uint32_t* __restrict__ mask, uint32_t opts,
-                                                          uint32_t* out_bits) {
+// fp32 weights (small problems): one 16-element block per thread.
+__global__ void __launch_bounds__(256) weight_amax_f32_kernel(const float* __restrict__ W, int64_t N, int K, int64_t ldw,
+                                                              const uint32_t* __restrict__ mask, uint32_t opts,
+                                                              uint32_t* out_bits) {
   const bool residual = opts & FS_RESIDUAL;
   const int64_t total = N * (K / 16);
   float m = 0.0f;
@@ -322,7 +346,7 @@ __global__ void __launch_bounds__(256) weight_amax_kernel(const T* __restrict__ 
     const int64_t r = i / (K / 16);
     const int b = static_cast<int>(i % (K / 16));
     float x[16];
-    load_block<T>(W + r * ldw + static_cast<int64_t>(b) * 16, x);
+    load_block<float>(W + r * ldw + static_cast<int64_t>(b) * 16, x);
     const uint32_t mbits = (mask && !residual) ? ((__ldg(mask + (b >> 1)) >> ((b & 1) * 16)) & 0xFFFFu) : 0u;
 #pragma unroll
     for (int j = 0; j < 16; ++j)
@@ -332,6 +356,67 @@ __global__ void __launch_bounds__(256) weight_amax_kernel(const T* __restrict__ 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) bits = max(bits, __shfl_xor_sync(0xffffffffu, bits, o));
   if ((threadIdx.x & 31) == 0 && bits) atomicMax(out_bits, bits);
+}
+
+// bf16 weights: a streaming reduction.  Each warp takes whole rows, lane l the 8 columns
+// 8l..8l+7 of every 256-column stripe, four 16-byte loads in flight.  |w| of a bf16 value orders
+// like its low 15 bits, so the maximum is taken on packed 16-bit halves (max.u16x2) after
+// clearing sign bits and protected lanes; the result, shifted to the high half, is the float.
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__global__ void __launch_bounds__(256) weight_amax_bf16_kernel(const uint16_t* __restrict__ W, int64_t N, int K,
+                                                               int64_t ldw, const uint32_t* __restrict__ mask,
+                                                               uint32_t opts, uint32_t* out_bits) {
+  const bool use_mask = mask && !(opts & FS_RESIDUAL);
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int stripes = K / 256;                 // K % 64 == 0; a ragged last stripe is handled below
+  const int tail_cols = K - stripes * 256;
+  uint32_t m = 0;
+  // Clears the lanes of column c0..c0+7 that are protected, and every sign bit.
+  auto keep = [&](int c0) -> uint4 {
+    uint32_t k8 = 0;
+    if (use_mask) k8 = (__ldg(mask + (c0 >> 5)) >> (c0 & 31)) & 0xFFu;
+    uint4 r;
+    uint32_t* rw = &r.x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t two = (k8 >> (2 * j)) & 3u;
+      rw[j] = 0x7FFF7FFFu & ~(((two & 1u) | ((two & 2u) << 15)) * 0xFFFFu);
+    }
+    return r;
+  };
+  auto fold = [&](const uint4& v, const uint4& k) {
+    m = vmax_u16x2(m, v.x & k.x);
+    m = vmax_u16x2(m, v.y & k.y);
+    m = vmax_u16x2(m, v.z & k.z);
+    m = vmax_u16x2(m, v.w & k.w);
+  };
+  for (int64_t r = warp; r < N; r += nwarps) {
+    const uint16_t* row = W + r * ldw;
+    int s = 0;
+    for (; s + 4 <= stripes; s += 4) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(row + (s + u) * 256 + lane * 8));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) fold(v[u], keep((s + u) * 256 + lane * 8));
+    }
+    for (; s < stripes; ++s) fold(__ldg(reinterpret_cast<const uint4*>(row + s * 256 + lane * 8)), keep(s * 256 + lane * 8));
+    if (tail_cols && lane * 8 < tail_cols) {
+      const int c0 = stripes * 256 + lane * 8;
+      fold(__ldg(reinterpret_cast<const uint4*>(row + c0)), keep(c0));
+    }
+  }
+  uint32_t bits = max(m & 0xFFFFu, m >> 16) << 16;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) bits = max(bits, __shfl_xor_sync(0xffffffffu, bits, o));
+  if (lane == 0 && bits) atomicMax(out_bits, bits);
 }
 
 // gW from the reduced amax bits (stored in the gW slot), then alpha = fl32(1/fl32(gA*gW)).
@@ -361,7 +446,9 @@ fs_status launch_quantize(int dtype, QuantArgs& a, int64_t padded_rows, cudaStre
   a.rows_per_cta = rpc;
   const int64_t chunks = ceil_div(padded_rows, rpc);
   if (chunks == 0) return FS_OK;
-  auto kernel = dtype == FS_DTYPE_BF16 ? quantize_kernel<uint16_t, kSide, kGrouped> : quantize_kernel<float, kSide, kGrouped>;
+  auto kernel = dtype == FS_DTYPE_BF16
+                    ? (rpc == 1 ? quantize_kernel<uint16_t, kSide, kGrouped, true> : quantize_kernel<uint16_t, kSide, kGrouped, false>)
+                    : (rpc == 1 ? quantize_kernel<float, kSide, kGrouped, true> : quantize_kernel<float, kSide, kGrouped, false>);
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQThreads, 0) != cudaSuccess || per_sm < 1) per_sm = 2;
   const int64_t grid = std::min<int64_t>(chunks, static_cast<int64_t>(quant_sm_count()) * per_sm);
@@ -430,13 +517,16 @@ extern "C" fs_status fs_prepare_weights(const void* W, int32_t dtype, int32_t N,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(gW, 0, sizeof(float), s);
   if (e != cudaSuccess) return cuda_status(e, "fs_prepare_weights: memset");
-  const int64_t blocks = static_cast<int64_t>(N) * (K / 16);
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(blocks, 256), 148 * 8));
   const uint32_t* m = p > 0 ? mask : nullptr;
-  if (dtype == FS_DTYPE_BF16)
-    weight_amax_kernel<uint16_t><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), N, K, ldw, m, opts, reinterpret_cast<uint32_t*>(gW));
-  else
-    weight_amax_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(W), N, K, ldw, m, opts, reinterpret_cast<uint32_t*>(gW));
+  if (dtype == FS_DTYPE_BF16) {
+    // one warp per row, 8 warps per CTA, at most 8 CTAs per SM
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(N, 8), static_cast<int64_t>(quant_sm_count()) * 8));
+    weight_amax_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), N, K, ldw, m, opts, reinterpret_cast<uint32_t*>(gW));
+  } else {
+    const int64_t blocks = static_cast<int64_t>(N) * (K / 16);
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(blocks, 256), 148 * 8));
+    weight_amax_f32_kernel<<<grid, 256, 0, s>>>(static_cast<const float*>(W), N, K, ldw, m, opts, reinterpret_cast<uint32_t*>(gW));
+  }
   FS_CHECK_LAUNCH("fs_prepare_weights: amax");
   weight_gain_kernel<<<1, 1, 0, s>>>(gW, alpha, gA, opts);
   FS_CHECK_LAUNCH("fs_prepare_weights: gain");

@@ -57,6 +57,26 @@ __device__ __forceinline__ void add_bf16(SmallSums& a, float x, bool& bad) {
   a.d2 += __float_as_uint(__fmaf_rn(yl, 16384.0f, kMagic));
 }
 
+// NaN-propagating maximum (a NaN operand makes the result NaN).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// The same raw-bit terms as add_bf16 for an element known to be finite and in range.
+__device__ __forceinline__ void add_bf16_in_range(uint32_t& a1, uint32_t& b1, uint32_t& c2, uint32_t& d2, float x) {
+  const float t1 = __fadd_rn(x, kMagic);
+  a1 += __float_as_uint(t1);
+  const float frac = __fsub_rn(x, __fsub_rn(t1, kMagic));
+  b1 += __float_as_uint(__fmaf_rn(frac, 65536.0f, kMagic));
+  const float y = __fmul_rn(x, x);
+  const float u = __fadd_rn(y, kMagic8);
+  c2 += __float_as_uint(u);
+  const float yl = __fsub_rn(y, __fsub_rn(u, kMagic8));
+  d2 += __float_as_uint(__fmaf_rn(yl, 16384.0f, kMagic));
+}
+
 // fp32 inputs (small problems): convert directly.
 __device__ __forceinline__ void add_f32(long long& s1, long long& s2, float& amax, float x, bool& bad) {
   const float ax = fabsf(x);
@@ -76,7 +96,7 @@ __device__ __forceinline__ void add_f32(long long& s1, long long& s2, float& ama
 // 64-bit totals in its own shared-memory slots ([warp][v][lane], conflict-free); the CTA reduces
 // them over warps and adds to the global state with integer atomics.
 template <typename T, int VEC>
-__global__ void __launch_bounds__(kStatsWarps * 32)
+__global__ void __launch_bounds__(kStatsWarps * 32, 3)
 channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int row_stride,
                      unsigned long long* n, unsigned long long* s1, unsigned long long* s2,
                      uint32_t* amax, uint32_t* flags) {
@@ -97,6 +117,27 @@ channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int
   float am[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) am[v] = 0.0f;
+  // bf16: raw-bit sums of up to kRawRows rows in wrapping 32-bit registers.  The largest term,
+  // yh/2^8 < 2^22, keeps the exact sum of 256 rows inside int32.
+  constexpr int kRawRows = 256;
+  uint32_t ra1[VEC], rb1[VEC], rc2[VEC], rd2[VEC];
+  int raw_rows = 0;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) { ra1[v] = 0u; rb1[v] = 0u; rc2[v] = 0u; rd2[v] = 0u; }
+  auto flush_raw = [&]() {
+    const uint32_t n_rows = static_cast<uint32_t>(raw_rows);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      const int A1 = static_cast<int>(ra1[v] - n_rows * kMagicBits);
+      const int B1 = static_cast<int>(rb1[v] - n_rows * kMagicBits);
+      const int C2 = static_cast<int>(rc2[v] - n_rows * kMagic8Bits);
+      const int D2 = static_cast<int>(rd2[v] - n_rows * kMagicBits);
+      sh_s1[warp][v][lane] += static_cast<long long>(A1) * 65536 + B1;
+      sh_s2[warp][v][lane] += static_cast<long long>(C2) * 4194304 + D2;   // yh*2^14 = (yh/2^8)*2^22
+      ra1[v] = 0u; rb1[v] = 0u; rc2[v] = 0u; rd2[v] = 0u;
+    }
+    raw_rows = 0;
+  };
 
   const int64_t taken = (M + row_stride - 1) / row_stride;     // rows 0, s, 2s, ...
   const int64_t step = static_cast<int64_t>(gridDim.y) * kStatsWarps;
@@ -123,27 +164,37 @@ channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int
           for (int v = 0; v < 4; ++v) add_f32(sh_s1[warp][v][lane], sh_s2[warp][v][lane], am[v], xs[v], bad);
         }
       } else {
-        // zero rows past the end contribute rint(0) = 0 (their raw bits are the magic patterns,
-        // removed below with the count of kUnroll rows)
+        // Zero rows past the end contribute rint(0) = 0: their raw bits are the magic patterns,
+        // removed with the row count.  A batch of kUnroll rows of a channel whose NaN-propagating
+        // maximum is in range takes the select-free path; otherwise (rare) each element is
+        // checked, out-of-range ones add the zero pattern and raise the flag.
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
-          SmallSums a{0u, 0u, 0u, 0u, am[v]};
+          float xs[kUnroll];
+          float mx = 0.0f;
 #pragma unroll
           for (int u = 0; u < kUnroll; ++u) {
             const uint32_t w = (&q[u].x)[v >> 1];
-            add_bf16(a, (v & 1) ? bf16_hi(w) : bf16_lo(w), bad);
+            xs[u] = (v & 1) ? bf16_hi(w) : bf16_lo(w);
+            mx = fmax_nan(mx, fabsf(xs[u]));
           }
-          am[v] = a.amax;
-          const int A1 = static_cast<int>(a.a1 - kUnroll * kMagicBits);
-          const int B1 = static_cast<int>(a.b1 - kUnroll * kMagicBits);
-          const int C2 = static_cast<int>(a.c2 - kUnroll * kMagic8Bits);
-          const int D2 = static_cast<int>(a.d2 - kUnroll * kMagicBits);
-          sh_s1[warp][v][lane] += static_cast<long long>(A1) * 65536 + B1;
-          sh_s2[warp][v][lane] += static_cast<long long>(C2) * 4194304 + D2;   // yh*2^14 = (yh/2^8)*2^22
+          if (mx < kRangeLimit) {
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) add_bf16_in_range(ra1[v], rb1[v], rc2[v], rd2[v], xs[u]);
+            am[v] = fmaxf(am[v], mx);
+          } else {
+            SmallSums a{ra1[v], rb1[v], rc2[v], rd2[v], am[v]};
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) add_bf16(a, xs[u], bad);
+            ra1[v] = a.a1; rb1[v] = a.b1; rc2[v] = a.c2; rd2[v] = a.d2; am[v] = a.amax;
+          }
         }
+        raw_rows += kUnroll;
+        if (raw_rows + kUnroll > kRawRows) flush_raw();
       }
     }
   }
+  if constexpr (!kF32) flush_raw();
 #pragma unroll
   for (int v = 0; v < VEC; ++v) sh_am[warp][v][lane] = am[v];
   if (bad) atomicOr(&sh_bad, 1);
