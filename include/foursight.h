@@ -203,8 +203,10 @@ fs_status fs_plan_check(fs_plan plan, void* stream);
 
 /* Packed operands as written above (activation rows M; weight rows N = the plan's N), p <= the
  * plan's p_max; alpha: device float.  Y [M][ldy] fp32 (bf16 with FS_OUT_BF16 in the plan's
- * opts), ldy >= N, 16-byte aligned rows.  M <= 16 runs the weight-streaming decode kernel, larger
- * M the tcgen05 tensor-core kernel (FS_PATH_TENSOR / FS_PATH_DECODE in the plan's opts force one).
+ * opts), ldy >= N, 16-byte aligned rows.  M <= 16 runs the weight-streaming decode kernel (weights
+ * as the 128-row operand of tcgen05 block-scaled MMAs with the tokens as N = 16, K split over a
+ * thread-block cluster), larger M the tcgen05 prefill kernel (FS_PATH_TENSOR / FS_PATH_DECODE in
+ * the plan's opts force one).
  * Plan requirements: N % 16 == 0 and K % 256 == 0 (FS_ERR_UNSUPPORTED otherwise); the packed
  * operands must be 16-byte aligned.  The output is not accumulated into: Y is overwritten. */
 fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, const uint8_t* sfx,

@@ -93,8 +93,8 @@ extern "C" fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const ui
     d.M = static_cast<int>(M); d.N = plan->N; d.K = plan->K; d.pp = pp;
     d.kb4 = static_cast<int>(round_up(plan->K / 16, 4) / 4);
     d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha;
-    d.Y = Y; d.ldy = ldy; d.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0;
-    return launch_splice_gemm_decode(d, s);
+    d.Y = Y; d.ldy = ldy; d.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; d.err = plan->err;
+    return launch_splice_gemm_decode_tc(d, s);
   }
   if (M > (int64_t{1} << 31) - 256) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm: M too large");
   TcParams prm{};

@@ -1,5 +1,7 @@
 // Internal launch interface shared by the SpliceGEMM kernels and the ABI layer.
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace fs {
@@ -34,6 +36,11 @@ struct TcLaunch {
 
 fs_status launch_splice_gemm_tc(const TcLaunch& L, const TcParams& prm, cudaStream_t s);
 
+// 2D K-major tensor map, 128-byte swizzle, box `box_inner` elements x `box_rows` rows.
+fs_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner_elems, uint64_t rows,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows);
+int sm_count();
+
 struct DecodeParams {
   int M, N, K, pp, kb4;
   const uint8_t* xq;
@@ -46,8 +53,9 @@ struct DecodeParams {
   void* Y;
   int64_t ldy;
   int out_bf16;
+  uint32_t* err;      // device error word (bounded-wait timeouts of the tensor-core decode kernel)
 };
 
-fs_status launch_splice_gemm_decode(const DecodeParams& p, cudaStream_t s);
+fs_status launch_splice_gemm_decode_tc(const DecodeParams& p, cudaStream_t s);
 
 }  // namespace fs

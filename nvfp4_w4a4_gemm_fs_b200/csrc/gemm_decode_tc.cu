@@ -1,0 +1,326 @@
+// SpliceGEMM decode path (M <= 16 tokens) on the 5th-generation tensor cores.
+//
+// FourSight §5.1 "Dual-path execution": for small M the product is bound by streaming the packed
+// weights once.  Here the weights are the MMA's 128-row A operand and the (at most 16) tokens its
+// N = 16 B operand, so the block-scaled tcgen05 MMA (kind::mxf4nvf4) applies the UE4M3 scales in
+// hardware and the SMs only move bytes.  To put every SM on the weight stream, the K range of
+// each 128-row tile is split over the CTAs of a thread-block cluster (up to 8 along grid y); each
+// CTA accumulates its part in TMEM, and the partials are summed in a fixed order through
+// distributed shared memory, scaled by alpha once and stored.  The protected slice X_S W'_S^T
+// (§4.2 Eq. 5) runs as BF16 MMAs (kind::f16) into the TMEM accumulator of the cluster's last CTA.
+//   warp 0      TMA producer: per k-tile a 128 x 128-byte box of W and a 16 x 128-byte box of the
+//               packed activations (rows past M read as zero), plus both tiles' scale atoms (bulk
+//               copies); the BF16 side tiles use the same boxes, 64 bf16 wide
+//   warp 1      TMEM allocation; one thread copies the scale atoms to TMEM (tcgen05.cp, ordered
+//               before its MMAs) and issues the MMAs
+//   warps 2..5  epilogue: TMEM -> shared-memory partial; after a cluster barrier each CTA sums a
+//               contiguous share of the tile's outputs over all CTAs of the cluster, x alpha, store
+// Every mbarrier wait is bounded; on expiry the kernel records a timeout in the error word and
+// still reaches both cluster barriers and releases TMEM.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace fs {
+namespace {
+
+constexpr int kDThreads = 192;
+constexpr int kDRows = 128;          // weight rows per tile (MMA M)
+constexpr int kDTok = 16;            // token columns (MMA N)
+constexpr int kDStages = 4;
+constexpr int kDMaxSplit = 8;        // portable cluster size
+constexpr uint64_t kDWaitNs = 2000000000ull;
+constexpr uint64_t kDDrainNs = 50000000ull;
+
+struct DCfg {
+  static constexpr int W_BYTES = kDRows * 128;      // 256 fp4 or 64 bf16 per row
+  static constexpr int X_BYTES = kDTok * 128;
+  static constexpr int SFW_BYTES = 2048;            // four 512-byte atoms, one per MMA
+  static constexpr int SFX_BYTES = 2048;
+  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;   // multiple of 1024
+  static constexpr int RED_BYTES = kDRows * kDTok * 4;                           // partial [token][row]
+  static constexpr int SMEM_BYTES = 1024 + kDStages * STAGE_BYTES + RED_BYTES + 8 * (2 * kDStages + 2) + 16;
+  static constexpr int TMEM_COLS = 128;
+  static constexpr int SF_COL = 32;                 // scale buffer b: SFA at SF_COL+32b, SFB at SF_COL+32b+16
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the 128-byte swizzle");
+  static_assert(SF_COL + 64 <= TMEM_COLS, "TMEM budget");
+};
+
+struct DecTcParams {
+  int M, N, KT, ST, kb4, kt_per, S;
+  const uint8_t* sfw;
+  const uint8_t* sfx;
+  const float* alpha;
+  void* Y;
+  int64_t ldy;
+  int out_bf16;
+  uint32_t* err;
+};
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* err) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 0) {
+      if (*abort_flag) return false;
+      if (now_ns() - t0 > kDWaitNs) {
+        if (err) atomicOr(err, ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = now_ns();
+  while (!ptx::mbar_try_wait(bar, parity))
+    if (now_ns() - t0 > limit_ns) return;
+}
+
+__global__ void __launch_bounds__(kDThreads, 1)
+splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                             const __grid_constant__ CUtensorMap tmWS, const __grid_constant__ CUtensorMap tmXS,
+                             const DecTcParams p) {
+  using C = DCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* red = reinterpret_cast<float*>(smem + kDStages * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDStages * C::STAGE_BYTES + C::RED_BYTES);
+  uint64_t* empty = full + kDStages;
+  uint64_t* acc_full = empty + kDStages;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(ptx::cluster_ctarank());     // K split inside the tile's cluster
+  const int n0 = static_cast<int>(blockIdx.x) * kDRows;
+  const int kt0 = rank * p.kt_per;
+  const int kt1 = kt0 + p.kt_per < p.KT ? kt0 + p.kt_per : p.KT;
+  const int nf = kt1 - kt0;                                       // FP4 k-tiles of this CTA (>= 1)
+  const int nk = nf + (rank == p.S - 1 ? p.ST : 0);              // + the BF16 side k-tiles
+  auto W_at = [&](int s) { return smem + s * C::STAGE_BYTES; };
+  auto X_at = [&](int s) { return smem + s * C::STAGE_BYTES + C::W_BYTES; };
+  auto SFW_at = [&](int s) { return smem + s * C::STAGE_BYTES + C::W_BYTES + C::X_BYTES; };
+  auto SFX_at = [&](int s) { return smem + s * C::STAGE_BYTES + C::W_BYTES + C::X_BYTES + C::SFW_BYTES; };
+
+  // Programmatic dependent launch: the next kernel may start its prologue now.  Pulling this
+  // CTA's weight boxes into L2 is safe before the wait (an L2 prefetch only); every real load and
+  // store comes after griddepcontrol.wait.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kDStages; ++s) { ptx::mbar_init(full + s, 1); ptx::mbar_init(empty + s, 1); }
+    ptx::mbar_init(acc_full, 1);
+    ptx::mbar_init(drain, 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tensormap(&tmW); ptx::prefetch_tensormap(&tmX);
+    if (p.ST > 0) { ptx::prefetch_tensormap(&tmWS); ptx::prefetch_tensormap(&tmXS); }
+    for (int kt = kt0; kt < kt1; ++kt) ptx::tma_prefetch_2d(&tmW, kt * 128, n0);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc<1>(tmem_slot, C::TMEM_COLS);
+    ptx::tmem_relinquish<1>();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      for (int i = 0; i < nk; ++i) {
+        if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err)) break;
+        if (i < nf) {
+          const int kt = kt0 + i;
+          ptx::mbar_arrive_expect_tx(full + stage, C::STAGE_BYTES);
+          ptx::tma_load_2d(W_at(stage), &tmW, kt * 128, n0, full + stage);
+          ptx::tma_load_2d(X_at(stage), &tmX, kt * 128, 0, full + stage);
+          ptx::bulk_load(SFW_at(stage), p.sfw + (static_cast<int64_t>(n0 / kDRows) * p.kb4 + kt * 4) * 512,
+                         C::SFW_BYTES, full + stage);
+          ptx::bulk_load(SFX_at(stage), p.sfx + static_cast<int64_t>(kt) * 4 * 512, C::SFX_BYTES, full + stage);
+        } else {
+          const int sk = i - nf;
+          ptx::mbar_arrive_expect_tx(full + stage, C::W_BYTES + C::X_BYTES);
+          ptx::tma_load_2d(W_at(stage), &tmWS, sk * 64, n0, full + stage);
+          ptx::tma_load_2d(X_at(stage), &tmXS, sk * 64, 0, full + stage);
+        }
+        ++issued;
+        if (++stage == kDStages) { stage = 0; phase ^= 1; }
+      }
+      if (*abort_flag) {
+        // copies issued but possibly not landed: the last min(issued, stages) stages
+        int s = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < kDStages && i < issued; ++i) {
+          if (--s < 0) { s = kDStages - 1; ph ^= 1; }
+          drain_bar(full + s, ph, kDDrainNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ scale copies + MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_f4 = ptx::idesc_nvf4(kDRows, kDTok);
+      constexpr uint32_t idesc_bf = ptx::idesc_bf16(kDRows, kDTok);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; i < nk; ++i) {
+        if (!wait_bar(full + stage, phase, abort_flag, p.err)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint64_t adesc = ptx::desc_kmajor_sw128(ptx::smem_u32(W_at(stage)));
+        const uint64_t bdesc = ptx::desc_kmajor_sw128(ptx::smem_u32(X_at(stage)));
+        if (i < nf) {
+          const uint32_t sfa = tmem + C::SF_COL + 32 * (i & 1);
+          const uint32_t sfb = sfa + 16;
+          const uint32_t sw = ptx::smem_u32(SFW_at(stage)), sx = ptx::smem_u32(SFX_at(stage));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            ptx::tc_cp_32x128b_warpx4(sfa + 4 * j, ptx::desc_sf_block(sw + 512 * j));
+            ptx::tc_cp_32x128b_warpx4(sfb + 4 * j, ptx::desc_sf_block(sx + 512 * j));
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            ptx::tc_mma_nvf4<1>(tmem, adesc + 2 * j, bdesc + 2 * j, idesc_f4, sfa + 4 * j, sfb + 4 * j, (i | j) != 0);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) ptx::tc_mma_bf16<1>(tmem, adesc + 2 * j, bdesc + 2 * j, idesc_bf, (i | j) != 0);
+        }
+        ptx::tc_commit<1>(empty + stage);
+        if (++stage == kDStages) { stage = 0; phase ^= 1; }
+      }
+      if (ok) ptx::tc_commit<1>(acc_full);
+      ptx::tc_commit<1>(drain);                    // every MMA issued above has completed
+      drain_bar(drain, 0, kDWaitNs);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue: TMEM -> partial
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    if (wait_bar(acc_full, 0, abort_flag, p.err)) {
+      ptx::tc_fence_after();
+      uint32_t r[16];
+      ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16), r);
+      ptx::tmem_ld_wait();
+#pragma unroll
+      for (int t = 0; t < kDTok; ++t) red[t * kDRows + row] = __uint_as_float(r[t]);
+    } else {
+#pragma unroll
+      for (int t = 0; t < kDTok; ++t) red[t * kDRows + row] = 0.0f;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();                             // every CTA's partial is in its shared memory
+  if (warp >= 2) {
+    // This CTA's share of the tile's outputs (token-major: consecutive rows of one token), four
+    // consecutive outputs per thread, summed over the cluster in rank order.  The S remote loads
+    // of a group are all issued before the first add, so their latencies overlap.
+    const int e = threadIdx.x - 64;
+    constexpr int kOut = kDRows * kDTok;
+    const int share = ((kOut + p.S - 1) / p.S + 3) & ~3;
+    const int v0 = rank * share;
+    const int v1 = v0 + share < kOut ? v0 + share : kOut;
+    const float alpha = __ldg(p.alpha);
+    const uint32_t red_addr = ptx::smem_u32(red);
+    for (int v = v0 + 4 * e; v < v1; v += 4 * 128) {
+      const int t = v / kDRows, rr = v - t * kDRows;   // 4 rows rr..rr+3 of token t
+      if (t >= p.M || n0 + rr >= p.N) continue;
+      float4 part[kDMaxSplit];
+#pragma unroll
+      for (int s2 = 0; s2 < kDMaxSplit; ++s2)
+        if (s2 < p.S) part[s2] = ptx::ld_shared_cluster_v4(ptx::mapa_shared(red_addr + 4u * v, s2));
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s2 = 0; s2 < kDMaxSplit; ++s2)
+        if (s2 < p.S) { sum.x += part[s2].x; sum.y += part[s2].y; sum.z += part[s2].z; sum.w += part[s2].w; }
+      const float y[4] = {sum.x * alpha, sum.y * alpha, sum.z * alpha, sum.w * alpha};
+      const int64_t off = static_cast<int64_t>(t) * p.ldy + n0 + rr;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (n0 + rr + q >= p.N) break;
+        if (p.out_bf16) static_cast<uint16_t*>(p.Y)[off + q] = f32_to_bf16_bits(y[q]);
+        else static_cast<float*>(p.Y)[off + q] = y[q];
+      }
+    }
+  }
+  ptx::cluster_sync();                             // no CTA leaves while another reads its partial
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc<1>(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+fs_status launch_splice_gemm_decode_tc(const DecodeParams& d, cudaStream_t s) {
+  using C = DCfg;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(splice_gemm_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm (decode): smem attribute");
+    attr = true;
+  }
+  DecTcParams p{};
+  p.M = d.M; p.N = d.N; p.KT = d.K / 256; p.ST = static_cast<int>(ceil_div(d.pp, 64)); p.kb4 = d.kb4;
+  p.sfw = d.sfw; p.sfx = d.sfx; p.alpha = d.alpha; p.Y = d.Y; p.ldy = d.ldy; p.out_bf16 = d.out_bf16; p.err = d.err;
+  // K split: as many CTAs per 128-row tile as fill two per SM, at most 8 (a portable cluster);
+  // every split keeps at least one FP4 k-tile.
+  const int tiles = static_cast<int>(ceil_div(d.N, kDRows));
+  int S = static_cast<int>(std::max<int64_t>(1, (2 * static_cast<int64_t>(sm_count())) / tiles));
+  S = std::min(S, std::min(kDMaxSplit, p.KT));
+  p.kt_per = static_cast<int>(ceil_div(p.KT, S));
+  p.S = static_cast<int>(ceil_div(p.KT, p.kt_per));
+
+  CUtensorMap tmW, tmX, tmWS, tmXS;
+  const uint64_t kbytes = static_cast<uint64_t>(d.K) / 2;
+  fs_status st = make_map(&tmW, d.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, d.N, kbytes, 128, kDRows);
+  if (st == FS_OK) st = make_map(&tmX, d.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, d.M, kbytes, 128, kDTok);
+  if (st != FS_OK) return st;
+  if (p.ST > 0) {
+    const uint64_t pp = static_cast<uint64_t>(d.pp);
+    st = make_map(&tmWS, d.ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, d.N, pp * 2, 64, kDRows);
+    if (st == FS_OK) st = make_map(&tmXS, d.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, d.M, pp * 2, 64, kDTok);
+    if (st != FS_OK) return st;
+  } else {
+    tmWS = tmW;
+    tmXS = tmX;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(p.S), 1);
+  cfg.blockDim = dim3(kDThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = 1;
+  attrs[0].val.clusterDim.y = static_cast<unsigned>(p.S);
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, splice_gemm_decode_tc_kernel, tmW, tmX, tmWS, tmXS, p);
+  if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm (decode path)");
+  FS_CHECK_LAUNCH("fs_splice_gemm (decode path)");
+  return FS_OK;
+}
+
+}  // namespace fs

@@ -90,8 +90,8 @@ extern "C" fs_status fs_splice_gemm_noalloc(int32_t N, int32_t K, uint32_t opts,
     DecodeParams d{};
     d.M = static_cast<int>(M); d.N = N; d.K = K; d.pp = pp; d.kb4 = static_cast<int>(round_up(K / 16, 4) / 4);
     d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha;
-    d.Y = Y; d.ldy = ldy; d.out_bf16 = bf16 ? 1 : 0;
-    st = launch_splice_gemm_decode(d, s);
+    d.Y = Y; d.ldy = ldy; d.out_bf16 = bf16 ? 1 : 0; d.err = scratch;
+    st = launch_splice_gemm_decode_tc(d, s);
   } else {
     TcParams prm{};
     prm.M = M; prm.N = N; prm.K = K; prm.KT = K / 256; prm.ST = static_cast<int>(ceil_div(pp, 64));

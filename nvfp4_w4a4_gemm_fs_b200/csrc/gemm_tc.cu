@@ -33,6 +33,9 @@
 #include "ptx.cuh"
 
 namespace fs {
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
+
 namespace {
 
 constexpr int kBM = 128;
@@ -503,47 +506,6 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   }
 }
 
-// ------------------------------------------------------------------------------------------
-// Host: tensor maps and launch
-// ------------------------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// 2D K-major map with a 128-byte-wide, `box_rows`-high box and 128-byte swizzle.
-fs_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner_elems,
-                   uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return fail(FS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t dims[2] = {inner_elems, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(FS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-  return FS_OK;
-}
-
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <int BN, int CG>
 fs_status set_smem_attr() {
   static bool done = false;
@@ -639,6 +601,47 @@ fs_status launch_cfg(const TcLaunch& L, TcParams prm, int units, cudaStream_t s)
 }
 
 }  // namespace
+
+// ------------------------------------------------------------------------------------------
+// Host: tensor maps and launch
+// ------------------------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2D K-major map with a 128-byte-wide, `box_rows`-high box and 128-byte swizzle.
+fs_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner_elems,
+                   uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[2] = {inner_elems, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FS_OK;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
 
 fs_status launch_splice_gemm_tc(const TcLaunch& L, const TcParams& prm, cudaStream_t s) {
   if (prm.E > kMaxExperts) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm: at most %d experts", kMaxExperts);

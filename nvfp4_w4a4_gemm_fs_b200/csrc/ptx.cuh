@@ -1,6 +1,7 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA loads and stores (no multicast loads),
-// cluster addressing for CTA pairs, tcgen05 (TMEM allocation, block-scaled and BF16 MMA for one
-// CTA or a CTA pair, commit, loads, stores) and shared-memory / instruction descriptors.
+// cluster addressing and distributed shared memory, tcgen05 (TMEM allocation, SMEM->TMEM copy,
+// block-scaled and BF16 MMA for one CTA or a CTA pair, commit, loads, stores) and shared-memory /
+// instruction descriptors.
 #pragma once
 
 #include <cuda.h>
@@ -138,6 +139,12 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                  ::"r"(smem_u32(bar)), "h"(static_cast<uint16_t>(3)) : "memory");
 }
 
+// SMEM -> TMEM copy of one 32-row x 128-bit block (a 512-byte scale atom), replicated into the
+// four lane quadrants; ordered with the issuing thread's later tcgen05.mma.
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc));
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T with NVFP4 operands and UE4M3 block scales from TMEM.
 template <int CG>
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -167,6 +174,16 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uin
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// 32 lanes x 16 consecutive 32-bit columns: thread i of the warp receives lane (quadrant*32 + i).
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives lane (quadrant*32 + i).
@@ -208,9 +225,27 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 constexpr uint32_t kLayoutSw128 = 2;    // 128-byte swizzle
+constexpr uint32_t kLayoutNone = 0;
 
 // K-major operand tile written by TMA with 128-byte swizzle: 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) { return smem_desc(saddr, 16, 1024, kLayoutSw128); }
+// A 512-byte scale atom as the source of tcgen05.cp: 32 rows x 16 bytes, no swizzle.
+__device__ __forceinline__ uint64_t desc_sf_block(uint32_t saddr) { return smem_desc(saddr, 0, 128, kLayoutNone); }
+
+// Prefetch a tiled box of a tensor into L2 (no shared-memory destination, no completion).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
+}
+// Load 16 bytes from the shared memory of a CTA of the cluster (shared::cluster address).  No
+// memory clobber, so that several such loads can be in flight; callers order them after the
+// cluster barrier, which is itself a volatile asm with a memory clobber.
+__device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
 
 // Instruction descriptor: kind::mxf4nvf4 with E2M1 A/B, UE4M3 scales (16-element blocks), K-major.
 __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
