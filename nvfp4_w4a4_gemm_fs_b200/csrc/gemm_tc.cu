@@ -53,6 +53,9 @@ constexpr uint64_t kDrainNs = 50000000ull;      // 50 ms bound on each wait of t
 #ifndef FS_TC_SF_BUFS
 #define FS_TC_SF_BUFS 2
 #endif
+#ifndef FS_TC_SF_SPLIT
+#define FS_TC_SF_SPLIT 1
+#endif
 #ifndef FS_TC_OVERLAP_ACC
 #define FS_TC_OVERLAP_ACC 1
 #endif
@@ -75,18 +78,25 @@ struct Cfg {
   static constexpr bool OVERLAP = BN == 128 || FS_TC_OVERLAP_ACC;
   static constexpr int ACC_SLOTS = BN == 256 ? 1 : 2;  // accumulator barrier pairs
   static constexpr int ACC_SPAN = BN == 256 ? (OVERLAP ? 384 : 256) : 256;
-  // Scale factors in TMEM: a ring of SF_BUFS k-tile buffers, so that the scales of later k-tiles
-  // do not overwrite columns the MMAs of earlier k-tiles may still read.
+  // Scale factors in TMEM: SF_BUFS k-tiles' worth, handed over in units of MPU MMAs (SF_SPLIT
+  // units per k-tile) that rotate over a ring of SF_UNITS slots.  The scales of unit u may be
+  // written once the MMAs of unit u - SF_UNITS are done.  Finer units give the scale warps more
+  // slack but add handoffs; on B200 one unit per k-tile measured fastest (two: +13%, four: +40%
+  // on an 8192 x 4096 x 4096 GEMM).
   static constexpr int SF_BUFS = FS_TC_SF_BUFS;
-  static constexpr int SF_COLS = 16 + 4 * (BN / 32);   // SFA: 4 MMAs x 4 columns; SFB: 4 MMAs x BN/32
-  static constexpr int SFA_COL = ACC_SPAN;
-  static constexpr int SFB_COL = ACC_SPAN + 16;
+  static constexpr int SF_SPLIT = FS_TC_SF_SPLIT;
+  static constexpr int MPU = 4 / SF_SPLIT;                 // MMAs per scale unit
+  static constexpr int SF_COLS = 16 + 4 * (BN / 32);       // per k-tile: SFA 4 MMAs x 4 columns; SFB 4 MMAs x BN/32
+  static constexpr int UNIT_COLS = SF_COLS / SF_SPLIT;     // SFA MPU x 4, then SFB MPU x BN/32
+  static constexpr int SF_UNITS = SF_BUFS * SF_SPLIT;
+  static constexpr int SF_COL = ACC_SPAN;
   static constexpr int TMEM_COLS = 512;
-  static_assert(ACC_SPAN + SF_BUFS * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_SPLIT == 1 || SF_SPLIT == 2 || SF_SPLIT == 4, "scale units divide the k-tile's 4 MMAs");
+  static_assert(ACC_SPAN + SF_UNITS * UNIT_COLS <= TMEM_COLS, "TMEM budget");
   static constexpr int STAGING_BYTES = 4 * STAGING_BUFS * 4096;  // 4 warps x buffers x (32 rows x 128 B)
   // full, sf_loaded, empty per stage; acc_full, acc_empty per slot; sf_full, sf_empty per scale
-  // buffer; drain
-  static constexpr int NUM_BARS = 3 * STAGES + 2 * ACC_SLOTS + 2 * SF_BUFS + 1;
+  // unit slot; drain
+  static constexpr int NUM_BARS = 3 * STAGES + 2 * ACC_SLOTS + 2 * SF_UNITS + 1;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 8 * NUM_BARS + 16 +
                                     4 * (kMaxExperts + 1);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
@@ -178,9 +188,9 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   uint64_t* empty = sfl + C::STAGES;               // the MMAs reading a stage are done
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + C::ACC_SLOTS;   // leader: released by the epilogues of both CTAs
-  uint64_t* sf_full = acc_empty + C::ACC_SLOTS;    // leader: scales of a k-tile are in TMEM (both CTAs)
-  uint64_t* sf_empty = sf_full + C::SF_BUFS;       // the MMAs reading a scale buffer are done
-  uint64_t* drain = sf_empty + C::SF_BUFS;         // leader: all MMAs issued so far are done
+  uint64_t* sf_full = acc_empty + C::ACC_SLOTS;    // leader: scales of a unit are in TMEM (both CTAs)
+  uint64_t* sf_empty = sf_full + C::SF_UNITS;      // the MMAs reading a scale slot are done
+  uint64_t* drain = sf_empty + C::SF_UNITS;        // leader: all MMAs issued so far are done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* cum_m = reinterpret_cast<int*>(tmem_slot + 4);
@@ -213,7 +223,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       ptx::mbar_init(empty + s, 1);
     }
     for (int a = 0; a < C::ACC_SLOTS; ++a) { ptx::mbar_init(acc_full + a, 1); ptx::mbar_init(acc_empty + a, 4 * CG); }
-    for (int b = 0; b < C::SF_BUFS; ++b) { ptx::mbar_init(sf_full + b, 4 * CG); ptx::mbar_init(sf_empty + b, 1); }
+    for (int b = 0; b < C::SF_UNITS; ++b) { ptx::mbar_init(sf_full + b, 4 * CG); ptx::mbar_init(sf_empty + b, 1); }
     ptx::mbar_init(drain, 1);
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tmA); ptx::prefetch_tensormap(&tmB); ptx::prefetch_tensormap(&tmY);
@@ -292,7 +302,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc_f4 = ptx::idesc_nvf4(kBM * CG, BN);
       constexpr uint32_t idesc_bf = ptx::idesc_bf16(kBM * CG, BN);
-      int stage = 0, acc = 0, sf_count = 0, i = 0;
+      int stage = 0, acc = 0, sf_unit = 0, i = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int t = unit; t < total_tiles && ok; t += nunits, ++i) {
@@ -305,16 +315,22 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           const uint64_t adesc = ptx::desc_kmajor_sw128(ptx::smem_u32(A_at(stage)));
           const uint64_t bdesc = ptx::desc_kmajor_sw128(ptx::smem_u32(B_at(stage)));
           if (kt < p.KT) {
-            const int buf = sf_count % C::SF_BUFS;
-            if (!wait_bar(sf_full + buf, (sf_count / C::SF_BUFS) & 1, abort_flag, p.err)) { ok = false; break; }
-            ptx::tc_fence_after();
-            const uint32_t sf_off = buf * C::SF_COLS;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              ptx::tc_mma_nvf4<CG>(d, adesc + 2 * j, bdesc + 2 * j, idesc_f4, tmem + C::SFA_COL + sf_off + 4 * j,
-                                   tmem + C::SFB_COL + sf_off + (BN / 32) * j, (kt | j) != 0);
-            ptx::tc_commit<CG>(sf_empty + buf);
-            ++sf_count;
+            for (int h = 0; h < C::SF_SPLIT; ++h) {
+              const int slot = sf_unit % C::SF_UNITS;
+              if (!wait_bar(sf_full + slot, (sf_unit / C::SF_UNITS) & 1, abort_flag, p.err)) { ok = false; break; }
+              ptx::tc_fence_after();
+              const uint32_t sf = tmem + C::SF_COL + slot * C::UNIT_COLS;
+#pragma unroll
+              for (int jj = 0; jj < C::MPU; ++jj) {
+                const int j = h * C::MPU + jj;
+                ptx::tc_mma_nvf4<CG>(d, adesc + 2 * j, bdesc + 2 * j, idesc_f4, sf + 4 * jj,
+                                     sf + 4 * C::MPU + (BN / 32) * jj, (kt | j) != 0);
+              }
+              ptx::tc_commit<CG>(sf_empty + slot);
+              ++sf_unit;
+            }
+            if (!ok) break;
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) ptx::tc_mma_bf16<CG>(d, adesc + 2 * j, bdesc + 2 * j, idesc_bf, 1u);
@@ -335,45 +351,51 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     // Each warp owns one TMEM lane quadrant and writes, for every FP4 k-tile, the block scales
     // of its 32 lanes exactly as tcgen05.cp.32x128b.warpx4 would lay them out: lane l, columns
     // 4c..4c+3 of an atom's slot hold the atom's 16-byte row l (SFA: one atom per MMA; SFB: the
-    // BN/128 row-group atoms side by side).  The k-tiles' scales rotate over SF_BUFS buffers.
+    // BN/128 row-group atoms side by side).  A k-tile's atoms are read from shared memory first,
+    // then written unit by unit as each ring slot frees up.
     // The scale-atom barrier of a stage completes one phase per FP4 use of that stage only, so
     // its parity is tracked per stage (the producer keeps the same bits).
     const int quad = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    int stage = 0, sf_count = 0;
+    int stage = 0, sf_unit = 0;
     uint32_t sfl_bits = 0;
     bool ok = true;
     for (int t = unit; t < total_tiles && ok; t += nunits) {
       for (int kt = 0; kt < ktiles; ++kt) {
         if (kt < p.KT) {
-          const int buf = sf_count % C::SF_BUFS;
-          if (!wait_bar(sf_empty + buf, ((sf_count / C::SF_BUFS) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
           if (!wait_bar(sfl + stage, (sfl_bits >> stage) & 1, abort_flag, p.err)) { ok = false; break; }
           sfl_bits ^= 1u << stage;
           const uint8_t* sfa = SFA_at(stage);
           const uint8_t* sfb = SFB_at(stage);
-          const uint32_t col = tmem + lane_base + buf * C::SF_COLS;
+          uint4 a[4], b0[4], b1[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j + lane * 16);
-            ptx::tmem_st_32x32b_x4(col + C::SFA_COL + 4 * j, a.x, a.y, a.z, a.w);
-            if constexpr (BN == 256) {
-              const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j + lane * 16);
-              const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + 512 * j + lane * 16);
-              ptx::tmem_st_32x32b_x8(col + C::SFB_COL + 8 * j, b0, b1);
-            } else {
-              const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j + lane * 16);
-              ptx::tmem_st_32x32b_x4(col + C::SFB_COL + 4 * j, b0.x, b0.y, b0.z, b0.w);
+            a[j] = *reinterpret_cast<const uint4*>(sfa + 512 * j + lane * 16);
+            b0[j] = *reinterpret_cast<const uint4*>(sfb + 512 * j + lane * 16);
+            if constexpr (BN == 256) b1[j] = *reinterpret_cast<const uint4*>(sfb + 2048 + 512 * j + lane * 16);
+          }
+#pragma unroll
+          for (int h = 0; h < C::SF_SPLIT; ++h) {
+            const int slot = sf_unit % C::SF_UNITS;
+            if (!wait_bar(sf_empty + slot, ((sf_unit / C::SF_UNITS) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
+            const uint32_t col = tmem + lane_base + C::SF_COL + slot * C::UNIT_COLS;
+#pragma unroll
+            for (int jj = 0; jj < C::MPU; ++jj) {
+              const int j = h * C::MPU + jj;
+              ptx::tmem_st_32x32b_x4(col + 4 * jj, a[j].x, a[j].y, a[j].z, a[j].w);
+              if constexpr (BN == 256) ptx::tmem_st_32x32b_x8(col + 4 * C::MPU + 8 * jj, b0[j], b1[j]);
+              else ptx::tmem_st_32x32b_x4(col + 4 * C::MPU + 4 * jj, b0[j].x, b0[j].y, b0[j].z, b0[j].w);
             }
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if constexpr (CG == 1) ptx::mbar_arrive(sf_full + slot);
+              else ptx::mbar_arrive_remote(leader(sf_full + slot));
+            }
+            ++sf_unit;
           }
-          ptx::tmem_st_wait();
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            if constexpr (CG == 1) ptx::mbar_arrive(sf_full + buf);
-            else ptx::mbar_arrive_remote(leader(sf_full + buf));
-          }
-          ++sf_count;
+          if (!ok) break;
         }
         if (++stage == C::STAGES) stage = 0;
       }
