@@ -141,14 +141,16 @@ struct TileMap {
   int n0;          // first output column
 };
 
-// Tile t -> rows / columns.  cum_m[e] counts the (kBM * CG)-row M-tiles before expert e; M-tiles
-// vary fastest so that the CTAs of one wave share B tiles in L2.
+// Tile t -> rows / columns.  cum_m[e] counts the (kBM * CG)-row M-tiles before expert e.  The
+// operand whose tiles vary fastest is read whole by every wave of CTAs, so the order keeps the
+// smaller operand there (it stays in L2) and streams the larger one once: M-tiles fastest when A
+// is the smaller (or for experts), N-tiles fastest otherwise.
 template <int CG>
 __device__ __forceinline__ TileMap map_tile(int t, const TcParams& p, const int* cum_m, int rank) {
   TileMap m;
   const int total_m = cum_m[p.E];
-  const int mt = t % total_m;
-  const int nt = t / total_m;
+  const int mt = p.n_fast ? t / p.n_tiles : t % total_m;
+  const int nt = p.n_fast ? t % p.n_tiles : t / total_m;
   int lo = 0, hi = p.E - 1;                   // expert with cum_m[e] <= mt < cum_m[e+1]
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -572,6 +574,8 @@ fs_status launch_cfg(const TcLaunch& L, TcParams prm, int units, cudaStream_t s)
   if (st != FS_OK) return st;
   prm.BN = BN;
   prm.n_tiles = static_cast<int>(ceil_div(prm.N, BN));
+  // N-tiles fastest when the weights (B) are the smaller operand of a dense problem.
+  prm.n_fast = (!prm.offsets && prm.E == 1 && static_cast<int64_t>(prm.N) <= L.a_rows) ? 1 : 0;
   CUtensorMap tmA, tmB, tmSA, tmSB;
   const uint64_t kbytes = static_cast<uint64_t>(prm.K) / 2;
   st = make_map(&tmA, L.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, L.a_rows, kbytes, 128, kBM);
