@@ -375,10 +375,11 @@ def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20):
 # ------------------------------------------------------------------------------------------
 # reference arm / CPU baseline: the oracle as it stands on a bounded sample
 # ------------------------------------------------------------------------------------------
-def oracle_sample_step(rows=128, seed=0):
+def oracle_sample_step(rows=M_PREFILL, seed=0):
     """One bounded sample of the step through the CPU oracle: the q projection (4096 <- 4096) of
-    `rows` tokens: statistics, top-64 selection, weight pre-split, activation quantisation and the
-    float64 SpliceGEMM.  Returns (seconds, flops counted as 2*rows*N*K)."""
+    `rows` tokens (all 8192 by default, 1/11.5 of the step's FLOPs): statistics, top-64 selection,
+    weight pre-split, activation quantisation and the float64 SpliceGEMM.  Returns (seconds,
+    flops counted as 2*rows*N*K)."""
     import numpy as np
 
     import synth
@@ -407,7 +408,7 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(rows=128):
+def cpu_baseline(rows=M_PREFILL):
     dt, flops = oracle_sample_step(rows)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"q projection 4096x4096 of {rows} of the 8192 tokens, P=64: stats, select, "
@@ -423,7 +424,7 @@ def run_reference(args):
         oracle_sample_step(32)
     times, flops = [], 0.0
     for _ in range(args.steps):
-        dt, fl = oracle_sample_step(128)
+        dt, fl = oracle_sample_step(M_PREFILL)
         times.append(dt)
         flops = fl
     tot = sum(times)
@@ -431,10 +432,11 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * tot / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "Qwen3-8B-shaped prefill, M=8192 bf16, P=64 (oracle sample: q projection, 128 rows)",
+            "config": {"workload": "Qwen3-8B-shaped prefill, M=8192 bf16, P=64 (oracle sample: the q projection, all 8192 rows)",
                        "global_batch": M_PREFILL, "seq_len": 1024, "parallelism": "cpu"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": "q projection 4096x4096 of 128 tokens per step, P=64"},
+                             "sample": "q projection 4096x4096 of all 8192 tokens per step, P=64: stats, select, "
+                                       "weight pre-split, quantise, float64 SpliceGEMM"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
@@ -465,26 +467,28 @@ def prep_case(F, args, device):
 
 
 def kernel_case(F, args, device):
-    """fs_splice_gemm alone on the q projection (4096 <- 4096), for profiling one kernel."""
+    """fs_splice_gemm alone on one projection shape (--shape; M=8192 for `gemm`, M=--decode-m for
+    `decode`), for profiling one kernel."""
     import torch
     if args.case == "prep":
         return prep_case(F, args, device)
-    M = M_PREFILL if args.case == "gemm" else 16
-    X = make_activations(M, 4096, 3, device)
-    W = make_weights(4096, 4096, 4, device)
-    st = F.StatsState(1, 4096, device=device)
-    F.fs_channel_stats(X, st)
+    N, K = {name: (n, k) for name, n, k, _ in PROJ}[args.shape]
+    M = M_PREFILL if args.case == "gemm" else args.decode_m
+    X = make_activations(M, K, 3, device)
+    W = make_weights(N, K, 4, device)
+    st = F.StatsState(1, K, device=device)
+    F.fs_channel_stats(make_activations(max(M, 2048), K, 3, device), st)
     _, mask, g = F.fs_select_topk(st, args.p)
     wq, _, alpha = F.fs_prepare_weights(W, mask[0], args.p, g)
     xq = F.fs_quantize_splice(X, mask[0], args.p, g)
-    plan = F.Plan(4096, 4096, max(args.p, 1))
-    Y = torch.empty(M, 4096, dtype=torch.float32, device=device)
+    plan = F.Plan(N, K, max(args.p, 1))
+    Y = torch.empty(M, N, dtype=torch.float32, device=device)
     for _ in range(args.warmup):
         F.fs_splice_gemm(plan, xq, wq, alpha, Y=Y)
     ms = timed(lambda: F.fs_splice_gemm(plan, xq, wq, alpha, Y=Y), args.steps) / args.steps
     plan.check()
-    print(json.dumps({"case": args.case, "M": M, "N": 4096, "K": 4096, "p": args.p, "us": ms * 1000.0,
-                      "tflops": 2.0 * M * 4096 * 4096 / (ms * 1e-3) / 1e12}))
+    print(json.dumps({"case": args.case, "shape": args.shape, "M": M, "N": N, "K": K, "p": args.p,
+                      "us": ms * 1000.0, "tflops": 2.0 * M * N * K / (ms * 1e-3) / 1e12}))
 
 
 # ------------------------------------------------------------------------------------------
@@ -499,8 +503,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--serial", action="store_true", help="one stream for the whole step (no group concurrency)")
     ap.add_argument("--case", default="step", choices=["step", "gemm", "decode", "prep"],
-                    help="step: the full benchmark; gemm / decode: only fs_splice_gemm on the q projection "
-                         "(M=8192, or M=16) for profiling one kernel")
+                    help="step: the full benchmark; gemm / decode: only fs_splice_gemm on one projection "
+                         "shape (M=8192, or M=--decode-m) for profiling one kernel; prep: the preparation "
+                         "kernels on the q projection")
+    ap.add_argument("--shape", default="q", choices=[name for name, _, _, _ in PROJ],
+                    help="projection shape of --case gemm / decode")
+    ap.add_argument("--decode-m", type=int, default=16, help="tokens of --case decode (1..16)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -631,7 +639,8 @@ def main():
         l0 = PrefillLayer(F, M_PREFILL, 0, seed=2 + rank, device=device)
         for _ in range(3):
             l0.step()
-        g0s = capture(l0.step)
+        # the P = 0 step is captured the same way as the timed step (4 streams unless --serial)
+        g0s = capture(l0.step if args.serial else (lambda: l0.step_streams(streams)))
         for _ in range(3):
             g0s.replay()
         ms0 = timed(g0s.replay, args.steps) / args.steps
