@@ -16,6 +16,9 @@ namespace fs {
 namespace {
 
 constexpr int kQThreads = 256;
+#ifndef FS_Q_PASS_ROWS
+#define FS_Q_PASS_ROWS 4
+#endif
 
 enum class Side { Activation, Weight };
 
@@ -112,7 +115,7 @@ struct ChunkLoc {
 // tables of the scale value and its reciprocal in shared memory; for bf16 input under a
 // power-of-two gain the division is replaced by one multiply and a 12-bit snap (snap12), which
 // yields the same codes.
-template <typename T, Side kSide, bool kGrouped, bool kOneRow>
+template <typename T, Side kSide, bool kGrouped, bool kRowPasses>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_t nchunks) {
   __shared__ uint16_t sh_mbits[16384 / 16];             // protected lanes of each 16-element block
   __shared__ uint4 sh_kill[sizeof(T) == 2 ? 2 * 16384 / 16 : 1];   // bf16: per block, 8 words of lanes to clear
@@ -172,19 +175,25 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
   if constexpr (kSide == Side::Weight) alpha_v = __ldg(a.alpha);
   const float inv6 = __frcp_rn(6.0f);
 
-  constexpr bool one_row = kOneRow;                   // rows_per_cta == 1: chunk = one row
+  // General chunks: block i of the chunk is (row i / nb, block i % nb).  kRowPasses (nb a multiple
+  // of the CTA size): every pass covers kQThreads blocks of one row, its row and first block kept
+  // incrementally, so a pass costs no division and its row addresses are uniform.
   auto load_one = [&](const ChunkLoc& L, int i0, RawBlock<T>& x) {
     const int i = i0 + tid;
-    const int r = one_row ? 0 : i / a.nb;
+    const int r = i / a.nb;
     if (L.e >= 0 && i < total && r < L.valid) {
-      const int b = one_row ? i : i % a.nb;
+      const int b = i % a.nb;
       load_raw<T>(X + (L.src_row0 + r) * a.ldx + static_cast<int64_t>(b) * 16, x);
     }
+  };
+  auto load_pass = [&](const ChunkLoc& L, int r, int b0, RawBlock<T>& x) {
+    if (L.e >= 0 && r < L.valid) load_raw<T>(X + (L.src_row0 + r) * a.ldx + static_cast<int64_t>(b0 + tid) * 16, x);
   };
 
   ChunkLoc L = locate(blockIdx.x);
   RawBlock<T> xc;
-  load_one(L, 0, xc);
+  if constexpr (kRowPasses) load_pass(L, 0, 0, xc);
+  else load_one(L, 0, xc);
   int cur_e = -1;
   const uint32_t* mask = nullptr;
   float g = 1.0f;
@@ -248,15 +257,29 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
       }
     }
     const ChunkLoc Ln = locate(chunk + gridDim.x);
+    int r_cur = 0, b_cur = 0;                      // kRowPasses: row and first block of this pass
     for (int i0 = 0; i0 < total; i0 += kQThreads) {
       RawBlock<T> xn;
-      if (i0 + kQThreads < total) load_one(L, i0 + kQThreads, xn);   // prefetch the next pass
-      else load_one(Ln, 0, xn);                                       // or the next chunk's first
+      int r_nxt = r_cur, b_nxt = b_cur + kQThreads;
+      if constexpr (kRowPasses) {
+        if (b_nxt == a.nb) { b_nxt = 0; ++r_nxt; }
+        if (i0 + kQThreads < total) load_pass(L, r_nxt, b_nxt, xn);   // prefetch the next pass
+        else load_pass(Ln, 0, 0, xn);                                  // or the next chunk's first
+      } else {
+        if (i0 + kQThreads < total) load_one(L, i0 + kQThreads, xn);
+        else load_one(Ln, 0, xn);
+      }
       const RawBlock<T>& x = xc;
-      const int i = i0 + tid;
-      const bool in_range = i < total;
-      const int r = (!in_range || one_row) ? 0 : i / a.nb;
-      const int b = !in_range ? 0 : (one_row ? i : i % a.nb);
+      int r, b;
+      bool in_range;
+      if constexpr (kRowPasses) {
+        r = r_cur; b = b_cur + tid; in_range = true;
+      } else {
+        const int i = i0 + tid;
+        in_range = i < total;
+        r = in_range ? i / a.nb : 0;
+        b = in_range ? i % a.nb : 0;
+      }
       const int64_t prow = L.prow0 + r;
       const bool has_data = in_range && r < L.valid;
       uint32_t sfc = 0;
@@ -304,6 +327,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
       if (in_range && (b & 3) == 0)
         *reinterpret_cast<uint32_t*>(a.sf + sf_offset(prow, b, a.kb4)) = sfc | (s1 << 8) | (s2 << 16) | (s3 << 24);
       xc = xn;
+      r_cur = r_nxt;
+      b_cur = b_nxt;
     }
     // Extract X_S: side column c of each row is channel sh_pidx[c] (the block data is still in
     // L1/L2), zero in the padding columns p..pp-1 and in the padding rows of a grouped buffer.
@@ -440,15 +465,19 @@ int quant_sm_count() {
 
 template <Side kSide, bool kGrouped>
 fs_status launch_quantize(int dtype, QuantArgs& a, int64_t padded_rows, cudaStream_t s) {
-  // rows per chunk: a power of two dividing 128, so a chunk never straddles a 128-row tile
+  // rows per chunk: a power of two dividing 128, so a chunk never straddles a 128-row tile.  With
+  // nb a multiple of the CTA size, 4 rows (4 or more passes) per chunk amortise the per-chunk work.
+  const bool passes = a.nb % kQThreads == 0;
   int rpc = 1;
-  while (rpc < 128 && rpc * a.nb < kQThreads) rpc *= 2;
+  if (passes) rpc = FS_Q_PASS_ROWS;
+  else
+    while (rpc < 128 && rpc * a.nb < kQThreads) rpc *= 2;
   a.rows_per_cta = rpc;
   const int64_t chunks = ceil_div(padded_rows, rpc);
   if (chunks == 0) return FS_OK;
   auto kernel = dtype == FS_DTYPE_BF16
-                    ? (rpc == 1 ? quantize_kernel<uint16_t, kSide, kGrouped, true> : quantize_kernel<uint16_t, kSide, kGrouped, false>)
-                    : (rpc == 1 ? quantize_kernel<float, kSide, kGrouped, true> : quantize_kernel<float, kSide, kGrouped, false>);
+                    ? (passes ? quantize_kernel<uint16_t, kSide, kGrouped, true> : quantize_kernel<uint16_t, kSide, kGrouped, false>)
+                    : (passes ? quantize_kernel<float, kSide, kGrouped, true> : quantize_kernel<float, kSide, kGrouped, false>);
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQThreads, 0) != cudaSuccess || per_sm < 1) per_sm = 2;
   const int64_t grid = std::min<int64_t>(chunks, static_cast<int64_t>(quant_sm_count()) * per_sm);
