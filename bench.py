@@ -45,6 +45,22 @@ P_DEFAULT = 64
 DECODE_LAYERS = 36
 
 
+# DRAM traffic of the tensor-core SpliceGEMM over one step (2 x q/o + 2 x k/v + 2 x gate/up + down,
+# M = 8192, P = 64): one ncu capture per shape of the current kernel (profiles/splice_gemm_tc_m8192_p64.md).
+GEMM_DRAM_BYTES_PER_STEP = 1310896896
+
+
+def gemm_alg_bytes(p):
+    """Operand and output bytes the 7 GEMMs of a step must move: A and B codes, scales and side
+    columns, and the fp32 output."""
+    pp = (p + 15) // 16 * 16
+    tot = 0
+    for _, N, K, _ in PROJ:
+        M = M_PREFILL
+        tot += M * K // 2 + M * K // 16 + 2 * M * pp + N * K // 2 + N * K // 16 + 2 * N * pp + 4 * M * N
+    return tot
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -300,6 +316,114 @@ def timed(fn, steps, dist=None):
 # ------------------------------------------------------------------------------------------
 # decode sweep (M <= 16), CUDA-graph replay over 36 distinct layers
 # ------------------------------------------------------------------------------------------
+def moe_case(F, p, device, reps=10):
+    """Mixture-of-experts projections (grouped path): 64 experts, top-8 routing of 4096 tokens with
+    Zipf(1.2) expert popularity (32768 routed rows, expert-contiguous), the up projection (gate and
+    up fused, 4096 <- 4096) and the down projection (4096 <- 2048), P = 64 per expert with its own
+    statistics, protected set, gains and packed weights.  Times the grouped quantise + grouped
+    GEMM and the grouped GEMM alone (graph replays), TFLOP/s = sum over experts of 2*rows*N*K / t."""
+    import numpy as np
+    import torch
+
+    import synth
+    counts = synth.moe_routing_counts(0)
+    E, total = len(counts), int(counts.sum())
+    offs = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int64, device=device)
+    out = {"experts": E, "routed_rows": total, "rows_min_median_max": [int(counts.min()), int(np.median(counts)),
+                                                                         int(counts.max())]}
+    for name, N, K in (("up", 4096, 4096), ("down", 4096, 2048)):
+        X = make_activations(total, K, 31 if name == "up" else 32, device)
+        st = F.StatsState(E, K, device=device)
+        for e in range(E):
+            F.fs_channel_stats(X[int(counts[:e].sum()):int(counts[:e + 1].sum())], st, group=e)
+        _, masks, gA = F.fs_select_topk(st, p)
+        pp = F.side_cols(p)
+        wq = F.Packed(torch.empty(E * N, K // 2, dtype=torch.uint8, device=device),
+                      torch.empty(F.sf_bytes(E * N, K), dtype=torch.uint8, device=device),
+                      torch.zeros(E * N, max(pp, 8), dtype=torch.bfloat16, device=device)[:, :pp], E * N, K, p)
+        alpha = torch.empty(E, dtype=torch.float32, device=device)
+        gW = torch.empty(E, dtype=torch.float32, device=device)
+        sfb = F.sf_bytes(N, K)
+        for e in range(E):
+            W = make_weights(N, K, 7000 + e, device)
+            F.fs_prepare_weights(W, masks[e], p, gA[e:e + 1], gW=gW[e:e + 1], alpha=alpha[e:e + 1],
+                                 out=F.Packed(wq.q[e * N:(e + 1) * N], wq.sf[e * sfb:(e + 1) * sfb],
+                                              wq.side[e * N:(e + 1) * N], N, K, p))
+            del W
+        xq = F.alloc_packed(F.grouped_rows(total, E), K, p, device)
+        plan = F.Plan(N, K, max(p, 1))
+        Y = torch.empty(total, N, dtype=torch.float32, device=device)
+
+        def gemm():
+            F.fs_splice_gemm_grouped(plan, offs, total, xq, wq, alpha, Y=Y)
+
+        def quant_gemm():
+            F.fs_quantize_splice_grouped(X, offs, masks, p, gA, out=xq, max_rows=total)
+            gemm()
+        quant_gemm()
+        torch.cuda.synchronize()
+        plan.check()
+        flops = 2.0 * total * N * K
+        res = {"N": N, "K": K}
+        for tag, fn in (("gemm", gemm), ("quant+gemm", quant_gemm)):
+            g = capture(fn)
+            for _ in range(3):
+                g.replay()
+            ms = timed(g.replay, reps) / reps
+            res[tag] = {"us": ms * 1000.0, "TFLOPs": flops / (ms * 1e-3) / 1e12}
+            del g
+        plan.check()
+        out[name] = res
+        del X, xq, wq, Y, st
+        torch.cuda.empty_cache()
+    return out
+
+
+def rollout_case(F, device, reps=20):
+    """The rollout-batch configuration: statistics over 16384 x 4096 bf16 activations (1% channels
+    x30), top-64 reselection, and the dual-gate filter over 1024 x 4096 float32 train-engine
+    log-probs with groups of G = 16 sequences (tau = 1e-4, K1 = ceil(0.01 * 4096) = 41, K2 = 5,
+    35% of sequences with injected tail tokens and runs).  GB/s = bytes read / time."""
+    import numpy as np
+    import torch
+
+    import synth
+    res = {}
+    X = make_activations(16384, 4096, 41, device)
+    st = F.StatsState(1, 4096, device=device)
+    P = torch.empty(1, 64, dtype=torch.int32, device=device)
+    mask = torch.empty(1, 128, dtype=torch.int32, device=device)
+    gA = torch.empty(1, dtype=torch.float32, device=device)
+    g = capture(lambda: F.fs_channel_stats(X, st))
+    for _ in range(3):
+        g.replay()
+    ms = timed(g.replay, reps) / reps
+    res["stats"] = {"us": ms * 1000.0, "GBps": X.numel() * 2 / (ms * 1e-3) / 1e9}
+    g = capture(lambda: F.fs_select_topk(st, 64, reset=False, P=P, mask=mask, gA=gA))
+    for _ in range(3):
+        g.replay()
+    ms = timed(g.replay, reps) / reps
+    res["select"] = {"us": ms * 1000.0, "K": 4096, "p": 64}
+    del g, X
+    lp, lengths, rewards, _ = synth.rollout_logprobs(5)
+    S, T = lp.shape
+    logp = torch.from_numpy(lp).to(device)
+    lens = torch.from_numpy(lengths).to(device)
+    rew = torch.from_numpy(rewards).to(device)
+    log_tau = float(np.float32(np.log(1e-4)))
+    K1 = int(np.ceil(0.01 * T))
+    adv = torch.empty(S, dtype=torch.float32, device=device)
+    outs = F.fs_seq_filter(logp, log_tau, K1, 5, lengths=lens, G=16, rewards=rew, adv=adv)
+    g = capture(lambda: F.fs_seq_filter(logp, log_tau, K1, 5, lengths=lens, G=16, rewards=rew, adv=adv))
+    for _ in range(3):
+        g.replay()
+    ms = timed(g.replay, reps) / reps
+    nbytes = S * T * 4 + S * (4 + 4 + 4 + 1 + 4 + 4)
+    res["filter"] = {"us": ms * 1000.0, "GBps": nbytes / (ms * 1e-3) / 1e9, "S": S, "T": T, "K1": K1, "K2": 5,
+                     "G": 16, "kept": int(outs[0].sum().item())}
+    return res
+
+
 def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20):
     import torch
     res = {}
@@ -619,9 +743,13 @@ def main():
                    "global_batch": world * M_PREFILL, "seq_len": 1024, "parallelism": f"dp{world}",
                    "p": p, "l2": "inputs larger than L2 (0.85 GB of bf16 activations and weights per step)"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp4_peak, "traffic": None,
-                     "kernel": "splice_gemm_tc_kernel (all 7 projections; 2MNK per launch / CUDA-event time)",
-                     "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16 ratio)"},
+                     "frac": gemm_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_STEP,
+                     "traffic_unit": "DRAM bytes per step (the 7 GEMM launches; ncu dram__bytes_read.sum + "
+                                     "dram__bytes_write.sum per shape, profiles/splice_gemm_tc_m8192_p64.md)",
+                     "algorithmic_bytes": gemm_alg_bytes(p),
+                     "kernel": "splice_gemm_tc_kernel (all 7 projections; sum 2MNK / sum of CUDA-event times)",
+                     "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16 ratio), "
+                                    "of measured"},
         "gemm_us": per_proj,
         "phase_us": phase_us,
         "clocks": clk.summary(),
@@ -670,6 +798,17 @@ def main():
         line["decode"]["weight_bytes_per_layer"] = wbytes
         line["decode"]["overhead_vs_p0_M16"] = dec["M16"]["gemm"]["us_per_layer"] / dec0["M16"]["gemm"]["us_per_layer"] - 1.0
         line["decode"]["hbm_peak_gbs"] = hbm
+        torch.cuda.empty_cache()
+        moe = moe_case(F, p, device)
+        moe["fp4_peak_tflops"] = fp4_peak
+        for nm in ("up", "down"):
+            moe[nm]["gemm"]["frac_fp4_peak"] = moe[nm]["gemm"]["TFLOPs"] / fp4_peak
+        line["moe"] = moe
+        torch.cuda.empty_cache()
+        ro = rollout_case(F, device)
+        for nm in ("stats", "filter"):
+            ro[nm]["frac_hbm"] = ro[nm]["GBps"] / hbm
+        line["rollout"] = ro
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

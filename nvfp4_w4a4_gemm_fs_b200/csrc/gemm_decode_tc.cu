@@ -29,7 +29,19 @@ namespace {
 constexpr int kDThreads = 192;
 constexpr int kDRows = 128;          // weight rows per tile (MMA M)
 constexpr int kDTok = 16;            // token columns (MMA N)
-constexpr int kDStages = 4;
+#ifndef FS_DEC_STAGES
+#define FS_DEC_STAGES 3
+#endif
+#ifndef FS_DEC_CTAS_PER_SM
+#define FS_DEC_CTAS_PER_SM 3
+#endif
+// Three stages of 22 KB (the partial sums reuse stage 0) let three CTAs share an SM, so the K
+// split can be wider without a second wave; against four stages at two CTAs per SM this measured
+// 14.9 -> 8.6 us for the 12288 x 4096 projection at M = 1.
+constexpr int kDStages = FS_DEC_STAGES;
+constexpr int kDCtasPerSm = FS_DEC_CTAS_PER_SM;   // residency the shared-memory budget allows
+static_assert(kDCtasPerSm * (1024 + 1024 + kDStages * (128 * 128 + 16 * 128 + 4096) + 8 * (2 * kDStages + 2) + 16) <= 233472,
+              "CTAs per SM must fit the SM's shared memory");
 constexpr int kDMaxSplit = 8;        // portable cluster size
 constexpr uint64_t kDWaitNs = 2000000000ull;
 constexpr uint64_t kDDrainNs = 50000000ull;
@@ -40,8 +52,9 @@ struct DCfg {
   static constexpr int SFW_BYTES = 2048;            // four 512-byte atoms, one per MMA
   static constexpr int SFX_BYTES = 2048;
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;   // multiple of 1024
-  static constexpr int RED_BYTES = kDRows * kDTok * 4;                           // partial [token][row]
-  static constexpr int SMEM_BYTES = 1024 + kDStages * STAGE_BYTES + RED_BYTES + 8 * (2 * kDStages + 2) + 16;
+  static constexpr int RED_BYTES = kDRows * kDTok * 4;   // partial [token][row], in stage 0 after the MMAs
+  static_assert(RED_BYTES <= STAGE_BYTES, "the partial fits in a stage");
+  static constexpr int SMEM_BYTES = 1024 + kDStages * STAGE_BYTES + 8 * (2 * kDStages + 2) + 16;
   static constexpr int TMEM_COLS = 128;
   static constexpr int SF_COL = 32;                 // scale buffer b: SFA at SF_COL+32b, SFB at SF_COL+32b+16
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the 128-byte swizzle");
@@ -94,8 +107,10 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
   using C = DCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* red = reinterpret_cast<float*>(smem + kDStages * C::STAGE_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDStages * C::STAGE_BYTES + C::RED_BYTES);
+  // The partial sums reuse stage 0: it is written only after every MMA (hence every stage's use)
+  // has completed (acc_full), and every load this CTA issues is consumed by one of those MMAs.
+  float* red = reinterpret_cast<float*>(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDStages * C::STAGE_BYTES);
   uint64_t* empty = full + kDStages;
   uint64_t* acc_full = empty + kDStages;
   uint64_t* drain = acc_full + 1;
@@ -281,10 +296,11 @@ fs_status launch_splice_gemm_decode_tc(const DecodeParams& d, cudaStream_t s) {
   DecTcParams p{};
   p.M = d.M; p.N = d.N; p.KT = d.K / 256; p.ST = static_cast<int>(ceil_div(d.pp, 64)); p.kb4 = d.kb4;
   p.sfw = d.sfw; p.sfx = d.sfx; p.alpha = d.alpha; p.Y = d.Y; p.ldy = d.ldy; p.out_bf16 = d.out_bf16; p.err = d.err;
-  // K split: as many CTAs per 128-row tile as fill two per SM, at most 8 (a portable cluster);
+  // K split: as many CTAs per 128-row tile as fill the SMs at the resident CTAs per SM, at most 8
+  // (a portable cluster);
   // every split keeps at least one FP4 k-tile.
   const int tiles = static_cast<int>(ceil_div(d.N, kDRows));
-  int S = static_cast<int>(std::max<int64_t>(1, (2 * static_cast<int64_t>(sm_count())) / tiles));
+  int S = static_cast<int>(std::max<int64_t>(1, (kDCtasPerSm * static_cast<int64_t>(sm_count())) / tiles));
   S = std::min(S, std::min(kDMaxSplit, p.KT));
   p.kt_per = static_cast<int>(ceil_div(p.KT, S));
   p.S = static_cast<int>(ceil_div(p.KT, p.kt_per));
