@@ -40,24 +40,30 @@ METRIC = "SpliceGEMM prefill TFLOPS & decode GB/s at P=64, % of roofline, overhe
 PROJ = (("q", 4096, 4096, 0), ("k", 1024, 4096, 0), ("v", 1024, 4096, 0), ("o", 4096, 4096, 1),
         ("gate", 12288, 4096, 2), ("up", 12288, 4096, 2), ("down", 4096, 12288, 3))
 GROUP_K = (4096, 4096, 4096, 12288)          # input groups: qkv, o, gate/up, down
+GROUP_NAMES = ("qkv", "o", "gate_up", "down")
+GROUP_PROJ = tuple(tuple(j for j, pr in enumerate(PROJ) if pr[3] == gi) for gi in range(4))
 M_PREFILL = 8192
 P_DEFAULT = 64
 DECODE_LAYERS = 36
 
 
-# DRAM traffic of the tensor-core SpliceGEMM over one step (2 x q/o + 2 x k/v + 2 x gate/up + down,
-# M = 8192, P = 64): one ncu capture per shape of the current kernel (profiles/splice_gemm_tc_m8192_p64.md).
-GEMM_DRAM_BYTES_PER_STEP = 1310896896
+# DRAM traffic of the tensor-core SpliceGEMM over one step (M = 8192, P = 64): ncu
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch per shape of the current kernel, summed
+# over a step's launches (fused: qkv, o, gate_up, down; unfused: q, k, v, o, gate, up, down);
+# profiles/splice_gemm_tc_dram_m8192_p64.md.
+GEMM_DRAM_BYTES_PER_STEP = {"fused": 1365232640, "unfused": 1298154752}
 
 
-def gemm_alg_bytes(p):
-    """Operand and output bytes the 7 GEMMs of a step must move: A and B codes, scales and side
-    columns, and the fp32 output."""
+def gemm_alg_bytes(p, fused=True):
+    """Operand and output bytes the GEMMs of a step must move: A and B codes, scales and side
+    columns, and the fp32 output.  Fused, each input group's packed activations are read once;
+    unfused, once per projection."""
     pp = (p + 15) // 16 * 16
-    tot = 0
+    M = M_PREFILL
+    a_bytes = lambda K: M * K // 2 + M * K // 16 + 2 * M * pp
+    tot = sum(a_bytes(K) for K in GROUP_K) if fused else sum(a_bytes(K) for _, _, K, _ in PROJ)
     for _, N, K, _ in PROJ:
-        M = M_PREFILL
-        tot += M * K // 2 + M * K // 16 + 2 * M * pp + N * K // 2 + N * K // 16 + 2 * N * pp + 4 * M * N
+        tot += N * K // 2 + N * K // 16 + 2 * N * pp + 4 * M * N
     return tot
 
 
@@ -140,9 +146,9 @@ def make_weights(N, K, seed, device):
 class PrefillLayer:
     """Buffers and launches of one per-step pass over a Qwen3-8B layer."""
 
-    def __init__(self, F, M, p, seed, device, out_bf16=False):
+    def __init__(self, F, M, p, seed, device, out_bf16=False, fused=True):
         import torch
-        self.F, self.M, self.p = F, M, p
+        self.F, self.M, self.p, self.fused = F, M, p, fused
         self.X = [make_activations(M, K, seed * 100 + i, device) for i, K in enumerate(GROUP_K)]
         self.W = [make_weights(N, K, seed * 100 + 10 + j, device) for j, (_, N, K, _) in enumerate(PROJ)]
         self.st4 = F.StatsState(3, 4096, device=device)
@@ -154,13 +160,26 @@ class PrefillLayer:
         self.m12 = torch.empty(1, 384, dtype=torch.int32, device=device)
         self.g12 = torch.empty(1, dtype=torch.float32, device=device)
         self.xq = [F.alloc_packed(M, K, p, device) for K in GROUP_K]
-        self.wq = [F.alloc_packed(N, K, p, device) for (_, N, K, _) in PROJ]
         self.gW = torch.empty(len(PROJ), dtype=torch.float32, device=device)
-        self.alpha = torch.empty(len(PROJ), dtype=torch.float32, device=device)
+        self.alpha = torch.empty(len(PROJ), dtype=torch.float32, device=device)   # PROJ order: a group's are adjacent
         popts = F.FS_OUT_BF16 if out_bf16 else 0
-        self.plans = [F.Plan(N, K, max(p, 1), popts) for (_, N, K, _) in PROJ]
         dt = torch.bfloat16 if out_bf16 else torch.float32
-        self.Y = [torch.empty(M, N, dtype=dt, device=device) for (_, N, K, _) in PROJ]
+        if fused:
+            # projections of one input group stacked by rows: one segmented GEMM per group
+            self.wq, self.wq_group, self.seg = [None] * len(PROJ), [], []
+            for gi, js in enumerate(GROUP_PROJ):
+                rows = [PROJ[j][1] for j in js]
+                allp, views = F.stacked_packed(rows, GROUP_K[gi], p, device)
+                self.wq_group.append(allp)
+                for j, v in zip(js, views):
+                    self.wq[j] = v
+                self.seg.append([0] + [sum(rows[:i + 1]) for i in range(len(rows))])
+            self.plans = [F.Plan(self.seg[gi][-1], GROUP_K[gi], max(p, 1), popts) for gi in range(4)]
+            self.Y = [torch.empty(M, self.seg[gi][-1], dtype=dt, device=device) for gi in range(4)]
+        else:
+            self.wq = [F.alloc_packed(N, K, p, device) for (_, N, K, _) in PROJ]
+            self.plans = [F.Plan(N, K, max(p, 1), popts) for (_, N, K, _) in PROJ]
+            self.Y = [torch.empty(M, N, dtype=dt, device=device) for (_, N, K, _) in PROJ]
         self.flops = sum(2.0 * M * N * K for (_, N, K, _) in PROJ)
         # per-group views for the multi-stream step (one selection problem per group)
         self.gstate = []
@@ -174,7 +193,12 @@ class PrefillLayer:
         self.gP = [self.P4[i:i + 1] for i in range(3)] + [self.P12]
         self.gm = [self.m4[i:i + 1] for i in range(3)] + [self.m12]
         self.gg = [self.g4[i:i + 1] for i in range(3)] + [self.g12]
-        self.launches_per_step = 4 + 4 + 3 * len(PROJ) + 4 + len(PROJ)   # select per group; prepare = amax + gain + quantise
+
+    def launches_per_step(self, serial=False):
+        """Kernel launches of one step: statistics per group, selection (one launch per statistics
+        state when serial, one per group on streams), weight pre-split = amax + gain + quantise per
+        projection, activation quantise per group, the GEMMs."""
+        return 4 + (2 if serial else 4) + 3 * len(PROJ) + 4 + len(self.gemm_fns())
 
     def mask_gain(self, gi):
         if gi < 3:
@@ -203,9 +227,8 @@ class PrefillLayer:
                 F.fs_prepare_weights(self.W[j], mask, self.p, gA, out=self.wq[j], gW=self.gW[j:j + 1],
                                      alpha=self.alpha[j:j + 1])
         F.fs_quantize_splice(self.X[gi], mask, self.p, gA, out=self.xq[gi])
-        for j, (_, N, K, pg) in enumerate(PROJ):
-            if pg == gi:
-                F.fs_splice_gemm(self.plans[j], self.xq[gi], self.wq[j], self.alpha[j:j + 1], Y=self.Y[j])
+        for fn in self.gemm_fns(gi):
+            fn()
 
     def step_streams(self, streams, allreduce=None):
         """The same work as step(), with the four independent input-group chains on four streams."""
@@ -251,12 +274,24 @@ class PrefillLayer:
                 fn()
         return [stats, select, prepare, quantize, gemm]
 
-    def gemm_fns(self):
+    def gemm_fns(self, group=None):
+        """The GEMM launches (of one input group, or all): one segmented launch per group when
+        fused, else one per projection."""
         F = self.F
+        groups = range(4) if group is None else (group,)
+        if self.fused:
+            def make_g(gi):
+                js = GROUP_PROJ[gi]
+                return lambda: F.fs_splice_gemm_segmented(self.plans[gi], self.xq[gi], self.wq_group[gi],
+                                                          self.alpha[js[0]:js[-1] + 1], self.seg[gi], Y=self.Y[gi])
+            return [make_g(gi) for gi in groups]
 
         def make(j, gi):
             return lambda: F.fs_splice_gemm(self.plans[j], self.xq[gi], self.wq[j], self.alpha[j:j + 1], Y=self.Y[j])
-        return [make(j, gi) for j, (_, N, K, gi) in enumerate(PROJ)]
+        return [make(j, gi) for j, (_, N, K, gi) in enumerate(PROJ) if gi in groups]
+
+    def gemm_names(self):
+        return list(GROUP_NAMES) if self.fused else [name for name, _, _, _ in PROJ]
 
     def check(self):
         for pl in self.plans:
@@ -424,10 +459,11 @@ def rollout_case(F, device, reps=20):
     return res
 
 
-def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20):
+def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20, fused=True):
+    """Decode GEMMs over `layers` distinct layers' weights (larger than L2 together), M tokens per
+    layer: one segmented launch per input group (fused) or one launch per projection."""
     import torch
     res = {}
-    packed = []          # per layer: list of (wq, alpha) per projection
     st = F.StatsState(1, 4096, device=device)
     calib = make_activations(4096, 4096, 999, device)
     F.fs_channel_stats(calib, st)
@@ -435,22 +471,29 @@ def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20):
     st12 = F.StatsState(1, 12288, device=device)
     F.fs_channel_stats(make_activations(4096, 12288, 998, device), st12)
     _, m12, g12 = F.fs_select_topk(st12, p)
+    units = [list(js) for js in GROUP_PROJ] if fused else [[j] for j in range(len(PROJ))]
+    packed = []          # per layer: list of (stacked weights, alpha, segment starts) per launch
     for layer in range(layers):
         row = []
-        for j, (_, N, K, gi) in enumerate(PROJ):
-            W = make_weights(N, K, 5000 + layer * 10 + j, device)
+        for js in units:
+            rows, K = [PROJ[j][1] for j in js], PROJ[js[0]][2]
             mask, g = (m4[0], g4[0:1]) if K == 4096 else (m12[0], g12[0:1])
-            wq, gW, alpha = F.fs_prepare_weights(W, mask, p, g)
-            row.append((wq, alpha))
-            del W
+            wall, views = F.stacked_packed(rows, K, p, device)
+            alpha = torch.empty(len(js), dtype=torch.float32, device=device)
+            for i, (j, v) in enumerate(zip(js, views)):
+                W = make_weights(PROJ[j][1], K, 5000 + layer * 10 + j, device)
+                F.fs_prepare_weights(W, mask, p, g, out=v, alpha=alpha[i:i + 1])
+                del W
+            row.append((wall, alpha, [0] + [sum(rows[:i + 1]) for i in range(len(rows))]))
         packed.append(row)
     torch.cuda.synchronize()
-    wbytes = sum(wq.q.numel() + N * (K // 16) + N * F.side_cols(p) * 2 for (wq, _), (_, N, K, _) in zip(packed[0], PROJ))
+    wbytes = sum(N * K // 2 + N * (K // 16) + N * F.side_cols(p) * 2 for (_, N, K, _) in PROJ)
     for M in Ms:
         Xs = [make_activations(M, K, 77 + gi, device) for gi, K in enumerate(GROUP_K)]
         xq = [F.alloc_packed(M, K, p, device) for K in GROUP_K]
-        plans = [F.Plan(N, K, max(p, 1)) for (_, N, K, _) in PROJ]
-        Ys = [torch.empty(M, N, dtype=torch.float32, device=device) for (_, N, K, _) in PROJ]
+        plans = [F.Plan(sum(PROJ[j][1] for j in js), PROJ[js[0]][2], max(p, 1)) for js in units]
+        Ys = [torch.empty(M, pl_n, dtype=torch.float32, device=device)
+              for pl_n in (sum(PROJ[j][1] for j in js) for js in units)]
 
         def run_layers(with_quant: bool):
             for layer in range(layers):
@@ -458,9 +501,13 @@ def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20):
                     for gi, K in enumerate(GROUP_K):
                         mask, g = (m4[0], g4[0:1]) if K == 4096 else (m12[0], g12[0:1])
                         F.fs_quantize_splice(Xs[gi], mask, p, g, out=xq[gi])
-                for j, (_, N, K, gi) in enumerate(PROJ):
-                    wq, alpha = packed[layer][j]
-                    F.fs_splice_gemm(plans[j], xq[gi], wq, alpha, Y=Ys[j])
+                for u, js in enumerate(units):
+                    wall, alpha, seg = packed[layer][u]
+                    gi = PROJ[js[0]][3]
+                    if len(js) == 1:
+                        F.fs_splice_gemm(plans[u], xq[gi], wall, alpha, Y=Ys[u])
+                    else:
+                        F.fs_splice_gemm_segmented(plans[u], xq[gi], wall, alpha, seg, Y=Ys[u])
 
         out = {}
         for tag, wq_flag in (("gemm", False), ("quant+gemm", True)):
@@ -484,11 +531,13 @@ def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20):
             e1.record()
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / reps
+            # the byte count is the per-projection one in both forms: weights once, packed
+            # activations once per projection, fp32 outputs
             xbytes = sum(M * K * 2 + M * (K // 2 + K // 16 + F.side_cols(p) * 2) for K in GROUP_K) if wq_flag else 0
             abytes = sum(M * (K // 2 + K // 16 + F.side_cols(p) * 2) + M * N * 4 for (_, N, K, _) in PROJ)
             total = layers * (wbytes + abytes + xbytes)
             out[tag] = {"us_per_layer": 1000.0 * ms / layers, "GBps": total / (ms * 1e-3) / 1e9,
-                        "bytes_per_layer": wbytes + abytes + xbytes}
+                        "bytes_per_layer": wbytes + abytes + xbytes, "launches_per_layer": len(units)}
             del graph
         for pl in plans:
             pl.check()
@@ -592,24 +641,39 @@ def prep_case(F, args, device):
 
 def kernel_case(F, args, device):
     """fs_splice_gemm alone on one projection shape (--shape; M=8192 for `gemm`, M=--decode-m for
-    `decode`), for profiling one kernel."""
+    `decode`), or fs_splice_gemm_segmented on one fused input group (--shape qkv / gate_up), for
+    profiling one kernel."""
     import torch
     if args.case == "prep":
         return prep_case(F, args, device)
-    N, K = {name: (n, k) for name, n, k, _ in PROJ}[args.shape]
+    if args.shape in GROUP_NAMES:
+        gi = GROUP_NAMES.index(args.shape)
+        rows = [PROJ[j][1] for j in GROUP_PROJ[gi]]
+        K = GROUP_K[gi]
+    else:
+        N, K = {name: (n, k) for name, n, k, _ in PROJ}[args.shape]
+        rows = [N]
+    N = sum(rows)
     M = M_PREFILL if args.case == "gemm" else args.decode_m
     X = make_activations(M, K, 3, device)
-    W = make_weights(N, K, 4, device)
     st = F.StatsState(1, K, device=device)
     F.fs_channel_stats(make_activations(max(M, 2048), K, 3, device), st)
     _, mask, g = F.fs_select_topk(st, args.p)
-    wq, _, alpha = F.fs_prepare_weights(W, mask[0], args.p, g)
+    wall, views = F.stacked_packed(rows, K, args.p, device)
+    alpha = torch.empty(len(rows), dtype=torch.float32, device=device)
+    for i, (n, v) in enumerate(zip(rows, views)):
+        F.fs_prepare_weights(make_weights(n, K, 4 + i, device), mask[0], args.p, g, out=v, alpha=alpha[i:i + 1])
+    seg = [0] + [sum(rows[:i + 1]) for i in range(len(rows))]
     xq = F.fs_quantize_splice(X, mask[0], args.p, g)
     plan = F.Plan(N, K, max(args.p, 1))
     Y = torch.empty(M, N, dtype=torch.float32, device=device)
+    if len(rows) == 1:
+        run = lambda: F.fs_splice_gemm(plan, xq, wall, alpha, Y=Y)
+    else:
+        run = lambda: F.fs_splice_gemm_segmented(plan, xq, wall, alpha, seg, Y=Y)
     for _ in range(args.warmup):
-        F.fs_splice_gemm(plan, xq, wq, alpha, Y=Y)
-    ms = timed(lambda: F.fs_splice_gemm(plan, xq, wq, alpha, Y=Y), args.steps) / args.steps
+        run()
+    ms = timed(run, args.steps) / args.steps
     plan.check()
     print(json.dumps({"case": args.case, "shape": args.shape, "M": M, "N": N, "K": K, "p": args.p,
                       "us": ms * 1000.0, "tflops": 2.0 * M * N * K / (ms * 1e-3) / 1e12}))
@@ -630,9 +694,11 @@ def main():
                     help="step: the full benchmark; gemm / decode: only fs_splice_gemm on one projection "
                          "shape (M=8192, or M=--decode-m) for profiling one kernel; prep: the preparation "
                          "kernels on the q projection")
-    ap.add_argument("--shape", default="q", choices=[name for name, _, _, _ in PROJ],
+    ap.add_argument("--shape", default="q", choices=[name for name, _, _, _ in PROJ] + list(GROUP_NAMES[::2]),
                     help="projection shape of --case gemm / decode")
     ap.add_argument("--decode-m", type=int, default=16, help="tokens of --case decode (1..16)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="one GEMM launch per projection instead of one segmented launch per input group")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -661,14 +727,14 @@ def main():
     if args.case != "step":
         return kernel_case(F, args, device)
 
-    layer = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device)
+    layer = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device, fused=not args.unfused)
     allreduce = stats_allreduce_fn(dist) if use_dist else None
     for _ in range(args.warmup):
         layer.step(allreduce)
     torch.cuda.synchronize()
     layer.check()
 
-    # The step is captured once into a CUDA graph and replayed: host launch latency of the 38
+    # The step is captured once into a CUDA graph and replayed: host launch latency of the 35-38
     # small library calls would otherwise show up as GPU idle time.  Each phase (and each GEMM)
     # is also captured on its own, replayed back to back with events in between, to attribute
     # time per kernel on the device.
@@ -691,7 +757,8 @@ def main():
     phase_graphs = [capture(fn) for fn in layer.phase_fns(allreduce)]
     gemm_graphs = [capture(fn) for fn in layer.gemm_fns()]
     phase_us = {name: 0.0 for name in PrefillLayer.PHASES}
-    gemm_ms = [[0.0] * len(PROJ) for _ in range(args.steps)]
+    gemm_names = layer.gemm_names()
+    gemm_ms = [[0.0] * len(gemm_names) for _ in range(args.steps)]
     for it_ in range(args.steps):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(phase_graphs) + len(gemm_graphs) + 1)]
         evs[0].record()
@@ -704,13 +771,13 @@ def main():
         for i, name in enumerate(PrefillLayer.PHASES[:-1]):
             phase_us[name] += evs[i].elapsed_time(evs[i + 1]) * 1000.0 / args.steps
         base = len(phase_graphs) - 1
-        for j in range(len(PROJ)):
+        for j in range(len(gemm_names)):
             gemm_ms[it_][j] = evs[base + j].elapsed_time(evs[base + j + 1])
     layer.check()
     gemm_total_ms = sum(sum(r) for r in gemm_ms) / args.steps
     phase_us["gemm"] = gemm_total_ms * 1000.0
     gemm_tflops = layer.flops / (gemm_total_ms * 1e-3) / 1e12
-    per_proj = {name: statistics.mean(r[j] for r in gemm_ms) * 1000.0 for j, (name, _, _, _) in enumerate(PROJ)}
+    per_proj = {name: statistics.mean(r[j] for r in gemm_ms) * 1000.0 for j, name in enumerate(gemm_names)}
     fp4_peak = peaks["bf16_tflops"] * 4.0         # dense NVFP4 = 4x dense BF16 (nominal 9 vs 2.25 PFLOP/s)
     del phase_graphs, gemm_graphs
 
@@ -733,6 +800,7 @@ def main():
     ms_e2e = timed(e2e_step, e2e_steps, dist if use_dist else None) / e2e_steps
     e2e_value = world * layer.flops / (ms_e2e * 1e-3) / 1e12
 
+    fkey = "fused" if layer.fused else "unfused"
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -743,11 +811,13 @@ def main():
                    "global_batch": world * M_PREFILL, "seq_len": 1024, "parallelism": f"dp{world}",
                    "p": p, "l2": "inputs larger than L2 (0.85 GB of bf16 activations and weights per step)"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_STEP,
-                     "traffic_unit": "DRAM bytes per step (the 7 GEMM launches; ncu dram__bytes_read.sum + "
-                                     "dram__bytes_write.sum per shape, profiles/splice_gemm_tc_m8192_p64.md)",
-                     "algorithmic_bytes": gemm_alg_bytes(p),
-                     "kernel": "splice_gemm_tc_kernel (all 7 projections; sum 2MNK / sum of CUDA-event times)",
+                     "frac": gemm_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_STEP[fkey],
+                     "traffic_unit": f"DRAM bytes per step (the {len(gemm_names)} GEMM launches; ncu "
+                                     "dram__bytes_read.sum + dram__bytes_write.sum per shape, "
+                                     "profiles/splice_gemm_tc_dram_m8192_p64.md)",
+                     "algorithmic_bytes": gemm_alg_bytes(p, layer.fused),
+                     "kernel": f"splice_gemm_tc_kernel ({len(gemm_names)} launches: {', '.join(gemm_names)}; "
+                               "sum 2MNK / sum of CUDA-event times)",
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16 ratio), "
                                     "of measured"},
         "gemm_us": per_proj,
@@ -755,7 +825,7 @@ def main():
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": ms_e2e},
-        "gpu_launches": (38 if args.serial else layer.launches_per_step) * args.steps,
+        "gpu_launches": layer.launches_per_step(args.serial) * args.steps,
         "graph": "each timed step is one CUDA-graph replay of the step's launches" +
                  ("" if args.serial else "; the 4 independent input-group chains run on 4 streams"),
     }
@@ -764,7 +834,7 @@ def main():
         # overhead against P = 0: the same step and the GEMMs alone
         del host_x, host_y
         torch.cuda.empty_cache()
-        l0 = PrefillLayer(F, M_PREFILL, 0, seed=2 + rank, device=device)
+        l0 = PrefillLayer(F, M_PREFILL, 0, seed=2 + rank, device=device, fused=not args.unfused)
         for _ in range(3):
             l0.step()
         # the P = 0 step is captured the same way as the timed step (4 streams unless --serial)
@@ -788,8 +858,8 @@ def main():
         del g0s, gg0
         del l0
         torch.cuda.empty_cache()
-        dec, wbytes = decode_sweep(F, p, device)
-        dec0, wbytes0 = decode_sweep(F, 0, device, Ms=(16,))
+        dec, wbytes = decode_sweep(F, p, device, fused=not args.unfused)
+        dec0, wbytes0 = decode_sweep(F, 0, device, Ms=(16,), fused=not args.unfused)
         hbm = peaks["hbm_gbs"]
         line["decode"] = {k: {**v["gemm"], "frac_hbm": v["gemm"]["GBps"] / hbm,
                               "with_quantise": {**v["quant+gemm"], "frac_hbm": v["quant+gemm"]["GBps"] / hbm}}

@@ -213,6 +213,28 @@ fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, 
                          const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
                          const float* alpha, void* Y, int64_t ldy, void* stream);
 
+/* Segmented SpliceGEMM: one launch over several projections that read the same activations (q,
+ * k and v; gate and up), their packed weights stacked as adjacent row ranges of one operand.
+ * FourSight §5.2 applies SpliceGEMM to every linear projection; computing projections that share
+ * an input in one launch gives each of them the same result as its own fs_splice_gemm call, up to
+ * the order of FP32 partial sums.
+ *   plan        N = the total rows (output columns) of all segments; p_max and opts as usual.
+ *   nseg        1..8 segments; seg_start: HOST array of nseg + 1 int32, 0 = seg_start[0] < ... <
+ *               seg_start[nseg] = N, interior boundaries multiples of 256 (of 128 when N % 256 != 0)
+ *               so that every tile of either path lies in one segment.
+ *   wq, sfw, ws segment s occupies rows [seg_start[s], seg_start[s+1]) of wq and ws and the scale
+ *               bytes from fs_sf_bytes(seg_start[s], K) on, exactly as fs_prepare_weights writes a
+ *               projection of seg_start[s+1] - seg_start[s] rows at those offsets; all segments are
+ *               prepared with the mask and gain of the shared activations.
+ *   alpha       device, nseg floats: segment s's alpha from its fs_prepare_weights.
+ *   Y           [M][ldy]: columns [seg_start[s], seg_start[s+1]) are projection s's output.
+ * Otherwise (operands, paths, alignment, errors) as fs_splice_gemm; argument errors are returned
+ * before anything launches. */
+fs_status fs_splice_gemm_segmented(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, const uint8_t* sfx,
+                                   const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
+                                   int32_t nseg, const int32_t* seg_start, const float* alpha, void* Y,
+                                   int64_t ldy, void* stream);
+
 /* Grouped SpliceGEMM over E experts (the mixture-of-experts projections).  Activations are the
  * padded-row outputs of fs_quantize_splice_grouped (row_offsets as given there); expert e's
  * weights are rows [e*N, (e+1)*N) of stacked wq [E*N][K/2], sfw (tiled over E*N rows) and

@@ -36,6 +36,7 @@ SIGNATURES = {
     "fs_plan_destroy": (C.c_int, [P]),
     "fs_plan_check": (C.c_int, [P, P]),
     "fs_splice_gemm": (C.c_int, [P, i64, i32, P, P, P, P, P, P, P, P, i64, P]),
+    "fs_splice_gemm_segmented": (C.c_int, [P, i64, i32, P, P, P, P, P, P, i32, P, P, P, i64, P]),
     "fs_splice_gemm_grouped": (C.c_int, [P, i32, P, i64, i32, P, P, P, P, P, P, P, P, i64, P]),
     "fs_seq_filter": (C.c_int, [P, i64, P, i32, i32, f32, i32, i32, i32, P, P, P, P, P, P]),
     "fs_splice_gemm_noalloc": (C.c_int, [i32, i32, u32, i64, i32, P, P, P, P, P, P, P, P, i64, i32, P]),

@@ -77,35 +77,80 @@ extern "C" fs_status fs_plan_check(fs_plan plan, void* stream) {
   return FS_OK;
 }
 
-extern "C" fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, const uint8_t* sfx,
-                                    const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
-                                    const float* alpha, void* Y, int64_t ldy, void* stream) {
-  if (M < 0) return fail(FS_ERR_INVALID_ARGUMENT, "fs_splice_gemm: M < 0");
-  fs_status st = check_operands("fs_splice_gemm", plan, p, xq, sfx, xs, wq, sfw, ws, alpha, Y, ldy);
+namespace {
+
+fs_status splice_gemm(const char* who, fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, const uint8_t* sfx,
+                      const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
+                      const Segments& seg, const float* alpha, void* Y, int64_t ldy, void* stream) {
+  if (M < 0) return fail(FS_ERR_INVALID_ARGUMENT, "%s: M < 0", who);
+  fs_status st = check_operands(who, plan, p, xq, sfx, xs, wq, sfw, ws, alpha, Y, ldy);
   if (st != FS_OK) return st;
   if (M == 0) return FS_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int pp = side_cols(p);
   const bool decode = (plan->opts & FS_PATH_DECODE) || (!(plan->opts & FS_PATH_TENSOR) && M <= 16);
   if (decode) {
-    if (M > 16) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm: the decode path takes M <= 16 (M=%lld)", (long long)M);
+    if (M > 16) return fail(FS_ERR_UNSUPPORTED, "%s: the decode path takes M <= 16 (M=%lld)", who, (long long)M);
     DecodeParams d{};
     d.M = static_cast<int>(M); d.N = plan->N; d.K = plan->K; d.pp = pp;
     d.kb4 = static_cast<int>(round_up(plan->K / 16, 4) / 4);
-    d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha;
+    d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha; d.seg = seg;
     d.Y = Y; d.ldy = ldy; d.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; d.err = plan->err;
     return launch_splice_gemm_decode_tc(d, s);
   }
-  if (M > (int64_t{1} << 31) - 256) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm: M too large");
+  if (M > (int64_t{1} << 31) - 256) return fail(FS_ERR_UNSUPPORTED, "%s: M too large", who);
   TcParams prm{};
   prm.M = M; prm.N = plan->N; prm.K = plan->K; prm.KT = plan->K / 256; prm.ST = static_cast<int>(ceil_div(pp, 64));
   prm.E = 1; prm.kb4 = plan->K / 64; prm.offsets = nullptr; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
-  prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
+  prm.seg = seg; prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
   TcLaunch L{};
   L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = M; L.b_rows = plan->N; L.y_rows = M; L.pp = pp;
   L.bn = (plan->N % 256 == 0) ? 256 : 128;
   L.max_tiles = ceil_div(M, 128) * ceil_div(plan->N, L.bn);
   return launch_splice_gemm_tc(L, prm, s);
+}
+
+Segments one_segment(int N) {
+  Segments sg{};
+  sg.n = 1;
+  sg.n0[0] = 0;
+  sg.n0[1] = N;
+  return sg;
+}
+
+}  // namespace
+
+extern "C" fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, const uint8_t* sfx,
+                                    const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
+                                    const float* alpha, void* Y, int64_t ldy, void* stream) {
+  if (!plan) return fail(FS_ERR_INVALID_ARGUMENT, "fs_splice_gemm: null plan");
+  return splice_gemm("fs_splice_gemm", plan, M, p, xq, sfx, xs, wq, sfw, ws, one_segment(plan->N), alpha, Y, ldy,
+                     stream);
+}
+
+extern "C" fs_status fs_splice_gemm_segmented(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq,
+                                              const uint8_t* sfx, const uint16_t* xs, const uint8_t* wq,
+                                              const uint8_t* sfw, const uint16_t* ws, int32_t nseg,
+                                              const int32_t* seg_start, const float* alpha, void* Y, int64_t ldy,
+                                              void* stream) {
+  const char* who = "fs_splice_gemm_segmented";
+  if (!plan) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null plan", who);
+  if (nseg < 1 || nseg > kMaxSegments || !seg_start)
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: need 1 <= nseg <= %d and seg_start", who, kMaxSegments);
+  // every tile of either path must lie in one segment
+  const int gran = (plan->N % 256 == 0) ? 256 : 128;
+  if (seg_start[0] != 0 || seg_start[nseg] != plan->N)
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: segments must start at 0 and end at N=%d", who, plan->N);
+  Segments sg{};
+  sg.n = nseg;
+  for (int i = 0; i <= nseg; ++i) {
+    if (i > 0 && seg_start[i] <= seg_start[i - 1])
+      return fail(FS_ERR_INVALID_ARGUMENT, "%s: segment starts must increase", who);
+    if (i > 0 && i < nseg && seg_start[i] % gran != 0)
+      return fail(FS_ERR_INVALID_ARGUMENT, "%s: segment boundaries must be multiples of %d", who, gran);
+    sg.n0[i] = seg_start[i];
+  }
+  return splice_gemm(who, plan, M, p, xq, sfx, xs, wq, sfw, ws, sg, alpha, Y, ldy, stream);
 }
 
 extern "C" fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64_t* row_offsets, int64_t max_rows,
@@ -123,6 +168,7 @@ extern "C" fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64
   TcParams prm{};
   prm.M = 0; prm.N = plan->N; prm.K = plan->K; prm.KT = plan->K / 256; prm.ST = static_cast<int>(ceil_div(pp, 64));
   prm.E = E; prm.kb4 = plan->K / 64; prm.offsets = row_offsets; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
+  prm.seg = one_segment(plan->N);
   prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
   TcLaunch L{};
   L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = a_rows; L.b_rows = static_cast<int64_t>(E) * plan->N; L.y_rows = max_rows; L.pp = pp;

@@ -6,6 +6,23 @@
 
 namespace fs {
 
+// Output segments of one launch: weight rows (= output columns) [seg_n0[s], seg_n0[s+1]) use
+// alpha[s] (projections that share an input, packed as adjacent row ranges).
+constexpr int kMaxSegments = 8;
+struct Segments {
+  int n;                           // 1 .. kMaxSegments
+  int n0[kMaxSegments + 1];        // first row of each segment, n0[n] = N
+};
+
+// Segment holding row `row` (segments are whole tiles, so any row of a tile will do).
+__device__ __forceinline__ int segment_of(int row, const Segments& sg) {
+  int s = 0;
+#pragma unroll
+  for (int i = 1; i < kMaxSegments; ++i)
+    if (i < sg.n && row >= sg.n0[i]) s = i;
+  return s;
+}
+
 // Kernel parameters of the tensor-core path (plain: E = 1, offsets = null).
 struct TcParams {
   int64_t M;
@@ -14,7 +31,8 @@ struct TcParams {
   const int64_t* offsets;
   const uint8_t* sfa;
   const uint8_t* sfb;
-  const float* alpha;
+  const float* alpha;     // [E] for experts, else [segments]
+  Segments seg;
   void* Y;
   int64_t ldy;
   int out_bf16;
@@ -50,7 +68,8 @@ struct DecodeParams {
   const uint8_t* wq;
   const uint8_t* sfw;
   const uint16_t* ws;
-  const float* alpha;
+  const float* alpha;  // [segments]
+  Segments seg;
   void* Y;
   int64_t ldy;
   int out_bf16;

@@ -66,6 +66,7 @@ struct DecTcParams {
   const uint8_t* sfw;
   const uint8_t* sfx;
   const float* alpha;
+  Segments seg;
   void* Y;
   int64_t ldy;
   int out_bf16;
@@ -252,7 +253,7 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
     const int share = ((kOut + p.S - 1) / p.S + 3) & ~3;
     const int v0 = rank * share;
     const int v1 = v0 + share < kOut ? v0 + share : kOut;
-    const float alpha = __ldg(p.alpha);
+    const float alpha = __ldg(p.alpha + segment_of(n0, p.seg));
     const uint32_t red_addr = ptx::smem_u32(red);
     for (int v = v0 + 4 * e; v < v1; v += 4 * 128) {
       const int t = v / kDRows, rr = v - t * kDRows;   // 4 rows rr..rr+3 of token t
@@ -295,7 +296,8 @@ fs_status launch_splice_gemm_decode_tc(const DecodeParams& d, cudaStream_t s) {
   }
   DecTcParams p{};
   p.M = d.M; p.N = d.N; p.KT = d.K / 256; p.ST = static_cast<int>(ceil_div(d.pp, 64)); p.kb4 = d.kb4;
-  p.sfw = d.sfw; p.sfx = d.sfx; p.alpha = d.alpha; p.Y = d.Y; p.ldy = d.ldy; p.out_bf16 = d.out_bf16; p.err = d.err;
+  p.sfw = d.sfw; p.sfx = d.sfx; p.alpha = d.alpha; p.seg = d.seg; p.Y = d.Y; p.ldy = d.ldy; p.out_bf16 = d.out_bf16;
+  p.err = d.err;
   // K split: as many CTAs per 128-row tile as fill the SMs at the resident CTAs per SM, at most 8
   // (a portable cluster);
   // every split keeps at least one FP4 k-tile.

@@ -91,12 +91,14 @@ extern "C" fs_status fs_splice_gemm_noalloc(int32_t N, int32_t K, uint32_t opts,
     d.M = static_cast<int>(M); d.N = N; d.K = K; d.pp = pp; d.kb4 = static_cast<int>(round_up(K / 16, 4) / 4);
     d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha;
     d.Y = Y; d.ldy = ldy; d.out_bf16 = bf16 ? 1 : 0; d.err = scratch;
+    d.seg.n = 1; d.seg.n0[0] = 0; d.seg.n0[1] = N;
     st = launch_splice_gemm_decode_tc(d, s);
   } else {
     TcParams prm{};
     prm.M = M; prm.N = N; prm.K = K; prm.KT = K / 256; prm.ST = static_cast<int>(ceil_div(pp, 64));
     prm.E = 1; prm.kb4 = K / 64; prm.offsets = nullptr; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
     prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = bf16 ? 1 : 0; prm.err = scratch;
+    prm.seg.n = 1; prm.seg.n0[0] = 0; prm.seg.n0[1] = N;
     TcLaunch L{};
     L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = M; L.b_rows = N; L.y_rows = M; L.pp = pp;
     L.bn = (N % 256 == 0) ? 256 : 128;

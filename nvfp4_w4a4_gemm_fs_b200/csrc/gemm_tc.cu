@@ -420,7 +420,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       const TileMap m = map_tile<CG>(t, p, cum_m, rank);
       if (!wait_bar(acc_full + acc, acc_phase, abort_flag, p.err)) break;
       ptx::tc_fence_after();
-      const float alpha = __ldg(p.alpha + m.e);
+      const float alpha = __ldg(p.alpha + (p.offsets ? m.e : segment_of(m.n0, p.seg)));
       const bool use_tma = !(p.offsets && m.rows < kBM);
       const bool row_ok = row < m.rows;
       const int64_t yrow = m.yrow + row;

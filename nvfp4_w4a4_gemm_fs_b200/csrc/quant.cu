@@ -384,9 +384,15 @@ __global__ void __launch_bounds__(256) weight_amax_f32_kernel(const float* __res
 }
 
 // bf16 weights: a streaming reduction.  Each warp takes whole rows, lane l the 8 columns
-// 8l..8l+7 of every 256-column stripe, four 16-byte loads in flight.  |w| of a bf16 value orders
+// 8l..8l+7 of every 256-column stripe, kAmaxDepth 16-byte loads in flight (the grid holds only a
+// few warps per SM for N = 4096, so each warp carries the memory parallelism).  |w| of a bf16 value orders
 // like its low 15 bits, so the maximum is taken on packed 16-bit halves (max.u16x2) after
 // clearing sign bits and protected lanes; the result, shifted to the high half, is the float.
+#ifndef FS_AMAX_DEPTH
+#define FS_AMAX_DEPTH 8
+#endif
+constexpr int kAmaxDepth = FS_AMAX_DEPTH;
+
 __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -425,12 +431,12 @@ __global__ void __launch_bounds__(256) weight_amax_bf16_kernel(const uint16_t* _
   for (int64_t r = warp; r < N; r += nwarps) {
     const uint16_t* row = W + r * ldw;
     int s = 0;
-    for (; s + 4 <= stripes; s += 4) {
-      uint4 v[4];
+    for (; s + kAmaxDepth <= stripes; s += kAmaxDepth) {
+      uint4 v[kAmaxDepth];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(row + (s + u) * 256 + lane * 8));
+      for (int u = 0; u < kAmaxDepth; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(row + (s + u) * 256 + lane * 8));
 #pragma unroll
-      for (int u = 0; u < 4; ++u) fold(v[u], keep((s + u) * 256 + lane * 8));
+      for (int u = 0; u < kAmaxDepth; ++u) fold(v[u], keep((s + u) * 256 + lane * 8));
     }
     for (; s < stripes; ++s) fold(__ldg(reinterpret_cast<const uint4*>(row + s * 256 + lane * 8)), keep(s * 256 + lane * 8));
     if (tail_cols && lane * 8 < tail_cols) {

@@ -7,12 +7,23 @@
 //
 // Moments are exact integers (s1 = sum rint(x 2^16), s2 = sum rint(x^2 2^14)), so every
 // reduction order gives the same state and the selection is reproducible bit for bit.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace fs {
 namespace {
 
 constexpr int kStatsWarps = 8;
+#ifndef FS_STATS_MIN_CTAS
+#define FS_STATS_MIN_CTAS 3
+#endif
+#ifndef FS_STATS_VEC
+#define FS_STATS_VEC 8
+#endif
+// bf16 channels per lane: 8 (16-byte loads).  4 channels with 4 CTAs per SM was faster on an
+// L2-resident input but 10% slower on a 16384 x 4096 input read from HBM.
+constexpr int kStatsVecBf16 = FS_STATS_VEC;
 constexpr double kS1Scale = 65536.0;
 constexpr double kS2Scale = 16384.0;
 constexpr float kRangeLimit = 32768.0f;
@@ -96,7 +107,7 @@ __device__ __forceinline__ void add_f32(long long& s1, long long& s2, float& ama
 // 64-bit totals in its own shared-memory slots ([warp][v][lane], conflict-free); the CTA reduces
 // them over warps and adds to the global state with integer atomics.
 template <typename T, int VEC>
-__global__ void __launch_bounds__(kStatsWarps * 32, 3)
+__global__ void __launch_bounds__(kStatsWarps * 32, FS_STATS_MIN_CTAS)
 channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int row_stride,
                      unsigned long long* n, unsigned long long* s1, unsigned long long* s2,
                      uint32_t* amax, uint32_t* flags) {
@@ -143,16 +154,17 @@ channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int
   const int64_t step = static_cast<int64_t>(gridDim.y) * kStatsWarps;
   if (active) {
     for (int64_t i = static_cast<int64_t>(blockIdx.y) * kStatsWarps + warp; i < taken; i += kUnroll * step) {
-      uint4 q[kUnroll];
+      using Load = typename std::conditional<sizeof(T) * VEC == 16, uint4, uint2>::type;   // VEC elements
+      Load q[kUnroll];
       int rows = 0;
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int64_t idx = i + u * step;
         if (idx < taken) {
-          q[u] = __ldg(reinterpret_cast<const uint4*>(X + idx * row_stride * ldx + c0));
+          q[u] = __ldg(reinterpret_cast<const Load*>(X + idx * row_stride * ldx + c0));
           ++rows;
         } else {
-          q[u] = make_uint4(0, 0, 0, 0);
+          q[u] = Load{};
         }
       }
       if constexpr (kF32) {
@@ -427,7 +439,7 @@ extern "C" fs_status fs_channel_stats(const void* X, int32_t dtype, int64_t M, i
   if (!aligned(s1, 8) || !aligned(s2, 8) || !aligned(n, 8) || !aligned(amax, 4) || !aligned(flags, 4)) return fail(FS_ERR_INVALID_ARGUMENT, "fs_channel_stats: misaligned state");
   if (M == 0) return FS_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int vec = dtype == FS_DTYPE_BF16 ? 8 : 4;
+  const int vec = dtype == FS_DTYPE_BF16 ? kStatsVecBf16 : 4;
   const int chunks = static_cast<int>(ceil_div(K, 32 * vec));
   const int64_t taken = ceil_div(M, row_stride);
   // Enough CTAs for ~4 per SM, each reading at least 64 rows.
@@ -439,7 +451,7 @@ extern "C" fs_status fs_channel_stats(const void* X, int32_t dtype, int64_t M, i
   auto* u1 = reinterpret_cast<unsigned long long*>(s1);
   auto* u2 = reinterpret_cast<unsigned long long*>(s2);
   if (dtype == FS_DTYPE_BF16)
-    channel_stats_kernel<uint16_t, 8><<<grid, kStatsWarps * 32, 0, s>>>(static_cast<const uint16_t*>(X), M, K, ldx, row_stride, un, u1, u2, amax, flags);
+    channel_stats_kernel<uint16_t, kStatsVecBf16><<<grid, kStatsWarps * 32, 0, s>>>(static_cast<const uint16_t*>(X), M, K, ldx, row_stride, un, u1, u2, amax, flags);
   else
     channel_stats_kernel<float, 4><<<grid, kStatsWarps * 32, 0, s>>>(static_cast<const float*>(X), M, K, ldx, row_stride, un, u1, u2, amax, flags);
   FS_CHECK_LAUNCH("fs_channel_stats");

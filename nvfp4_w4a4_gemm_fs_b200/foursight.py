@@ -16,6 +16,7 @@ __all__ = [
     "fs_channel_stats", "fs_stats_check", "fs_select_topk", "fs_prepare_weights",
     "fs_quantize_splice", "fs_quantize_splice_grouped", "fs_splice_gemm", "fs_splice_gemm_grouped",
     "fs_seq_filter", "Plan", "StatsState", "Packed", "side_cols", "sf_bytes", "grouped_rows",
+    "fs_splice_gemm_segmented", "stacked_packed",
     "alloc_packed", "stream_handle",
 ]
 
@@ -178,6 +179,41 @@ def fs_splice_gemm(plan: Plan, xq: Packed, wq: Packed, alpha: torch.Tensor, Y: t
                              _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, _ptr(alpha), _ptr(Y),
                              Y.stride(0), stream_handle(stream)), "fs_splice_gemm")
     return Y
+
+
+def fs_splice_gemm_segmented(plan: Plan, xq: Packed, wq: Packed, alpha: torch.Tensor, seg_start,
+                             Y: torch.Tensor | None = None, stream=None):
+    """Projections sharing the activations xq, stacked as row ranges seg_start[s]..seg_start[s+1]
+    of wq, each with its own alpha[s]; returns Y [M, N] with projection s in those columns."""
+    lib = _lib.load()
+    M = xq.rows
+    seg = [int(v) for v in seg_start]
+    arr = (C.c_int32 * len(seg))(*seg)
+    if Y is None:
+        dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
+        Y = torch.empty(M, plan.N, dtype=dt, device=xq.q.device)
+    check(lib.fs_splice_gemm_segmented(plan.handle, M, xq.p, _ptr(xq.q), _ptr(xq.sf), _ptr(xq.side) if xq.p else None,
+                                       _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, len(seg) - 1, arr,
+                                       _ptr(alpha), _ptr(Y), Y.stride(0), stream_handle(stream)),
+          "fs_splice_gemm_segmented")
+    return Y
+
+
+def stacked_packed(rows_per_segment, K: int, p: int, device="cuda") -> tuple:
+    """One packed weight operand for projections stacked by rows, and per-segment views of it that
+    fs_prepare_weights can write (rows of each segment must be a multiple of 128)."""
+    total = sum(rows_per_segment)
+    pp = side_cols(p)
+    q = torch.empty(total, K // 2, dtype=torch.uint8, device=device)
+    sf = torch.empty(sf_bytes(total, K), dtype=torch.uint8, device=device)
+    side = torch.zeros(total, max(pp, 8), dtype=torch.bfloat16, device=device)[:, :pp]
+    views, r0 = [], 0
+    for n in rows_per_segment:
+        if n % 128:
+            raise ValueError("segment rows must be a multiple of 128")
+        views.append(Packed(q[r0:r0 + n], sf[sf_bytes(r0, K):sf_bytes(r0 + n, K)], side[r0:r0 + n], n, K, p))
+        r0 += n
+    return Packed(q, sf, side, total, K, p), views
 
 
 def fs_splice_gemm_grouped(plan: Plan, row_offsets: torch.Tensor, max_rows: int, xq: Packed, wq: Packed,

@@ -135,6 +135,40 @@ def test_tensor_core_pairs_several_tiles_sampled_rows(M, N, K, p):
     _assert_close(Y[torch.from_numpy(rows).cuda()], Yr, mag)
 
 
+@pytest.mark.parametrize("path,M", [("decode", 8), ("tensor", 300)])
+def test_segmented_projections_match_each_projection(path, M):
+    """Three projections sharing X and P (a q/k/v-like group), stacked by rows (512, 256, 256),
+    each with its own weights and weight gain: one segmented launch reproduces every projection's
+    own oracle result in its columns of Y."""
+    K, p, seg_rows = 1024, 64, [512, 256, 256]
+    x, _ = synth.outlier_activations(201, M, K)
+    X = splice.as_f32(x, True)
+    st = stats.accumulate(stats.new_state(K), X)
+    P = stats.select_topk(st, p)
+    gA = stats.next_gain(st, P)
+    mask = mask_tensor(stats.protect_mask(P, K))
+    g = torch.tensor([float(gA)], device="cuda")
+    xq = F.fs_quantize_splice(bf16_tensor(x), mask, p, g)
+    wq_all, views = F.stacked_packed(seg_rows, K, p)
+    alphas = torch.empty(len(seg_rows), device="cuda")
+    Ws = []
+    for j, (n, view) in enumerate(zip(seg_rows, views)):
+        w = synth.gaussian_weights(300 + j, n, K)
+        Ws.append(splice.as_f32(w, True))
+        F.fs_prepare_weights(bf16_tensor(w), mask, p, g, out=view, alpha=alphas[j:j + 1])
+    seg = np.concatenate([[0], np.cumsum(seg_rows)]).tolist()
+    plan = F.Plan(seg[-1], K, p, F.FS_PATH_DECODE if path == "decode" else F.FS_PATH_TENSOR)
+    Y = F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, seg)
+    plan.check()
+    for j in range(len(seg_rows)):
+        Yr, mag = _ref(X, Ws[j], P, gA)
+        _assert_close(Y[:, seg[j]:seg[j + 1]], Yr, mag)
+    # boundaries must keep every tile inside one segment, start at 0 and end at N
+    for bad in ([0, 384, 768, 1024], [0, 512, 768, 1000], [256, 512, 768, 1024]):
+        with pytest.raises(F.FoursightError):
+            F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, bad)
+
+
 def test_repeatable_and_overwrites_output():
     X, W, Xt, Wt, P, gA = _problem(92, 256, 512, 1024, 64)
     Y1, _ = _run_gpu(Xt, Wt, P, gA, 64, 512, 1024)
