@@ -646,6 +646,9 @@ def kernel_case(F, args, device):
     import torch
     if args.case == "prep":
         return prep_case(F, args, device)
+    if args.case == "moe":
+        print(json.dumps({"case": "moe", **moe_case(F, args.p, device, reps=args.steps)}))
+        return
     if args.shape in GROUP_NAMES:
         gi = GROUP_NAMES.index(args.shape)
         rows = [PROJ[j][1] for j in GROUP_PROJ[gi]]
@@ -690,10 +693,10 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--serial", action="store_true", help="one stream for the whole step (no group concurrency)")
-    ap.add_argument("--case", default="step", choices=["step", "gemm", "decode", "prep"],
+    ap.add_argument("--case", default="step", choices=["step", "gemm", "decode", "prep", "moe"],
                     help="step: the full benchmark; gemm / decode: only fs_splice_gemm on one projection "
                          "shape (M=8192, or M=--decode-m) for profiling one kernel; prep: the preparation "
-                         "kernels on the q projection")
+                         "kernels on the q projection; moe: the grouped 64-expert projections alone")
     ap.add_argument("--shape", default="q", choices=[name for name, _, _, _ in PROJ] + list(GROUP_NAMES[::2]),
                     help="projection shape of --case gemm / decode")
     ap.add_argument("--decode-m", type=int, default=16, help="tokens of --case decode (1..16)")

@@ -407,9 +407,10 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     // Part 1: the 128 accumulator columns the next tile will overwrite are loaded into registers
     // and released at once (BN = 128: the whole tile).  Part 2 (BN = 256): the other 128 columns,
     // 32 at a time, while the next tile's MMAs run.  Each 32 x 32 chunk is scaled by alpha,
-    // staged in shared memory with the TMA swizzle and written by a TMA store.  Partial tiles of
-    // an expert (rows that end inside the output) use direct stores instead, since a box would
-    // cross into the next expert's rows.
+    // staged in shared memory with the TMA swizzle and written by a TMA store.  In a partial tile
+    // of an expert (rows that end inside the output) the warp whose 32 rows hold the expert's last
+    // row stores directly, since its box would cross into the next expert's rows; warps whose rows
+    // all belong to the expert still use TMA.
     const int quad = warp & 3;                  // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;           // row of the tile held by this thread
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
@@ -421,7 +422,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       if (!wait_bar(acc_full + acc, acc_phase, abort_flag, p.err)) break;
       ptx::tc_fence_after();
       const float alpha = __ldg(p.alpha + (p.offsets ? m.e : segment_of(m.n0, p.seg)));
-      const bool use_tma = !(p.offsets && m.rows < kBM);
+      const bool use_tma = !p.offsets || (quad + 1) * 32 <= m.rows;
       const bool row_ok = row < m.rows;
       const int64_t yrow = m.yrow + row;
       const int base = C::OVERLAP ? (i & 1) * 128 : 0;
@@ -465,16 +466,39 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           }
           ++nbuf;
         } else if (row_ok) {
+          // Y's base and row pitch are 16-byte aligned (the Y tensor map requires it) and col0 is
+          // a multiple of 32, so whole 32-column chunks go out as 16-byte stores.
+          const bool whole = col0 + 32 <= p.N;
           if (p.out_bf16) {
             uint16_t* y = static_cast<uint16_t*>(p.Y) + yrow * p.ldy + col0;
+            if (whole) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (col0 + c < p.N) y[c] = f32_to_bf16_bits(__uint_as_float(r[c]) * alpha);
+              for (int j = 0; j < 4; ++j) {
+                uint32_t w[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                  w[h] = static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[8 * j + 2 * h]) * alpha)) |
+                         (static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[8 * j + 2 * h + 1]) * alpha)) << 16);
+                *reinterpret_cast<uint4*>(y + 8 * j) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                if (col0 + c < p.N) y[c] = f32_to_bf16_bits(__uint_as_float(r[c]) * alpha);
+            }
           } else {
             float* y = static_cast<float*>(p.Y) + yrow * p.ldy + col0;
+            if (whole) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (col0 + c < p.N) y[c] = __uint_as_float(r[c]) * alpha;
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(y + 4 * j) =
+                    make_float4(__uint_as_float(r[4 * j]) * alpha, __uint_as_float(r[4 * j + 1]) * alpha,
+                                __uint_as_float(r[4 * j + 2]) * alpha, __uint_as_float(r[4 * j + 3]) * alpha);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                if (col0 + c < p.N) y[c] = __uint_as_float(r[c]) * alpha;
+            }
           }
         }
       };

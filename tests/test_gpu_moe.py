@@ -33,7 +33,7 @@ def _build(counts, N, K, p, seed=0):
     return E, offs, Xs, Ws, Ps, gAs
 
 
-def _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p):
+def _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p, plan_opts=0):
     total = int(offs[-1])
     X_all = np.concatenate([x for x in Xs if len(x)]) if total else np.zeros((0, K), np.uint16)
     Xt = bf16_tensor(X_all.reshape(total, K))
@@ -53,14 +53,15 @@ def _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p):
         F.fs_prepare_weights(bf16_tensor(Ws[e]), masks[e], p, gA[e:e + 1], out=out, gW=gW[e:e + 1],
                              alpha=alpha[e:e + 1])
     wq = F.Packed(wq_all, sf_all, ws_all, E * N, K, p)
-    plan = F.Plan(N, K, max(p, 1))
+    plan = F.Plan(N, K, max(p, 1), plan_opts)
     Y = F.fs_splice_gemm_grouped(plan, offs_t, total, xq, wq, alpha)
     plan.check()
     return xq, Y
 
 
 def _check_expert_outputs(offs, Xs, Ws, Ps, gAs, Y, rows_per_expert=None):
-    Yc = Y.cpu().numpy().astype(np.float64)
+    bf16_out = Y.dtype == torch.bfloat16
+    Yc = Y.float().cpu().numpy().astype(np.float64)
     for e in range(len(Xs)):
         r0, r1 = int(offs[e]), int(offs[e + 1])
         if r1 == r0:
@@ -73,7 +74,8 @@ def _check_expert_outputs(offs, Xs, Ws, Ps, gAs, Y, rows_per_expert=None):
         wq = splice.prepare_weights(W, Ps[e], gAs[e])
         Yr, mag = splice.splice_gemm(xq, wq, wq["alpha"])
         got = Yc[r0 + sel]
-        assert np.all(np.abs(got - Yr) <= 1e-5 * mag), f"expert {e}: outside tolerance"
+        tol = 1e-5 * mag + (2.0 ** -8 * np.abs(Yr) if bf16_out else 0.0)   # + half an ulp of bf16
+        assert np.all(np.abs(got - Yr) <= tol), f"expert {e}: outside tolerance"
 
 
 def test_grouped_small_experts_and_packed_layout():
@@ -127,3 +129,16 @@ def test_grouped_more_tiles_than_sms_side_heavy(N):
     E, offs, Xs, Ws, Ps, gAs = _build(counts, N, K, p, seed=3)
     _, Y = _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p)
     _check_expert_outputs(offs, Xs, Ws, Ps, gAs, Y, rows_per_expert=6)
+
+
+@pytest.mark.parametrize("N", [256, 384])
+def test_grouped_partial_tiles_bf16_output(N):
+    """Experts whose last tile ends inside a 32-row warp group, at a warp boundary and after one
+    row, with bf16 output: warps whose rows all belong to the expert store whole boxes, the warp
+    holding the expert's last row stores row by row, and nothing spills into the next expert."""
+    counts = [1, 127, 129, 32, 0, 64, 95, 160, 31]
+    K, p = 512, 16
+    E, offs, Xs, Ws, Ps, gAs = _build(counts, N, K, p, seed=4)
+    _, Y = _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p, plan_opts=F.FS_OUT_BF16)
+    assert Y.dtype == torch.bfloat16
+    _check_expert_outputs(offs, Xs, Ws, Ps, gAs, Y)
