@@ -31,6 +31,8 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 inline int side_cols(int p) { return (p + 15) / 16 * 16; }
 inline int64_t sf_bytes(int64_t rows, int K) { return round_up(rows, 128) * round_up(K / 16, 4); }
+// Streaming multiprocessors of the current device (queried once).
+int sm_count();
 
 #define FS_CHECK_LAUNCH(what)                                         \
   do {                                                                \

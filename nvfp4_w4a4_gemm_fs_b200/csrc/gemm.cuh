@@ -58,7 +58,6 @@ fs_status launch_splice_gemm_tc(const TcLaunch& L, const TcParams& prm, cudaStre
 // 2D K-major tensor map, 128-byte swizzle, box `box_inner` elements x `box_rows` rows.
 fs_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner_elems, uint64_t rows,
                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows);
-int sm_count();
 
 struct DecodeParams {
   int M, N, K, pp, kb4;

@@ -383,15 +383,17 @@ __global__ void __launch_bounds__(256) weight_amax_f32_kernel(const float* __res
   if ((threadIdx.x & 31) == 0 && bits) atomicMax(out_bits, bits);
 }
 
-// bf16 weights: a streaming reduction.  Each warp takes whole rows, lane l the 8 columns
-// 8l..8l+7 of every 256-column stripe, kAmaxDepth 16-byte loads in flight (the grid holds only a
-// few warps per SM for N = 4096, so each warp carries the memory parallelism).  |w| of a bf16 value orders
-// like its low 15 bits, so the maximum is taken on packed 16-bit halves (max.u16x2) after
-// clearing sign bits and protected lanes; the result, shifted to the high half, is the float.
+// bf16 weights: a streaming reduction over the whole matrix (the gain needs one maximum, so rows
+// play no role): the work is the N x K/256 stripes of 256 columns, dealt round-robin to the
+// warps, kAmaxDepth stripes (16-byte loads, lane l the 8 columns 8l..8l+7) in flight per warp.
+// |w| of a bf16 value orders like its low 15 bits, so the maximum is taken on packed 16-bit
+// halves (max.u16x2) after clearing sign bits and protected lanes; the result, shifted to the
+// high half, is the float.  One atomic per CTA.
 #ifndef FS_AMAX_DEPTH
 #define FS_AMAX_DEPTH 8
 #endif
 constexpr int kAmaxDepth = FS_AMAX_DEPTH;
+constexpr int kAmaxThreads = 256;
 
 __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
   uint32_t r;
@@ -399,9 +401,11 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
   return r;
 }
 
-__global__ void __launch_bounds__(256) weight_amax_bf16_kernel(const uint16_t* __restrict__ W, int64_t N, int K,
-                                                               int64_t ldw, const uint32_t* __restrict__ mask,
-                                                               uint32_t opts, uint32_t* out_bits) {
+__global__ void __launch_bounds__(kAmaxThreads) weight_amax_bf16_kernel(const uint16_t* __restrict__ W, int64_t N,
+                                                                        int K, int64_t ldw,
+                                                                        const uint32_t* __restrict__ mask,
+                                                                        uint32_t opts, uint32_t* out_bits) {
+  __shared__ uint32_t sh_max[kAmaxThreads / 32];
   const bool use_mask = mask && !(opts & FS_RESIDUAL);
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -428,26 +432,46 @@ __global__ void __launch_bounds__(256) weight_amax_bf16_kernel(const uint16_t* _
     m = vmax_u16x2(m, v.z & k.z);
     m = vmax_u16x2(m, v.w & k.w);
   };
-  for (int64_t r = warp; r < N; r += nwarps) {
-    const uint16_t* row = W + r * ldw;
-    int s = 0;
-    for (; s + kAmaxDepth <= stripes; s += kAmaxDepth) {
+  if (stripes > 0) {
+    // stripe u = r * stripes + s; this warp takes u = warp, warp + nwarps, ...
+    int64_t r = warp / stripes;
+    int s = static_cast<int>(warp - r * stripes);
+    const int64_t dr = nwarps / stripes;
+    const int ds = static_cast<int>(nwarps - dr * stripes);
+    while (r < N) {
       uint4 v[kAmaxDepth];
+      int c[kAmaxDepth];
 #pragma unroll
-      for (int u = 0; u < kAmaxDepth; ++u) v[u] = __ldg(reinterpret_cast<const uint4*>(row + (s + u) * 256 + lane * 8));
+      for (int d = 0; d < kAmaxDepth; ++d) {
+        c[d] = 0;
+        v[d] = make_uint4(0u, 0u, 0u, 0u);
+        if (r < N) {
+          c[d] = s * 256 + lane * 8;
+          v[d] = __ldg(reinterpret_cast<const uint4*>(W + r * ldw + c[d]));
+          r += dr;
+          s += ds;
+          if (s >= stripes) { s -= stripes; ++r; }
+        }
+      }
 #pragma unroll
-      for (int u = 0; u < kAmaxDepth; ++u) fold(v[u], keep((s + u) * 256 + lane * 8));
+      for (int d = 0; d < kAmaxDepth; ++d) fold(v[d], keep(c[d]));
     }
-    for (; s < stripes; ++s) fold(__ldg(reinterpret_cast<const uint4*>(row + s * 256 + lane * 8)), keep(s * 256 + lane * 8));
-    if (tail_cols && lane * 8 < tail_cols) {
-      const int c0 = stripes * 256 + lane * 8;
-      fold(__ldg(reinterpret_cast<const uint4*>(row + c0)), keep(c0));
-    }
+  }
+  if (tail_cols && lane * 8 < tail_cols) {
+    const int c0 = stripes * 256 + lane * 8;
+    for (int64_t r = warp; r < N; r += nwarps) fold(__ldg(reinterpret_cast<const uint4*>(W + r * ldw + c0)), keep(c0));
   }
   uint32_t bits = max(m & 0xFFFFu, m >> 16) << 16;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) bits = max(bits, __shfl_xor_sync(0xffffffffu, bits, o));
-  if (lane == 0 && bits) atomicMax(out_bits, bits);
+  if (lane == 0) sh_max[threadIdx.x >> 5] = bits;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0;
+#pragma unroll
+    for (int w = 0; w < kAmaxThreads / 32; ++w) b = max(b, sh_max[w]);
+    if (b) atomicMax(out_bits, b);
+  }
 }
 
 // gW from the reduced amax bits (stored in the gW slot), then alpha = fl32(1/fl32(gA*gW)).
@@ -456,17 +480,6 @@ __global__ void weight_gain_kernel(float* gW, float* alpha, const float* gA, uin
   const float g = (opts & FS_GAIN_EXACT) ? gain_exact(amax) : gain_pow2(amax);
   *gW = g;
   *alpha = __fdiv_rn(1.0f, __fmul_rn(*gA, g));
-}
-
-int quant_sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
 }
 
 template <Side kSide, bool kGrouped>
@@ -486,7 +499,7 @@ fs_status launch_quantize(int dtype, QuantArgs& a, int64_t padded_rows, cudaStre
                     : (passes ? quantize_kernel<float, kSide, kGrouped, true> : quantize_kernel<float, kSide, kGrouped, false>);
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQThreads, 0) != cudaSuccess || per_sm < 1) per_sm = 2;
-  const int64_t grid = std::min<int64_t>(chunks, static_cast<int64_t>(quant_sm_count()) * per_sm);
+  const int64_t grid = std::min<int64_t>(chunks, static_cast<int64_t>(sm_count()) * per_sm);
   kernel<<<static_cast<unsigned>(grid), kQThreads, 0, s>>>(a, chunks);
   FS_CHECK_LAUNCH("quantize kernel");
   return FS_OK;
@@ -554,9 +567,15 @@ extern "C" fs_status fs_prepare_weights(const void* W, int32_t dtype, int32_t N,
   if (e != cudaSuccess) return cuda_status(e, "fs_prepare_weights: memset");
   const uint32_t* m = p > 0 ? mask : nullptr;
   if (dtype == FS_DTYPE_BF16) {
-    // one warp per row, 8 warps per CTA, at most 8 CTAs per SM
-    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(N, 8), static_cast<int64_t>(quant_sm_count()) * 8));
-    weight_amax_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), N, K, ldw, m, opts, reinterpret_cast<uint32_t*>(gW));
+    // one wave of resident CTAs, each warp with at least kAmaxDepth stripes
+    static int per_sm = 0;
+    if (per_sm == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, weight_amax_bf16_kernel, kAmaxThreads, 0) !=
+                            cudaSuccess || per_sm < 1))
+      per_sm = 1;
+    const int64_t work = static_cast<int64_t>(N) * std::max(1, K / 256);
+    const unsigned grid = static_cast<unsigned>(std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div(work, (kAmaxThreads / 32) * kAmaxDepth), static_cast<int64_t>(sm_count()) * per_sm)));
+    weight_amax_bf16_kernel<<<grid, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(W), N, K, ldw, m, opts, reinterpret_cast<uint32_t*>(gW));
   } else {
     const int64_t blocks = static_cast<int64_t>(N) * (K / 16);
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(blocks, 256), 148 * 8));

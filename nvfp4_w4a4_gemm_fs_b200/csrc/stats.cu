@@ -439,18 +439,27 @@ extern "C" fs_status fs_channel_stats(const void* X, int32_t dtype, int64_t M, i
   if (!aligned(s1, 8) || !aligned(s2, 8) || !aligned(n, 8) || !aligned(amax, 4) || !aligned(flags, 4)) return fail(FS_ERR_INVALID_ARGUMENT, "fs_channel_stats: misaligned state");
   if (M == 0) return FS_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int vec = dtype == FS_DTYPE_BF16 ? kStatsVecBf16 : 4;
+  const bool bf16 = dtype == FS_DTYPE_BF16;
+  const int vec = bf16 ? kStatsVecBf16 : 4;
   const int chunks = static_cast<int>(ceil_div(K, 32 * vec));
   const int64_t taken = ceil_div(M, row_stride);
-  // Enough CTAs for ~4 per SM, each reading at least 64 rows.
-  int64_t gy = ceil_div(148 * 4, chunks);
+  // One wave: as many row groups per channel chunk as fill the resident CTA slots (a second,
+  // partial wave would run at a fraction of the occupancy), each reading at least 128 rows.
+  const void* kernel = bf16 ? reinterpret_cast<const void*>(channel_stats_kernel<uint16_t, kStatsVecBf16>)
+                            : reinterpret_cast<const void*>(channel_stats_kernel<float, 4>);
+  static int per_sm[2] = {0, 0};
+  int& slots = per_sm[bf16 ? 0 : 1];
+  if (slots == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&slots, kernel, kStatsWarps * 32, 0) != cudaSuccess ||
+                     slots < 1))
+    slots = 1;
+  int64_t gy = std::max<int64_t>(1, static_cast<int64_t>(slots) * sm_count() / chunks);
   gy = std::min<int64_t>(gy, std::max<int64_t>(1, ceil_div(taken, 128)));
   gy = std::min<int64_t>(gy, 65535);
   dim3 grid(chunks, static_cast<unsigned>(gy));
   auto* un = reinterpret_cast<unsigned long long*>(n);
   auto* u1 = reinterpret_cast<unsigned long long*>(s1);
   auto* u2 = reinterpret_cast<unsigned long long*>(s2);
-  if (dtype == FS_DTYPE_BF16)
+  if (bf16)
     channel_stats_kernel<uint16_t, kStatsVecBf16><<<grid, kStatsWarps * 32, 0, s>>>(static_cast<const uint16_t*>(X), M, K, ldx, row_stride, un, u1, u2, amax, flags);
   else
     channel_stats_kernel<float, 4><<<grid, kStatsWarps * 32, 0, s>>>(static_cast<const float*>(X), M, K, ldx, row_stride, un, u1, u2, amax, flags);

@@ -173,6 +173,27 @@ def test_prepare_weights_bit_exact(dtype, N, K, p, opts):
     check_packed(out, ref, N, K, p)
 
 
+@pytest.mark.parametrize("opts", [0, 1])
+def test_prepare_weights_gain_sees_every_element(opts):
+    """One planted large weight decides the gain, wherever it sits: first and last element, the
+    ragged last 64 columns (K = 576 is not a multiple of 256), a middle row; a larger one in a
+    protected column is ignored by the split form and counted by the residual form."""
+    N, K, p = 300, 576, 16
+    _, _, P, st = _prep_inputs(5, 64, K, p, "bf16")
+    gA = stats.next_gain(st, P, residual=bool(opts & 1))
+    mask = mask_tensor(stats.protect_mask(P, K))
+    unprot = [c for c in range(K) if c not in set(int(v) for v in P)]
+    spots = [(0, unprot[0], 0x40A0), (N - 1, unprot[-1], 0xC0F0), (N // 2, unprot[len(unprot) // 2], 0x4110),
+             (N - 1, unprot[200], 0x40E0)]
+    for r, c, bits in spots:
+        w = synth.gaussian_weights(11, N, K, as_bf16=True).copy()
+        w[r, c] = bits
+        w[N // 3, int(P[0])] = 0x42C8                      # 100.0 in a protected column
+        ref = splice.prepare_weights(splice.as_f32(w, True), P, gA, splice.RESIDUAL if opts & 1 else splice.SPLIT)
+        _, gW, alpha = F.fs_prepare_weights(bf16_tensor(w), mask, p, torch.tensor([float(gA)], device="cuda"), opts=opts)
+        assert gW.item() == float(ref["gW"]) and alpha.item() == float(ref["alpha"]), (r, c)
+
+
 # ----------------------------------------------------------------------------- filter
 def test_seq_filter_hand_built_cases():
     lt = seqfilter.log_tau(1e-4)
