@@ -49,9 +49,9 @@ DECODE_LAYERS = 36
 
 # DRAM traffic of the tensor-core SpliceGEMM over one step (M = 8192, P = 64): ncu
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch per shape of the current kernel, summed
-# over a step's launches (fused: qkv, o, gate_up, down; unfused: q, k, v, o, gate, up, down);
-# profiles/splice_gemm_tc_dram_m8192_p64.md.
-GEMM_DRAM_BYTES_PER_STEP = {"fused": 1365232640, "unfused": 1298154752}
+# over the step's launches (qkv, o, gate_up, down; profiles/splice_gemm_tc_dram_m8192_p64.md).  The
+# one-launch-per-projection form (--unfused) has no capture of the current kernel.
+GEMM_DRAM_BYTES_PER_STEP = {"fused": 1367799296, "unfused": None}
 
 
 def gemm_alg_bytes(p, fused=True):

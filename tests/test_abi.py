@@ -65,6 +65,11 @@ def test_host_validation_rejects_bad_arguments(lib):
     # weights: N == 0, missing alpha
     assert lib.fs_prepare_weights(dummy, 0, 0, 64, 64, None, 0, 0, dummy, dummy, dummy, None, dummy, dummy, None) == 1
     assert lib.fs_prepare_weights(dummy, 0, 4, 64, 64, None, 0, 0, dummy, dummy, dummy, None, dummy, None, None) == 1
+    # segmented GEMM: a plan is required before the segments are looked at
+    seg = (C.c_int32 * 3)(0, 128, 256)
+    assert lib.fs_splice_gemm_segmented(None, 8, 0, dummy, dummy, None, dummy, dummy, None, 2, seg, dummy, dummy, 256,
+                                        None) == 1
+    assert b"plan" in lib.fs_last_error()
     # filter: K1 < 1, rewards without G
     assert lib.fs_seq_filter(dummy, 64, None, 4, 64, -9.0, 0, 5, 0, None, None, dummy, dummy, dummy, None) == 1
     assert lib.fs_seq_filter(dummy, 64, None, 4, 64, -9.0, 3, 5, 3, dummy, dummy, dummy, dummy, dummy, None) == 1
