@@ -784,24 +784,60 @@ def main():
     fp4_peak = peaks["bf16_tflops"] * 4.0         # dense NVFP4 = 4x dense BF16 (nominal 9 vs 2.25 PFLOP/s)
     del phase_graphs, gemm_graphs
 
-    # end to end: host (pinned) activations in, all projection outputs back to host, every step
+    # End to end: every step copies its activations in from pinned host memory, runs the step
+    # through the library calls and copies all outputs back.  Two buffer sets alternate so that
+    # the host->device copy of step i+1, the step i itself and the device->host copy of step i-1
+    # run at once on three streams (the copies use the two DMA directions).
+    layer2 = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device, fused=not args.unfused)
+    sets = [layer, layer2]
     host_x = [x.cpu().pin_memory() for x in layer.X]
-    host_y = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in layer.Y]
+    host_y = [[torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in L.Y] for L in sets]
     h2d = sum(x.numel() * x.element_size() for x in host_x)
-    d2h = sum(y.numel() * y.element_size() for y in host_y)
+    d2h = sum(y.numel() * y.element_size() for y in host_y[0])
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in sets]
+    ev_run = [torch.cuda.Event() for _ in sets]
+    ev_out = [torch.cuda.Event() for _ in sets]
+    e2e_i = [0]
 
     def e2e_step():
-        for dx, hx in zip(layer.X, host_x):
-            dx.copy_(hx, non_blocking=True)
-        layer.step(allreduce)
-        for hy, dy in zip(host_y, layer.Y):
-            hy.copy_(dy, non_blocking=True)
+        i = e2e_i[0]
+        e2e_i[0] += 1
+        b = i % 2
+        L = sets[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_run[b])          # step i-2 has read this set's activations
+            for dx, hx in zip(L.X, host_x):
+                dx.copy_(hx, non_blocking=True)
+            ev_in[b].record()
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(ev_in[b])
+            if i >= 2:
+                s_run.wait_event(ev_out[b])         # step i-2's outputs have left this set
+            L.step(allreduce)
+            ev_run[b].record()
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_run[b])
+            for hy, dy in zip(host_y[b], L.Y):
+                hy.copy_(dy, non_blocking=True)
+            ev_out[b].record()
 
-    e2e_steps = max(3, min(args.steps, 5))
-    for _ in range(2):
-        e2e_step()
-    ms_e2e = timed(e2e_step, e2e_steps, dist if use_dist else None) / e2e_steps
+    def e2e_run(n):
+        main = torch.cuda.current_stream()
+        for s_ in (s_in, s_run, s_out):             # after the start event on the main stream ...
+            s_.wait_stream(main)
+        for _ in range(n):
+            e2e_step()
+        for s_ in (s_in, s_run, s_out):             # ... and before its end event
+            main.wait_stream(s_)
+
+    e2e_steps = max(3, min(args.steps, 6))
+    e2e_run(2)
+    ms_e2e = timed(lambda: e2e_run(e2e_steps), 1, dist if use_dist else None) / e2e_steps
     e2e_value = world * layer.flops / (ms_e2e * 1e-3) / 1e12
+    layer2.check()
+    del layer2, sets
 
     fkey = "fused" if layer.fused else "unfused"
     line = {
@@ -827,7 +863,8 @@ def main():
         "phase_us": phase_us,
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": ms_e2e},
+                "ms_per_step": ms_e2e,
+                "schedule": "two buffer sets; copy-in of step i+1, step i and copy-out of step i-1 on three streams"},
         "gpu_launches": layer.launches_per_step(args.serial) * args.steps,
         "graph": "each timed step is one CUDA-graph replay of the step's launches" +
                  ("" if args.serial else "; the 4 independent input-group chains run on 4 streams"),

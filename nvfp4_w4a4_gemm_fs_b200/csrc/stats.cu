@@ -262,7 +262,7 @@ select_topk_kernel(int K, long long* n_all, long long* s1_all, long long* s2_all
   extern __shared__ unsigned long long sh_keys[];         // [K]
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long sh_prefix;
-  __shared__ int sh_need;
+  __shared__ int sh_need, sh_binc, sh_ties;
   __shared__ int sh_scan[kSelThreads / 32];
   __shared__ uint32_t sh_amax[kSelThreads / 32];
 
@@ -283,7 +283,9 @@ select_topk_kernel(int K, long long* n_all, long long* s1_all, long long* s2_all
 
   // Radix select of the p-th largest ordered key, 8 bits at a time from the top.  Histogram
   // updates are aggregated per warp (lanes with the same digit add once), and warp 0 finds the
-  // threshold digit with a suffix scan over 8 bins per lane.
+  // threshold digit with a suffix scan over 8 bins per lane.  Once the bin holding the p-th key
+  // is taken whole (its count equals the keys still needed), every key at or above the bin's
+  // prefix is selected: the passes stop with T = that prefix and `need` = the keys equal to it.
   unsigned long long prefix = 0;
   int need = p;
   const int lane = tid & 31, warp_id = tid >> 5;
@@ -315,18 +317,29 @@ select_topk_kernel(int K, long long* n_all, long long* s1_all, long long* s2_all
         }
         const int above = incl - local;
         if (above < need && need <= incl) {
-          int r = need - above, d = 8 * lane;
+          int r = need - above, d = 8 * lane, bc = 0;
+#pragma unroll
           for (int i = 7; i >= 0; --i) {
-            if (c[i] >= r) { d = 8 * lane + i; break; }
+            if (c[i] >= r) { d = 8 * lane + i; bc = c[i]; break; }
             r -= c[i];
           }
           sh_prefix = prefix | (static_cast<unsigned long long>(d) << shift);
           sh_need = r;
+          sh_binc = bc;
         }
       }
+      if (tid == 0) sh_ties = 0;
       __syncthreads();
       prefix = sh_prefix;
       need = sh_need;
+      if (shift > 0 && sh_binc == need) {          // uniform: the whole bin is selected
+        int eq = 0;
+        for (int j = tid; j < K; j += blockDim.x) eq += sh_keys[j] == prefix;
+        if (eq) atomicAdd(&sh_ties, eq);
+        __syncthreads();
+        need = sh_ties;
+        break;
+      }
       __syncthreads();
     }
   }
