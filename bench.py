@@ -8,7 +8,8 @@ one pass of the per-step path over one layer:
   fs_select_topk     top-64 reselection (batched per K)
   fs_prepare_weights pre-split of the 7 projections with the new protected set
   fs_quantize_splice the 4 activation groups
-  fs_splice_gemm     q, k, v, o, gate, up, down
+  fs_splice_gemm_segmented  one launch per input group: q|k|v, o, gate|up, down
+                     (--unfused: fs_splice_gemm per projection)
 
 `value` is the whole-step throughput in TFLOP/s, counting 2*M*N*K per projection (the same
 numerator for every P).  Inputs (activations and bf16 weights, about 0.85 GB) are larger than the
@@ -16,6 +17,7 @@ numerator for every P).  Inputs (activations and bf16 weights, about 0.85 GB) ar
 {1,4,16}, 36 distinct layers per CUDA-graph replay) in GB/s and the overhead against P = 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extras]
+                  [--case step|gemm|decode|prep|moe] [--shape ...] [--unfused]
 
 Under torchrun each rank runs its own batch (weak scaling); the only exchange is an all-reduce of
 the integer channel statistics before reselection, so every rank selects the same channels.
