@@ -88,6 +88,54 @@ __device__ __forceinline__ void add_bf16_in_range(uint32_t& a1, uint32_t& b1, ui
   d2 += __float_as_uint(__fmaf_rn(yl, 16384.0f, kMagic));
 }
 
+// Two elements of one channel at once with the packed fp32 instructions of sm_100a: each lane of
+// add/sub/mul/fma.rn.f32x2 is the IEEE single-precision RN operation of add_bf16_in_range, in the
+// same order, so the raw-bit terms are identical; the two lanes' bits are summed with one 3-input
+// add per term.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t lanes_sum(uint64_t v) {
+  return static_cast<uint32_t>(v) + static_cast<uint32_t>(v >> 32);
+}
+__device__ __forceinline__ void add_bf16_pair_in_range(uint32_t& a1, uint32_t& b1, uint32_t& c2, uint32_t& d2,
+                                                       float x0, float x1) {
+  constexpr uint64_t kM2 = (static_cast<uint64_t>(kMagicBits) << 32) | kMagicBits;
+  constexpr uint64_t kM8x2 = (static_cast<uint64_t>(kMagic8Bits) << 32) | kMagic8Bits;
+  constexpr uint64_t k2p16 = 0x4780000047800000ull;    // 65536.0f in both lanes
+  constexpr uint64_t k2p14 = 0x4680000046800000ull;    // 16384.0f in both lanes
+  const uint64_t X = pack_f32x2(x0, x1);
+  const uint64_t T1 = add_f32x2(X, kM2);
+  a1 += lanes_sum(T1);
+  const uint64_t F = sub_f32x2(X, sub_f32x2(T1, kM2));
+  b1 += lanes_sum(fma_f32x2(F, k2p16, kM2));
+  const uint64_t Y = mul_f32x2(X, X);
+  const uint64_t U = add_f32x2(Y, kM8x2);
+  c2 += lanes_sum(U);
+  const uint64_t YL = sub_f32x2(Y, sub_f32x2(U, kM8x2));
+  d2 += lanes_sum(fma_f32x2(YL, k2p14, kM2));
+}
+
 // fp32 inputs (small problems): convert directly.
 __device__ __forceinline__ void add_f32(long long& s1, long long& s2, float& amax, float x, bool& bad) {
   const float ax = fabsf(x);
@@ -180,20 +228,28 @@ channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int
         // removed with the row count.  A batch of kUnroll rows of a channel whose NaN-propagating
         // maximum is in range takes the select-free path; otherwise (rare) each element is
         // checked, out-of-range ones add the zero pattern and raise the flag.
+        // The batch maximum of |x| per channel comes from the bf16 bits: the low 15 bits order
+        // like |x| (NaN above infinity), and |x| < 2^15 exactly when they are below 0x4700.
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
+          uint32_t m2 = 0;                         // both channels of the word, packed
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) {
+            const uint32_t w = (&q[u].x)[v >> 1] & 0x7FFF7FFFu;
+            asm("max.u16x2 %0, %1, %2;" : "=r"(m2) : "r"(m2), "r"(w));
+          }
           float xs[kUnroll];
-          float mx = 0.0f;
 #pragma unroll
           for (int u = 0; u < kUnroll; ++u) {
             const uint32_t w = (&q[u].x)[v >> 1];
             xs[u] = (v & 1) ? bf16_hi(w) : bf16_lo(w);
-            mx = fmax_nan(mx, fabsf(xs[u]));
           }
-          if (mx < kRangeLimit) {
+          const uint32_t mag = (v & 1) ? (m2 >> 16) : (m2 & 0xFFFFu);
+          if (mag < 0x4700u) {
+            static_assert(kUnroll % 2 == 0, "rows are taken in pairs");
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) add_bf16_in_range(ra1[v], rb1[v], rc2[v], rd2[v], xs[u]);
-            am[v] = fmaxf(am[v], mx);
+            for (int u = 0; u < kUnroll; u += 2) add_bf16_pair_in_range(ra1[v], rb1[v], rc2[v], rd2[v], xs[u], xs[u + 1]);
+            am[v] = fmaxf(am[v], __uint_as_float(mag << 16));
           } else {
             SmallSums a{ra1[v], rb1[v], rc2[v], rd2[v], am[v]};
 #pragma unroll

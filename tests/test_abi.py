@@ -33,6 +33,26 @@ def test_every_declared_symbol_is_exported(lib):
         assert n in _lib.SIGNATURES, f"binding lacks {n}"
 
 
+def _declared_arity():
+    """Parameter count of every function the header declares (FS_API prototypes)."""
+    src = open(os.path.join(ROOT, "include", "foursight.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    out = {}
+    for name, params in re.findall(r"\b(fs_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src, flags=re.S):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    from nvfp4_w4a4_gemm_fs_b200 import _lib
+    arity = _declared_arity()
+    assert len(arity) >= 15
+    for name, n in arity.items():
+        assert len(_lib.SIGNATURES[name][1]) == n, f"{name}: header {n} parameters, binding {len(_lib.SIGNATURES[name][1])}"
+
+
 def test_status_strings_and_sizes(lib):
     assert lib.fs_status_string(0) == b"FS_OK"
     assert lib.fs_status_string(5) == b"FS_ERR_TIMEOUT"
