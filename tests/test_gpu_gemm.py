@@ -169,6 +169,38 @@ def test_segmented_projections_match_each_projection(path, M):
             F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, bad)
 
 
+@pytest.mark.parametrize("seg_rows", [[4096, 1024, 1024], [12288, 12288]])
+def test_full_size_segmented_sampled_rows(seg_rows):
+    """The launches bench.py times: M = 8192 tokens, K = 4096, the q/k/v (or gate/up) weights
+    stacked in one segmented launch; the oracle checks 40 sampled rows of every projection."""
+    M, K, p = 8192, 4096, 64
+    x, _ = synth.outlier_activations(211, M, K)
+    X = splice.as_f32(x, True)
+    st = stats.accumulate(stats.new_state(K), X)
+    P = stats.select_topk(st, p)
+    gA = stats.next_gain(st, P)
+    mask = mask_tensor(stats.protect_mask(P, K))
+    g = torch.tensor([float(gA)], device="cuda")
+    xq = F.fs_quantize_splice(bf16_tensor(x), mask, p, g)
+    wq_all, views = F.stacked_packed(seg_rows, K, p)
+    alphas = torch.empty(len(seg_rows), device="cuda")
+    Ws = []
+    for j, (n, view) in enumerate(zip(seg_rows, views)):
+        w = synth.gaussian_weights(400 + j, n, K)
+        Ws.append(splice.as_f32(w, True))
+        F.fs_prepare_weights(bf16_tensor(w), mask, p, g, out=view, alpha=alphas[j:j + 1])
+    seg = np.concatenate([[0], np.cumsum(seg_rows)]).tolist()
+    plan = F.Plan(seg[-1], K, p)
+    Y = F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, seg)
+    plan.check()
+    rows = np.sort(np.random.default_rng(seg[-1]).choice(M, 40, replace=False))
+    rows[0], rows[-1] = 0, M - 1
+    rows_t = torch.from_numpy(rows).cuda()
+    for j in range(len(seg_rows)):
+        Yr, mag = _ref(X, Ws[j], P, gA, rows=rows)
+        _assert_close(Y[rows_t, seg[j]:seg[j + 1]], Yr, mag)
+
+
 def test_repeatable_and_overwrites_output():
     X, W, Xt, Wt, P, gA = _problem(92, 256, 512, 1024, 64)
     Y1, _ = _run_gpu(Xt, Wt, P, gA, 64, 512, 1024)
