@@ -169,11 +169,12 @@ def test_segmented_projections_match_each_projection(path, M):
             F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, bad)
 
 
-@pytest.mark.parametrize("seg_rows", [[4096, 1024, 1024], [12288, 12288]])
-def test_full_size_segmented_sampled_rows(seg_rows):
-    """The launches bench.py times: M = 8192 tokens, K = 4096, the q/k/v (or gate/up) weights
-    stacked in one segmented launch; the oracle checks 40 sampled rows of every projection."""
-    M, K, p = 8192, 4096, 64
+@pytest.mark.parametrize("M,seg_rows", [(8192, [4096, 1024, 1024]), (8192, [12288, 12288]), (16, [4096, 1024, 1024])])
+def test_full_size_segmented_sampled_rows(M, seg_rows):
+    """The launches bench.py times: M = 8192 tokens (tensor-core path) or 16 (decode path), K =
+    4096, the q/k/v (or gate/up) weights stacked in one segmented launch; the oracle checks 40
+    sampled rows (all rows at M = 16) of every projection."""
+    K, p = 4096, 64
     x, _ = synth.outlier_activations(211, M, K)
     X = splice.as_f32(x, True)
     st = stats.accumulate(stats.new_state(K), X)
@@ -193,8 +194,11 @@ def test_full_size_segmented_sampled_rows(seg_rows):
     plan = F.Plan(seg[-1], K, p)
     Y = F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, seg)
     plan.check()
-    rows = np.sort(np.random.default_rng(seg[-1]).choice(M, 40, replace=False))
-    rows[0], rows[-1] = 0, M - 1
+    if M <= 40:
+        rows = np.arange(M)
+    else:
+        rows = np.sort(np.random.default_rng(seg[-1]).choice(M, 40, replace=False))
+        rows[0], rows[-1] = 0, M - 1
     rows_t = torch.from_numpy(rows).cuda()
     for j in range(len(seg_rows)):
         Yr, mag = _ref(X, Ws[j], P, gA, rows=rows)
