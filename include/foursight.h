@@ -208,7 +208,9 @@ fs_status fs_plan_check(fs_plan plan, void* stream);
  * thread-block cluster), larger M the tcgen05 prefill kernel (FS_PATH_TENSOR / FS_PATH_DECODE in
  * the plan's opts force one).
  * Plan requirements: N % 16 == 0 and K % 256 == 0 (FS_ERR_UNSUPPORTED otherwise); the packed
- * operands must be 16-byte aligned.  The output is not accumulated into: Y is overwritten. */
+ * operands must be 16-byte aligned.  The output is not accumulated into: Y is overwritten.
+ * M = 0 (an empty batch) returns FS_OK without reading any operand pointer (the plan must still
+ * be valid); the same holds for the segmented, grouped (max_rows = 0) and allocation-free calls. */
 fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq, const uint8_t* sfx,
                          const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
                          const float* alpha, void* Y, int64_t ldy, void* stream);

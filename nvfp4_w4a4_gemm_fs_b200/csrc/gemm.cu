@@ -83,9 +83,10 @@ fs_status splice_gemm(const char* who, fs_plan plan, int64_t M, int32_t p, const
                       const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
                       const Segments& seg, const float* alpha, void* Y, int64_t ldy, void* stream) {
   if (M < 0) return fail(FS_ERR_INVALID_ARGUMENT, "%s: M < 0", who);
+  if (!plan) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null plan", who);
+  if (M == 0) return FS_OK;                        // an empty batch reads no operand
   fs_status st = check_operands(who, plan, p, xq, sfx, xs, wq, sfw, ws, alpha, Y, ldy);
   if (st != FS_OK) return st;
-  if (M == 0) return FS_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int pp = side_cols(p);
   const bool decode = (plan->opts & FS_PATH_DECODE) || (!(plan->opts & FS_PATH_TENSOR) && M <= 16);
@@ -158,10 +159,11 @@ extern "C" fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64
                                             const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
                                             const float* alpha, void* Y, int64_t ldy, void* stream) {
   if (E <= 0 || !row_offsets || max_rows < 0) return fail(FS_ERR_INVALID_ARGUMENT, "fs_splice_gemm_grouped: need E > 0, row_offsets, max_rows >= 0");
+  if (!plan) return fail(FS_ERR_INVALID_ARGUMENT, "fs_splice_gemm_grouped: null plan");
+  if (max_rows == 0) return FS_OK;                 // no routed rows: nothing is read or written
   fs_status st = check_operands("fs_splice_gemm_grouped", plan, p, xq, sfx, xs, wq, sfw, ws, alpha, Y, ldy);
   if (st != FS_OK) return st;
   if (plan->N % 128 != 0) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm_grouped: need N %% 128 == 0");
-  if (max_rows == 0) return FS_OK;
   const int64_t a_rows = fs_grouped_rows(max_rows, E);
   if (a_rows > (int64_t{1} << 31) - 256) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm_grouped: too many rows");
   const int pp = side_cols(p);

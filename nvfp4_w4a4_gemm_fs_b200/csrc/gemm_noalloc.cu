@@ -64,6 +64,7 @@ extern "C" fs_status fs_splice_gemm_noalloc(int32_t N, int32_t K, uint32_t opts,
   if (p < 0 || p > 256 || p > K) return fail(FS_ERR_INVALID_ARGUMENT, "%s: need 0 <= p <= min(K, 256)", who);
   if ((opts & (FS_PATH_TENSOR | FS_PATH_DECODE)) == (FS_PATH_TENSOR | FS_PATH_DECODE))
     return fail(FS_ERR_INVALID_ARGUMENT, "%s: FS_PATH_TENSOR and FS_PATH_DECODE are exclusive", who);
+  if (M == 0) return FS_OK;                        // an empty batch reads no operand
   if (!xq || !sfx || !wq || !sfw || !alpha || !Y || (p > 0 && (!xs || !ws)))
     return fail(FS_ERR_INVALID_ARGUMENT, "%s: null pointer", who);
   if (!aligned(xq, 16) || !aligned(sfx, 16) || !aligned(wq, 16) || !aligned(sfw, 16) ||
@@ -74,7 +75,6 @@ extern "C" fs_status fs_splice_gemm_noalloc(int32_t N, int32_t K, uint32_t opts,
     return fail(FS_ERR_INVALID_ARGUMENT, "%s: Y must be 16-byte aligned with ldy >= N and 16-byte rows", who);
   // The kernels need exactly kNoAllocScratchWords words of scratch; no problem size needs more.
   static_assert(kNoAllocScratchWords >= 1, "one error word");
-  if (M == 0) return FS_OK;
 
   uint32_t* scratch = nullptr;
   fs_status st = scratch_for_current_device(&scratch);

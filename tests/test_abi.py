@@ -85,6 +85,10 @@ def test_host_validation_rejects_bad_arguments(lib):
     # weights: N == 0, missing alpha
     assert lib.fs_prepare_weights(dummy, 0, 0, 64, 64, None, 0, 0, dummy, dummy, dummy, None, dummy, dummy, None) == 1
     assert lib.fs_prepare_weights(dummy, 0, 4, 64, 64, None, 0, 0, dummy, dummy, dummy, None, dummy, None, None) == 1
+    # an empty batch is a no-op that reads no operand (allocation-free entry: no plan needed)
+    assert lib.fs_splice_gemm_noalloc(256, 512, 0, 0, 64, None, None, None, None, None, None, None, None, 256, 0,
+                                      None) == 0
+    assert lib.fs_splice_gemm(None, 0, 0, None, None, None, None, None, None, None, None, 256, None) == 1   # null plan
     # segmented GEMM: a plan is required before the segments are looked at
     seg = (C.c_int32 * 3)(0, 128, 256)
     assert lib.fs_splice_gemm_segmented(None, 8, 0, dummy, dummy, None, dummy, dummy, None, 2, seg, dummy, dummy, 256,

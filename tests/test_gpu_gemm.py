@@ -205,6 +205,28 @@ def test_full_size_segmented_sampled_rows(M, seg_rows):
         _assert_close(Y[rows_t, seg[j]:seg[j + 1]], Yr, mag)
 
 
+def test_empty_batches_are_no_ops():
+    """M = 0 tokens (and a grouped call with no routed rows): every call succeeds, reads nothing and
+    returns an empty output; the statistics state is untouched."""
+    K, N, p = 512, 512, 64
+    X, W, Xt, Wt, P, gA = _problem(5, 8, N, K, p)
+    mask = mask_tensor(stats.protect_mask(P, K))
+    g = torch.tensor([float(gA)], device="cuda")
+    wq, _, alpha = F.fs_prepare_weights(Wt, mask, p, g)
+    empty = torch.empty(0, K, dtype=torch.bfloat16, device="cuda")
+    st = F.StatsState(1, K)
+    F.fs_channel_stats(empty, st)
+    assert int(st.n.item()) == 0 and not st.s1.any() and not st.s2.any()
+    xq = F.fs_quantize_splice(empty, mask, p, g)
+    assert xq.rows == 0
+    plan = F.Plan(N, K, p)
+    assert F.fs_splice_gemm(plan, xq, wq, alpha).shape == (0, N)
+    assert F.fs_splice_gemm_segmented(plan, xq, wq, alpha.repeat(2), [0, 256, N]).shape == (0, N)
+    offs = torch.zeros(3, dtype=torch.int64, device="cuda")
+    assert F.fs_splice_gemm_grouped(plan, offs, 0, xq, wq, alpha.repeat(2)).shape == (0, N)
+    plan.check()
+
+
 def test_repeatable_and_overwrites_output():
     X, W, Xt, Wt, P, gA = _problem(92, 256, 512, 1024, 64)
     Y1, _ = _run_gpu(Xt, Wt, P, gA, 64, 512, 1024)
