@@ -68,30 +68,10 @@ __device__ __forceinline__ void add_bf16(SmallSums& a, float x, bool& bad) {
   a.d2 += __float_as_uint(__fmaf_rn(yl, 16384.0f, kMagic));
 }
 
-// NaN-propagating maximum (a NaN operand makes the result NaN).
-__device__ __forceinline__ float fmax_nan(float a, float b) {
-  float r;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
-  return r;
-}
-
-// The same raw-bit terms as add_bf16 for an element known to be finite and in range.
-__device__ __forceinline__ void add_bf16_in_range(uint32_t& a1, uint32_t& b1, uint32_t& c2, uint32_t& d2, float x) {
-  const float t1 = __fadd_rn(x, kMagic);
-  a1 += __float_as_uint(t1);
-  const float frac = __fsub_rn(x, __fsub_rn(t1, kMagic));
-  b1 += __float_as_uint(__fmaf_rn(frac, 65536.0f, kMagic));
-  const float y = __fmul_rn(x, x);
-  const float u = __fadd_rn(y, kMagic8);
-  c2 += __float_as_uint(u);
-  const float yl = __fsub_rn(y, __fsub_rn(u, kMagic8));
-  d2 += __float_as_uint(__fmaf_rn(yl, 16384.0f, kMagic));
-}
-
 // Two elements of one channel at once with the packed fp32 instructions of sm_100a: each lane of
-// add/sub/mul/fma.rn.f32x2 is the IEEE single-precision RN operation of add_bf16_in_range, in the
-// same order, so the raw-bit terms are identical; the two lanes' bits are summed with one 3-input
-// add per term.
+// add/sub/mul/fma.rn.f32x2 is the IEEE single-precision RN operation add_bf16 performs on an
+// in-range element, in the same order, so the raw-bit terms are identical; the two lanes' bits are
+// summed with one 3-input add per term.
 __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
 }
@@ -225,11 +205,11 @@ channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int
         }
       } else {
         // Zero rows past the end contribute rint(0) = 0: their raw bits are the magic patterns,
-        // removed with the row count.  A batch of kUnroll rows of a channel whose NaN-propagating
-        // maximum is in range takes the select-free path; otherwise (rare) each element is
+        // removed with the row count.  The batch maximum of |x| per channel comes from the bf16
+        // bits: the low 15 bits order like |x| (infinity and NaN above every finite value), and
+        // |x| < 2^15 exactly when they are below 0x4700.  A batch of kUnroll rows of a channel
+        // whose maximum is in range takes the select-free path; otherwise (rare) each element is
         // checked, out-of-range ones add the zero pattern and raise the flag.
-        // The batch maximum of |x| per channel comes from the bf16 bits: the low 15 bits order
-        // like |x| (NaN above infinity), and |x| < 2^15 exactly when they are below 0x4700.
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
           uint32_t m2 = 0;                         // both channels of the word, packed
