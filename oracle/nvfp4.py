@@ -19,7 +19,8 @@ Readings taken where the paper is silent:
 * the sign of zero is kept (-0 encodes as 0x8); a zero block scale gives every
   element the code 0 with its own sign; masked lanes are +0 (code 0x0);
 * the gain: largest power of two g with ``amax*g <= 6*448``, or fl32(2688/amax)
-  under the exact-gain option; amax = 0 gives g = 1.
+  (saturated to the largest finite float32) under the exact-gain option; amax = 0
+  gives g = 1.
 """
 from __future__ import annotations
 
@@ -115,12 +116,22 @@ def gain_pow2(amax: float) -> np.float32:
     return np.float32(2.0 ** E)
 
 
+FLOAT32_MAX = np.float32(np.finfo(np.float32).max)
+
+
 def gain_exact(amax: float) -> np.float32:
-    """fl32(2688 / amax); 1 if amax == 0 (the common NVFP4 tensor-scale recipe)."""
+    """fl32(2688 / amax), saturated to the largest finite float32; 1 if amax == 0 or not finite.
+
+    The common NVFP4 tensor-scale recipe.  The gain must be a finite FP32 value: for amax below
+    2688 / FLT_MAX (every subnormal amax) the IEEE quotient overflows, and the gain saturates, as
+    the power-of-two rule clamps its exponent at 127.
+    """
     a = np.float32(amax)
     if a == 0 or not np.isfinite(a):
         return np.float32(1.0)
-    return np.float32(np.float32(GAIN_TARGET) / a)
+    with np.errstate(over="ignore"):
+        q = np.float32(np.float32(GAIN_TARGET) / a)
+    return np.float32(min(q, FLOAT32_MAX))
 
 
 def alpha_from_gains(gA, gW) -> np.float32:

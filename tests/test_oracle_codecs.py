@@ -133,3 +133,49 @@ def test_gain_pow2_is_the_largest_fitting_power(amax):
     assert Fraction(a) * Fraction(g) <= 2688
     assert Fraction(a) * Fraction(2 * g) > 2688
     assert nvfp4.gain_pow2(0.0) == 1.0
+
+
+def _fl32(q: Fraction) -> float:
+    """The binary32 value nearest to the positive rational q (ties to even), or inf past the
+    largest finite one: written from the format's definition (24-bit significands, minimum normal
+    exponent -126, subnormal spacing 2^-149), independent of numpy's division."""
+    e = q.numerator.bit_length() - q.denominator.bit_length()    # 2^e <= q < 2^(e+2)
+    while Fraction(2) ** e > q:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= q:
+        e += 1
+    unit = Fraction(2) ** (max(e, -126) - 23)
+    n, r = divmod(q, unit)
+    n = int(n)
+    if r > unit / 2 or (r == unit / 2 and n % 2 == 1):
+        n += 1
+    v = n * unit
+    return float("inf") if v >= Fraction(2) ** 128 else float(v)
+
+
+@pytest.mark.parametrize("amax", [1.0, 3.0, 7.0, 2688.0, 0.1, 1e-3, 123.456, 5e4, 1e30, 6.0 * 448 / 1024,
+                                  8e-36, 7.9e-36])
+def test_gain_exact_is_the_correctly_rounded_quotient(amax):
+    """gain_exact(a) is 2688/a rounded once to binary32 (the exact rational quotient, rounded by
+    the format's definition), and lies within half an ulp of it."""
+    a = float(np.float32(amax))
+    g = float(nvfp4.gain_exact(a))
+    ref = _fl32(Fraction(2688) / Fraction(a))
+    assert ref != float("inf")
+    assert g == ref
+    ulp = float(np.spacing(np.float32(g)))
+    assert abs(Fraction(a) * Fraction(g) - 2688) <= Fraction(a) * Fraction(ulp) / 2
+
+
+def test_gain_exact_degenerate_inputs():
+    """amax = 0 and non-finite amax give g = 1; an amax whose quotient overflows (every subnormal,
+    and normals below 2688 / FLT_MAX) saturates to the largest finite float32."""
+    fmax = float(np.finfo(np.float32).max)
+    assert nvfp4.gain_exact(0.0) == 1.0 and nvfp4.gain_exact(float("inf")) == 1.0 and nvfp4.gain_exact(float("nan")) == 1.0
+    for a in (float(np.float32(1e-40)), float(np.float32(2.0 ** -149)), float(np.float32(2.0 ** -126)),
+              float(np.float32(7.8e-36))):
+        assert _fl32(Fraction(2688) / Fraction(a)) == float("inf")
+        assert float(nvfp4.gain_exact(a)) == fmax
+    # the smallest amax with a finite quotient is not clamped
+    a = float(np.nextafter(np.float32(2688.0 / fmax), np.float32(1)))
+    assert float(nvfp4.gain_exact(a)) == _fl32(Fraction(2688) / Fraction(a)) <= fmax
