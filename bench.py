@@ -51,8 +51,8 @@ DECODE_LAYERS = 36
 
 # DRAM traffic of the tensor-core SpliceGEMM over one step (M = 8192, P = 64): ncu
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch per shape of the current kernel, summed
-# over the step's launches (qkv, o, gate_up, down; profiles/splice_gemm_tc_dram_m8192_p64.md).  The
-# one-launch-per-projection form (--unfused) has no capture of the current kernel.
+# over the step's launches (qkv, o, gate_up, down).  None where no capture of the current kernel
+# exists (the one-launch-per-projection form, --unfused).
 GEMM_DRAM_BYTES_PER_STEP = {"fused": 1367799296, "unfused": None}
 
 
@@ -316,16 +316,10 @@ def capture(fn):
 
 
 def stats_allreduce_fn(dist):
-    """The DP exchange: sum the integer moments and counts, max the per-channel maxima."""
-    import torch
-
-    def f(st):
-        dist.all_reduce(st.s1, op=dist.ReduceOp.SUM)
-        dist.all_reduce(st.s2, op=dist.ReduceOp.SUM)
-        dist.all_reduce(st.n, op=dist.ReduceOp.SUM)
-        dist.all_reduce(st.amax, op=dist.ReduceOp.MAX)      # non-negative float bits order as ints
-        dist.all_reduce(st.flags, op=dist.ReduceOp.MAX)
-    return f
+    """The DP exchange: sum the integer moments and counts, max the per-channel maxima
+    (nvfp4_w4a4_gemm_fs_b200.dp.allreduce_stats)."""
+    from nvfp4_w4a4_gemm_fs_b200 import dp
+    return dp.allreduce_stats
 
 
 def timed(fn, steps, dist=None):
@@ -539,12 +533,50 @@ def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20, fus
             abytes = sum(M * (K // 2 + K // 16 + F.side_cols(p) * 2) + M * N * 4 for (_, N, K, _) in PROJ)
             total = layers * (wbytes + abytes + xbytes)
             out[tag] = {"us_per_layer": 1000.0 * ms / layers, "GBps": total / (ms * 1e-3) / 1e9,
-                        "bytes_per_layer": wbytes + abytes + xbytes, "launches_per_layer": len(units)}
+                        "bytes_per_layer": wbytes + abytes + xbytes,
+                        "launches_per_layer": len(units) + (len(GROUP_K) if wq_flag else 0)}
             del graph
         for pl in plans:
             pl.check()
         res[f"M{M}"] = out
     return res, wbytes
+
+
+def side_slice_bound(p):
+    """Lower bound of the GEMM time added by p protected channels: the BF16 slice's 2*M*N*Pp flops
+    at a quarter of the NVFP4 rate, against the step's 2*M*N*K NVFP4 flops (4*Pp/K per projection,
+    weighted by N*K over the layer)."""
+    pp = (p + 15) // 16 * 16
+    return sum(4.0 * N * pp for _, N, K, _ in PROJ) / sum(float(N) * K for _, N, K, _ in PROJ)
+
+
+def p_variant(F, p, device, streams, args, rank):
+    """The timed step and its GEMMs at another protected-channel count p: step time (one graph
+    replay, captured as the main step) and the sum of the GEMM launches' times."""
+    import torch
+    lay = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device, fused=not args.unfused)
+    for _ in range(3):
+        lay.step()
+    gs = capture(lay.step if args.serial else (lambda: lay.step_streams(streams)))
+    for _ in range(3):
+        gs.replay()
+    ms = timed(gs.replay, args.steps) / args.steps
+    gg = [capture(fn) for fn in lay.gemm_fns()]
+    for g_ in gg:
+        g_.replay()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(args.steps):
+        for g_ in gg:
+            g_.replay()
+    ev[1].record()
+    torch.cuda.synchronize()
+    gms = ev[0].elapsed_time(ev[1]) / args.steps
+    lay.check()
+    out = {"step_ms": ms, "gemm_ms": gms, "gemm_tflops": lay.flops / (gms * 1e-3) / 1e12,
+           "step_tflops": lay.flops / (ms * 1e-3) / 1e12}
+    del gs, gg, lay
+    return out
 
 
 # ------------------------------------------------------------------------------------------
@@ -635,10 +667,27 @@ def prep_case(F, args, device):
         F.fs_select_topk(st, args.p, reset=True, P=P, mask=mask, gA=g)
         F.fs_prepare_weights(W, mask[0], args.p, g, out=wq, gW=gW, alpha=alpha)
         F.fs_quantize_splice(X, mask[0], args.p, g, out=xq)
-    for _ in range(args.warmup):
-        run()
-    ms = timed(run, args.steps) / args.steps
-    print(json.dumps({"case": "prep", "us_per_pass": ms * 1000.0}))
+
+    def run_fused():
+        F.fs_select_topk(st, args.p, reset=True, P=P, mask=mask, gA=g)
+        F.fs_prepare_weights(W, mask[0], args.p, g, out=wq, gW=gW, alpha=alpha)
+        F.fs_quantize_splice_stats(X, mask[0], args.p, g, st, out=xq)
+    res = {"case": "prep"}
+    for name, fn in (("separate", run), ("fused", run_fused)):
+        for _ in range(args.warmup):
+            fn()
+        res[name + "_us_per_pass"] = timed(fn, args.steps) / args.steps * 1000.0
+    # the statistics + quantise part alone, each form as one graph replay
+    parts = {"stats+quantize": lambda: (F.fs_channel_stats(X, st), F.fs_quantize_splice(X, mask[0], args.p, g, out=xq)),
+             "quantize_stats_fused": lambda: F.fs_quantize_splice_stats(X, mask[0], args.p, g, st, out=xq)}
+    for name, fn in parts.items():
+        gr = capture(fn)
+        for _ in range(3):
+            gr.replay()
+        us = timed(gr.replay, args.steps) / args.steps * 1000.0
+        res[name + "_us"] = us
+        res[name + "_GBps"] = (X.numel() * 2 + X.shape[0] * (X.shape[1] // 2 + X.shape[1] // 16)) / (us * 1e-6) / 1e9
+    print(json.dumps(res))
 
 
 def kernel_case(F, args, device):
@@ -854,8 +903,8 @@ def main():
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_STEP[fkey],
                      "traffic_unit": f"DRAM bytes per step (the {len(gemm_names)} GEMM launches; ncu "
-                                     "dram__bytes_read.sum + dram__bytes_write.sum per shape, "
-                                     "profiles/splice_gemm_tc_dram_m8192_p64.md)",
+                                     "dram__bytes_read.sum + dram__bytes_write.sum per shape of the "
+                                     "current kernel)",
                      "algorithmic_bytes": gemm_alg_bytes(p, layer.fused),
                      "kernel": f"splice_gemm_tc_kernel ({len(gemm_names)} launches: {', '.join(gemm_names)}; "
                                "sum 2MNK / sum of CUDA-event times)",
@@ -873,33 +922,26 @@ def main():
     }
 
     if not args.no_extras and rank == 0:
-        # overhead against P = 0: the same step and the GEMMs alone
+        # the protected-channel budget: the same step and its GEMMs at P = 0 (the overhead
+        # reference) and at P = 256 (FourSight §6.4's larger budget), each captured like the timed step
         del host_x, host_y
         torch.cuda.empty_cache()
-        l0 = PrefillLayer(F, M_PREFILL, 0, seed=2 + rank, device=device, fused=not args.unfused)
-        for _ in range(3):
-            l0.step()
-        # the P = 0 step is captured the same way as the timed step (4 streams unless --serial)
-        g0s = capture(l0.step if args.serial else (lambda: l0.step_streams(streams)))
-        for _ in range(3):
-            g0s.replay()
-        ms0 = timed(g0s.replay, args.steps) / args.steps
-        gg0 = [capture(fn) for fn in l0.gemm_fns()]
-        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        ev0[0].record()
-        for _ in range(args.steps):
-            for g_ in gg0:
-                g_.replay()
-        ev0[1].record()
-        torch.cuda.synchronize()
-        g0 = ev0[0].elapsed_time(ev0[1]) / args.steps
-        l0.check()
-        line["overhead_vs_p0"] = {"step_ms_p0": ms0, "step_ms_p": ms_step, "step_overhead": ms_step / ms0 - 1.0,
-                                  "gemm_ms_p0": g0, "gemm_ms_p": gemm_total_ms, "gemm_overhead": gemm_total_ms / g0 - 1.0,
-                                  "gemm_tflops_p0": l0.flops / (g0 * 1e-3) / 1e12}
-        del g0s, gg0
-        del l0
-        torch.cuda.empty_cache()
+        sweep = {}
+        for pv in sorted({0, 256} - {p}):
+            sweep[pv] = p_variant(F, pv, device, streams, args, rank)
+            torch.cuda.empty_cache()
+        sweep[p] = {"step_ms": ms_step, "gemm_ms": gemm_total_ms, "gemm_tflops": gemm_tflops,
+                    "step_tflops": value / world}
+        s0 = sweep[0]
+        line["overhead_vs_p0"] = {"step_ms_p0": s0["step_ms"], "step_ms_p": ms_step,
+                                  "step_overhead": ms_step / s0["step_ms"] - 1.0,
+                                  "gemm_ms_p0": s0["gemm_ms"], "gemm_ms_p": gemm_total_ms,
+                                  "gemm_overhead": gemm_total_ms / s0["gemm_ms"] - 1.0,
+                                  "gemm_tflops_p0": s0["gemm_tflops"]}
+        line["p_sweep"] = {str(pv): {**r, "step_overhead_vs_p0": r["step_ms"] / s0["step_ms"] - 1.0,
+                                     "gemm_overhead_vs_p0": r["gemm_ms"] / s0["gemm_ms"] - 1.0,
+                                     "gemm_overhead_lower_bound": side_slice_bound(pv)}
+                           for pv, r in sorted(sweep.items())}
         dec, wbytes = decode_sweep(F, p, device, fused=not args.unfused)
         dec0, wbytes0 = decode_sweep(F, 0, device, Ms=(16,), fused=not args.unfused)
         hbm = peaks["hbm_gbs"]

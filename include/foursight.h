@@ -27,8 +27,8 @@
  *   returned early and its output is undefined).
  * - dtype codes: FS_DTYPE_BF16 (row-major bf16), FS_DTYPE_F32 (row-major fp32).
  * - Leading dimensions (ldx, ldw, ldy) are in elements and must make every row
- *   start on a 16-byte boundary; base pointers must be 16-byte aligned (256-byte
- *   for the packed operands of fs_splice_gemm, which are read by TMA).
+ *   start on a 16-byte boundary; base pointers must be 16-byte aligned (the packed
+ *   operands of fs_splice_gemm are read by TMA, whose tensor maps need exactly that).
  *
  * Packed NVFP4 operand layout (written by fs_quantize_splice / fs_prepare_weights,
  * read by fs_splice_gemm):
@@ -74,7 +74,12 @@ enum {
   FS_GAIN_EXACT = 1u << 2, /* encode gain fl32(2688/amax) instead of the power-of-two gain */
   FS_OUT_BF16 = 1u << 3,   /* fs_splice_gemm writes bf16 Y instead of fp32 */
   FS_PATH_TENSOR = 1u << 4, /* plan option: always use the tcgen05 tensor-core kernel */
-  FS_PATH_DECODE = 1u << 5  /* plan option: always use the weight-streaming decode kernel (M <= 16) */
+  FS_PATH_DECODE = 1u << 5, /* plan option: always use the weight-streaming decode kernel (M <= 16) */
+  FS_FAULT_NO_COPIES = 1u << 6 /* plan (and fs_splice_gemm_noalloc) option for tests of failure detection:
+                              the GEMM kernels' producers issue no copies and every bounded wait is
+                              limited to 20 ms, so each launch gives up its waits, takes its abort path
+                              (no copy in flight, TMEM released) and reports FS_ERR_TIMEOUT through
+                              fs_plan_check; the output is left undefined.  Never set in production. */
 };
 
 /* Readable name of a status code (static storage). */
@@ -171,6 +176,20 @@ fs_status fs_prepare_weights(const void* W, int32_t dtype, int32_t N, int32_t K,
 fs_status fs_quantize_splice(const void* X, int32_t dtype, int64_t M, int32_t K, int64_t ldx,
                              const uint32_t* mask, int32_t p, const float* gA, uint32_t opts,
                              uint8_t* xq, uint8_t* sfx, uint16_t* xs, void* stream);
+
+/* Activation preparation and channel statistics in ONE pass over X — FourSight §5.2 (the forward
+ * hook accumulates running channel moments of the token rows BEFORE masking) together with §5.1
+ * "Data preparation".  Equivalent, bit for bit, to
+ *     fs_channel_stats(X, dtype, M, K, ldx, row_stride, n, s1, s2, amax, flags)
+ *     fs_quantize_splice(X, dtype, M, K, ldx, mask, p, gA, opts, xq, sfx, xs)
+ * but X is read once.  The moments go into the state that the NEXT reselection reads, while mask,
+ * p and gA are the CURRENT protected set and gain (the paper's order: reselect after each step from
+ * the moments gathered during it).  Arguments, layouts and requirements as for the two calls;
+ * dtype must be FS_DTYPE_BF16 (FS_ERR_UNSUPPORTED for fp32 input). */
+fs_status fs_quantize_splice_stats(const void* X, int32_t dtype, int64_t M, int32_t K, int64_t ldx,
+                                   const uint32_t* mask, int32_t p, const float* gA, uint32_t opts,
+                                   uint8_t* xq, uint8_t* sfx, uint16_t* xs, int32_t row_stride, int64_t* n,
+                                   int64_t* s1, int64_t* s2, uint32_t* amax, uint32_t* flags, void* stream);
 
 /* Grouped (mixture-of-experts) form: E experts, expert e owning rows
  * [row_offsets[e], row_offsets[e+1]) of X (row_offsets: device int64 [E+1], row_offsets[0] == 0,

@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(HERE, "libfoursight.so")
 FS_OK, FS_ERR_INVALID_ARGUMENT, FS_ERR_UNSUPPORTED, FS_ERR_CUDA, FS_ERR_RANGE, FS_ERR_TIMEOUT = range(6)
 FS_DTYPE_BF16, FS_DTYPE_F32 = 0, 1
 FS_RESIDUAL, FS_KEY_M2, FS_GAIN_EXACT, FS_OUT_BF16, FS_PATH_TENSOR, FS_PATH_DECODE = 1, 2, 4, 8, 16, 32
+FS_FAULT_NO_COPIES = 64
 
 P = C.c_void_p
 i32, i64, u32, f32 = C.c_int32, C.c_int64, C.c_uint32, C.c_float
@@ -32,6 +33,7 @@ SIGNATURES = {
     "fs_prepare_weights": (C.c_int, [P, i32, i32, i32, i64, P, i32, u32, P, P, P, P, P, P, P]),
     "fs_quantize_splice": (C.c_int, [P, i32, i64, i32, i64, P, i32, P, u32, P, P, P, P]),
     "fs_quantize_splice_grouped": (C.c_int, [P, i32, i32, P, i64, i32, i64, P, i32, P, u32, P, P, P, P]),
+    "fs_quantize_splice_stats": (C.c_int, [P, i32, i64, i32, i64, P, i32, P, u32, P, P, P, i32, P, P, P, P, P, P]),
     "fs_plan_create": (C.c_int, [C.POINTER(P), i32, i32, i32, u32]),
     "fs_plan_destroy": (C.c_int, [P]),
     "fs_plan_check": (C.c_int, [P, P]),

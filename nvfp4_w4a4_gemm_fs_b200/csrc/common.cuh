@@ -16,6 +16,7 @@
 #include <algorithm>
 
 #include "foursight.h"
+#include "per_device.h"
 
 namespace fs {
 
@@ -31,8 +32,13 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 inline int side_cols(int p) { return (p + 15) / 16 * 16; }
 inline int64_t sf_bytes(int64_t rows, int K) { return round_up(rows, 128) * round_up(K / 16, 4); }
-// Streaming multiprocessors of the current device (queried once).
+// Index of the current device (cudaGetDevice), -1 if it cannot be read.
+int current_device();
+// Streaming multiprocessors of the current device (queried once per device).
 int sm_count();
+// Sets a kernel's dynamic shared-memory limit once per device (the attribute belongs to the
+// device's context); `cache` is the caller's static per-device flag.
+fs_status set_max_dynamic_smem(PerDevice<int>& cache, const void* kernel, int bytes, const char* who);
 
 #define FS_CHECK_LAUNCH(what)                                         \
   do {                                                                \
@@ -167,9 +173,11 @@ __device__ __forceinline__ float gain_pow2(float amax) {
   return __uint_as_float(static_cast<uint32_t>(E + 127) << 23);
 }
 
+// fl32(2688/amax) saturated to the largest finite float (the quotient overflows for every
+// subnormal amax); 1 for amax == 0 or non-finite.
 __device__ __forceinline__ float gain_exact(float amax) {
   if (!(amax > 0.0f) || !isfinite(amax)) return 1.0f;
-  return __fdiv_rn(2688.0f, amax);
+  return fminf(__fdiv_rn(2688.0f, amax), 3.40282346638528859812e+38f);
 }
 
 // Byte offset of (row r, 16-block b) in the tiled scale array; kb4 = roundup(K/16,4)/4.

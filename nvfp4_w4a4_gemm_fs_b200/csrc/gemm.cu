@@ -97,6 +97,7 @@ fs_status splice_gemm(const char* who, fs_plan plan, int64_t M, int32_t p, const
     d.kb4 = static_cast<int>(round_up(plan->K / 16, 4) / 4);
     d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha; d.seg = seg;
     d.Y = Y; d.ldy = ldy; d.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; d.err = plan->err;
+    d.wait_ns = wait_limit_ns(plan->opts); d.no_copies = (plan->opts & FS_FAULT_NO_COPIES) ? 1 : 0;
     return launch_splice_gemm_decode_tc(d, s);
   }
   if (M > (int64_t{1} << 31) - 256) return fail(FS_ERR_UNSUPPORTED, "%s: M too large", who);
@@ -104,6 +105,7 @@ fs_status splice_gemm(const char* who, fs_plan plan, int64_t M, int32_t p, const
   prm.M = M; prm.N = plan->N; prm.K = plan->K; prm.KT = plan->K / 256; prm.ST = static_cast<int>(ceil_div(pp, 64));
   prm.E = 1; prm.kb4 = plan->K / 64; prm.offsets = nullptr; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
   prm.seg = seg; prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
+  prm.wait_ns = wait_limit_ns(plan->opts); prm.no_copies = (plan->opts & FS_FAULT_NO_COPIES) ? 1 : 0;
   TcLaunch L{};
   L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = M; L.b_rows = plan->N; L.y_rows = M; L.pp = pp;
   L.bn = (plan->N % 256 == 0) ? 256 : 128;
@@ -172,6 +174,7 @@ extern "C" fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64
   prm.E = E; prm.kb4 = plan->K / 64; prm.offsets = row_offsets; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
   prm.seg = one_segment(plan->N);
   prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
+  prm.wait_ns = wait_limit_ns(plan->opts); prm.no_copies = (plan->opts & FS_FAULT_NO_COPIES) ? 1 : 0;
   TcLaunch L{};
   L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = a_rows; L.b_rows = static_cast<int64_t>(E) * plan->N; L.y_rows = max_rows; L.pp = pp;
   L.bn = (plan->N % 256 == 0) ? 256 : 128;

@@ -37,6 +37,8 @@ struct TcParams {
   int64_t ldy;
   int out_bf16;
   uint32_t* err;
+  uint64_t wait_ns;   // limit of every bounded wait
+  int no_copies;      // failure-detection test hook: the producer issues no copies
 };
 
 // Host-side description of the operand buffers for tensor-map encoding.
@@ -73,7 +75,15 @@ struct DecodeParams {
   int64_t ldy;
   int out_bf16;
   uint32_t* err;      // device error word (bounded-wait timeouts of the tensor-core decode kernel)
+  uint64_t wait_ns;   // limit of every bounded wait
+  int no_copies;      // failure-detection test hook: the producer issues no copies
 };
+
+// Wait limits: the normal bound, and the short one of the failure-detection test option
+// (FS_FAULT_NO_COPIES), under which every launch gives up its waits and reports a timeout.
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+constexpr uint64_t kFaultWaitLimitNs = 20000000ull;
+inline uint64_t wait_limit_ns(uint32_t opts) { return (opts & FS_FAULT_NO_COPIES) ? kFaultWaitLimitNs : kWaitLimitNs; }
 
 fs_status launch_splice_gemm_decode_tc(const DecodeParams& p, cudaStream_t s);
 

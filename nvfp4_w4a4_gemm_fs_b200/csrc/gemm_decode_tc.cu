@@ -43,7 +43,6 @@ constexpr int kDCtasPerSm = FS_DEC_CTAS_PER_SM;   // residency the shared-memory
 static_assert(kDCtasPerSm * (1024 + 1024 + kDStages * (128 * 128 + 16 * 128 + 4096) + 8 * (2 * kDStages + 2) + 16) <= 233472,
               "CTAs per SM must fit the SM's shared memory");
 constexpr int kDMaxSplit = 8;        // portable cluster size
-constexpr uint64_t kDWaitNs = 2000000000ull;
 constexpr uint64_t kDDrainNs = 50000000ull;
 
 struct DCfg {
@@ -71,6 +70,8 @@ struct DecTcParams {
   int64_t ldy;
   int out_bf16;
   uint32_t* err;
+  uint64_t wait_ns;
+  int no_copies;
 };
 
 __device__ __forceinline__ uint64_t now_ns() {
@@ -79,14 +80,15 @@ __device__ __forceinline__ uint64_t now_ns() {
   return t;
 }
 
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* err) {
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* err,
+                                         uint64_t limit_ns) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   for (uint32_t i = 1;; ++i) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if ((i & 255) == 0) {
       if (*abort_flag) return false;
-      if (now_ns() - t0 > kDWaitNs) {
+      if (now_ns() - t0 > limit_ns) {
         if (err) atomicOr(err, ERR_TIMEOUT);
         *abort_flag = 1;
         return false;
@@ -142,7 +144,8 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&tmW); ptx::prefetch_tensormap(&tmX);
     if (p.ST > 0) { ptx::prefetch_tensormap(&tmWS); ptx::prefetch_tensormap(&tmXS); }
-    for (int kt = kt0; kt < kt1; ++kt) ptx::tma_prefetch_2d(&tmW, kt * 128, n0);
+    if (!p.no_copies)
+      for (int kt = kt0; kt < kt1; ++kt) ptx::tma_prefetch_2d(&tmW, kt * 128, n0);
   }
   if (warp == 1) {
     ptx::tmem_alloc<1>(tmem_slot, C::TMEM_COLS);
@@ -156,11 +159,13 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // (p.no_copies, the failure-detection test hook: nothing is issued; the MMA and epilogue
+    // waits run out and every CTA still reaches both cluster barriers)
+    if (lane == 0 && !p.no_copies) {
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       for (int i = 0; i < nk; ++i) {
-        if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err)) break;
+        if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err, p.wait_ns)) break;
         if (i < nf) {
           const int kt = kt0 + i;
           ptx::mbar_arrive_expect_tx(full + stage, C::STAGE_BYTES);
@@ -197,7 +202,7 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
       uint32_t phase = 0;
       bool ok = true;
       for (int i = 0; i < nk; ++i) {
-        if (!wait_bar(full + stage, phase, abort_flag, p.err)) { ok = false; break; }
+        if (!wait_bar(full + stage, phase, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint64_t adesc = ptx::desc_kmajor_sw128(ptx::smem_u32(W_at(stage)));
         const uint64_t bdesc = ptx::desc_kmajor_sw128(ptx::smem_u32(X_at(stage)));
@@ -222,13 +227,13 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
       }
       if (ok) ptx::tc_commit<1>(acc_full);
       ptx::tc_commit<1>(drain);                    // every MMA issued above has completed
-      drain_bar(drain, 0, kDWaitNs);
+      drain_bar(drain, 0, p.wait_ns);
     }
   } else {
     // ------------------------------------------------------------------ epilogue: TMEM -> partial
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    if (wait_bar(acc_full, 0, abort_flag, p.err)) {
+    if (wait_bar(acc_full, 0, abort_flag, p.err, p.wait_ns)) {
       ptx::tc_fence_after();
       uint32_t r[16];
       ptx::tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16), r);
@@ -287,17 +292,14 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
 
 fs_status launch_splice_gemm_decode_tc(const DecodeParams& d, cudaStream_t s) {
   using C = DCfg;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(splice_gemm_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm (decode): smem attribute");
-    attr = true;
-  }
+  static PerDevice<int> attr;
+  fs_status ast = set_max_dynamic_smem(attr, reinterpret_cast<const void*>(splice_gemm_decode_tc_kernel),
+                                       C::SMEM_BYTES, "fs_splice_gemm (decode): smem attribute");
+  if (ast != FS_OK) return ast;
   DecTcParams p{};
   p.M = d.M; p.N = d.N; p.KT = d.K / 256; p.ST = static_cast<int>(ceil_div(d.pp, 64)); p.kb4 = d.kb4;
   p.sfw = d.sfw; p.sfx = d.sfx; p.alpha = d.alpha; p.seg = d.seg; p.Y = d.Y; p.ldy = d.ldy; p.out_bf16 = d.out_bf16;
-  p.err = d.err;
+  p.err = d.err; p.wait_ns = d.wait_ns; p.no_copies = d.no_copies;
   // K split: as many CTAs per 128-row tile as fill the SMs at the resident CTAs per SM, at most 8
   // (a portable cluster);
   // every split keeps at least one FP4 k-tile.

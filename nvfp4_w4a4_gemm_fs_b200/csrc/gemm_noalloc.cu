@@ -12,8 +12,6 @@
 // clears it (cudaMemsetAsync on the caller's stream, no allocation) before its kernel starts.  Two
 // calls that overlap on the GPU (different streams, no ordering between them) race on it: a
 // timeout reported by one may then come from the other.
-#include <mutex>
-
 #include "common.cuh"
 #include "gemm.cuh"
 
@@ -25,25 +23,17 @@ namespace {
 constexpr int kNoAllocScratchWords = 1;
 static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocScratchWords];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-uint32_t* g_scratch_ptr[kMaxDevices] = {};
-
-// Once per device, with that device current: the device address of the scratch array.  In host
-// code the array's name is only a host-side stand-in, so kernels must be given this address.
-fs_status scratch_for_current_device(uint32_t** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm_noalloc: cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm_noalloc: device %d >= %d", dev, kMaxDevices);
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm_noalloc: cudaGetSymbolAddress");
-    g_scratch_ptr[dev] = static_cast<uint32_t*>(ptr);
-  }
-  *out = g_scratch_ptr[dev];
+// The device address of the scratch array in the context current on this thread.  In host code
+// the array's name is only a host-side stand-in, so kernels must be given this address.  It is
+// looked up on every call (cudaGetSymbolAddress allocates nothing): an address cached per device
+// number would go stale after cudaDeviceReset or under another context of the same device.  The
+// first lookup in a context may load the library's module there, which is why the first call on a
+// device should come before any stream capture.
+fs_status scratch_for_current_context(uint32_t** out) {
+  void* ptr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm_noalloc: cudaGetSymbolAddress");
+  *out = static_cast<uint32_t*>(ptr);
   return FS_OK;
 }
 
@@ -73,24 +63,25 @@ extern "C" fs_status fs_splice_gemm_noalloc(int32_t N, int32_t K, uint32_t opts,
   const bool bf16 = opts & FS_OUT_BF16;
   if (ldy < N || !aligned(Y, 16) || (ldy % (bf16 ? 8 : 4)) != 0)
     return fail(FS_ERR_INVALID_ARGUMENT, "%s: Y must be 16-byte aligned with ldy >= N and 16-byte rows", who);
+  const bool decode = (opts & FS_PATH_DECODE) || (!(opts & FS_PATH_TENSOR) && M <= 16);
+  if (decode && M > 16) return fail(FS_ERR_UNSUPPORTED, "%s: the decode path takes M <= 16", who);
   // The kernels need exactly kNoAllocScratchWords words of scratch; no problem size needs more.
   static_assert(kNoAllocScratchWords >= 1, "one error word");
 
   uint32_t* scratch = nullptr;
-  fs_status st = scratch_for_current_device(&scratch);
+  fs_status st = scratch_for_current_context(&scratch);
   if (st != FS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(scratch, 0, kNoAllocScratchWords * sizeof(uint32_t), s);
   if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm_noalloc: clearing scratch");
 
   const int pp = side_cols(p);
-  const bool decode = (opts & FS_PATH_DECODE) || (!(opts & FS_PATH_TENSOR) && M <= 16);
   if (decode) {
-    if (M > 16) return fail(FS_ERR_UNSUPPORTED, "%s: the decode path takes M <= 16", who);
     DecodeParams d{};
     d.M = static_cast<int>(M); d.N = N; d.K = K; d.pp = pp; d.kb4 = static_cast<int>(round_up(K / 16, 4) / 4);
     d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha;
     d.Y = Y; d.ldy = ldy; d.out_bf16 = bf16 ? 1 : 0; d.err = scratch;
+    d.wait_ns = wait_limit_ns(opts); d.no_copies = (opts & FS_FAULT_NO_COPIES) ? 1 : 0;
     d.seg.n = 1; d.seg.n0[0] = 0; d.seg.n0[1] = N;
     st = launch_splice_gemm_decode_tc(d, s);
   } else {
@@ -98,6 +89,7 @@ extern "C" fs_status fs_splice_gemm_noalloc(int32_t N, int32_t K, uint32_t opts,
     prm.M = M; prm.N = N; prm.K = K; prm.KT = K / 256; prm.ST = static_cast<int>(ceil_div(pp, 64));
     prm.E = 1; prm.kb4 = K / 64; prm.offsets = nullptr; prm.sfa = sfx; prm.sfb = sfw; prm.alpha = alpha;
     prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = bf16 ? 1 : 0; prm.err = scratch;
+    prm.wait_ns = wait_limit_ns(opts); prm.no_copies = (opts & FS_FAULT_NO_COPIES) ? 1 : 0;
     prm.seg.n = 1; prm.seg.n0[0] = 0; prm.seg.n0[1] = N;
     TcLaunch L{};
     L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = M; L.b_rows = N; L.y_rows = M; L.pp = pp;

@@ -41,7 +41,6 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kThreads = 320;                  // producer, MMA, 4 epilogue and 4 scale warps
 constexpr int kMaxExperts = 256;
-constexpr uint64_t kWaitNs = 4000000000ull;     // 4 s bound on any single wait
 constexpr uint64_t kDrainNs = 50000000ull;      // 50 ms bound on each wait of the abort path
 
 #ifndef FS_TC_PAIR_STAGES
@@ -108,15 +107,16 @@ __device__ __forceinline__ uint64_t now_ns() {
   return t;
 }
 
-// Wait with a deadline and an abort flag shared by the CTA's roles.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* err) {
+// Wait with a deadline (`limit_ns`) and an abort flag shared by the CTA's roles.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* err,
+                                         uint64_t limit_ns) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   for (uint32_t i = 1;; ++i) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if ((i & 255) == 0) {
       if (*abort_flag) return false;
-      if (now_ns() - t0 > kWaitNs) {
+      if (now_ns() - t0 > limit_ns) {
         atomicOr(err, ERR_TIMEOUT);
         *abort_flag = 1;
         return false;
@@ -246,7 +246,9 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // (p.no_copies, the failure-detection test hook: nothing is issued, so every other role's
+    // first wait runs out and the kernel takes its abort path with no copy in flight)
+    if (lane == 0 && !p.no_copies) {
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       uint32_t sfl_bits = 0, last_fp4 = 0;   // per stage: parity of its next FP4 use; last use was FP4
@@ -258,7 +260,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         const bool sfa_ok = p.offsets || (m.arow / kBM) < m_groups;
         const int64_t brow = m.brow + rank * C::B_ROWS;
         for (int kt = 0; kt < ktiles; ++kt) {
-          if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err)) { ok = false; break; }
+          if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
           const bool fp4 = kt < p.KT;
           last_fp4 = (last_fp4 & ~(1u << stage)) | (static_cast<uint32_t>(fp4) << stage);
           if (fp4) {
@@ -308,11 +310,11 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int t = unit; t < total_tiles && ok; t += nunits, ++i) {
-        if (!wait_bar(acc_empty + acc, acc_phase ^ 1, abort_flag, p.err)) break;
+        if (!wait_bar(acc_empty + acc, acc_phase ^ 1, abort_flag, p.err, p.wait_ns)) break;
         ptx::tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(C::OVERLAP ? (i & 1) * 128 : 0);
         for (int kt = 0; kt < ktiles; ++kt) {
-          if (!wait_bar(full + stage, phase, abort_flag, p.err)) { ok = false; break; }
+          if (!wait_bar(full + stage, phase, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint64_t adesc = ptx::desc_kmajor_sw128(ptx::smem_u32(A_at(stage)));
           const uint64_t bdesc = ptx::desc_kmajor_sw128(ptx::smem_u32(B_at(stage)));
@@ -320,7 +322,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 #pragma unroll
             for (int h = 0; h < C::SF_SPLIT; ++h) {
               const int slot = sf_unit % C::SF_UNITS;
-              if (!wait_bar(sf_full + slot, (sf_unit / C::SF_UNITS) & 1, abort_flag, p.err)) { ok = false; break; }
+              if (!wait_bar(sf_full + slot, (sf_unit / C::SF_UNITS) & 1, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
               ptx::tc_fence_after();
               const uint32_t sf = tmem + C::SF_COL + slot * C::UNIT_COLS;
 #pragma unroll
@@ -346,7 +348,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       }
       // Every MMA issued above has completed before TMEM can be released.
       ptx::tc_commit<CG>(drain);
-      drain_bar(drain, 0, kWaitNs);
+      drain_bar(drain, 0, p.wait_ns);
     }
   } else if (warp >= 6) {
     // ------------------------------------------------------------------ scale warps
@@ -365,7 +367,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     for (int t = unit; t < total_tiles && ok; t += nunits) {
       for (int kt = 0; kt < ktiles; ++kt) {
         if (kt < p.KT) {
-          if (!wait_bar(sfl + stage, (sfl_bits >> stage) & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!wait_bar(sfl + stage, (sfl_bits >> stage) & 1, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
           sfl_bits ^= 1u << stage;
           const uint8_t* sfa = SFA_at(stage);
           const uint8_t* sfb = SFB_at(stage);
@@ -379,7 +381,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 #pragma unroll
           for (int h = 0; h < C::SF_SPLIT; ++h) {
             const int slot = sf_unit % C::SF_UNITS;
-            if (!wait_bar(sf_empty + slot, ((sf_unit / C::SF_UNITS) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
+            if (!wait_bar(sf_empty + slot, ((sf_unit / C::SF_UNITS) & 1) ^ 1, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
             const uint32_t col = tmem + lane_base + C::SF_COL + slot * C::UNIT_COLS;
 #pragma unroll
             for (int jj = 0; jj < C::MPU; ++jj) {
@@ -419,7 +421,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     uint32_t acc_phase = 0;
     for (int t = unit; t < total_tiles; t += nunits, ++i) {
       const TileMap m = map_tile<CG>(t, p, cum_m, rank);
-      if (!wait_bar(acc_full + acc, acc_phase, abort_flag, p.err)) break;
+      if (!wait_bar(acc_full + acc, acc_phase, abort_flag, p.err, p.wait_ns)) break;
       ptx::tc_fence_after();
       const float alpha = __ldg(p.alpha + (p.offsets ? m.e : segment_of(m.n0, p.seg)));
       const bool use_tma = !p.offsets || (quad + 1) * 32 <= m.rows;
@@ -556,23 +558,19 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 
 template <int BN, int CG>
 fs_status set_smem_attr() {
-  static bool done = false;
-  if (!done) {
-    cudaError_t e = cudaFuncSetAttribute(splice_gemm_tc_kernel<BN, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<BN, CG>::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm: smem attribute");
-    done = true;
-  }
-  return FS_OK;
+  static PerDevice<int> cache;
+  return set_max_dynamic_smem(cache, reinterpret_cast<const void*>(splice_gemm_tc_kernel<BN, CG>),
+                              Cfg<BN, CG>::SMEM_BYTES, "fs_splice_gemm: smem attribute");
 }
 
-// Number of CTA pairs that can be resident at once (clusters must fit inside a GPC, so this can
-// be below half the SM count); 0 when the query fails.
+// Number of CTA pairs that can be resident at once on the current device (clusters must fit
+// inside a GPC, so this can be below half the SM count); 0 when the query fails.
 int pair_slots() {
-  static int n = -1;
-  if (n < 0) {
-    n = 0;
-    if (set_smem_attr<256, 2>() != FS_OK) return n;
+  static PerDevice<int> cache;
+  int n = 0;
+  if (cache.get(current_device(), &n, [](int* out) {
+    *out = 0;
+    if (set_smem_attr<256, 2>() != FS_OK) return false;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(sm_count() & ~1));
     cfg.blockDim = dim3(kThreads);
@@ -585,10 +583,12 @@ int pair_slots() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, splice_gemm_tc_kernel<256, 2>, &cfg) == cudaSuccess && c > 0) n = c;
+    if (cudaOccupancyMaxActiveClusters(&c, splice_gemm_tc_kernel<256, 2>, &cfg) == cudaSuccess && c > 0) *out = c;
     else cudaGetLastError();
-  }
-  return n;
+    return true;
+  }))
+    return n;
+  return 0;
 }
 
 template <int BN, int CG>
@@ -680,17 +680,6 @@ fs_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, u
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return FS_OK;
-}
-
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
 }
 
 fs_status launch_splice_gemm_tc(const TcLaunch& L, const TcParams& prm, cudaStream_t s) {

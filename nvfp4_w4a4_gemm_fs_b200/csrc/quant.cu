@@ -568,9 +568,12 @@ extern "C" fs_status fs_prepare_weights(const void* W, int32_t dtype, int32_t N,
   const uint32_t* m = p > 0 ? mask : nullptr;
   if (dtype == FS_DTYPE_BF16) {
     // one wave of resident CTAs, each warp with at least kAmaxDepth stripes
-    static int per_sm = 0;
-    if (per_sm == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, weight_amax_bf16_kernel, kAmaxThreads, 0) !=
-                            cudaSuccess || per_sm < 1))
+    static PerDevice<int> occ;
+    int per_sm = 1;
+    if (!occ.get(current_device(), &per_sm, [](int* v) {
+          return cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, weight_amax_bf16_kernel, kAmaxThreads, 0) ==
+                     cudaSuccess && *v >= 1;
+        }))
       per_sm = 1;
     const int64_t work = static_cast<int64_t>(N) * std::max(1, K / 256);
     const unsigned grid = static_cast<unsigned>(std::max<int64_t>(

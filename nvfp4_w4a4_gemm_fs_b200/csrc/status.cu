@@ -28,6 +28,36 @@ fs_status cuda_status(cudaError_t e, const char* what) {
   return fail(FS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+int sm_count() {
+  static PerDevice<int> cache;
+  int n = 0;
+  const int dev = current_device();
+  if (cache.get(dev, &n, [dev](int* v) {
+        return cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && *v > 0;
+      }))
+    return n;
+  return 148;
+}
+
+fs_status set_max_dynamic_smem(PerDevice<int>& cache, const void* kernel, int bytes, const char* who) {
+  int done = 0;
+  cudaError_t err = cudaSuccess;
+  if (cache.get(current_device(), &done, [&](int* v) {
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        *v = 1;
+        return err == cudaSuccess;
+      }))
+    return FS_OK;
+  if (err != cudaSuccess) return cuda_status(err, who);
+  return fail(FS_ERR_CUDA, "%s: no current device", who);
+}
+
 }  // namespace fs
 
 extern "C" {

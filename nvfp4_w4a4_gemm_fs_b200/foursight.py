@@ -14,7 +14,7 @@ from ._lib import FS_DTYPE_BF16, FS_DTYPE_F32, check
 
 __all__ = [
     "fs_channel_stats", "fs_stats_check", "fs_select_topk", "fs_prepare_weights",
-    "fs_quantize_splice", "fs_quantize_splice_grouped", "fs_splice_gemm", "fs_splice_gemm_grouped",
+    "fs_quantize_splice", "fs_quantize_splice_grouped", "fs_quantize_splice_stats", "fs_splice_gemm", "fs_splice_gemm_grouped",
     "fs_seq_filter", "Plan", "StatsState", "Packed", "side_cols", "sf_bytes", "grouped_rows",
     "fs_splice_gemm_segmented", "stacked_packed",
     "alloc_packed", "stream_handle",
@@ -127,6 +127,21 @@ def fs_quantize_splice(X: torch.Tensor, mask, p: int, gA: torch.Tensor, opts: in
     check(lib.fs_quantize_splice(_ptr(X), _dtype_code(X), M, K, X.stride(0), _ptr(mask) if p else None, p,
                                  _ptr(gA), opts, _ptr(out.q), _ptr(out.sf), _ptr(out.side) if p else None,
                                  stream_handle(stream)), "fs_quantize_splice")
+    return out
+
+
+def fs_quantize_splice_stats(X: torch.Tensor, mask, p: int, gA: torch.Tensor, state: StatsState, group: int = 0,
+                             row_stride: int = 1, opts: int = 0, out: Packed | None = None, stream=None):
+    """fs_quantize_splice with the CURRENT protected set (mask, p, gA) and fs_channel_stats into
+    ``state`` (for the NEXT reselection) in one pass over the bf16 activations X."""
+    lib = _lib.load()
+    M, K = X.shape
+    out = alloc_packed(M, K, p, X.device) if out is None else out
+    n, s1, s2, amax, flags = state.group(group)
+    check(lib.fs_quantize_splice_stats(_ptr(X), _dtype_code(X), M, K, X.stride(0), _ptr(mask) if p else None, p,
+                                       _ptr(gA), opts, _ptr(out.q), _ptr(out.sf), _ptr(out.side) if p else None,
+                                       row_stride, _ptr(n), _ptr(s1), _ptr(s2), _ptr(amax), _ptr(flags),
+                                       stream_handle(stream)), "fs_quantize_splice_stats")
     return out
 
 

@@ -31,13 +31,18 @@ def _problem(seed, M, N, K, p, dtype="bf16", residual=False, calib_rows=None):
     return X, W, Xt, Wt, P, gA
 
 
+def nan_output(M, N, bf16=False):
+    """Output buffer prefilled with NaN, so that an element the kernel never writes fails the check."""
+    return torch.full((M, N), float("nan"), dtype=torch.bfloat16 if bf16 else torch.float32, device="cuda")
+
+
 def _run_gpu(Xt, Wt, P, gA, p, N, K, opts=0, plan_opts=0):
     mask = mask_tensor(stats.protect_mask(P, K))
     g = torch.tensor([float(gA)], device="cuda")
     wq, gW, alpha = F.fs_prepare_weights(Wt, mask, p, g, opts=opts)
     xq = F.fs_quantize_splice(Xt, mask, p, g, opts=opts)
     plan = F.Plan(N, K, max(p, 1), plan_opts)
-    Y = F.fs_splice_gemm(plan, xq, wq, alpha)
+    Y = F.fs_splice_gemm(plan, xq, wq, alpha, Y=nan_output(Xt.shape[0], N, bool(plan_opts & F.FS_OUT_BF16)))
     plan.check()
     return Y, plan
 
@@ -51,8 +56,9 @@ def _ref(X, W, P, gA, residual=False, rows=None):
 
 def _assert_close(Y, Yr, mag, bf16_out=False):
     Yg = Y.float().cpu().numpy().astype(np.float64)
+    assert np.isfinite(Yg).all(), f"{(~np.isfinite(Yg)).sum()} outputs not finite (unwritten or overflowed)"
     tol = REL * mag + (2.0 ** -8 * np.abs(Yr) if bf16_out else 0.0)
-    bad = np.abs(Yg - Yr) > tol
+    bad = ~(np.abs(Yg - Yr) <= tol)
     assert not bad.any(), (f"{bad.sum()} of {bad.size} outside tolerance; worst excess "
                            f"{np.max(np.abs(Yg - Yr) - tol):.3e} at {np.unravel_index(np.argmax(np.abs(Yg - Yr) - tol), Yr.shape)}")
 
@@ -109,14 +115,33 @@ def test_paths_agree_on_the_same_inputs():
     _assert_close(Yt, Yr, mag)
 
 
-@pytest.mark.parametrize("N,K", [(4096, 4096), (1024, 4096), (12288, 4096), (4096, 12288)])
-def test_full_size_prefill_sampled_rows(N, K):
-    """M = 8192 tokens as timed; the oracle checks 48 sampled rows spread over all row tiles."""
-    M, p = 8192, 64
+def _row_per_tile(M, seed):
+    """One random row in every 128-row tile (first and last rows included): each output tile of
+    the launch, and each CTA of a pair, contributes a checked row."""
+    rng = np.random.default_rng(seed)
+    rows = np.array([t + rng.integers(0, min(128, M - t)) for t in range(0, M, 128)])
+    return np.unique(np.concatenate([[0, M - 1], rows]))
+
+
+def test_full_size_prefill_all_rows_q():
+    """The q projection as timed (M = 8192, N = K = 4096, P = 64): every one of the 8192 x 4096
+    outputs against the oracle's float64 Eq. 5."""
+    M, N, K, p = 8192, 4096, 4096, 64
     X, W, Xt, Wt, P, gA = _problem(7, M, N, K, p)
     Y, _ = _run_gpu(Xt, Wt, P, gA, p, N, K)
-    rows = np.sort(np.random.default_rng(N + K).choice(M, 48, replace=False))
-    rows[0], rows[-1] = 0, M - 1
+    Yr, mag = _ref(X, W, P, gA)
+    _assert_close(Y, Yr, mag)
+
+
+@pytest.mark.parametrize("N,K,p", [(1024, 4096, 64), (12288, 4096, 64), (4096, 12288, 64), (4096, 4096, 256),
+                                   (4096, 12288, 256)])
+def test_full_size_prefill_rows_of_every_tile(N, K, p):
+    """M = 8192 tokens as timed (P = 64, and the P = 256 budget); the oracle checks one row of
+    every 128-row tile, so every row tile and both CTAs of every pair are covered."""
+    M = 8192
+    X, W, Xt, Wt, P, gA = _problem(7, M, N, K, p)
+    Y, _ = _run_gpu(Xt, Wt, P, gA, p, N, K)
+    rows = _row_per_tile(M, N + K + p)
     Yr, mag = _ref(X, W, P, gA, rows=rows)
     _assert_close(Y[torch.from_numpy(rows).cuda()], Yr, mag)
 
@@ -158,7 +183,7 @@ def test_segmented_projections_match_each_projection(path, M):
         F.fs_prepare_weights(bf16_tensor(w), mask, p, g, out=view, alpha=alphas[j:j + 1])
     seg = np.concatenate([[0], np.cumsum(seg_rows)]).tolist()
     plan = F.Plan(seg[-1], K, p, F.FS_PATH_DECODE if path == "decode" else F.FS_PATH_TENSOR)
-    Y = F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, seg)
+    Y = F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, seg, Y=nan_output(M, seg[-1]))
     plan.check()
     for j in range(len(seg_rows)):
         Yr, mag = _ref(X, Ws[j], P, gA)
@@ -172,8 +197,8 @@ def test_segmented_projections_match_each_projection(path, M):
 @pytest.mark.parametrize("M,seg_rows", [(8192, [4096, 1024, 1024]), (8192, [12288, 12288]), (16, [4096, 1024, 1024])])
 def test_full_size_segmented_sampled_rows(M, seg_rows):
     """The launches bench.py times: M = 8192 tokens (tensor-core path) or 16 (decode path), K =
-    4096, the q/k/v (or gate/up) weights stacked in one segmented launch; the oracle checks 40
-    sampled rows (all rows at M = 16) of every projection."""
+    4096, the q/k/v (or gate/up) weights stacked in one segmented launch; the oracle checks one
+    row of every 128-row tile (all rows at M = 16) of every projection."""
     K, p = 4096, 64
     x, _ = synth.outlier_activations(211, M, K)
     X = splice.as_f32(x, True)
@@ -192,13 +217,9 @@ def test_full_size_segmented_sampled_rows(M, seg_rows):
         F.fs_prepare_weights(bf16_tensor(w), mask, p, g, out=view, alpha=alphas[j:j + 1])
     seg = np.concatenate([[0], np.cumsum(seg_rows)]).tolist()
     plan = F.Plan(seg[-1], K, p)
-    Y = F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, seg)
+    Y = F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, seg, Y=nan_output(M, seg[-1]))
     plan.check()
-    if M <= 40:
-        rows = np.arange(M)
-    else:
-        rows = np.sort(np.random.default_rng(seg[-1]).choice(M, 40, replace=False))
-        rows[0], rows[-1] = 0, M - 1
+    rows = np.arange(M) if M <= 40 else _row_per_tile(M, seg[-1])
     rows_t = torch.from_numpy(rows).cuda()
     for j in range(len(seg_rows)):
         Yr, mag = _ref(X, Ws[j], P, gA, rows=rows)
@@ -232,3 +253,4 @@ def test_repeatable_and_overwrites_output():
     Y1, _ = _run_gpu(Xt, Wt, P, gA, 64, 512, 1024)
     Y2, _ = _run_gpu(Xt, Wt, P, gA, 64, 512, 1024)
     assert torch.equal(Y1, Y2)
+    assert torch.isfinite(Y1).all()

@@ -118,6 +118,56 @@ def test_quantize_splice_bit_exact(dtype, M, K, p, residual):
         check_packed(out, ref, M, K, p)
 
 
+@pytest.mark.parametrize("M,K,p,stride,residual", [(1, 64, 0, 1, False), (8, 512, 64, 1, False), (130, 576, 5, 1, True),
+                                                   (300, 4096, 64, 3, False), (16, 12288, 256, 1, False),
+                                                   (1000, 2048, 64, 2, True), (8192, 4096, 64, 1, False),
+                                                   (2049, 12288, 64, 1, False), (257, 4096, 0, 1, False)])
+def test_quantize_splice_stats_bit_exact(M, K, p, stride, residual):
+    """The fused pass (NEXT-1): moments of the raw rows into a state that already holds a previous
+    batch, and the packed operand under the current protected set, both bit-exact against the
+    oracle's statistics and activation preparation; a second call is repeatable."""
+    X, T, P, st = _prep_inputs(17 + M + K, M, K, p, "bf16")
+    Xprev, Tprev = _x(5 + K, 33, K, "bf16")
+    gA = stats.next_gain(st, P, residual=residual)
+    mask = mask_tensor(stats.protect_mask(P, K))
+    g = torch.tensor([float(gA)], dtype=torch.float32, device="cuda")
+    opts = F.FS_RESIDUAL if residual else 0
+    ref = splice.quantize_splice(X, P, gA, splice.RESIDUAL if residual else splice.SPLIT)
+    for rep in range(2):
+        state = F.StatsState(1, K)
+        F.fs_channel_stats(Tprev, state)                                  # earlier batch of the window
+        out = F.fs_quantize_splice_stats(T, mask, p, g, state, row_stride=stride, opts=opts)
+        torch.cuda.synchronize()
+        check_packed(out, ref, M, K, p)
+        want = stats.accumulate(stats.accumulate(stats.new_state(K), Xprev), X, stride)
+        got = _state_np(state)
+        assert got["n"] == want["n"] and got["flags"] == want["flags"] == 0, rep
+        assert np.array_equal(got["s1"], want["s1"]) and np.array_equal(got["s2"], want["s2"]), rep
+        assert np.array_equal(got["amax"], want["amax"]), rep
+
+
+def test_quantize_splice_stats_range_flag_and_outliers():
+    """Elements at and past the statistics range (|x| >= 2^15) raise the flag and add nothing to the
+    moments, values just below it are counted; the quantised operand is unaffected by the flag."""
+    K, M = 512, 64
+    X, T, P, st = _prep_inputs(3, M, K, 16, "bf16")
+    x = nvfp4.bf16_bits(X)
+    x[5, 7] = 0x4700                                                     # 2^15: out of range
+    x[9, 100] = 0xC700                                                   # -2^15
+    x[10, 101] = 0x46FF                                                  # just below 2^15: counted
+    X = nvfp4.bf16_value(x)
+    gA = stats.next_gain(stats.accumulate(stats.new_state(K), X), P)
+    state = F.StatsState(1, K)
+    out = F.fs_quantize_splice_stats(bf16_tensor(x), mask_tensor(stats.protect_mask(P, K)), 16,
+                                     torch.tensor([float(gA)], device="cuda"), state)
+    want = stats.accumulate(stats.new_state(K), X)
+    got = _state_np(state)
+    assert got["flags"] == want["flags"] == 1
+    assert np.array_equal(got["s1"], want["s1"]) and np.array_equal(got["s2"], want["s2"])
+    assert np.array_equal(got["amax"], want["amax"])
+    check_packed(out, splice.quantize_splice(X, P, gA), M, K, 16)
+
+
 def test_quantize_every_scale_code_and_rounding_boundary():
     """Blocks built so that every normal UE4M3 scale is hit and elements sit on E2M1 midpoints +-1 ulp."""
     mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.0, 6.5, 0.1, 0.0], np.float32)
@@ -169,6 +219,22 @@ def test_prepare_weights_bit_exact(dtype, N, K, p, opts):
     out, gW, alpha = F.fs_prepare_weights(Wt, mask_tensor(stats.protect_mask(P, K)), p,
                                           torch.tensor([float(gA)], device="cuda"), opts=opts)
     ref = splice.prepare_weights(W, P, gA, splice.RESIDUAL if residual else splice.SPLIT, exact_gain=exact)
+    assert gW.item() == float(ref["gW"]) and alpha.item() == float(ref["alpha"])
+    check_packed(out, ref, N, K, p)
+
+
+def test_exact_gain_saturates_for_subnormal_weights():
+    """FS_GAIN_EXACT on weights whose largest magnitude is subnormal: fl32(2688/amax) overflows and
+    the gain saturates to the largest finite float32; codes, scales and side columns stay bit-exact."""
+    N, K, p = 256, 512, 16
+    _, _, P, st = _prep_inputs(5, 64, K, p, "bf16")
+    w = (synth.gaussian_weights(13, N, K, as_bf16=False) * np.float32(2.0 ** -130)).astype(np.float32)
+    assert 0 < np.abs(w).max() < np.finfo(np.float32).tiny
+    gA = np.float32(2.0 ** -100)
+    out, gW, alpha = F.fs_prepare_weights(f32_tensor(w), mask_tensor(stats.protect_mask(P, K)), p,
+                                          torch.tensor([float(gA)], device="cuda"), opts=F.FS_GAIN_EXACT)
+    ref = splice.prepare_weights(w, P, gA, exact_gain=True)
+    assert float(ref["gW"]) == float(np.finfo(np.float32).max)
     assert gW.item() == float(ref["gW"]) and alpha.item() == float(ref["alpha"])
     check_packed(out, ref, N, K, p)
 

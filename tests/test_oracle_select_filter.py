@@ -190,6 +190,23 @@ def test_group_advantage_and_original_denominator():
     assert r2["adv"].tolist() == [0, 0, 2, 3, 4, 5, 6, 7]
 
 
-def test_default_K1_reading():
-    """K1 = 0.01 x output_len with output_len the response-length limit: 4096 -> ceil(40.96) = 41."""
-    assert math.ceil(0.01 * 4096) == 41
+def test_gates_at_the_rollout_defaults():
+    """§4.1: G1 drops a trajectory with AT LEAST K1 tail tokens, G2 one with AT LEAST K2
+    consecutive ones (Eq. 3 keeps count < K1 and run < K2).  At the rollout defaults (K1 = 41 for a
+    4096-token response limit, K2 = 5) a sequence with 40 isolated tail tokens and runs of 4 is kept;
+    one more isolated tail token, or one run of 5, drops it."""
+    lt = np.float32(-9.0)
+    T = 4096
+
+    def seq(isolated, run):
+        lp = np.full(T, np.float32(-0.5))
+        lp[np.arange(isolated) * 50] = -20                 # isolated tails, 49 normal tokens apart
+        if run:
+            lp[3000:3000 + run] = -20
+        return lp
+
+    batch = np.stack([seq(40, 0), seq(41, 0), seq(36, 4), seq(36, 5), seq(0, 4), seq(0, 5)])
+    r = seqfilter.seq_filter(batch, None, lt, K1=41, K2=5)
+    assert r["tail_count"].tolist() == [40, 41, 40, 41, 4, 5]
+    assert r["max_run"].tolist() == [1, 1, 4, 5, 4, 5]
+    assert r["keep"].tolist() == [1, 0, 1, 0, 1, 0]
