@@ -148,9 +148,20 @@ def make_weights(N, K, seed, device):
 class PrefillLayer:
     """Buffers and launches of one per-step pass over a Qwen3-8B layer."""
 
-    def __init__(self, F, M, p, seed, device, out_bf16=False, fused=True):
+    def __init__(self, F, M, p, seed, device, out_bf16=False, fused=True, compact=False, fused_prep=False):
         import torch
         self.F, self.M, self.p, self.fused = F, M, p, fused
+        # fused_prep: the paper's order within a step -- reselect from the moments gathered during
+        # the previous step, pre-split the weights, then one pass over X that quantises with the
+        # new set and gathers the moments for the next step (fs_quantize_splice_stats); otherwise
+        # statistics, reselection, pre-split and quantise run as four separate passes
+        self.fused_prep = fused_prep and not compact
+        self.PHASES = (("select", "prepare_weights", "quantize_stats", "gemm") if self.fused_prep
+                       else ("stats", "select", "prepare_weights", "quantize", "gemm"))
+        # compacted-K operands (FS_COMPACT_K): the NVFP4 operands hold the K - p unprotected
+        # channels, padded to a multiple of 256; the GEMMs run with K = that width
+        self.qopts = F.FS_COMPACT_K if compact else 0
+        self.KQ = [F.compact_cols(K, p) if compact else K for K in GROUP_K]
         self.X = [make_activations(M, K, seed * 100 + i, device) for i, K in enumerate(GROUP_K)]
         self.W = [make_weights(N, K, seed * 100 + 10 + j, device) for j, (_, N, K, _) in enumerate(PROJ)]
         self.st4 = F.StatsState(3, 4096, device=device)
@@ -161,7 +172,7 @@ class PrefillLayer:
         self.P12 = torch.empty(1, max(p, 1), dtype=torch.int32, device=device)[:, :p]
         self.m12 = torch.empty(1, 384, dtype=torch.int32, device=device)
         self.g12 = torch.empty(1, dtype=torch.float32, device=device)
-        self.xq = [F.alloc_packed(M, K, p, device) for K in GROUP_K]
+        self.xq = [F.alloc_packed(M, Kq, p, device) for Kq in self.KQ]
         self.gW = torch.empty(len(PROJ), dtype=torch.float32, device=device)
         self.alpha = torch.empty(len(PROJ), dtype=torch.float32, device=device)   # PROJ order: a group's are adjacent
         popts = F.FS_OUT_BF16 if out_bf16 else 0
@@ -171,16 +182,16 @@ class PrefillLayer:
             self.wq, self.wq_group, self.seg = [None] * len(PROJ), [], []
             for gi, js in enumerate(GROUP_PROJ):
                 rows = [PROJ[j][1] for j in js]
-                allp, views = F.stacked_packed(rows, GROUP_K[gi], p, device)
+                allp, views = F.stacked_packed(rows, self.KQ[gi], p, device)
                 self.wq_group.append(allp)
                 for j, v in zip(js, views):
                     self.wq[j] = v
                 self.seg.append([0] + [sum(rows[:i + 1]) for i in range(len(rows))])
-            self.plans = [F.Plan(self.seg[gi][-1], GROUP_K[gi], max(p, 1), popts) for gi in range(4)]
+            self.plans = [F.Plan(self.seg[gi][-1], self.KQ[gi], max(p, 1), popts) for gi in range(4)]
             self.Y = [torch.empty(M, self.seg[gi][-1], dtype=dt, device=device) for gi in range(4)]
         else:
-            self.wq = [F.alloc_packed(N, K, p, device) for (_, N, K, _) in PROJ]
-            self.plans = [F.Plan(N, K, max(p, 1), popts) for (_, N, K, _) in PROJ]
+            self.wq = [F.alloc_packed(N, self.KQ[gi], p, device) for (_, N, K, gi) in PROJ]
+            self.plans = [F.Plan(N, self.KQ[gi], max(p, 1), popts) for (_, N, K, gi) in PROJ]
             self.Y = [torch.empty(M, N, dtype=dt, device=device) for (_, N, K, _) in PROJ]
         self.flops = sum(2.0 * M * N * K for (_, N, K, _) in PROJ)
         # per-group views for the multi-stream step (one selection problem per group)
@@ -200,14 +211,13 @@ class PrefillLayer:
         """Kernel launches of one step: statistics per group, selection (one launch per statistics
         state when serial, one per group on streams), weight pre-split = amax + gain + quantise per
         projection, activation quantise per group, the GEMMs."""
-        return 4 + (2 if serial else 4) + 3 * len(PROJ) + 4 + len(self.gemm_fns())
+        stats = 0 if self.fused_prep else 4
+        return stats + (2 if serial else 4) + 3 * len(PROJ) + 4 + len(self.gemm_fns())
 
     def mask_gain(self, gi):
         if gi < 3:
             return self.m4[gi], self.g4[gi:gi + 1]
         return self.m12[0], self.g12[0:1]
-
-    PHASES = ("stats", "select", "prepare_weights", "quantize", "gemm")
 
     def step(self, allreduce=None):
         for fn in self.phase_fns(allreduce):
@@ -218,7 +228,8 @@ class PrefillLayer:
         pre-split of its projections, activation quantise, its GEMMs."""
         F = self.F
         st, gidx = (self.st4, gi) if gi < 3 else (self.st12, 0)
-        F.fs_channel_stats(self.X[gi], st, group=gidx)
+        if not self.fused_prep:
+            F.fs_channel_stats(self.X[gi], st, group=gidx)
         if allreduce is not None:
             allreduce(self.gstate[gi])
         g = self.gstate[gi]
@@ -227,8 +238,11 @@ class PrefillLayer:
         for j, (_, N, K, pg) in enumerate(PROJ):
             if pg == gi:
                 F.fs_prepare_weights(self.W[j], mask, self.p, gA, out=self.wq[j], gW=self.gW[j:j + 1],
-                                     alpha=self.alpha[j:j + 1])
-        F.fs_quantize_splice(self.X[gi], mask, self.p, gA, out=self.xq[gi])
+                                     alpha=self.alpha[j:j + 1], opts=self.qopts)
+        if self.fused_prep:
+            F.fs_quantize_splice_stats(self.X[gi], mask, self.p, gA, st, group=gidx, out=self.xq[gi])
+        else:
+            F.fs_quantize_splice(self.X[gi], mask, self.p, gA, out=self.xq[gi], opts=self.qopts)
         for fn in self.gemm_fns(gi):
             fn()
 
@@ -264,16 +278,30 @@ class PrefillLayer:
             for j, (_, N, K, gi) in enumerate(PROJ):
                 mask, g = self.mask_gain(gi)
                 F.fs_prepare_weights(self.W[j], mask, self.p, g, out=self.wq[j], gW=self.gW[j:j + 1],
-                                     alpha=self.alpha[j:j + 1])
+                                     alpha=self.alpha[j:j + 1], opts=self.qopts)
 
         def quantize():
             for gi in range(4):
                 mask, g = self.mask_gain(gi)
-                F.fs_quantize_splice(self.X[gi], mask, self.p, g, out=self.xq[gi])
+                F.fs_quantize_splice(self.X[gi], mask, self.p, g, out=self.xq[gi], opts=self.qopts)
+
+        def quantize_stats():
+            for gi in range(4):
+                mask, g = self.mask_gain(gi)
+                st, gidx = (self.st4, gi) if gi < 3 else (self.st12, 0)
+                F.fs_quantize_splice_stats(self.X[gi], mask, self.p, g, st, group=gidx, out=self.xq[gi])
 
         def gemm():
             for fn in self.gemm_fns():
                 fn()
+        if self.fused_prep:
+            # the moments the reselection reads come from the previous step's pass
+            def select_after_exchange():
+                if allreduce is not None:
+                    allreduce(self.st4)
+                    allreduce(self.st12)
+                select()
+            return [select_after_exchange, prepare, quantize_stats, gemm]
         return [stats, select, prepare, quantize, gemm]
 
     def gemm_fns(self, group=None):
@@ -455,6 +483,55 @@ def rollout_case(F, device, reps=20):
     return res
 
 
+def training_case(F, device, reps=10):
+    """The training-side kernels: the straight-through backward of the q projection at M = 8192
+    (dX = dY W, dW = dY^T X in BF16 on the tensor-core kernel, three operand transposes), and the
+    Eq. 4 objective with gradient and the K3 metric over 1024 x 4096 fp32 log-probs."""
+    import numpy as np
+    import torch
+    out = {}
+    M, N, K = M_PREFILL, 4096, 4096
+    g = torch.Generator(device=device).manual_seed(77)
+    dY = (torch.randn(M, N, generator=g, device=device) * 1e-3).to(torch.bfloat16)
+    X = make_activations(M, K, 78, device)
+    W = make_weights(N, K, 79, device)
+    plan = F.Plan(256, 256, 1)
+    work = torch.empty(F.load().fs_ste_backward_work_bytes(M, N, K), dtype=torch.uint8, device=device)
+    dX = torch.empty(M, K, device=device)
+    dW = torch.empty(N, K, device=device)
+    run = lambda: F.fs_ste_backward(plan, dY, X, W, work=work, dX=dX, dW=dW)
+    gr = capture(run)
+    for _ in range(3):
+        gr.replay()
+    ms = timed(gr.replay, reps) / reps
+    flops = 2 * 2.0 * M * N * K
+    out["ste_backward_q"] = {"us": ms * 1000.0, "TFLOPs": flops / (ms * 1e-3) / 1e12, "M": M, "N": N, "K": K}
+    gg = capture(lambda: F.fs_gemm_bf16(plan, dY, W, Y=dX))        # one GEMM alone (W untransposed: timing only)
+    for _ in range(3):
+        gg.replay()
+    ms = timed(gg.replay, reps) / reps
+    out["gemm_bf16_8192x4096x4096"] = {"us": ms * 1000.0, "TFLOPs": 2.0 * M * N * K / (ms * 1e-3) / 1e12}
+    plan.check()
+    del gr, gg, work, dX, dW, dY, X, W
+    S, T = 1024, 4096
+    rng = np.random.default_rng(5)
+    lo = torch.from_numpy((-rng.exponential(0.5, (S, T))).astype(np.float32)).to(device)
+    lp = lo + torch.randn(S, T, generator=g, device=device) * 0.1
+    adv = torch.randn(S, generator=g, device=device)
+    lengths = torch.full((S,), T, dtype=torch.int32, device=device)
+    gobj = capture(lambda: F.fs_grpo_objective(lp, lo, adv, 0.2, lengths=lengths))
+    for _ in range(3):
+        gobj.replay()
+    ms = timed(gobj.replay, reps) / reps
+    out["grpo_objective"] = {"us": ms * 1000.0, "GBps": 12.0 * S * T / (ms * 1e-3) / 1e9, "S": S, "T": T}
+    gk3 = capture(lambda: F.fs_k3_kl(lp, lo, lengths=lengths))
+    for _ in range(3):
+        gk3.replay()
+    ms = timed(gk3.replay, reps) / reps
+    out["k3_kl"] = {"us": ms * 1000.0, "GBps": 8.0 * S * T / (ms * 1e-3) / 1e9, "S": S, "T": T}
+    return out
+
+
 def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20, fused=True):
     """Decode GEMMs over `layers` distinct layers' weights (larger than L2 together), M tokens per
     layer: one segmented launch per input group (fused) or one launch per projection."""
@@ -543,18 +620,21 @@ def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20, fus
 
 
 def side_slice_bound(p):
-    """Lower bound of the GEMM time added by p protected channels: the BF16 slice's 2*M*N*Pp flops
-    at a quarter of the NVFP4 rate, against the step's 2*M*N*K NVFP4 flops (4*Pp/K per projection,
-    weighted by N*K over the layer)."""
+    """Tensor time of the BF16 slice relative to the NVFP4 product when both run at their peak
+    rates: 2*M*N*Pp flops at a quarter of the NVFP4 rate against 2*M*N*K (4*Pp/K per projection,
+    weighted by N*K over the layer).  A kernel whose NVFP4 part runs below peak pays less than this
+    in relative terms, since its BF16 slice is the smaller share of a longer loop."""
     pp = (p + 15) // 16 * 16
     return sum(4.0 * N * pp for _, N, K, _ in PROJ) / sum(float(N) * K for _, N, K, _ in PROJ)
 
 
-def p_variant(F, p, device, streams, args, rank):
-    """The timed step and its GEMMs at another protected-channel count p: step time (one graph
-    replay, captured as the main step) and the sum of the GEMM launches' times."""
+def p_variant(F, p, device, streams, args, rank, compact=False):
+    """The timed step and its GEMMs at another protected-channel count p (compact: the
+    compacted-K operands): step time (one graph replay, captured as the main step) and the sum of
+    the GEMM launches' times."""
     import torch
-    lay = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device, fused=not args.unfused)
+    lay = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device, fused=not args.unfused, compact=compact,
+                       fused_prep=args.prep == "fused")
     for _ in range(3):
         lay.step()
     gs = capture(lay.step if args.serial else (lambda: lay.step_streams(streams)))
@@ -751,6 +831,10 @@ def main():
     ap.add_argument("--shape", default="q", choices=[name for name, _, _, _ in PROJ] + list(GROUP_NAMES[::2]),
                     help="projection shape of --case gemm / decode")
     ap.add_argument("--decode-m", type=int, default=16, help="tokens of --case decode (1..16)")
+    ap.add_argument("--prep", default="fused", choices=["fused", "separate"],
+                    help="fused: reselect from the previous step's moments, then one pass over X for the "
+                         "quantise and the next moments (fs_quantize_splice_stats); separate: statistics, "
+                         "reselection and quantise as their own passes")
     ap.add_argument("--unfused", action="store_true",
                     help="one GEMM launch per projection instead of one segmented launch per input group")
     args = ap.parse_args()
@@ -781,7 +865,8 @@ def main():
     if args.case != "step":
         return kernel_case(F, args, device)
 
-    layer = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device, fused=not args.unfused)
+    layer = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device, fused=not args.unfused,
+                         fused_prep=args.prep == "fused")
     allreduce = stats_allreduce_fn(dist) if use_dist else None
     for _ in range(args.warmup):
         layer.step(allreduce)
@@ -810,7 +895,7 @@ def main():
 
     phase_graphs = [capture(fn) for fn in layer.phase_fns(allreduce)]
     gemm_graphs = [capture(fn) for fn in layer.gemm_fns()]
-    phase_us = {name: 0.0 for name in PrefillLayer.PHASES}
+    phase_us = {name: 0.0 for name in layer.PHASES}
     gemm_names = layer.gemm_names()
     gemm_ms = [[0.0] * len(gemm_names) for _ in range(args.steps)]
     for it_ in range(args.steps):
@@ -822,7 +907,7 @@ def main():
         for g_ in gemm_graphs:
             g_.replay(); evs[k].record(); k += 1
         torch.cuda.synchronize()
-        for i, name in enumerate(PrefillLayer.PHASES[:-1]):
+        for i, name in enumerate(layer.PHASES[:-1]):
             phase_us[name] += evs[i].elapsed_time(evs[i + 1]) * 1000.0 / args.steps
         base = len(phase_graphs) - 1
         for j in range(len(gemm_names)):
@@ -839,7 +924,8 @@ def main():
     # through the library calls and copies all outputs back.  Two buffer sets alternate so that
     # the host->device copy of step i+1, the step i itself and the device->host copy of step i-1
     # run at once on three streams (the copies use the two DMA directions).
-    layer2 = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device, fused=not args.unfused)
+    layer2 = PrefillLayer(F, M_PREFILL, p, seed=2 + rank, device=device, fused=not args.unfused,
+                          fused_prep=args.prep == "fused")
     sets = [layer, layer2]
     host_x = [x.cpu().pin_memory() for x in layer.X]
     host_y = [[torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in L.Y] for L in sets]
@@ -899,7 +985,8 @@ def main():
         "config": {"workload": "Qwen3-8B-shaped prefill layer: M=8192 bf16 tokens (8x1024), 7 projections, P=64; "
                                "per step stats + top-64 reselect + weight pre-split + quantise + SpliceGEMM",
                    "global_batch": world * M_PREFILL, "seq_len": 1024, "parallelism": f"dp{world}",
-                   "p": p, "l2": "inputs larger than L2 (0.85 GB of bf16 activations and weights per step)"},
+                   "p": p, "prep": args.prep,
+                   "l2": "inputs larger than L2 (0.85 GB of bf16 activations and weights per step)"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_STEP[fkey],
                      "traffic_unit": f"DRAM bytes per step (the {len(gemm_names)} GEMM launches; ncu "
@@ -940,8 +1027,13 @@ def main():
                                   "gemm_tflops_p0": s0["gemm_tflops"]}
         line["p_sweep"] = {str(pv): {**r, "step_overhead_vs_p0": r["step_ms"] / s0["step_ms"] - 1.0,
                                      "gemm_overhead_vs_p0": r["gemm_ms"] / s0["gemm_ms"] - 1.0,
-                                     "gemm_overhead_lower_bound": side_slice_bound(pv)}
+                                     "side_slice_tensor_time": side_slice_bound(pv)}
                            for pv, r in sorted(sweep.items())}
+        # compacted-K operands at P = 256 (whole k-tiles of NVFP4 work removed)
+        rc = p_variant(F, 256, device, streams, args, rank, compact=True)
+        line["p_sweep"]["256_compact_k"] = {**rc, "step_overhead_vs_p0": rc["step_ms"] / s0["step_ms"] - 1.0,
+                                            "gemm_overhead_vs_p0": rc["gemm_ms"] / s0["gemm_ms"] - 1.0}
+        torch.cuda.empty_cache()
         dec, wbytes = decode_sweep(F, p, device, fused=not args.unfused)
         dec0, wbytes0 = decode_sweep(F, 0, device, Ms=(16,), fused=not args.unfused)
         hbm = peaks["hbm_gbs"]
@@ -963,6 +1055,13 @@ def main():
         for nm in ("stats", "filter"):
             ro[nm]["frac_hbm"] = ro[nm]["GBps"] / hbm
         line["rollout"] = ro
+        torch.cuda.empty_cache()
+        tr = training_case(F, device)
+        for nm in ("ste_backward_q", "gemm_bf16_8192x4096x4096"):
+            tr[nm]["frac_bf16_peak"] = tr[nm]["TFLOPs"] / peaks["bf16_tflops"]
+        for nm in ("grpo_objective", "k3_kl"):
+            tr[nm]["frac_hbm"] = tr[nm]["GBps"] / hbm
+        line["training"] = tr
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

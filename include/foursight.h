@@ -75,6 +75,7 @@ enum {
   FS_OUT_BF16 = 1u << 3,   /* fs_splice_gemm writes bf16 Y instead of fp32 */
   FS_PATH_TENSOR = 1u << 4, /* plan option: always use the tcgen05 tensor-core kernel */
   FS_PATH_DECODE = 1u << 5, /* plan option: always use the weight-streaming decode kernel (M <= 16) */
+  FS_COMPACT_K = 1u << 7,   /* fs_quantize_splice / fs_prepare_weights: compacted-K operand (below) */
   FS_FAULT_NO_COPIES = 1u << 6 /* plan (and fs_splice_gemm_noalloc) option for tests of failure detection:
                               the GEMM kernels' producers issue no copies and every bounded wait is
                               limited to 20 ms, so each launch gives up its waits, takes its abort path
@@ -91,6 +92,14 @@ const char* fs_version(void);
 
 /* Pp = roundup(p, 16): the column count of the packed side buffers. */
 int32_t fs_side_cols(int32_t p);
+/* Kc = roundup(K - p, 256): the columns of a compacted-K NVFP4 operand (FS_COMPACT_K).  In that
+ * form the protected channels are REMOVED from the NVFP4 operand rather than zeroed in place: its
+ * columns are the K - p unprotected channels in ascending order followed by zero columns, so the
+ * 16-element blocks (and their scales) are re-formed over the unprotected channels.  Gains, side
+ * buffers and alpha are those of the split form.  A SpliceGEMM of compacted operands runs with a
+ * plan of K = Kc; it saves whole 256-wide k-tiles of NVFP4 work once p reaches 256.  The
+ * residual form cannot be compacted (FS_ERR_INVALID_ARGUMENT). */
+int32_t fs_compact_cols(int32_t K, int32_t p);
 /* Bytes of the tiled scale array for R rows and K channels. */
 int64_t fs_sf_bytes(int64_t R, int32_t K);
 
@@ -153,7 +162,7 @@ fs_status fs_select_topk(int32_t nprob, int32_t K, int64_t* n, int64_t* s1, int6
  *       FS_RESIDUAL), same rule as gA;
  *   alpha [1] float: fl32(1 / fl32(gA*gW)).
  * Protected lanes are zeroed before the block scales are computed (split form) unless
- * FS_RESIDUAL.  Block quantisation: t = fl32(fl32(a_b*g)/6), sf = UE4M3 round-to-nearest-even
+ * FS_RESIDUAL; with FS_COMPACT_K they are removed (wq [N][Kc/2], sfw fs_sf_bytes(N,Kc)).  Block quantisation: t = fl32(fl32(a_b*g)/6), sf = UE4M3 round-to-nearest-even
  * (saturating at 448), v = fl32(fl32(w*g)/sf), code = E2M1 round-to-nearest-even (saturating at
  * 6, sign kept; sf == 0 gives code 0 with the sign of w).
  * Requirements: K % 64 == 0, 0 <= p <= min(K, 256), N >= 1.
@@ -170,7 +179,8 @@ fs_status fs_prepare_weights(const void* W, int32_t dtype, int32_t N, int32_t K,
  *
  * X [M][K] (ldx, bf16 or fp32); mask/p as for fs_prepare_weights; gA: device float (frozen gain).
  * Writes xq [M][K/2], sfx (tiled, fs_sf_bytes(M,K)), xs [M][Pp] bf16 (bf16 of X_S, rounded to
- * nearest even for fp32 input).  Same block rule as fs_prepare_weights.
+ * nearest even for fp32 input).  Same block rule as fs_prepare_weights.  With FS_COMPACT_K in
+ * opts the NVFP4 operand is compacted (see fs_compact_cols): xq [M][Kc/2], sfx fs_sf_bytes(M,Kc).
  * Requirements: K % 64 == 0, M >= 0, 0 <= p <= min(K, 256).
  * ---------------------------------------------------------------------------------------- */
 fs_status fs_quantize_splice(const void* X, int32_t dtype, int64_t M, int32_t K, int64_t ldx,
@@ -211,7 +221,8 @@ int64_t fs_grouped_rows(int64_t max_rows, int32_t E);
  * protected slice accumulated into the same FP32 accumulator, scaled once by alpha.
  *
  * A plan caches the kernel choice for one weight shape (N, K, p_max) and owns a device error
- * word; creating it is the only call that allocates.  fs_plan_check synchronises `stream` and
+ * word and the decode kernel's workspace (split-tile partial sums and arrival counters, about
+ * 2.4 MB plus 16 bytes per 128 rows of N); creating it is the only call that allocates.  fs_plan_check synchronises `stream` and
  * returns FS_ERR_TIMEOUT if a kernel launched with the plan gave up a bounded wait (the word is
  * then cleared).  A plan may be used from one stream at a time.
  * ---------------------------------------------------------------------------------------- */
@@ -223,9 +234,12 @@ fs_status fs_plan_check(fs_plan plan, void* stream);
 /* Packed operands as written above (activation rows M; weight rows N = the plan's N), p <= the
  * plan's p_max; alpha: device float.  Y [M][ldy] fp32 (bf16 with FS_OUT_BF16 in the plan's
  * opts), ldy >= N, 16-byte aligned rows.  M <= 16 runs the weight-streaming decode kernel (weights
- * as the 128-row operand of tcgen05 block-scaled MMAs with the tokens as N = 16, K split over a
- * thread-block cluster), larger M the tcgen05 prefill kernel (FS_PATH_TENSOR / FS_PATH_DECODE in
- * the plan's opts force one).
+ * as the 128-row operand of tcgen05 block-scaled MMAs with the tokens as N = 16; one persistent CTA
+ * per SM takes a balanced range of the k-tiles of all output tiles, and tiles split between CTAs
+ * are summed in a fixed order through the plan's workspace), larger M the tcgen05 prefill kernel
+ * (FS_PATH_TENSOR / FS_PATH_DECODE in the plan's opts force one).  The plan's workspace makes
+ * calls with the same plan ordered on one stream; calls that overlap on the GPU need their own
+ * plans.
  * Plan requirements: N % 16 == 0 and K % 256 == 0 (FS_ERR_UNSUPPORTED otherwise); the packed
  * operands must be 16-byte aligned.  The output is not accumulated into: Y is overwritten.
  * M = 0 (an empty batch) returns FS_OK without reading any operand pointer (the plan must still
@@ -273,7 +287,9 @@ fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64_t* row_off
  * reserved at start-up, a plugin whose host forbids allocations) calls this instead: same
  * operands, same results, no plan.  Its only scratch is one 32-bit error word in a file-scope
  * __device__ array of the library (1 word, 256-byte aligned); every GPU that loads the library
- * holds it until the process exits.  No problem size needs more scratch than that; shapes beyond
+ * holds it until the process exits.  No problem size needs more scratch than that (for M <= 16 it
+ * runs the workspace-free decode kernel: K split over a thread-block cluster, partials summed
+ * through distributed shared memory); shapes beyond
  * the kernels' limits (N % 16, K % 256 or 256 <= K <= 65536, M < 2^31 - 256, p <= min(K, 256)) are
  * rejected with FS_ERR_INVALID_ARGUMENT / FS_ERR_UNSUPPORTED.
  *   N, K, opts  as for fs_plan_create (FS_OUT_BF16, FS_PATH_TENSOR, FS_PATH_DECODE apply);
@@ -311,6 +327,57 @@ fs_status fs_splice_gemm_noalloc(int32_t N, int32_t K, uint32_t opts, int64_t M,
 fs_status fs_seq_filter(const float* logp, int64_t ld, const int32_t* lengths, int32_t S, int32_t T,
                         float log_tau, int32_t K1, int32_t K2, int32_t G, const float* rewards,
                         float* adv, uint8_t* keep, int32_t* tail_count, int32_t* max_run, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Training side — FourSight §5.2 "System Implementation" (backward passes run in BF16 with the
+ * straight-through estimator), §4.1 Eq. 4 (GRPO objective with filtered advantages and the original
+ * 1/G denominator) and §6.1 (TIM measured by sampled K3 estimates of the KL divergence).
+ * ---------------------------------------------------------------------------------------- */
+
+/* Y [M][N] = alpha * A [M][K] . B [N][K]^T with BF16 operands (row-major, K contiguous, leading
+ * dimensions lda/ldb in elements, 16-byte aligned rows) and FP32 accumulation on the tcgen05
+ * kernel of fs_splice_gemm (every k-tile through its BF16 path).  alpha: device float or NULL
+ * (1).  The plan supplies only the error word and FS_OUT_BF16 / FS_FAULT_NO_COPIES (its N and K
+ * are not used).  Requirements: N % 16 == 0, K >= 1, M < 2^31 - 256. */
+fs_status fs_gemm_bf16(fs_plan plan, int64_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda,
+                       const uint16_t* B, int64_t ldb, const float* alpha, void* Y, int64_t ldy, void* stream);
+
+/* dst [C][ldd] = src [R][lds]^T for bf16 matrices (16-byte vector accesses when both are 16-byte
+ * aligned with ld % 8 == 0). */
+fs_status fs_transpose_bf16(int64_t R, int64_t C, const uint16_t* src, int64_t lds, uint16_t* dst, int64_t ldd,
+                            void* stream);
+
+/* Straight-through backward of Y = SpliceGEMM(X, W): the quantiser's Jacobian is taken as the
+ * identity, so the gradients use the BF16 operands:  dX [M][K] = dY [M][N] . W [N][K]  and
+ * dW [N][K] = dY^T . X [M][K], FP32 accumulation, FP32 outputs (bf16 with FS_OUT_BF16 in the plan).
+ * dY, X, W bf16 row-major with leading dimensions in elements.  work: device scratch of
+ * fs_ste_backward_work_bytes(M, N, K) bytes, 256-byte aligned (the transposes dY^T, X^T, W^T).
+ * Requirements: N, K multiples of 16, M <= 2^24.  Two fs_gemm_bf16 launches and three transposes. */
+int64_t fs_ste_backward_work_bytes(int64_t M, int32_t N, int32_t K);
+fs_status fs_ste_backward(fs_plan plan, int64_t M, int32_t N, int32_t K, const uint16_t* dY, int64_t lddy,
+                          const uint16_t* X, int64_t ldx, const uint16_t* W, int64_t ldw, void* work,
+                          int64_t work_bytes, void* dX, int64_t lddx, void* dW, int64_t lddw, void* stream);
+
+/* GRPO objective of Eq. 4 with the advantages A'_i already filtered (fs_seq_filter's adv: f_i A_i):
+ *   rho_it = exp(logp_it - logp_old_it),  l_it = min(rho A', clip(rho, 1 - eps, 1 + eps) A'),
+ *   seq_obj [S] = (1/|y_i|) sum_{t < |y_i|} l_it   (|y_i| = lengths[i], or T when lengths == NULL),
+ *   J (optional, device float) = (1/S) sum_i seq_obj_i: the mean over groups of (1/G) sum over the
+ *     group, so a dropped sequence still counts in the denominator (the original 1/G),
+ *   grad [S][ldg] (optional) = dJ/dlogp_it = rho A' / (S |y_i|) where the unclipped term is the
+ *     minimum (rho A' <= clip(rho) A'), else 0; positions >= |y_i| get 0.
+ * logp, logp_old: fp32 [S][ld].  Sums run in float64 in a fixed order (reproducible).
+ * Requirements: 0 <= eps < 1, ld >= T. */
+fs_status fs_grpo_objective(const float* logp, const float* logp_old, int64_t ld, const int32_t* lengths,
+                            int32_t S, int32_t T, const float* adv, float eps, float* seq_obj, float* J,
+                            float* grad, int64_t ldg, void* stream);
+
+/* TIM metric: per token d = logp_train - logp_rollout (fp32 [S][ld], tokens sampled by the rollout
+ * engine) and k3 = exp(d) - 1 - d >= 0, the K3 estimate of KL(pi_rollout || pi_train).
+ * seq_k3 [S]: mean over each sequence's tokens (0 for an empty one); batch_k3 (optional, device
+ * float): mean over all tokens of the batch, which needs work of fs_k3_work_bytes(S) bytes. */
+int64_t fs_k3_work_bytes(int32_t S);
+fs_status fs_k3_kl(const float* logp_train, const float* logp_roll, int64_t ld, const int32_t* lengths, int32_t S,
+                   int32_t T, float* seq_k3, float* batch_k3, void* work, void* stream);
 
 #ifdef __cplusplus
 }

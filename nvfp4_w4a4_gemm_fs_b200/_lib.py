@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(HERE, "libfoursight.so")
 FS_OK, FS_ERR_INVALID_ARGUMENT, FS_ERR_UNSUPPORTED, FS_ERR_CUDA, FS_ERR_RANGE, FS_ERR_TIMEOUT = range(6)
 FS_DTYPE_BF16, FS_DTYPE_F32 = 0, 1
 FS_RESIDUAL, FS_KEY_M2, FS_GAIN_EXACT, FS_OUT_BF16, FS_PATH_TENSOR, FS_PATH_DECODE = 1, 2, 4, 8, 16, 32
-FS_FAULT_NO_COPIES = 64
+FS_FAULT_NO_COPIES, FS_COMPACT_K = 64, 128
 
 P = C.c_void_p
 i32, i64, u32, f32 = C.c_int32, C.c_int64, C.c_uint32, C.c_float
@@ -25,6 +25,7 @@ SIGNATURES = {
     "fs_last_error": (C.c_char_p, []),
     "fs_version": (C.c_char_p, []),
     "fs_side_cols": (i32, [i32]),
+    "fs_compact_cols": (i32, [i32, i32]),
     "fs_sf_bytes": (i64, [i64, i32]),
     "fs_grouped_rows": (i64, [i64, i32]),
     "fs_channel_stats": (C.c_int, [P, i32, i64, i32, i64, i32, P, P, P, P, P, P]),
@@ -42,6 +43,13 @@ SIGNATURES = {
     "fs_splice_gemm_grouped": (C.c_int, [P, i32, P, i64, i32, P, P, P, P, P, P, P, P, i64, P]),
     "fs_seq_filter": (C.c_int, [P, i64, P, i32, i32, f32, i32, i32, i32, P, P, P, P, P, P]),
     "fs_splice_gemm_noalloc": (C.c_int, [i32, i32, u32, i64, i32, P, P, P, P, P, P, P, P, i64, i32, P]),
+    "fs_gemm_bf16": (C.c_int, [P, i64, i32, i32, P, i64, P, i64, P, P, i64, P]),
+    "fs_transpose_bf16": (C.c_int, [i64, i64, P, i64, P, i64, P]),
+    "fs_ste_backward_work_bytes": (i64, [i64, i32, i32]),
+    "fs_ste_backward": (C.c_int, [P, i64, i32, i32, P, i64, P, i64, P, i64, P, i64, P, i64, P, i64, P]),
+    "fs_grpo_objective": (C.c_int, [P, P, i64, P, i32, i32, P, f32, P, P, P, i64, P]),
+    "fs_k3_work_bytes": (i64, [i32]),
+    "fs_k3_kl": (C.c_int, [P, P, i64, P, i32, i32, P, P, P, P]),
 }
 
 _lib = None

@@ -9,6 +9,8 @@ struct fs_plan_s {
   uint32_t opts;
   uint32_t* err;      // device error word (bounded-wait timeouts)
   int device;
+  void* ws;           // decode workspace: split-tile partials and their arrival counters
+  int64_t ws_bytes;
 };
 
 using namespace fs;
@@ -42,12 +44,16 @@ extern "C" fs_status fs_plan_create(fs_plan* out, int32_t N, int32_t K, int32_t 
   if (K < 256 || K % 256 != 0 || K > 65536) return fail(FS_ERR_UNSUPPORTED, "fs_plan_create: need K %% 256 == 0, 256 <= K <= 65536 (K=%d)", K);
   if (p_max < 0 || p_max > 256 || p_max > K) return fail(FS_ERR_INVALID_ARGUMENT, "fs_plan_create: need 0 <= p_max <= min(K, 256)");
   if ((opts & kPathMask) == kPathMask) return fail(FS_ERR_INVALID_ARGUMENT, "fs_plan_create: FS_PATH_TENSOR and FS_PATH_DECODE are exclusive");
-  auto* pl = new fs_plan_s{N, K, p_max, opts, nullptr, 0};
+  auto* pl = new fs_plan_s{N, K, p_max, opts, nullptr, 0, nullptr, 0};
   cudaGetDevice(&pl->device);
+  pl->ws_bytes = decode_sk_workspace_bytes(N);
   cudaError_t e = cudaMalloc(&pl->err, sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(pl->err, 0, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMalloc(&pl->ws, pl->ws_bytes);
+  if (e == cudaSuccess) e = cudaMemset(pl->ws, 0, pl->ws_bytes);
   if (e != cudaSuccess) {
     if (pl->err) cudaFree(pl->err);
+    if (pl->ws) cudaFree(pl->ws);
     delete pl;
     return cuda_status(e, "fs_plan_create");
   }
@@ -58,6 +64,7 @@ extern "C" fs_status fs_plan_create(fs_plan* out, int32_t N, int32_t K, int32_t 
 extern "C" fs_status fs_plan_destroy(fs_plan plan) {
   if (!plan) return FS_OK;
   cudaFree(plan->err);
+  cudaFree(plan->ws);
   delete plan;
   return FS_OK;
 }
@@ -70,7 +77,9 @@ extern "C" fs_status fs_plan_check(fs_plan plan, void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_status(e, "fs_plan_check");
   if (w) {
+    // an aborted decode launch may leave split-tile arrival counters behind: clear them too
     cudaMemsetAsync(plan->err, 0, sizeof(uint32_t), s);
+    cudaMemsetAsync(plan->ws, 0, plan->ws_bytes, s);
     cudaStreamSynchronize(s);
     return fail(FS_ERR_TIMEOUT, "a SpliceGEMM kernel gave up a bounded wait (error word 0x%x)", w);
   }
@@ -98,7 +107,7 @@ fs_status splice_gemm(const char* who, fs_plan plan, int64_t M, int32_t p, const
     d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha; d.seg = seg;
     d.Y = Y; d.ldy = ldy; d.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; d.err = plan->err;
     d.wait_ns = wait_limit_ns(plan->opts); d.no_copies = (plan->opts & FS_FAULT_NO_COPIES) ? 1 : 0;
-    return launch_splice_gemm_decode_tc(d, s);
+    return launch_splice_gemm_decode_sk(d, plan->ws, plan->ws_bytes, s);
   }
   if (M > (int64_t{1} << 31) - 256) return fail(FS_ERR_UNSUPPORTED, "%s: M too large", who);
   TcParams prm{};
@@ -180,4 +189,81 @@ extern "C" fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64
   L.bn = (plan->N % 256 == 0) ? 256 : 128;
   L.max_tiles = ceil_div(a_rows, 128) * (plan->N / L.bn);
   return launch_splice_gemm_tc(L, prm, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------------------------------
+// BF16 GEMM on the same tensor-core kernel: no NVFP4 k-tiles, every k-tile through the BF16
+// path that carries the protected slice of a SpliceGEMM (kind::f16 MMAs, FP32 accumulation in
+// TMEM).  Used by the straight-through backward of FourSight §5.2 ("backward passes run in BF16
+// with STE").
+// ------------------------------------------------------------------------------------------
+namespace fs {
+
+fs_status gemm_bf16(const char* who, fs_plan plan, int64_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda,
+                    const uint16_t* B, int64_t ldb, const float* alpha, void* Y, int64_t ldy, cudaStream_t s) {
+  if (!plan) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null plan", who);
+  if (M < 0 || N < 16 || N % 16 != 0 || K < 1)
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: need M >= 0, N %% 16 == 0 (N >= 16), K >= 1", who);
+  if (M == 0) return FS_OK;
+  if (M > (int64_t{1} << 31) - 256 || K > (1 << 24)) return fail(FS_ERR_UNSUPPORTED, "%s: problem too large", who);
+  if (!A || !B || !Y) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null pointer", who);
+  if (lda < K || ldb < K || lda % 8 != 0 || ldb % 8 != 0 || !aligned(A, 16) || !aligned(B, 16))
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: A and B need 16-byte aligned rows with ld >= K", who);
+  const bool bf16 = plan->opts & FS_OUT_BF16;
+  if (ldy < N || !aligned(Y, 16) || (ldy % (bf16 ? 8 : 4)) != 0)
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: Y must be 16-byte aligned with ldy >= N and 16-byte rows", who);
+  TcParams prm{};
+  prm.M = M; prm.N = N; prm.K = 0; prm.KT = 0; prm.ST = static_cast<int>(ceil_div(K, 64));
+  prm.E = 1; prm.kb4 = 0; prm.offsets = nullptr; prm.sfa = nullptr; prm.sfb = nullptr; prm.alpha = alpha;
+  prm.seg = one_segment(N); prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = bf16 ? 1 : 0; prm.err = plan->err;
+  prm.wait_ns = wait_limit_ns(plan->opts); prm.no_copies = (plan->opts & FS_FAULT_NO_COPIES) ? 1 : 0;
+  TcLaunch L{};
+  L.xq = A; L.wq = B; L.xs = A; L.ws = B; L.a_rows = M; L.b_rows = N; L.y_rows = M; L.pp = K;
+  L.xs_ld = lda; L.ws_ld = ldb;
+  L.bn = (N % 256 == 0) ? 256 : 128;
+  L.max_tiles = ceil_div(M, 128) * ceil_div(N, L.bn);
+  return launch_splice_gemm_tc(L, prm, s);
+}
+
+}  // namespace fs
+
+extern "C" fs_status fs_gemm_bf16(fs_plan plan, int64_t M, int32_t N, int32_t K, const uint16_t* A, int64_t lda,
+                                  const uint16_t* B, int64_t ldb, const float* alpha, void* Y, int64_t ldy,
+                                  void* stream) {
+  return gemm_bf16("fs_gemm_bf16", plan, M, N, K, A, lda, B, ldb, alpha, Y, ldy, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int64_t fs_ste_backward_work_bytes(int64_t M, int32_t N, int32_t K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  const int64_t ldm = round_up(M, 8);
+  return 2 * (static_cast<int64_t>(N) * ldm + static_cast<int64_t>(K) * ldm + static_cast<int64_t>(K) * N) + 3 * 256;
+}
+
+extern "C" fs_status fs_ste_backward(fs_plan plan, int64_t M, int32_t N, int32_t K, const uint16_t* dY, int64_t lddy,
+                                     const uint16_t* X, int64_t ldx, const uint16_t* W, int64_t ldw, void* work,
+                                     int64_t work_bytes, void* dX, int64_t lddx, void* dW, int64_t lddw, void* stream) {
+  const char* who = "fs_ste_backward";
+  if (!plan) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null plan", who);
+  if (M < 0 || N < 16 || N % 16 != 0 || K < 16 || K % 16 != 0)
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: need M >= 0 and N, K multiples of 16", who);
+  if (M == 0) return FS_OK;
+  if (M > (int64_t{1} << 24)) return fail(FS_ERR_UNSUPPORTED, "%s: M > 2^24 (the reduction length of dW)", who);
+  if (!dY || !X || !W || !work || !dX || !dW) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null pointer", who);
+  if (work_bytes < fs_ste_backward_work_bytes(M, N, K) || !aligned(work, 256))
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: work must be 256-byte aligned with fs_ste_backward_work_bytes bytes", who);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t ldm = round_up(M, 8);
+  auto* base = static_cast<uint8_t*>(work);
+  auto* dYt = reinterpret_cast<uint16_t*>(base);                                            // [N][ldm]
+  auto* Xt = reinterpret_cast<uint16_t*>(base + round_up(2 * N * ldm, 256));                 // [K][ldm]
+  auto* Wt = reinterpret_cast<uint16_t*>(base + round_up(2 * N * ldm, 256) + round_up(2 * K * ldm, 256));   // [K][N]
+  fs_status st = fs_transpose_bf16(M, N, dY, lddy, dYt, ldm, stream);
+  if (st == FS_OK) st = fs_transpose_bf16(M, K, X, ldx, Xt, ldm, stream);
+  if (st == FS_OK) st = fs_transpose_bf16(N, K, W, ldw, Wt, N, stream);
+  if (st != FS_OK) return st;
+  // dX [M][K] = dY [M][N] . W [N][K]: A = dY (reduction over N), B = W^T [K][N]
+  st = gemm_bf16(who, plan, M, K, N, dY, lddy, Wt, N, nullptr, dX, lddx, s);
+  if (st != FS_OK) return st;
+  // dW [N][K] = dY^T [N][M] . X [M][K]: A = dY^T (reduction over M), B = X^T [K][M]
+  return gemm_bf16(who, plan, N, K, static_cast<int32_t>(M), dYt, ldm, Xt, ldm, nullptr, dW, lddw, s);
 }

@@ -50,7 +50,8 @@ struct TcLaunch {
   int64_t a_rows;     // rows of the activation buffers (padded rows for experts)
   int64_t b_rows;     // rows of the weight buffers (E * N for experts)
   int64_t y_rows;     // rows of Y
-  int pp;
+  int pp;               // columns of the side (BF16) operands
+  int64_t xs_ld, ws_ld; // their leading dimensions in elements (0: pp)
   int bn;
   int64_t max_tiles;
 };
@@ -85,6 +86,11 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kFaultWaitLimitNs = 20000000ull;
 inline uint64_t wait_limit_ns(uint32_t opts) { return (opts & FS_FAULT_NO_COPIES) ? kFaultWaitLimitNs : kWaitLimitNs; }
 
+// Workspace-free decode kernel (K split over a thread-block cluster, DSMEM reduction).
 fs_status launch_splice_gemm_decode_tc(const DecodeParams& p, cudaStream_t s);
+// Persistent stream-K decode kernel; needs decode_sk_workspace_bytes(N) bytes of workspace whose
+// counters are zero (the kernel leaves them zero after every completed launch).
+int64_t decode_sk_workspace_bytes(int N);
+fs_status launch_splice_gemm_decode_sk(const DecodeParams& p, void* workspace, int64_t ws_bytes, cudaStream_t s);
 
 }  // namespace fs

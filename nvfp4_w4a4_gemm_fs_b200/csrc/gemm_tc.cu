@@ -337,7 +337,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             if (!ok) break;
           } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) ptx::tc_mma_bf16<CG>(d, adesc + 2 * j, bdesc + 2 * j, idesc_bf, 1u);
+            for (int j = 0; j < 4; ++j) ptx::tc_mma_bf16<CG>(d, adesc + 2 * j, bdesc + 2 * j, idesc_bf, (kt | j) != 0);
           }
           ptx::tc_commit<CG>(empty + stage);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -423,7 +423,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       const TileMap m = map_tile<CG>(t, p, cum_m, rank);
       if (!wait_bar(acc_full + acc, acc_phase, abort_flag, p.err, p.wait_ns)) break;
       ptx::tc_fence_after();
-      const float alpha = __ldg(p.alpha + (p.offsets ? m.e : segment_of(m.n0, p.seg)));
+      const float alpha = p.alpha ? __ldg(p.alpha + (p.offsets ? m.e : segment_of(m.n0, p.seg))) : 1.0f;
       const bool use_tma = !p.offsets || (quad + 1) * 32 <= m.rows;
       const bool row_ok = row < m.rows;
       const int64_t yrow = m.yrow + row;
@@ -602,15 +602,22 @@ fs_status launch_cfg(const TcLaunch& L, TcParams prm, int units, cudaStream_t s)
   prm.n_fast = (!prm.offsets && prm.E == 1 && static_cast<int64_t>(prm.N) <= L.a_rows) ? 1 : 0;
   CUtensorMap tmA, tmB, tmSA, tmSB;
   const uint64_t kbytes = static_cast<uint64_t>(prm.K) / 2;
-  st = make_map(&tmA, L.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, L.a_rows, kbytes, 128, kBM);
-  if (st == FS_OK) st = make_map(&tmB, L.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, L.b_rows, kbytes, 128, C::B_ROWS);
-  if (st != FS_OK) return st;
+  if (prm.KT > 0) {
+    st = make_map(&tmA, L.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, L.a_rows, kbytes, 128, kBM);
+    if (st == FS_OK) st = make_map(&tmB, L.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, L.b_rows, kbytes, 128, C::B_ROWS);
+    if (st != FS_OK) return st;
+  }
   if (prm.ST > 0) {
     const uint64_t pp = static_cast<uint64_t>(L.pp);
-    st = make_map(&tmSA, L.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, L.a_rows, pp * 2, 64, kBM);
-    if (st == FS_OK) st = make_map(&tmSB, L.ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, L.b_rows, pp * 2, 64, C::B_ROWS);
+    const uint64_t lds = static_cast<uint64_t>(L.xs_ld ? L.xs_ld : L.pp), ldw = static_cast<uint64_t>(L.ws_ld ? L.ws_ld : L.pp);
+    st = make_map(&tmSA, L.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, L.a_rows, lds * 2, 64, kBM);
+    if (st == FS_OK) st = make_map(&tmSB, L.ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, L.b_rows, ldw * 2, 64, C::B_ROWS);
     if (st != FS_OK) return st;
-  } else {
+  }
+  if (prm.KT == 0) {            // BF16 only: the FP4 maps are never used for loads
+    tmA = tmSA;
+    tmB = tmSB;
+  } else if (prm.ST == 0) {
     tmSA = tmA;
     tmSB = tmB;
   }

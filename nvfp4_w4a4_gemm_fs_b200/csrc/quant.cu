@@ -13,6 +13,12 @@
 #include "common.cuh"
 
 namespace fs {
+
+// Row-streaming quantiser (quant_stats.cu) used for bf16 batches of at most kSmallBatchRows rows.
+constexpr int64_t kSmallBatchRows = 64;
+fs_status quantize_rows_bf16(const void* X, int64_t M, int32_t K, int64_t ldx, const uint32_t* mask, int32_t p,
+                             const float* gA, uint32_t opts, uint8_t* xq, uint8_t* sfx, uint16_t* xs, cudaStream_t s);
+
 namespace {
 
 constexpr int kQThreads = 256;
@@ -358,6 +364,136 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
   }
 }
 
+// Compacted-K form (FS_COMPACT_K): the NVFP4 operand holds the unprotected channels in ascending
+// order, so the 16-element blocks are re-formed over them, zero padded to Kc = roundup(K - p, 256)
+// columns; the side buffer is the same as in the split form.  One thread per (row, compacted
+// block): its 16 elements are gathered through a table of source channels built once per CTA by
+// a block-wide scan of the mask.  Same block arithmetic as quantize_kernel.
+template <typename T, Side kSide>
+__global__ void __launch_bounds__(kQThreads) quantize_compact_kernel(QuantArgs a, int Kc, int64_t rows_padded) {
+  __shared__ uint16_t sh_src[16384];                  // source channel of compacted column j
+  __shared__ uint16_t sh_pidx[256];                   // protected channels, ascending
+  __shared__ int sh_scan[kQThreads / 32][2];
+  __shared__ float sh_val[128], sh_rcp[128];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid < 128) {
+    const bool real = tid > 0 && tid < 127;
+    const float d = real ? ue4m3_value(tid) : 1.0f;
+    sh_val[tid] = d;
+    sh_rcp[tid] = real ? __frcp_rn(d) : 0.0f;
+  }
+  // channel lists: thread t scans channels [t*per, (t+1)*per); exclusive scans of both counts
+  const int per = (a.K + kQThreads - 1) / kQThreads;
+  const int c0 = tid * per, c1 = min(a.K, c0 + per);
+  auto is_prot = [&](int ch) { return a.masks && ((__ldg(a.masks + (ch >> 5)) >> (ch & 31)) & 1u); };
+  int nu = 0, np = 0;
+  for (int ch = c0; ch < c1; ++ch) { if (is_prot(ch)) ++np; else ++nu; }
+  int xu = nu, xp = np;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int yu = __shfl_up_sync(0xffffffffu, xu, o), yp = __shfl_up_sync(0xffffffffu, xp, o);
+    if (lane >= o) { xu += yu; xp += yp; }
+  }
+  if (lane == 31) { sh_scan[warp][0] = xu; sh_scan[warp][1] = xp; }
+  __syncthreads();
+  int bu = xu - nu, bp = xp - np;
+  for (int w = 0; w < warp; ++w) { bu += sh_scan[w][0]; bp += sh_scan[w][1]; }
+  for (int ch = c0; ch < c1; ++ch) {
+    if (is_prot(ch)) { if (bp < 256) sh_pidx[bp] = static_cast<uint16_t>(ch); ++bp; }
+    else sh_src[bu++] = static_cast<uint16_t>(ch);
+  }
+  __syncthreads();
+  const int nkeep = a.K - a.p;
+  const int nbc = Kc / 16;
+  const T* X = static_cast<const T*>(a.X);
+  const float g = __ldg(a.gains);
+  const bool fast = sizeof(T) == 2 && pow2_gain_in_fast_range(g);
+  const float inv6 = __frcp_rn(6.0f);
+  const int64_t items = rows_padded * nbc;          // nbc % 4 == 0: a warp's aligned groups of 4 share a row
+  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * kQThreads; i0 < items; i0 += static_cast<int64_t>(gridDim.x) * kQThreads) {
+    const int64_t i = i0 + tid;
+    const bool in_range = i < items;
+    const int64_t r = in_range ? i / nbc : 0;
+    const int jb = in_range ? static_cast<int>(i - r * nbc) : 0;
+    uint32_t sfc = 0;
+    if (in_range && r < a.rows) {
+      float x[16];
+      const T* row = X + r * a.ldx;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int jc = jb * 16 + e;
+        float v = 0.0f;
+        if (jc < nkeep) {
+          if constexpr (sizeof(T) == 2) v = __uint_as_float(static_cast<uint32_t>(__ldg(row + sh_src[jc])) << 16);
+          else v = __ldg(row + sh_src[jc]);
+        }
+        x[e] = v;
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[e]));
+      const float t = div_markstein(__fmul_rn(amax, g), 6.0f, inv6);
+      sfc = ue4m3_rne(t);
+      const float sd = sh_val[sfc], sr = sh_rcp[sfc];
+      float v[16];
+      if (fast) {
+        const float R = __fmul_rn(g, sr);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = snap12(__fmul_rn(x[e], R));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = div_markstein(__fmul_rn(x[e], g), sd, sr);
+      }
+      const uint32_t lo = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+      const uint32_t hi = e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+      *reinterpret_cast<uint2*>(a.q + r * (Kc / 2) + static_cast<int64_t>(jb) * 8) = make_uint2(lo, hi);
+    }
+    const uint32_t s1 = __shfl_down_sync(0xffffffffu, sfc, 1);
+    const uint32_t s2 = __shfl_down_sync(0xffffffffu, sfc, 2);
+    const uint32_t s3 = __shfl_down_sync(0xffffffffu, sfc, 3);
+    if (in_range && (jb & 3) == 0)
+      *reinterpret_cast<uint32_t*>(a.sf + sf_offset(r, jb, a.kb4)) = sfc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+  // side columns (as in the split form): the protected channels in ascending order, zero padded
+  if (a.pp > 0) {
+    const float alpha_v = kSide == Side::Weight ? __ldg(a.alpha) : 1.0f;
+    const int64_t sitems = a.rows * a.pp;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kQThreads + tid; i < sitems;
+         i += static_cast<int64_t>(gridDim.x) * kQThreads) {
+      const int64_t r = i / a.pp;
+      const int c = static_cast<int>(i - r * a.pp);
+      uint16_t hv = 0;
+      if (c < a.p) {
+        const T* src = X + r * a.ldx + sh_pidx[c];
+        float xv;
+        if constexpr (sizeof(T) == 2) xv = __uint_as_float(static_cast<uint32_t>(__ldg(src)) << 16);
+        else xv = __ldg(src);
+        if constexpr (kSide == Side::Activation) {
+          hv = f32_to_bf16_bits(xv);
+        } else {
+          const float wb = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_bits(xv)) << 16);
+          hv = f32_to_bf16_bits(__fdiv_rn(wb, alpha_v));
+        }
+      }
+      a.side[r * a.pp + c] = hv;
+    }
+  }
+}
+
+template <Side kSide>
+fs_status launch_quantize_compact(int dtype, QuantArgs& a, cudaStream_t s) {
+  const int Kc = static_cast<int>(round_up(a.K - a.p, 256));
+  a.kb4 = Kc / 64;
+  const int64_t rows_padded = round_up(a.rows, 128);
+  const int64_t items = rows_padded * (Kc / 16);
+  if (items == 0) return FS_OK;
+  auto kernel = dtype == FS_DTYPE_BF16 ? quantize_compact_kernel<uint16_t, kSide> : quantize_compact_kernel<float, kSide>;
+  const int64_t grid = std::min<int64_t>(ceil_div(items, kQThreads), static_cast<int64_t>(sm_count()) * 4);
+  kernel<<<static_cast<unsigned>(grid), kQThreads, 0, s>>>(a, Kc, rows_padded);
+  FS_CHECK_LAUNCH("quantize (compacted K)");
+  return FS_OK;
+}
+
 // Max |W| over the unprotected columns (all columns in the residual form) as float bits.
 // fp32 weights (small problems): one 16-element block per thread.
 __global__ void __launch_bounds__(256) weight_amax_f32_kernel(const float* __restrict__ W, int64_t N, int K, int64_t ldw,
@@ -507,14 +643,18 @@ fs_status launch_quantize(int dtype, QuantArgs& a, int64_t padded_rows, cudaStre
 
 fs_status check_common(const char* who, int32_t dtype, int32_t K, int64_t ld, const void* X, int32_t p,
                        const uint32_t* mask, const void* gain, const uint8_t* q, const uint8_t* sf,
-                       const uint16_t* side) {
+                       const uint16_t* side, uint32_t opts = 0) {
   if (dtype != FS_DTYPE_BF16 && dtype != FS_DTYPE_F32) return fail(FS_ERR_INVALID_ARGUMENT, "%s: bad dtype %d", who, dtype);
   if (K <= 0 || K % 64 != 0 || K > 16384) return fail(FS_ERR_INVALID_ARGUMENT, "%s: need K %% 64 == 0 and 0 < K <= 16384 (K=%d)", who, K);
   if (p < 0 || p > K || p > 256) return fail(FS_ERR_INVALID_ARGUMENT, "%s: need 0 <= p <= min(K,256) (p=%d)", who, p);
   const int esz = dtype == FS_DTYPE_BF16 ? 2 : 4;
   if (ld < K || (ld * esz) % 16 != 0) return fail(FS_ERR_INVALID_ARGUMENT, "%s: leading dimension must be >= K with 16-byte rows", who);
-  if (!X || !gain || !q || !sf || (p > 0 && (!mask || !side))) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null pointer", who);
-  if (!aligned(X, 16) || !aligned(q, 16) || !aligned(sf, 16) || (side && !aligned(side, 16)) || (mask && !aligned(mask, 4)))
+  // a compacted operand of no columns (FS_COMPACT_K with p == K) has no codes or scales
+  const bool need_q = !((opts & FS_COMPACT_K) && p == K);
+  if (!X || !gain || (need_q && (!q || !sf)) || (p > 0 && (!mask || !side)))
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: null pointer", who);
+  if (!aligned(X, 16) || (q && !aligned(q, 16)) || (sf && !aligned(sf, 16)) || (side && !aligned(side, 16)) ||
+      (mask && !aligned(mask, 4)))
     return fail(FS_ERR_INVALID_ARGUMENT, "%s: misaligned pointer", who);
   return FS_OK;
 }
@@ -529,12 +669,18 @@ extern "C" fs_status fs_quantize_splice(const void* X, int32_t dtype, int64_t M,
                                         uint8_t* xq, uint8_t* sfx, uint16_t* xs, void* stream) {
   if (M < 0) return fail(FS_ERR_INVALID_ARGUMENT, "fs_quantize_splice: M < 0");
   if (M == 0) return FS_OK;
-  fs_status st = check_common("fs_quantize_splice", dtype, K, ldx, X, p, mask, gA, xq, sfx, xs);
+  fs_status st = check_common("fs_quantize_splice", dtype, K, ldx, X, p, mask, gA, xq, sfx, xs, opts);
   if (st != FS_OK) return st;
   QuantArgs a{};
   a.X = X; a.ldx = ldx; a.K = K; a.nb = K / 16; a.kb4 = static_cast<int>(round_up(K / 16, 4) / 4);
   a.p = p; a.pp = side_cols(p); a.opts = opts; a.masks = mask; a.gains = gA; a.alpha = nullptr;
   a.q = xq; a.sf = sfx; a.side = xs; a.E = 1; a.offsets = nullptr; a.rows = M;
+  if (opts & FS_COMPACT_K) {
+    if (opts & FS_RESIDUAL) return fail(FS_ERR_INVALID_ARGUMENT, "fs_quantize_splice: FS_COMPACT_K excludes FS_RESIDUAL");
+    return launch_quantize_compact<Side::Activation>(dtype, a, static_cast<cudaStream_t>(stream));
+  }
+  if (dtype == FS_DTYPE_BF16 && M <= kSmallBatchRows)       // decode-sized batches
+    return quantize_rows_bf16(X, M, K, ldx, mask, p, gA, opts, xq, sfx, xs, static_cast<cudaStream_t>(stream));
   return launch_quantize<Side::Activation, false>(dtype, a, round_up(M, 128), static_cast<cudaStream_t>(stream));
 }
 
@@ -559,9 +705,11 @@ extern "C" fs_status fs_prepare_weights(const void* W, int32_t dtype, int32_t N,
                                         uint8_t* wq, uint8_t* sfw, uint16_t* ws, float* gW, float* alpha,
                                         void* stream) {
   if (N <= 0) return fail(FS_ERR_INVALID_ARGUMENT, "fs_prepare_weights: N must be >= 1");
-  fs_status st = check_common("fs_prepare_weights", dtype, K, ldw, W, p, mask, gA, wq, sfw, ws);
+  fs_status st = check_common("fs_prepare_weights", dtype, K, ldw, W, p, mask, gA, wq, sfw, ws, opts);
   if (st != FS_OK) return st;
   if (!gW || !alpha) return fail(FS_ERR_INVALID_ARGUMENT, "fs_prepare_weights: null gW/alpha");
+  if ((opts & FS_COMPACT_K) && (opts & FS_RESIDUAL))
+    return fail(FS_ERR_INVALID_ARGUMENT, "fs_prepare_weights: FS_COMPACT_K excludes FS_RESIDUAL");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(gW, 0, sizeof(float), s);
   if (e != cudaSuccess) return cuda_status(e, "fs_prepare_weights: memset");
@@ -591,5 +739,6 @@ extern "C" fs_status fs_prepare_weights(const void* W, int32_t dtype, int32_t N,
   a.X = W; a.ldx = ldw; a.K = K; a.nb = K / 16; a.kb4 = static_cast<int>(round_up(K / 16, 4) / 4);
   a.p = p; a.pp = side_cols(p); a.opts = opts; a.masks = mask; a.gains = gW; a.alpha = alpha;
   a.q = wq; a.sf = sfw; a.side = ws; a.E = 1; a.offsets = nullptr; a.rows = N;
+  if (opts & FS_COMPACT_K) return launch_quantize_compact<Side::Weight>(dtype, a, s);
   return launch_quantize<Side::Weight, false>(dtype, a, round_up(N, 128), s);
 }

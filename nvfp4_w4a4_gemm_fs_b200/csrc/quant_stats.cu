@@ -55,6 +55,7 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
   return r;
 }
 
+template <bool kStats>
 __global__ void __launch_bounds__(kQSThreads, 2) quantize_stats_kernel(const QSArgs a) {
   __shared__ unsigned long long sh_s1[kSlab];      // per channel of the slab, summed over the warps
   __shared__ unsigned long long sh_s2[kSlab];
@@ -215,6 +216,10 @@ __global__ void __launch_bounds__(kQSThreads, 2) quantize_stats_kernel(const QSA
 #pragma unroll
   for (int d = 0; d < kDepth - 1; ++d) issue(first + d * step, d);
   int slot = 0;
+  // r0 % row_stride, kept incrementally (a 64-bit division per row would dominate the loop)
+  const int64_t stride = a.row_stride;
+  int64_t mod0 = first % stride;
+  const int64_t dmod = step % stride;
   for (int64_t r0 = first; r0 < a.Mp; r0 += step) {
     issue(r0 + (kDepth - 1) * step, (slot + kDepth - 1) % kDepth);
     asm volatile("cp.async.wait_group %0;" ::"n"(kDepth - 1) : "memory");
@@ -224,9 +229,12 @@ __global__ void __launch_bounds__(kQSThreads, 2) quantize_stats_kernel(const QSA
     if (active && r1 < a.M) xb = ring[warp][slot][1][lane];
     slot = slot + 1 == kDepth ? 0 : slot + 1;
     // moments of the raw (unmasked) values of the rows the statistics take
-    const bool ta = r0 < a.M && (r0 % a.row_stride) == 0;
-    const bool tb = r1 < a.M && (r1 % a.row_stride) == 0;
-    if (active && (ta || tb)) {
+    const int64_t mod1 = mod0 + 1 == stride ? 0 : mod0 + 1;
+    const bool ta = r0 < a.M && mod0 == 0;
+    const bool tb = r1 < a.M && mod1 == 0;
+    mod0 += dmod;
+    if (mod0 >= stride) mod0 -= stride;
+    if (kStats && active && (ta || tb)) {
       const uint32_t wa[4] = {ta ? xa.x : 0u, ta ? xa.y : 0u, ta ? xa.z : 0u, ta ? xa.w : 0u};
       const uint32_t wb[4] = {tb ? xb.x : 0u, tb ? xb.y : 0u, tb ? xb.z : 0u, tb ? xb.w : 0u};
 #pragma unroll
@@ -258,6 +266,7 @@ __global__ void __launch_bounds__(kQSThreads, 2) quantize_stats_kernel(const QSA
     quantise_row(r1, xb);
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");   // nothing left in flight (all past the end)
+  if constexpr (!kStats) return;
   flush_raw();
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -281,6 +290,39 @@ __global__ void __launch_bounds__(kQSThreads, 2) quantize_stats_kernel(const QSA
 }
 
 }  // namespace
+
+// One wave: as many row groups per slab as fill the resident CTA slots, each with at least 16 row
+// pairs per warp when the batch is large enough.
+fs_status launch_quantize_rows(const QSArgs& a, bool with_stats, cudaStream_t s, const char* who) {
+  static PerDevice<int> occ;
+  int slots = 1;
+  if (!occ.get(current_device(), &slots, [](int* v) {
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, quantize_stats_kernel<true>, kQSThreads, 0) ==
+                   cudaSuccess && *v >= 1;
+      }))
+    slots = 1;
+  const int chunks = static_cast<int>(ceil_div(a.K, kSlab));
+  int64_t gy = std::max<int64_t>(1, static_cast<int64_t>(slots) * sm_count() / chunks);
+  gy = std::min<int64_t>(gy, std::max<int64_t>(1, ceil_div(a.Mp, 2 * kQSWarps * 16)));
+  gy = std::min<int64_t>(gy, 65535);
+  const dim3 grid(chunks, static_cast<unsigned>(gy));
+  if (with_stats) quantize_stats_kernel<true><<<grid, kQSThreads, 0, s>>>(a);
+  else quantize_stats_kernel<false><<<grid, kQSThreads, 0, s>>>(a);
+  FS_CHECK_LAUNCH(who);
+  return FS_OK;
+}
+
+// fs_quantize_splice for decode-sized bf16 batches: the same row-streaming kernel without the
+// moments (no per-CTA mask tables; each lane derives its protected lanes from the mask directly).
+fs_status quantize_rows_bf16(const void* X, int64_t M, int32_t K, int64_t ldx, const uint32_t* mask, int32_t p,
+                             const float* gA, uint32_t opts, uint8_t* xq, uint8_t* sfx, uint16_t* xs, cudaStream_t s) {
+  QSArgs a{};
+  a.X = static_cast<const uint16_t*>(X); a.ldx = ldx; a.M = M; a.Mp = round_up(M, 128); a.K = K;
+  a.kb4 = static_cast<int>(round_up(K / 16, 4) / 4); a.p = p; a.pp = side_cols(p); a.opts = opts;
+  a.mask = p > 0 ? mask : nullptr; a.gain = gA; a.q = xq; a.sf = sfx; a.side = xs; a.row_stride = 1;
+  return launch_quantize_rows(a, false, s, "fs_quantize_splice");
+}
+
 }  // namespace fs
 
 using namespace fs;
@@ -310,20 +352,5 @@ extern "C" fs_status fs_quantize_splice_stats(const void* X, int32_t dtype, int6
   a.mask = p > 0 ? mask : nullptr; a.gain = gA; a.q = xq; a.sf = sfx; a.side = xs; a.row_stride = row_stride;
   a.n = reinterpret_cast<unsigned long long*>(n); a.s1 = reinterpret_cast<unsigned long long*>(s1);
   a.s2 = reinterpret_cast<unsigned long long*>(s2); a.amax = amax; a.flags = flags;
-  // One wave: as many row groups per slab as fill the resident CTA slots, each with at least 16
-  // row pairs per warp when the batch is large enough.
-  static PerDevice<int> occ;
-  int slots = 1;
-  if (!occ.get(current_device(), &slots, [](int* v) {
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, quantize_stats_kernel, kQSThreads, 0) == cudaSuccess &&
-               *v >= 1;
-      }))
-    slots = 1;
-  const int chunks = static_cast<int>(ceil_div(K, kSlab));
-  int64_t gy = std::max<int64_t>(1, static_cast<int64_t>(slots) * sm_count() / chunks);
-  gy = std::min<int64_t>(gy, std::max<int64_t>(1, ceil_div(a.Mp, 2 * kQSWarps * 16)));
-  gy = std::min<int64_t>(gy, 65535);
-  quantize_stats_kernel<<<dim3(chunks, static_cast<unsigned>(gy)), kQSThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
-  FS_CHECK_LAUNCH(who);
-  return FS_OK;
+  return launch_quantize_rows(a, true, static_cast<cudaStream_t>(stream), who);
 }

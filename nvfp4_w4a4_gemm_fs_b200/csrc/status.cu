@@ -80,6 +80,10 @@ const char* fs_version(void) { return "foursight-splicegemm 0.1 (sm_100a)"; }
 
 int32_t fs_side_cols(int32_t p) { return p < 0 ? 0 : fs::side_cols(p); }
 
+int32_t fs_compact_cols(int32_t K, int32_t p) {
+  return (K < 0 || p < 0 || p > K) ? 0 : static_cast<int32_t>(fs::round_up(K - p, 256));
+}
+
 int64_t fs_sf_bytes(int64_t R, int32_t K) { return (R < 0 || K < 0) ? 0 : fs::sf_bytes(R, K); }
 
 int64_t fs_grouped_rows(int64_t max_rows, int32_t E) {

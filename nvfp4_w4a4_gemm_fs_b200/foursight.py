@@ -15,8 +15,9 @@ from ._lib import FS_DTYPE_BF16, FS_DTYPE_F32, check
 __all__ = [
     "fs_channel_stats", "fs_stats_check", "fs_select_topk", "fs_prepare_weights",
     "fs_quantize_splice", "fs_quantize_splice_grouped", "fs_quantize_splice_stats", "fs_splice_gemm", "fs_splice_gemm_grouped",
-    "fs_seq_filter", "Plan", "StatsState", "Packed", "side_cols", "sf_bytes", "grouped_rows",
-    "fs_splice_gemm_segmented", "stacked_packed",
+    "fs_seq_filter", "Plan", "StatsState", "Packed", "side_cols", "sf_bytes", "grouped_rows", "compact_cols",
+    "fs_splice_gemm_segmented", "stacked_packed", "fs_gemm_bf16", "fs_transpose_bf16", "fs_ste_backward",
+    "fs_grpo_objective", "fs_k3_kl",
     "alloc_packed", "stream_handle",
 ]
 
@@ -106,11 +107,20 @@ def fs_select_topk(state: StatsState, p: int, opts: int = 0, reset: bool = False
     return P, mask, gA
 
 
+def compact_cols(K: int, p: int) -> int:
+    return _lib.load().fs_compact_cols(K, p)
+
+
+def _packed_cols(K: int, p: int, opts: int) -> int:
+    """Columns of the NVFP4 operand: K, or the compacted width with FS_COMPACT_K."""
+    return compact_cols(K, p) if opts & _lib.FS_COMPACT_K else K
+
+
 def fs_prepare_weights(W: torch.Tensor, mask, p: int, gA: torch.Tensor, opts: int = 0, out: Packed | None = None,
                        gW=None, alpha=None, stream=None):
     lib = _lib.load()
     N, K = W.shape
-    out = alloc_packed(N, K, p, W.device) if out is None else out
+    out = alloc_packed(N, _packed_cols(K, p, opts), p, W.device) if out is None else out
     gW = torch.empty(1, dtype=torch.float32, device=W.device) if gW is None else gW
     alpha = torch.empty(1, dtype=torch.float32, device=W.device) if alpha is None else alpha
     check(lib.fs_prepare_weights(_ptr(W), _dtype_code(W), N, K, W.stride(0), _ptr(mask) if p else None, p, opts,
@@ -123,7 +133,7 @@ def fs_quantize_splice(X: torch.Tensor, mask, p: int, gA: torch.Tensor, opts: in
                        stream=None):
     lib = _lib.load()
     M, K = X.shape
-    out = alloc_packed(M, K, p, X.device) if out is None else out
+    out = alloc_packed(M, _packed_cols(K, p, opts), p, X.device) if out is None else out
     check(lib.fs_quantize_splice(_ptr(X), _dtype_code(X), M, K, X.stride(0), _ptr(mask) if p else None, p,
                                  _ptr(gA), opts, _ptr(out.q), _ptr(out.sf), _ptr(out.side) if p else None,
                                  stream_handle(stream)), "fs_quantize_splice")
@@ -259,3 +269,76 @@ def fs_seq_filter(logp: torch.Tensor, log_tau: float, K1: int, K2: int, lengths=
                             _ptr(rewards), _ptr(adv), _ptr(keep), _ptr(cnt), _ptr(run), stream_handle(stream)),
           "fs_seq_filter")
     return keep, cnt, run, adv
+
+
+# ------------------------------------------------------------------------------------------ training side
+def _bits16(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype != torch.bfloat16:
+        raise TypeError("bf16 tensor expected")
+    return t
+
+
+def fs_gemm_bf16(plan: Plan, A: torch.Tensor, B: torch.Tensor, alpha: torch.Tensor | None = None,
+                 Y: torch.Tensor | None = None, stream=None):
+    """Y [M, N] = alpha * A [M, K] @ B [N, K]^T (bf16 operands, fp32 accumulation)."""
+    lib = _lib.load()
+    M, K = A.shape
+    N = B.shape[0]
+    if Y is None:
+        dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
+        Y = torch.empty(M, N, dtype=dt, device=A.device)
+    check(lib.fs_gemm_bf16(plan.handle, M, N, K, _ptr(_bits16(A)), A.stride(0), _ptr(_bits16(B)), B.stride(0),
+                           _ptr(alpha), _ptr(Y), Y.stride(0), stream_handle(stream)), "fs_gemm_bf16")
+    return Y
+
+
+def fs_transpose_bf16(src: torch.Tensor, dst: torch.Tensor | None = None, stream=None):
+    lib = _lib.load()
+    R, C_ = src.shape
+    dst = torch.empty(C_, R, dtype=torch.bfloat16, device=src.device) if dst is None else dst
+    check(lib.fs_transpose_bf16(R, C_, _ptr(_bits16(src)), src.stride(0), _ptr(dst), dst.stride(0),
+                                stream_handle(stream)), "fs_transpose_bf16")
+    return dst
+
+
+def fs_ste_backward(plan: Plan, dY: torch.Tensor, X: torch.Tensor, W: torch.Tensor, work: torch.Tensor | None = None,
+                    dX: torch.Tensor | None = None, dW: torch.Tensor | None = None, stream=None):
+    """Straight-through backward of the SpliceGEMM forward: (dX, dW) = (dY @ W, dY^T @ X) on bf16 operands."""
+    lib = _lib.load()
+    M, N = dY.shape
+    K = X.shape[1]
+    dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
+    nbytes = lib.fs_ste_backward_work_bytes(M, N, K)
+    work = torch.empty(nbytes, dtype=torch.uint8, device=dY.device) if work is None else work
+    dX = torch.empty(M, K, dtype=dt, device=dY.device) if dX is None else dX
+    dW = torch.empty(N, K, dtype=dt, device=dY.device) if dW is None else dW
+    check(lib.fs_ste_backward(plan.handle, M, N, K, _ptr(_bits16(dY)), dY.stride(0), _ptr(_bits16(X)), X.stride(0),
+                              _ptr(_bits16(W)), W.stride(0), _ptr(work), work.numel(), _ptr(dX), dX.stride(0),
+                              _ptr(dW), dW.stride(0), stream_handle(stream)), "fs_ste_backward")
+    return dX, dW
+
+
+def fs_grpo_objective(logp: torch.Tensor, logp_old: torch.Tensor, adv: torch.Tensor, eps: float, lengths=None,
+                      with_grad: bool = True, stream=None):
+    """Eq. 4 with filtered advantages: returns (J [1], seq_obj [S], grad [S, T] or None)."""
+    lib = _lib.load()
+    S, T = logp.shape
+    seq = torch.empty(max(S, 1), dtype=torch.float32, device=logp.device)[:S]
+    J = torch.empty(1, dtype=torch.float32, device=logp.device)
+    grad = torch.empty(S, T, dtype=torch.float32, device=logp.device) if with_grad else None
+    check(lib.fs_grpo_objective(_ptr(logp), _ptr(logp_old), logp.stride(0), _ptr(lengths), S, T, _ptr(adv),
+                                float(eps), _ptr(seq), _ptr(J), _ptr(grad), grad.stride(0) if grad is not None else T,
+                                stream_handle(stream)), "fs_grpo_objective")
+    return J, seq, grad
+
+
+def fs_k3_kl(logp_train: torch.Tensor, logp_roll: torch.Tensor, lengths=None, stream=None):
+    """K3 estimates of KL(pi_rollout || pi_train): (per-sequence means [S], batch mean [1])."""
+    lib = _lib.load()
+    S, T = logp_train.shape
+    seq = torch.empty(max(S, 1), dtype=torch.float32, device=logp_train.device)[:S]
+    batch = torch.empty(1, dtype=torch.float32, device=logp_train.device)
+    work = torch.empty(max(lib.fs_k3_work_bytes(S), 8), dtype=torch.uint8, device=logp_train.device)
+    check(lib.fs_k3_kl(_ptr(logp_train), _ptr(logp_roll), logp_train.stride(0), _ptr(lengths), S, T, _ptr(seq),
+                       _ptr(batch), _ptr(work), stream_handle(stream)), "fs_k3_kl")
+    return seq, batch

@@ -14,6 +14,11 @@ Sparse Channel Compensation") computes on its data-parallel hot path:
 * ``seqfilter`` — dual-gate TIM-aware sequence filter and advantage masking
                 (§4.1 Eq. 3-4; §2.1 GRPO advantage).
 * ``bounds``  — the error-bound constants of §9.3 (Lemma 2, Lemma 3, Thm. 1).
+* ``train``   — the training side: STE backward in BF16, the Eq. 4 GRPO objective
+                with filtered advantages and its gradient, the K3 TIM metric
+                (§5.2, §4.1 Eq. 4, §6.1).
+``splice`` also holds the compacted-K variant (``COMPACT``): protected columns
+removed from the NVFP4 operand, blocks re-formed over the rest.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg may import this package.  It shares no code with the CUDA library and never
@@ -24,4 +29,4 @@ they live: the MoE routing synthesis (a workload choice, not a result) and the
 absolute accumulation error of the tensor cores (covered only by the stated
 tolerance).
 """
-from . import nvfp4, splice, stats, seqfilter, bounds  # noqa: F401
+from . import nvfp4, splice, stats, seqfilter, bounds, train  # noqa: F401

@@ -14,6 +14,12 @@ K coordinates.  Under power-of-two gains the Eq. 5 form equals the definition
 pin that identity.
 
 Side buffers are padded to Pp = roundup(p, 16) columns with zeros.
+
+Compacted-K variant (``COMPACT``, the "next" form the pages leave open): the protected columns
+are removed from the NVFP4 operand instead of zeroed in place, so the 16-element blocks are
+re-formed over the unprotected channels in ascending order; the operand has compact_cols(K, p)
+columns (zero padded to a multiple of 256).  Gains, the side buffers and alpha are those of the
+split form; only block membership (hence the block scales) changes.
 """
 from __future__ import annotations
 
@@ -23,10 +29,28 @@ from . import nvfp4
 
 SPLIT = "split"
 RESIDUAL = "residual"
+COMPACT = "compact"
 
 
 def padded_p(p: int) -> int:
     return (int(p) + 15) // 16 * 16
+
+
+def compact_cols(K: int, p: int) -> int:
+    """Columns of the compacted NVFP4 operand: the K - p unprotected channels, padded with zero
+    columns to a multiple of 256 (one NVFP4 k-tile of the GEMM kernels)."""
+    return (int(K) - int(p) + 255) // 256 * 256
+
+
+def compact(A, P) -> np.ndarray:
+    """A[:, ~P] (unprotected columns in ascending channel order) followed by zero columns up to
+    compact_cols(K, p): the compacted-K reading of x_R (§9.3.1), blocks re-formed over ~P."""
+    A = np.asarray(A, dtype=np.float32)
+    K = A.shape[1]
+    keep = keep_vector(P, K)
+    out = np.zeros((A.shape[0], compact_cols(K, int((~keep).sum()))), np.float32)
+    out[:, : int(keep.sum())] = A[:, keep]
+    return out
 
 
 def keep_vector(P, K) -> np.ndarray:
@@ -50,7 +74,11 @@ def quantize_splice(X, P, gA, mode: str = SPLIT):
     M, K = X.shape
     P = np.asarray(P, dtype=np.int64)
     keep = keep_vector(P, K)
-    codes, sf = nvfp4.quantize_blocks(X, keep, gA, scale_from_all_lanes=(mode == RESIDUAL))
+    if mode == COMPACT:
+        Xc = compact(X, P)
+        codes, sf = nvfp4.quantize_blocks(Xc, np.ones(Xc.shape[1], bool), gA)
+    else:
+        codes, sf = nvfp4.quantize_blocks(X, keep, gA, scale_from_all_lanes=(mode == RESIDUAL))
     xs = np.zeros((M, padded_p(len(P))), np.float32)
     xs[:, : len(P)] = nvfp4.bf16_round(X[:, P])
     return {"codes": codes, "sf": sf, "xs": xs}
@@ -59,7 +87,7 @@ def quantize_splice(X, P, gA, mode: str = SPLIT):
 def weight_gain(W, P, mode: str = SPLIT, exact: bool = False) -> np.float32:
     """g_W from the absolute maximum of W over the unprotected columns (all columns in residual form)."""
     W = np.asarray(W, dtype=np.float32)
-    cols = keep_vector(P, W.shape[1]) if mode == SPLIT else np.ones(W.shape[1], bool)
+    cols = keep_vector(P, W.shape[1]) if mode != RESIDUAL else np.ones(W.shape[1], bool)
     amax = np.float32(np.abs(W[:, cols]).max()) if cols.any() and W.size else np.float32(0)
     return nvfp4.gain_exact(amax) if exact else nvfp4.gain_pow2(amax)
 
@@ -74,7 +102,11 @@ def prepare_weights(W, P, gA, mode: str = SPLIT, exact_gain: bool = False):
     P = np.asarray(P, dtype=np.int64)
     gW = weight_gain(W, P, mode, exact_gain)
     alpha = nvfp4.alpha_from_gains(gA, gW)
-    codes, sf = nvfp4.quantize_blocks(W, keep_vector(P, K), gW, scale_from_all_lanes=(mode == RESIDUAL))
+    if mode == COMPACT:
+        Wc = compact(W, P)
+        codes, sf = nvfp4.quantize_blocks(Wc, np.ones(Wc.shape[1], bool), gW)
+    else:
+        codes, sf = nvfp4.quantize_blocks(W, keep_vector(P, K), gW, scale_from_all_lanes=(mode == RESIDUAL))
     ws = np.zeros((N, padded_p(len(P))), np.float32)
     wp = nvfp4.bf16_round(W[:, P])
     ws[:, : len(P)] = nvfp4.bf16_round((wp / alpha).astype(np.float32))

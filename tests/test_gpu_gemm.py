@@ -85,6 +85,29 @@ def test_decode_path(M, N, K, p):
     _assert_close(Y, Yr, mag)
 
 
+@pytest.mark.parametrize("M,N,K,p", [(16, 128, 12288, 64), (5, 384, 4096, 64), (1, 24576, 4096, 64),
+                                     (2, 1024, 4096, 256), (9, 144, 256, 16)])
+def test_decode_split_tiles_are_summed_in_order_and_repeatable(M, N, K, p):
+    """The decode kernel cuts the units of all tiles into one balanced range per SM, so tiles are
+    split between CTAs (one tile over 49 CTAs; three tiles over 51; 192 tiles at about 22 units per
+    CTA; the BF16 units of P = 256; a ragged last tile).  Split tiles are summed from the workspace
+    in CTA order: three launches in a row give bit-identical outputs (which also shows the arrival
+    counters return to zero), all within the oracle's bound."""
+    X, W, Xt, Wt, P, gA = _problem(60 + M + N, M, N, K, p)
+    mask = mask_tensor(stats.protect_mask(P, K))
+    g = torch.tensor([float(gA)], device="cuda")
+    wq, _, alpha = F.fs_prepare_weights(Wt, mask, p, g)
+    xq = F.fs_quantize_splice(Xt, mask, p, g)
+    plan = F.Plan(N, K, max(p, 1), F.FS_PATH_DECODE)
+    outs = []
+    for _ in range(3):
+        outs.append(F.fs_splice_gemm(plan, xq, wq, alpha, Y=nan_output(M, N)))
+    plan.check()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    Yr, mag = _ref(X, W, P, gA)
+    _assert_close(outs[0], Yr, mag)
+
+
 @pytest.mark.parametrize("M,N,K,p", [(128, 256, 256, 0), (128, 256, 512, 64), (300, 1024, 4096, 64),
                                      (17, 384, 1024, 64), (1000, 512, 2048, 256), (256, 128, 768, 16),
                                      (200, 768, 4096, 5), (129, 256, 12288, 64)])

@@ -250,3 +250,77 @@ def test_theorem1_bound_holds_per_row(golden_dir):
     # and in expectation over rows, with m_j the empirical second moments
     mj = (X[rows_ok].astype(np.float64) ** 2).mean(axis=0)
     assert lhs[rows_ok].mean() <= C * (W.astype(np.float64) ** 2).sum() * mj[keep].sum()
+
+
+# ----------------------------------------------------------------------------- compacted K
+def test_compact_with_no_protection_is_the_split_form():
+    """P = {}: nothing is removed, so the compacted operand is the split operand."""
+    rng = np.random.default_rng(20)
+    X = rng.standard_normal((6, 512)).astype(np.float32)
+    g = nvfp4.gain_pow2(np.abs(X).max())
+    a = splice.quantize_splice(X, [], g, splice.COMPACT)
+    b = splice.quantize_splice(X, [], g, splice.SPLIT)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["sf"], b["sf"])
+
+
+def test_compact_with_every_channel_protected_is_the_exact_bf16_gemm():
+    """P = all: the NVFP4 operand has no columns and Y is the BF16 product X W^T exactly."""
+    rng = np.random.default_rng(21)
+    X = nvfp4.bf16_round(rng.standard_normal((4, 64)).astype(np.float32))
+    W = nvfp4.bf16_round((rng.standard_normal((8, 64)) * 0.1).astype(np.float32))
+    P = np.arange(64)
+    assert splice.compact_cols(64, 64) == 0
+    xq = splice.quantize_splice(X, P, np.float32(1), splice.COMPACT)
+    wq = splice.prepare_weights(W, P, np.float32(1), splice.COMPACT)
+    assert xq["codes"].shape == (4, 0)
+    Y, _ = splice.splice_gemm(xq, wq, wq["alpha"])
+    assert np.array_equal(Y, X.astype(np.float64) @ W.astype(np.float64).T)
+
+
+def test_compact_blocks_are_formed_over_the_unprotected_channels():
+    """Channel j holds 2^(j // 16): in original coordinates block b has maximum 2^b; with channels
+    0 and 17 protected, compacted block 0 holds channels 1..16 (maximum 2) and block 1 channels
+    18..33 (maximum 4), block 2 channels 34..47 and zero padding (maximum 4).  The scale codes follow
+    from the pinned UE4M3 encoder at those maxima; the split form keeps 1, 2, 4."""
+    K = 48
+    X = np.array([[2.0 ** (j // 16) for j in range(K)]], np.float32)
+    P = [0, 17]
+    g = np.float32(1.0)
+    sf_of = lambda a: int(nvfp4.ue4m3_encode(np.float32(np.float32(a * g) / np.float32(6.0))))
+    c = splice.quantize_splice(X, P, g, splice.COMPACT)
+    assert c["codes"].shape == (1, 256)
+    assert c["sf"][0, :3].tolist() == [sf_of(2.0), sf_of(4.0), sf_of(4.0)]
+    assert not c["sf"][0, 3:].any() and not c["codes"][0, 46:].any()
+    s = splice.quantize_splice(X, P, g, splice.SPLIT)
+    assert s["sf"][0].tolist() == [sf_of(1.0), sf_of(2.0), sf_of(4.0)]
+
+
+def test_compact_lemma2_bound_and_gemm_against_brute_force():
+    """Every compacted block obeys Lemma 2's per-element bound, and the SpliceGEMM of compacted
+    operands equals a rational triple loop over the dequantised values plus the BF16 slice."""
+    from fractions import Fraction
+    rng = np.random.default_rng(22)
+    M, N, K = 3, 2, 96
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    X[:, [5, 40, 41]] *= 40
+    W = (rng.standard_normal((N, K)) * 0.05).astype(np.float32)
+    P = np.array([5, 40, 41])
+    gA = nvfp4.gain_pow2(np.abs(np.delete(X, P, axis=1)).max())
+    xq = splice.quantize_splice(X, P, gA, splice.COMPACT)
+    wq = splice.prepare_weights(W, P, gA, splice.COMPACT)
+    Xc = splice.compact(X, P)
+    xh = nvfp4.dequantize(xq["codes"], xq["sf"], gA)
+    nb = Xc.shape[1] // 16
+    a_b = np.abs(Xc).reshape(M, nb, 16).max(axis=2)
+    err = np.abs(xh - Xc).reshape(M, nb, 16).max(axis=2)
+    ok = (xq["sf"] >= 8) & (xq["sf"] < 126)          # normal, unsaturated scales (Lemma 2's premise)
+    assert ok[:, : (K - 3 + 15) // 16].all()
+    assert np.all(err[ok] <= bounds.c_elem() * a_b[ok] * (1 + 2.0 ** -20))
+    Y, _ = splice.splice_gemm(xq, wq, wq["alpha"])
+    xv = nvfp4.dequantize(xq["codes"], xq["sf"])
+    wv = nvfp4.dequantize(wq["codes"], wq["sf"])
+    for m in range(M):
+        for n in range(N):
+            acc = sum(Fraction(float(xv[m, k])) * Fraction(float(wv[n, k])) for k in range(xv.shape[1]))
+            acc += sum(Fraction(float(xq["xs"][m, j])) * Fraction(float(wq["ws"][n, j])) for j in range(xq["xs"].shape[1]))
+            assert Y[m, n] == float(Fraction(float(np.float32(wq["alpha"]))) * acc)

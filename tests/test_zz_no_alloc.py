@@ -49,17 +49,19 @@ def test_noalloc_matches_planned_call_twice(M, N, K, p):
     Y_ref = F.fs_splice_gemm(plan, xq, wq, alpha)
     plan.check()
     ref = Y_ref.cpu().numpy().astype(np.float64)
-    mag = np.abs(ref) + 1e-30
     xr = splice.quantize_splice(X, P, gA)
     wr = splice.prepare_weights(W, P, gA)
     Yo, mag_o = splice.splice_gemm(xr, wr, wr["alpha"])
+    # For M <= 16 the planned call runs the persistent decode kernel and this entry the
+    # workspace-free one: the FP32 partial sums are added in different orders, so the two agree
+    # within the bound every GEMM test uses, 1e-5 * sum_k |x_hat_k w_hat_k| (not bit for bit).
+    mag = mag_o
     for call in range(2):
         Y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
         st = _call(lib, N, K, 0, M, p, xq, wq, alpha, Y, 1)
         assert st == 0, lib.fs_last_error()
         got = Y.cpu().numpy().astype(np.float64)
-        # same kernels on the same operands: equal up to the 1e-5 relative tolerance the tests use
-        assert np.all(np.abs(got - ref) <= 1e-5 * mag), f"call {call} differs from fs_splice_gemm"
+        assert np.all(np.abs(got - ref) <= 2e-5 * mag), f"call {call} differs from fs_splice_gemm"
         # and within the oracle's bound, like every other GEMM parity test
         assert np.all(np.abs(got - Yo) <= 1e-5 * mag_o), f"call {call} outside the oracle bound"
 
@@ -72,7 +74,7 @@ def test_noalloc_timeout_is_reported_and_cleared(path):
     lib = F.load()
     M = 8 if path else 300
     N, K, p = 512, 1024, 64
-    xq, wq, alpha, _ = _packed(77 + M, M, N, K, p)
+    xq, wq, alpha, (X, W, P, gA) = _packed(77 + M, M, N, K, p)
     Y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
     assert _call(lib, N, K, path | F.FS_FAULT_NO_COPIES, M, p, xq, wq, alpha, Y, 1) == 5
     plan = F.Plan(N, K, p, path)
@@ -80,7 +82,11 @@ def test_noalloc_timeout_is_reported_and_cleared(path):
     plan.check()
     assert _call(lib, N, K, path, M, p, xq, wq, alpha, Y, 1) == 0, lib.fs_last_error()
     ref = Y_ref.cpu().numpy().astype(np.float64)
-    assert np.all(np.abs(Y.cpu().numpy().astype(np.float64) - ref) <= 1e-5 * (np.abs(ref) + 1e-30))
+    xr = splice.quantize_splice(X, P, gA)
+    wr = splice.prepare_weights(W, P, gA)
+    Yo, mag = splice.splice_gemm(xr, wr, wr["alpha"])
+    got = Y.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - Yo) <= 1e-5 * mag) and np.all(np.abs(got - ref) <= 2e-5 * mag)
 
 
 def test_noalloc_rejects_unsupported_shapes():
