@@ -53,7 +53,7 @@ DECODE_LAYERS = 36
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch per shape of the current kernel, summed
 # over the step's launches (qkv, o, gate_up, down).  None where no capture of the current kernel
 # exists (the one-launch-per-projection form, --unfused).
-GEMM_DRAM_BYTES_PER_STEP = {"fused": 1367799296, "unfused": None}
+GEMM_DRAM_BYTES_PER_STEP = {"fused": 1368882176, "unfused": None}
 
 
 def gemm_alg_bytes(p, fused=True):
@@ -780,6 +780,16 @@ def kernel_case(F, args, device):
     if args.case == "moe":
         print(json.dumps({"case": "moe", **moe_case(F, args.p, device, reps=args.steps)}))
         return
+    if args.case == "rollout":
+        print(json.dumps({"case": "rollout", **rollout_case(F, device, reps=args.steps)}))
+        return
+    if args.case == "training":
+        print(json.dumps({"case": "training", **training_case(F, device, reps=args.steps)}))
+        return
+    if args.case == "decode_sweep":
+        dec, wbytes = decode_sweep(F, args.p, device, fused=not args.unfused, reps=args.steps)
+        print(json.dumps({"case": "decode_sweep", "weight_bytes_per_layer": wbytes, **dec}))
+        return
     if args.shape in GROUP_NAMES:
         gi = GROUP_NAMES.index(args.shape)
         rows = [PROJ[j][1] for j in GROUP_PROJ[gi]]
@@ -824,14 +834,14 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--serial", action="store_true", help="one stream for the whole step (no group concurrency)")
-    ap.add_argument("--case", default="step", choices=["step", "gemm", "decode", "prep", "moe"],
+    ap.add_argument("--case", default="step", choices=["step", "gemm", "decode", "prep", "moe", "decode_sweep", "rollout", "training"],
                     help="step: the full benchmark; gemm / decode: only fs_splice_gemm on one projection "
                          "shape (M=8192, or M=--decode-m) for profiling one kernel; prep: the preparation "
                          "kernels on the q projection; moe: the grouped 64-expert projections alone")
     ap.add_argument("--shape", default="q", choices=[name for name, _, _, _ in PROJ] + list(GROUP_NAMES[::2]),
                     help="projection shape of --case gemm / decode")
     ap.add_argument("--decode-m", type=int, default=16, help="tokens of --case decode (1..16)")
-    ap.add_argument("--prep", default="fused", choices=["fused", "separate"],
+    ap.add_argument("--prep", default="separate", choices=["fused", "separate"],
                     help="fused: reselect from the previous step's moments, then one pass over X for the "
                          "quantise and the next moments (fs_quantize_splice_stats); separate: statistics, "
                          "reselection and quantise as their own passes")

@@ -221,8 +221,7 @@ int64_t fs_grouped_rows(int64_t max_rows, int32_t E);
  * protected slice accumulated into the same FP32 accumulator, scaled once by alpha.
  *
  * A plan caches the kernel choice for one weight shape (N, K, p_max) and owns a device error
- * word and the decode kernel's workspace (split-tile partial sums and arrival counters, about
- * 2.4 MB plus 16 bytes per 128 rows of N); creating it is the only call that allocates.  fs_plan_check synchronises `stream` and
+ * word; creating it is the only call that allocates.  fs_plan_check synchronises `stream` and
  * returns FS_ERR_TIMEOUT if a kernel launched with the plan gave up a bounded wait (the word is
  * then cleared).  A plan may be used from one stream at a time.
  * ---------------------------------------------------------------------------------------- */
@@ -234,12 +233,9 @@ fs_status fs_plan_check(fs_plan plan, void* stream);
 /* Packed operands as written above (activation rows M; weight rows N = the plan's N), p <= the
  * plan's p_max; alpha: device float.  Y [M][ldy] fp32 (bf16 with FS_OUT_BF16 in the plan's
  * opts), ldy >= N, 16-byte aligned rows.  M <= 16 runs the weight-streaming decode kernel (weights
- * as the 128-row operand of tcgen05 block-scaled MMAs with the tokens as N = 16; one persistent CTA
- * per SM takes a balanced range of the k-tiles of all output tiles, and tiles split between CTAs
- * are summed in a fixed order through the plan's workspace), larger M the tcgen05 prefill kernel
- * (FS_PATH_TENSOR / FS_PATH_DECODE in the plan's opts force one).  The plan's workspace makes
- * calls with the same plan ordered on one stream; calls that overlap on the GPU need their own
- * plans.
+ * as the 128-row operand of tcgen05 block-scaled MMAs with the tokens as N = 16, K split over a
+ * thread-block cluster), larger M the tcgen05 prefill kernel (FS_PATH_TENSOR / FS_PATH_DECODE in
+ * the plan's opts force one).
  * Plan requirements: N % 16 == 0 and K % 256 == 0 (FS_ERR_UNSUPPORTED otherwise); the packed
  * operands must be 16-byte aligned.  The output is not accumulated into: Y is overwritten.
  * M = 0 (an empty batch) returns FS_OK without reading any operand pointer (the plan must still
@@ -287,9 +283,7 @@ fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64_t* row_off
  * reserved at start-up, a plugin whose host forbids allocations) calls this instead: same
  * operands, same results, no plan.  Its only scratch is one 32-bit error word in a file-scope
  * __device__ array of the library (1 word, 256-byte aligned); every GPU that loads the library
- * holds it until the process exits.  No problem size needs more scratch than that (for M <= 16 it
- * runs the workspace-free decode kernel: K split over a thread-block cluster, partials summed
- * through distributed shared memory); shapes beyond
+ * holds it until the process exits.  No problem size needs more scratch than that; shapes beyond
  * the kernels' limits (N % 16, K % 256 or 256 <= K <= 65536, M < 2^31 - 256, p <= min(K, 256)) are
  * rejected with FS_ERR_INVALID_ARGUMENT / FS_ERR_UNSUPPORTED.
  *   N, K, opts  as for fs_plan_create (FS_OUT_BF16, FS_PATH_TENSOR, FS_PATH_DECODE apply);

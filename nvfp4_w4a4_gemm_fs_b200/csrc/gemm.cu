@@ -9,8 +9,6 @@ struct fs_plan_s {
   uint32_t opts;
   uint32_t* err;      // device error word (bounded-wait timeouts)
   int device;
-  void* ws;           // decode workspace: split-tile partials and their arrival counters
-  int64_t ws_bytes;
 };
 
 using namespace fs;
@@ -44,16 +42,12 @@ extern "C" fs_status fs_plan_create(fs_plan* out, int32_t N, int32_t K, int32_t 
   if (K < 256 || K % 256 != 0 || K > 65536) return fail(FS_ERR_UNSUPPORTED, "fs_plan_create: need K %% 256 == 0, 256 <= K <= 65536 (K=%d)", K);
   if (p_max < 0 || p_max > 256 || p_max > K) return fail(FS_ERR_INVALID_ARGUMENT, "fs_plan_create: need 0 <= p_max <= min(K, 256)");
   if ((opts & kPathMask) == kPathMask) return fail(FS_ERR_INVALID_ARGUMENT, "fs_plan_create: FS_PATH_TENSOR and FS_PATH_DECODE are exclusive");
-  auto* pl = new fs_plan_s{N, K, p_max, opts, nullptr, 0, nullptr, 0};
+  auto* pl = new fs_plan_s{N, K, p_max, opts, nullptr, 0};
   cudaGetDevice(&pl->device);
-  pl->ws_bytes = decode_sk_workspace_bytes(N);
   cudaError_t e = cudaMalloc(&pl->err, sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(pl->err, 0, sizeof(uint32_t));
-  if (e == cudaSuccess) e = cudaMalloc(&pl->ws, pl->ws_bytes);
-  if (e == cudaSuccess) e = cudaMemset(pl->ws, 0, pl->ws_bytes);
   if (e != cudaSuccess) {
     if (pl->err) cudaFree(pl->err);
-    if (pl->ws) cudaFree(pl->ws);
     delete pl;
     return cuda_status(e, "fs_plan_create");
   }
@@ -64,7 +58,6 @@ extern "C" fs_status fs_plan_create(fs_plan* out, int32_t N, int32_t K, int32_t 
 extern "C" fs_status fs_plan_destroy(fs_plan plan) {
   if (!plan) return FS_OK;
   cudaFree(plan->err);
-  cudaFree(plan->ws);
   delete plan;
   return FS_OK;
 }
@@ -77,9 +70,7 @@ extern "C" fs_status fs_plan_check(fs_plan plan, void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_status(e, "fs_plan_check");
   if (w) {
-    // an aborted decode launch may leave split-tile arrival counters behind: clear them too
     cudaMemsetAsync(plan->err, 0, sizeof(uint32_t), s);
-    cudaMemsetAsync(plan->ws, 0, plan->ws_bytes, s);
     cudaStreamSynchronize(s);
     return fail(FS_ERR_TIMEOUT, "a SpliceGEMM kernel gave up a bounded wait (error word 0x%x)", w);
   }
@@ -107,7 +98,7 @@ fs_status splice_gemm(const char* who, fs_plan plan, int64_t M, int32_t p, const
     d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha; d.seg = seg;
     d.Y = Y; d.ldy = ldy; d.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; d.err = plan->err;
     d.wait_ns = wait_limit_ns(plan->opts); d.no_copies = (plan->opts & FS_FAULT_NO_COPIES) ? 1 : 0;
-    return launch_splice_gemm_decode_sk(d, plan->ws, plan->ws_bytes, s);
+    return launch_splice_gemm_decode_tc(d, s);
   }
   if (M > (int64_t{1} << 31) - 256) return fail(FS_ERR_UNSUPPORTED, "%s: M too large", who);
   TcParams prm{};

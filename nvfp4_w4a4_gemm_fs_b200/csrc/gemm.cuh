@@ -86,11 +86,6 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint64_t kFaultWaitLimitNs = 20000000ull;
 inline uint64_t wait_limit_ns(uint32_t opts) { return (opts & FS_FAULT_NO_COPIES) ? kFaultWaitLimitNs : kWaitLimitNs; }
 
-// Workspace-free decode kernel (K split over a thread-block cluster, DSMEM reduction).
 fs_status launch_splice_gemm_decode_tc(const DecodeParams& p, cudaStream_t s);
-// Persistent stream-K decode kernel; needs decode_sk_workspace_bytes(N) bytes of workspace whose
-// counters are zero (the kernel leaves them zero after every completed launch).
-int64_t decode_sk_workspace_bytes(int N);
-fs_status launch_splice_gemm_decode_sk(const DecodeParams& p, void* workspace, int64_t ws_bytes, cudaStream_t s);
 
 }  // namespace fs

@@ -144,7 +144,7 @@ struct TileMap {
 // Tile t -> rows / columns.  cum_m[e] counts the (kBM * CG)-row M-tiles before expert e.  The
 // operand whose tiles vary fastest is read whole by every wave of CTAs, so the order keeps the
 // smaller operand there (it stays in L2) and streams the larger one once: M-tiles fastest when A
-// is the smaller (or for experts), N-tiles fastest otherwise.
+// is the smaller, N-tiles fastest otherwise and for experts.
 template <int CG>
 __device__ __forceinline__ TileMap map_tile(int t, const TcParams& p, const int* cum_m, int rank) {
   TileMap m;
@@ -598,8 +598,10 @@ fs_status launch_cfg(const TcLaunch& L, TcParams prm, int units, cudaStream_t s)
   if (st != FS_OK) return st;
   prm.BN = BN;
   prm.n_tiles = static_cast<int>(ceil_div(prm.N, BN));
-  // N-tiles fastest when the weights (B) are the smaller operand of a dense problem.
-  prm.n_fast = (!prm.offsets && prm.E == 1 && static_cast<int64_t>(prm.N) <= L.a_rows) ? 1 : 0;
+  // N-tiles fastest when the weights (B) are the smaller operand of a dense problem, and for experts:
+  // then the tiles in flight belong to a few consecutive experts, whose weights stay in L2 while
+  // each of their 128-row activation tiles meets every N-tile.
+  prm.n_fast = (prm.offsets || (prm.E == 1 && static_cast<int64_t>(prm.N) <= L.a_rows)) ? 1 : 0;
   CUtensorMap tmA, tmB, tmSA, tmSB;
   const uint64_t kbytes = static_cast<uint64_t>(prm.K) / 2;
   if (prm.KT > 0) {

@@ -29,7 +29,7 @@ def _inputs(seed, M, K, p, dtype):
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("M,K,p", [(8, 512, 64), (130, 576, 5), (300, 4096, 64), (64, 4096, 256), (16, 12288, 256),
-                                   (5, 256, 0), (3, 1024, 1024)])
+                                   (5, 256, 0), (3, 256, 256)])
 def test_compact_quantise_bit_exact(dtype, M, K, p):
     x, X, P, gA = _inputs(31 + M + K, M, K, p, dtype)
     T = bf16_tensor(x) if dtype == "bf16" else f32_tensor(x)

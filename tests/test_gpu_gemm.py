@@ -87,12 +87,11 @@ def test_decode_path(M, N, K, p):
 
 @pytest.mark.parametrize("M,N,K,p", [(16, 128, 12288, 64), (5, 384, 4096, 64), (1, 24576, 4096, 64),
                                      (2, 1024, 4096, 256), (9, 144, 256, 16)])
-def test_decode_split_tiles_are_summed_in_order_and_repeatable(M, N, K, p):
-    """The decode kernel cuts the units of all tiles into one balanced range per SM, so tiles are
-    split between CTAs (one tile over 49 CTAs; three tiles over 51; 192 tiles at about 22 units per
-    CTA; the BF16 units of P = 256; a ragged last tile).  Split tiles are summed from the workspace
-    in CTA order: three launches in a row give bit-identical outputs (which also shows the arrival
-    counters return to zero), all within the oracle's bound."""
+def test_decode_split_k_is_summed_in_order_and_repeatable(M, N, K, p):
+    """The decode kernel splits each tile's K range over the CTAs of a cluster and sums their
+    partials in rank order (one tile of K = 12288; three tiles; 192 tiles; the BF16 k-tiles of
+    P = 256; a ragged last tile): three launches in a row give bit-identical outputs, all within
+    the oracle's bound."""
     X, W, Xt, Wt, P, gA = _problem(60 + M + N, M, N, K, p)
     mask = mask_tensor(stats.protect_mask(P, K))
     g = torch.tensor([float(gA)], device="cuda")

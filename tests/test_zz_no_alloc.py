@@ -52,9 +52,8 @@ def test_noalloc_matches_planned_call_twice(M, N, K, p):
     xr = splice.quantize_splice(X, P, gA)
     wr = splice.prepare_weights(W, P, gA)
     Yo, mag_o = splice.splice_gemm(xr, wr, wr["alpha"])
-    # For M <= 16 the planned call runs the persistent decode kernel and this entry the
-    # workspace-free one: the FP32 partial sums are added in different orders, so the two agree
-    # within the bound every GEMM test uses, 1e-5 * sum_k |x_hat_k w_hat_k| (not bit for bit).
+    # the two calls run the same kernels; both are held to the bound every GEMM test uses,
+    # 1e-5 * sum_k |x_hat_k w_hat_k|, against the oracle and against each other
     mag = mag_o
     for call in range(2):
         Y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
