@@ -56,6 +56,12 @@ DECODE_LAYERS = 36
 GEMM_DRAM_BYTES_PER_STEP = {"fused": 1368882176, "unfused": None}
 
 
+# Issue rate of this kernel's block-scaled MMA alone (kind::mxf4nvf4, 256 x 256 x 64 on CTA pairs and
+# 128 x 256 on one CTA, no operand loads or stores), measured once on this machine's B200s: the
+# tensor cores' own ceiling for the instruction the SpliceGEMM issues, beside the 4 x BF16 estimate.
+FP4_MMA_ONLY_TFLOPS = 8900.0
+
+
 def gemm_alg_bytes(p, fused=True):
     """Operand and output bytes the GEMMs of a step must move: A and B codes, scales and side
     columns, and the fp32 output.  Fused, each input group's packed activations are read once;
@@ -652,10 +658,19 @@ def p_variant(F, p, device, streams, args, rank, compact=False):
     ev[1].record()
     torch.cuda.synchronize()
     gms = ev[0].elapsed_time(ev[1]) / args.steps
+    # per-phase device times (each phase one graph, replayed back to back)
+    pg = [capture(fn) for fn in lay.phase_fns()]
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(pg) + 1)]
+    evs[0].record()
+    for k, g_ in enumerate(pg):
+        g_.replay()
+        evs[k + 1].record()
+    torch.cuda.synchronize()
+    phase_us = {name: 1000.0 * evs[k].elapsed_time(evs[k + 1]) for k, name in enumerate(lay.PHASES)}
     lay.check()
     out = {"step_ms": ms, "gemm_ms": gms, "gemm_tflops": lay.flops / (gms * 1e-3) / 1e12,
-           "step_tflops": lay.flops / (ms * 1e-3) / 1e12}
-    del gs, gg, lay
+           "step_tflops": lay.flops / (ms * 1e-3) / 1e12, "phase_us": phase_us}
+    del gs, gg, pg, lay
     return out
 
 
@@ -1006,7 +1021,9 @@ def main():
                      "kernel": f"splice_gemm_tc_kernel ({len(gemm_names)} launches: {', '.join(gemm_names)}; "
                                "sum 2MNK / sum of CUDA-event times)",
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16 ratio), "
-                                    "of measured"},
+                                    "of measured",
+                     "peak_fp4_mma_only_tflops": FP4_MMA_ONLY_TFLOPS,
+                     "frac_vs_mma_only": gemm_tflops / FP4_MMA_ONLY_TFLOPS},
         "gemm_us": per_proj,
         "phase_us": phase_us,
         "clocks": clk.summary(),
@@ -1028,7 +1045,7 @@ def main():
             sweep[pv] = p_variant(F, pv, device, streams, args, rank)
             torch.cuda.empty_cache()
         sweep[p] = {"step_ms": ms_step, "gemm_ms": gemm_total_ms, "gemm_tflops": gemm_tflops,
-                    "step_tflops": value / world}
+                    "step_tflops": value / world, "phase_us": phase_us}
         s0 = sweep[0]
         line["overhead_vs_p0"] = {"step_ms_p0": s0["step_ms"], "step_ms_p": ms_step,
                                   "step_overhead": ms_step / s0["step_ms"] - 1.0,

@@ -18,10 +18,12 @@ namespace {
 constexpr int kTile = 64;
 
 // dst[c][r] = src[r][c] for a 64 x 64 tile per CTA: 16-byte loads along src rows into shared
-// memory (padded), 16-byte stores along dst rows.
+// memory, 16-byte stores along dst rows.  Rows of the tile are padded to 66 elements (33 words),
+// so the column reads of the store phase (8 consecutive rows per thread, 8 threads 8 rows apart)
+// fall in distinct banks.
 __global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t* __restrict__ src, int64_t lds, uint16_t* dst,
                                                              int64_t ldd, int64_t R, int64_t C, bool vec) {
-  __shared__ uint16_t tile[kTile][kTile + 8];
+  __shared__ uint16_t tile[kTile][kTile + 2];
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kTile, c0 = static_cast<int64_t>(blockIdx.x) * kTile;
   const int t = threadIdx.x;
   // load: 64 rows x 8 chunks of 8 elements; thread t takes chunk t % 8 of rows t / 8 and t / 8 + 32
@@ -134,15 +136,29 @@ __device__ __forceinline__ float k3_of(float d) {
 
 __global__ void __launch_bounds__(kSThreads)
 k3_kl_kernel(const float* __restrict__ logp_train, const float* __restrict__ logp_roll, int64_t ld,
-             const int32_t* __restrict__ lengths, int T, float* seq_k3, double* seq_sum) {
+             const int32_t* __restrict__ lengths, int T, float* seq_k3, double* seq_sum, bool vec) {
   __shared__ double sh[kSThreads / 32];
   const int s = blockIdx.x;
   int L = lengths ? __ldg(lengths + s) : T;
   L = L < 0 ? 0 : (L > T ? T : L);
   const float* a = logp_train + static_cast<int64_t>(s) * ld;
   const float* b = logp_roll + static_cast<int64_t>(s) * ld;
+  // per-thread partials in float over 4 tokens at a time (16-byte loads of both rows when the rows
+  // are 16-byte aligned), accumulated into a double per group of four
   double part = 0.0;
-  for (int t = threadIdx.x; t < L; t += kSThreads) part += static_cast<double>(k3_of(__fsub_rn(__ldg(a + t), __ldg(b + t))));
+  int t0 = 0;
+  if (vec) {
+    const int L4 = L & ~3;
+    for (int t = 4 * threadIdx.x; t < L4; t += 4 * kSThreads) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(a + t));
+      const float4 y = __ldg(reinterpret_cast<const float4*>(b + t));
+      const float q = (k3_of(__fsub_rn(x.x, y.x)) + k3_of(__fsub_rn(x.y, y.y))) +
+                      (k3_of(__fsub_rn(x.z, y.z)) + k3_of(__fsub_rn(x.w, y.w)));
+      part += static_cast<double>(q);
+    }
+    t0 = L4;
+  }
+  for (int t = t0 + threadIdx.x; t < L; t += kSThreads) part += static_cast<double>(k3_of(__fsub_rn(__ldg(a + t), __ldg(b + t))));
   const double tot = block_sum(part, sh);
   if (threadIdx.x == 0) {
     seq_k3[s] = L > 0 ? __double2float_rn(tot / static_cast<double>(L)) : 0.0f;
@@ -223,7 +239,8 @@ extern "C" fs_status fs_k3_kl(const float* logp_train, const float* logp_roll, i
   if (work && !aligned(work, 8)) return fail(FS_ERR_INVALID_ARGUMENT, "%s: work must be 8-byte aligned", who);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   double* sums = static_cast<double*>(work);      // per-sequence sums for the batch mean (may be null)
-  k3_kl_kernel<<<S, kSThreads, 0, s>>>(logp_train, logp_roll, ld, lengths, T, seq_k3, sums);
+  const bool vec = aligned(logp_train, 16) && aligned(logp_roll, 16) && ld % 4 == 0;
+  k3_kl_kernel<<<S, kSThreads, 0, s>>>(logp_train, logp_roll, ld, lengths, T, seq_k3, sums, vec);
   FS_CHECK_LAUNCH(who);
   if (batch_k3) {
     k3_batch_kernel<<<1, kSThreads, 0, s>>>(sums, lengths, S, T, batch_k3);
