@@ -216,12 +216,14 @@ def test_segmented_projections_match_each_projection(path, M):
             F.fs_splice_gemm_segmented(plan, xq, wq_all, alphas, bad)
 
 
-@pytest.mark.parametrize("M,seg_rows", [(8192, [4096, 1024, 1024]), (8192, [12288, 12288]), (16, [4096, 1024, 1024])])
-def test_full_size_segmented_sampled_rows(M, seg_rows):
+@pytest.mark.parametrize("M,seg_rows,p", [(8192, [4096, 1024, 1024], 64), (8192, [12288, 12288], 64),
+                                          (16, [4096, 1024, 1024], 64), (8192, [4096, 1024, 1024], 256)])
+def test_full_size_segmented_sampled_rows(M, seg_rows, p):
     """The launches bench.py times: M = 8192 tokens (tensor-core path) or 16 (decode path), K =
     4096, the q/k/v (or gate/up) weights stacked in one segmented launch; the oracle checks one
-    row of every 128-row tile (all rows at M = 16) of every projection."""
-    K, p = 4096, 64
+    row of every 128-row tile (all rows at M = 16) of every projection; the qkv launch also at the
+    P = 256 budget."""
+    K = 4096
     x, _ = synth.outlier_activations(211, M, K)
     X = splice.as_f32(x, True)
     st = stats.accumulate(stats.new_state(K), X)
