@@ -42,7 +42,10 @@ constexpr int kDStages = FS_DEC_STAGES;
 constexpr int kDCtasPerSm = FS_DEC_CTAS_PER_SM;   // residency the shared-memory budget allows
 static_assert(kDCtasPerSm * (1024 + 1024 + kDStages * (128 * 128 + 16 * 128 + 4096) + 8 * (2 * kDStages + 2) + 16) <= 233472,
               "CTAs per SM must fit the SM's shared memory");
-constexpr int kDMaxSplit = 8;        // portable cluster size
+#ifndef FS_DEC_MAX_SPLIT
+#define FS_DEC_MAX_SPLIT 8
+#endif
+constexpr int kDMaxSplit = FS_DEC_MAX_SPLIT;   // at most a portable cluster (8)
 constexpr uint64_t kDDrainNs = 50000000ull;
 
 struct DCfg {

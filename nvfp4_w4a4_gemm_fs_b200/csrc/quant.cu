@@ -11,6 +11,7 @@
 //   t   = fl32(fl32(a_b*g)/6);  sf = UE4M3_RNE_satfinite(t)
 //   v   = fl32(fl32(x*g)/sf);   q  = E2M1_RNE_satfinite(v)   (sf == 0: q = +-0)
 #include "common.cuh"
+#include "moments.cuh"
 
 namespace fs {
 
@@ -27,6 +28,12 @@ constexpr int kQThreads = 256;
 #endif
 
 enum class Side { Activation, Weight };
+
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
 
 struct QuantArgs {
   const void* X;
@@ -305,16 +312,36 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
         }
         const RawBlock<T>& xs = residual ? x : xm;    // lanes that set the block scale
         float amax = 0.0f;
+        if constexpr (sizeof(T) == 2) {
+          // bf16: |x| orders like its low 15 bits, so the block maximum is a packed 16-bit max of
+          // the magnitudes (finite inputs), shifted back into a float
+          uint32_t m = 0;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xs.get(j)));
+          for (int j = 0; j < 8; ++j) m = vmax_u16x2(m, xs.w[j] & 0x7FFF7FFFu);
+          amax = __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(xs.get(j)));
+        }
         const float t = div_markstein(__fmul_rn(amax, g), 6.0f, inv6);
         sfc = ue4m3_rne(t);
         const float sd = sh_val[sfc], sr = sh_rcp[sfc];
         float v[16];
         if (fast) {
           const float R = __fmul_rn(g, sr);        // exact: g is a power of two in range
+          if constexpr (sizeof(T) == 2) {
+            // two elements per packed multiply (each lane the IEEE RN product of the scalar form)
+            const uint64_t R2 = moments::pack_f32x2(R, R);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = snap12(__fmul_rn(xm.get(j), R));
+            for (int j = 0; j < 8; ++j) {
+              const uint64_t pr = moments::mul_f32x2(moments::pack_f32x2(bf16_lo(xm.w[j]), bf16_hi(xm.w[j])), R2);
+              v[2 * j] = snap12(__uint_as_float(static_cast<uint32_t>(pr)));
+              v[2 * j + 1] = snap12(__uint_as_float(static_cast<uint32_t>(pr >> 32)));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = snap12(__fmul_rn(xm.get(j), R));
+          }
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = div_markstein(__fmul_rn(xm.get(j), g), sd, sr);
@@ -530,12 +557,6 @@ __global__ void __launch_bounds__(256) weight_amax_f32_kernel(const float* __res
 #endif
 constexpr int kAmaxDepth = FS_AMAX_DEPTH;
 constexpr int kAmaxThreads = 256;
-
-__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
 
 __global__ void __launch_bounds__(kAmaxThreads) weight_amax_bf16_kernel(const uint16_t* __restrict__ W, int64_t N,
                                                                         int K, int64_t ldw,
