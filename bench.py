@@ -574,31 +574,38 @@ def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20, fus
         Ys = [torch.empty(M, pl_n, dtype=torch.float32, device=device)
               for pl_n in (sum(PROJ[j][1] for j in js) for js in units)]
 
-        def run_layers(with_quant: bool):
+        def run_layers(mode: str):
+            # packed: GEMMs on activations prepared beforehand; quant: fs_quantize_splice per input
+            # group, then the GEMMs; fused: fs_decode_splice_gemm, the preparation inside the GEMM
             for layer in range(layers):
-                if with_quant:
+                if mode == "quant":
                     for gi, K in enumerate(GROUP_K):
                         mask, g = (m4[0], g4[0:1]) if K == 4096 else (m12[0], g12[0:1])
                         F.fs_quantize_splice(Xs[gi], mask, p, g, out=xq[gi])
                 for u, js in enumerate(units):
                     wall, alpha, seg = packed[layer][u]
                     gi = PROJ[js[0]][3]
-                    if len(js) == 1:
+                    if mode == "fused":
+                        K = GROUP_K[gi]
+                        mask, g = (m4[0], g4[0:1]) if K == 4096 else (m12[0], g12[0:1])
+                        F.fs_decode_splice_gemm(plans[u], Xs[gi], mask, p, g, wall, alpha,
+                                                seg_start=seg if len(js) > 1 else None, Y=Ys[u])
+                    elif len(js) == 1:
                         F.fs_splice_gemm(plans[u], xq[gi], wall, alpha, Y=Ys[u])
                     else:
                         F.fs_splice_gemm_segmented(plans[u], xq[gi], wall, alpha, seg, Y=Ys[u])
 
         out = {}
-        for tag, wq_flag in (("gemm", False), ("quant+gemm", True)):
-            run_layers(True)
+        for tag, mode in (("gemm", "packed"), ("quant+gemm", "quant"), ("fused_prep", "fused")):
+            run_layers("quant")
             torch.cuda.synchronize()
             s = torch.cuda.Stream()
             s.wait_stream(torch.cuda.current_stream())
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.stream(s):
-                run_layers(wq_flag)          # warm (also sets kernel attributes before capture)
+                run_layers(mode)             # warm (also sets kernel attributes before capture)
                 with torch.cuda.graph(graph, stream=s):
-                    run_layers(wq_flag)
+                    run_layers(mode)
             torch.cuda.synchronize()
             for _ in range(3):
                 graph.replay()
@@ -610,14 +617,19 @@ def decode_sweep(F, p, device, Ms=(1, 4, 16), layers=DECODE_LAYERS, reps=20, fus
             e1.record()
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / reps
-            # the byte count is the per-projection one in both forms: weights once, packed
-            # activations once per projection, fp32 outputs
-            xbytes = sum(M * K * 2 + M * (K // 2 + K // 16 + F.side_cols(p) * 2) for K in GROUP_K) if wq_flag else 0
-            abytes = sum(M * (K // 2 + K // 16 + F.side_cols(p) * 2) + M * N * 4 for (_, N, K, _) in PROJ)
+            # algorithmic bytes: the weights once; packed activations once per projection (packed,
+            # quant) plus the quantiser's bf16 read and packed write per input group (quant), or the
+            # bf16 activations once per launch (fused); fp32 outputs
+            ybytes = sum(M * N * 4 for (_, N, _, _) in PROJ)
+            if mode == "fused":
+                abytes = sum(M * PROJ[js[0]][2] * 2 for js in units) + ybytes
+            else:
+                abytes = sum(M * (K // 2 + K // 16 + F.side_cols(p) * 2) for (_, _, K, _) in PROJ) + ybytes
+            xbytes = sum(M * K * 2 + M * (K // 2 + K // 16 + F.side_cols(p) * 2) for K in GROUP_K) if mode == "quant" else 0
             total = layers * (wbytes + abytes + xbytes)
             out[tag] = {"us_per_layer": 1000.0 * ms / layers, "GBps": total / (ms * 1e-3) / 1e9,
                         "bytes_per_layer": wbytes + abytes + xbytes,
-                        "launches_per_layer": len(units) + (len(GROUP_K) if wq_flag else 0)}
+                        "launches_per_layer": len(units) + (len(GROUP_K) if mode == "quant" else 0)}
             del graph
         for pl in plans:
             pl.check()
@@ -1065,7 +1077,8 @@ def main():
         dec0, wbytes0 = decode_sweep(F, 0, device, Ms=(16,), fused=not args.unfused)
         hbm = peaks["hbm_gbs"]
         line["decode"] = {k: {**v["gemm"], "frac_hbm": v["gemm"]["GBps"] / hbm,
-                              "with_quantise": {**v["quant+gemm"], "frac_hbm": v["quant+gemm"]["GBps"] / hbm}}
+                              "with_quantise": {**v["quant+gemm"], "frac_hbm": v["quant+gemm"]["GBps"] / hbm},
+                              "fused_prep": {**v["fused_prep"], "frac_hbm": v["fused_prep"]["GBps"] / hbm}}
                           for k, v in dec.items()}
         line["decode"]["layers"] = DECODE_LAYERS
         line["decode"]["weight_bytes_per_layer"] = wbytes

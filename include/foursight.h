@@ -266,6 +266,31 @@ fs_status fs_splice_gemm_segmented(fs_plan plan, int64_t M, int32_t p, const uin
                                    int32_t nseg, const int32_t* seg_start, const float* alpha, void* Y,
                                    int64_t ldy, void* stream);
 
+/* Decode-path SpliceGEMM with the activation preparation in the same launch — FourSight §5.1
+ * "Low-latency decode path" with its "Data preparation" (Mask S->0, FP4 Quant, Extract X_S).
+ * Equivalent, bit for bit, to
+ *     fs_quantize_splice(X, FS_DTYPE_BF16, M, K, ldx, mask, p, gA, xopts, xq, sfx, xs)
+ *     fs_splice_gemm_segmented(plan, M, p, xq, sfx, xs, wq, sfw, ws, nseg, seg_start, alpha, Y, ldy)
+ * on the decode kernel, without the packed activation buffers: every CTA of the weight-streaming
+ * kernel encodes its own K range of the (at most 16) token rows into its shared-memory stages, so
+ * the activations never make a round trip through global memory and no second kernel runs.
+ *   X          device bf16 [M][ldx], ldx >= K (the plan's K), 16-byte aligned rows; 0 <= M <= 16
+ *              (FS_ERR_UNSUPPORTED above 16).
+ *   mask, p    the protected set as for fs_quantize_splice (mask may be NULL when p == 0);
+ *              p <= the plan's p_max.
+ *   gA         device float, the frozen activation gain.
+ *   xopts      0 or FS_RESIDUAL (the activation encoding; FS_COMPACT_K is not available here).
+ *   wq .. ws   the prepared weights of the plan's N rows (fs_prepare_weights, same mask and gA).
+ *   nseg, seg_start  as for fs_splice_gemm_segmented; nseg <= 1 with seg_start NULL is one
+ *              projection with alpha[0].
+ *   alpha, Y, ldy    as for fs_splice_gemm.
+ * The plan must not force FS_PATH_TENSOR (FS_ERR_UNSUPPORTED).  Argument errors are returned
+ * before anything launches; M = 0 returns FS_OK without reading any operand. */
+fs_status fs_decode_splice_gemm(fs_plan plan, int64_t M, int32_t p, const void* X, int64_t ldx,
+                                const uint32_t* mask, const float* gA, uint32_t xopts, const uint8_t* wq,
+                                const uint8_t* sfw, const uint16_t* ws, int32_t nseg, const int32_t* seg_start,
+                                const float* alpha, void* Y, int64_t ldy, void* stream);
+
 /* Grouped SpliceGEMM over E experts (the mixture-of-experts projections).  Activations are the
  * padded-row outputs of fs_quantize_splice_grouped (row_offsets as given there); expert e's
  * weights are rows [e*N, (e+1)*N) of stacked wq [E*N][K/2], sfw (tiled over E*N rows) and

@@ -41,6 +41,7 @@ SIGNATURES = {
     "fs_splice_gemm": (C.c_int, [P, i64, i32, P, P, P, P, P, P, P, P, i64, P]),
     "fs_splice_gemm_segmented": (C.c_int, [P, i64, i32, P, P, P, P, P, P, i32, P, P, P, i64, P]),
     "fs_splice_gemm_grouped": (C.c_int, [P, i32, P, i64, i32, P, P, P, P, P, P, P, P, i64, P]),
+    "fs_decode_splice_gemm": (C.c_int, [P, i64, i32, P, i64, P, P, u32, P, P, P, i32, P, P, P, i64, P]),
     "fs_seq_filter": (C.c_int, [P, i64, P, i32, i32, f32, i32, i32, i32, P, P, P, P, P, P]),
     "fs_splice_gemm_noalloc": (C.c_int, [i32, i32, u32, i64, i32, P, P, P, P, P, P, P, P, i64, i32, P]),
     "fs_gemm_bf16": (C.c_int, [P, i64, i32, i32, P, i64, P, i64, P, P, i64, P]),

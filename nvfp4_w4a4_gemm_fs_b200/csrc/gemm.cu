@@ -131,6 +131,31 @@ extern "C" fs_status fs_splice_gemm(fs_plan plan, int64_t M, int32_t p, const ui
                      stream);
 }
 
+namespace {
+
+// Segments of a launch from the caller's seg_start: every tile of either path must lie in one
+// segment.
+fs_status build_segments(const char* who, const fs_plan_s* plan, int32_t nseg, const int32_t* seg_start,
+                         Segments* sg) {
+  if (nseg < 1 || nseg > kMaxSegments || !seg_start)
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: need 1 <= nseg <= %d and seg_start", who, kMaxSegments);
+  const int gran = (plan->N % 256 == 0) ? 256 : 128;
+  if (seg_start[0] != 0 || seg_start[nseg] != plan->N)
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: segments must start at 0 and end at N=%d", who, plan->N);
+  *sg = Segments{};
+  sg->n = nseg;
+  for (int i = 0; i <= nseg; ++i) {
+    if (i > 0 && seg_start[i] <= seg_start[i - 1])
+      return fail(FS_ERR_INVALID_ARGUMENT, "%s: segment starts must increase", who);
+    if (i > 0 && i < nseg && seg_start[i] % gran != 0)
+      return fail(FS_ERR_INVALID_ARGUMENT, "%s: segment boundaries must be multiples of %d", who, gran);
+    sg->n0[i] = seg_start[i];
+  }
+  return FS_OK;
+}
+
+}  // namespace
+
 extern "C" fs_status fs_splice_gemm_segmented(fs_plan plan, int64_t M, int32_t p, const uint8_t* xq,
                                               const uint8_t* sfx, const uint16_t* xs, const uint8_t* wq,
                                               const uint8_t* sfw, const uint16_t* ws, int32_t nseg,
@@ -138,22 +163,49 @@ extern "C" fs_status fs_splice_gemm_segmented(fs_plan plan, int64_t M, int32_t p
                                               void* stream) {
   const char* who = "fs_splice_gemm_segmented";
   if (!plan) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null plan", who);
-  if (nseg < 1 || nseg > kMaxSegments || !seg_start)
-    return fail(FS_ERR_INVALID_ARGUMENT, "%s: need 1 <= nseg <= %d and seg_start", who, kMaxSegments);
-  // every tile of either path must lie in one segment
-  const int gran = (plan->N % 256 == 0) ? 256 : 128;
-  if (seg_start[0] != 0 || seg_start[nseg] != plan->N)
-    return fail(FS_ERR_INVALID_ARGUMENT, "%s: segments must start at 0 and end at N=%d", who, plan->N);
-  Segments sg{};
-  sg.n = nseg;
-  for (int i = 0; i <= nseg; ++i) {
-    if (i > 0 && seg_start[i] <= seg_start[i - 1])
-      return fail(FS_ERR_INVALID_ARGUMENT, "%s: segment starts must increase", who);
-    if (i > 0 && i < nseg && seg_start[i] % gran != 0)
-      return fail(FS_ERR_INVALID_ARGUMENT, "%s: segment boundaries must be multiples of %d", who, gran);
-    sg.n0[i] = seg_start[i];
-  }
+  Segments sg;
+  const fs_status st = build_segments(who, plan, nseg, seg_start, &sg);
+  if (st != FS_OK) return st;
   return splice_gemm(who, plan, M, p, xq, sfx, xs, wq, sfw, ws, sg, alpha, Y, ldy, stream);
+}
+
+extern "C" fs_status fs_decode_splice_gemm(fs_plan plan, int64_t M, int32_t p, const void* X, int64_t ldx,
+                                           const uint32_t* mask, const float* gA, uint32_t xopts, const uint8_t* wq,
+                                           const uint8_t* sfw, const uint16_t* ws, int32_t nseg,
+                                           const int32_t* seg_start, const float* alpha, void* Y, int64_t ldy,
+                                           void* stream) {
+  const char* who = "fs_decode_splice_gemm";
+  if (!plan) return fail(FS_ERR_INVALID_ARGUMENT, "%s: null plan", who);
+  if (M < 0) return fail(FS_ERR_INVALID_ARGUMENT, "%s: M < 0", who);
+  if (M > 16) return fail(FS_ERR_UNSUPPORTED, "%s: the decode path takes M <= 16 (M=%lld)", who, (long long)M);
+  if (plan->opts & FS_PATH_TENSOR) return fail(FS_ERR_UNSUPPORTED, "%s: the plan forces the tensor-core path", who);
+  if (xopts & ~static_cast<uint32_t>(FS_RESIDUAL))
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: xopts may hold FS_RESIDUAL only (0x%x)", who, xopts);
+  if (p < 0 || p > plan->p_max) return fail(FS_ERR_INVALID_ARGUMENT, "%s: p=%d outside [0, p_max=%d]", who, p, plan->p_max);
+  Segments sg = one_segment(plan->N);
+  if (!(nseg <= 1 && !seg_start)) {
+    const fs_status st = build_segments(who, plan, nseg, seg_start, &sg);
+    if (st != FS_OK) return st;
+  }
+  if (M == 0) return FS_OK;                        // an empty batch reads no operand
+  if (!X || !gA || !wq || !sfw || !alpha || !Y || (p > 0 && (!mask || !ws)))
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: null pointer", who);
+  if (ldx < plan->K || (ldx * 2) % 16 != 0 || !aligned(X, 16))
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: X must be 16-byte aligned with ldx >= K and 16-byte rows", who);
+  if (!aligned(wq, 16) || !aligned(sfw, 16) || (p > 0 && (!aligned(ws, 16) || !aligned(mask, 4))) || !aligned(gA, 4))
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: misaligned operand", who);
+  const bool bf16 = plan->opts & FS_OUT_BF16;
+  if (ldy < plan->N || !aligned(Y, 16) || (ldy % (bf16 ? 8 : 4)) != 0)
+    return fail(FS_ERR_INVALID_ARGUMENT, "%s: Y must be 16-byte aligned with ldy >= N and 16-byte rows", who);
+  DecodeParams d{};
+  d.M = static_cast<int>(M); d.N = plan->N; d.K = plan->K; d.pp = side_cols(p);
+  d.kb4 = static_cast<int>(round_up(plan->K / 16, 4) / 4);
+  d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha; d.seg = sg;
+  d.Y = Y; d.ldy = ldy; d.out_bf16 = bf16 ? 1 : 0; d.err = plan->err;
+  d.wait_ns = wait_limit_ns(plan->opts); d.no_copies = (plan->opts & FS_FAULT_NO_COPIES) ? 1 : 0;
+  d.fuse = 1; d.x = static_cast<const uint16_t*>(X); d.ldx = ldx; d.mask = p > 0 ? mask : nullptr; d.p = p;
+  d.gA = gA; d.residual = (xopts & FS_RESIDUAL) ? 1 : 0;
+  return launch_splice_gemm_decode_tc(d, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64_t* row_offsets, int64_t max_rows,

@@ -78,6 +78,14 @@ struct DecodeParams {
   uint32_t* err;      // device error word (bounded-wait timeouts of the tensor-core decode kernel)
   uint64_t wait_ns;   // limit of every bounded wait
   int no_copies;      // failure-detection test hook: the producer issues no copies
+  // fuse != 0: the kernel prepares the activations itself from bf16 X (xq, sfx, xs unused)
+  int fuse;
+  const uint16_t* x;
+  int64_t ldx;
+  const uint32_t* mask;
+  int p;
+  const float* gA;
+  int residual;
 };
 
 // Wait limits: the normal bound, and the short one of the failure-detection test option

@@ -40,8 +40,6 @@ constexpr int kDTok = 16;            // token columns (MMA N)
 // 14.9 -> 8.6 us for the 12288 x 4096 projection at M = 1.
 constexpr int kDStages = FS_DEC_STAGES;
 constexpr int kDCtasPerSm = FS_DEC_CTAS_PER_SM;   // residency the shared-memory budget allows
-static_assert(kDCtasPerSm * (1024 + 1024 + kDStages * (128 * 128 + 16 * 128 + 4096) + 8 * (2 * kDStages + 2) + 16) <= 233472,
-              "CTAs per SM must fit the SM's shared memory");
 #ifndef FS_DEC_MAX_SPLIT
 #define FS_DEC_MAX_SPLIT 8
 #endif
@@ -56,12 +54,17 @@ struct DCfg {
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;   // multiple of 1024
   static constexpr int RED_BYTES = kDRows * kDTok * 4;   // partial [token][row], in stage 0 after the MMAs
   static_assert(RED_BYTES <= STAGE_BYTES, "the partial fits in a stage");
-  static constexpr int SMEM_BYTES = 1024 + kDStages * STAGE_BYTES + 8 * (2 * kDStages + 2) + 16;
+  // full, empty, xfull per stage; acc_full; drain; the TMEM slot and abort flag; the protected
+  // channel list of the fused activation preparation (at most 256 uint16)
+  static constexpr int BAR_BYTES = 8 * (3 * kDStages + 2);
+  static constexpr int SMEM_BYTES = 1024 + kDStages * STAGE_BYTES + BAR_BYTES + 16 + 2 * 256;
   static constexpr int TMEM_COLS = 128;
   static constexpr int SF_COL = 32;                 // scale buffer b: SFA at SF_COL+32b, SFB at SF_COL+32b+16
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the 128-byte swizzle");
   static_assert(SF_COL + 64 <= TMEM_COLS, "TMEM budget");
 };
+// (+ 1 KB the hardware reserves per CTA)
+static_assert(kDCtasPerSm * (DCfg::SMEM_BYTES + 1024) <= 233472, "CTAs per SM must fit the SM's shared memory");
 
 struct DecTcParams {
   int M, N, KT, ST, kb4, kt_per, S;
@@ -75,6 +78,14 @@ struct DecTcParams {
   uint32_t* err;
   uint64_t wait_ns;
   int no_copies;
+  // fused activation preparation (the kFuse kernel): bf16 X [M][ldx], the protected set as a
+  // bitmask of p channels, the frozen gain, the residual form
+  const uint16_t* x;
+  int64_t ldx;
+  const uint32_t* mask;
+  int p;
+  const float* gA;
+  int residual;
 };
 
 __device__ __forceinline__ uint64_t now_ns() {
@@ -106,6 +117,66 @@ __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity, uint64
     if (now_ns() - t0 > limit_ns) return;
 }
 
+// Fused activation preparation (kFuse): §5.1 "Data preparation" for this CTA's K range of the (at
+// most 16) token rows, written straight into the stage in the layout the TMA path would have
+// loaded: the E2M1 codes of row r as the 128-byte row r of the X box (128-byte swizzle: 16-byte
+// chunk c at position c ^ (r % 8)), the UE4M3 scales as bytes r*16 + (b % 4) of the b/4-th
+// 512-byte atom, and for the side k-tiles the bf16 values of the protected channels.  The block
+// rule is the library's (t = fl32(fl32(a_b g)/6), sf = UE4M3_RNE(t), v = fl32(fl32(x g)/sf),
+// q = E2M1_RNE(v)), so the stage bytes equal those fs_quantize_splice writes and the product is
+// bit-identical to the unfused call.
+struct PrepBlock {
+  uint32_t codes0, codes1;   // elements 0..7, 8..15
+  uint32_t sfc;
+};
+
+__device__ __forceinline__ uint32_t dec_vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// One 16-element block: w = its 8 bf16 pairs (element 2j in the low half of w[j]), kb = its 16
+// protected-lane bits.
+__device__ __forceinline__ PrepBlock prep_block(const uint32_t (&w)[8], uint32_t kb, bool residual, float g,
+                                                bool fast, float inv6) {
+  uint32_t xm[8];
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t two = (kb >> (2 * j)) & 3u;
+    const uint32_t kill = ((two & 1u) | ((two & 2u) << 15)) * 0xFFFFu;
+    xm[j] = w[j] & ~kill;
+    m = dec_vmax_u16x2(m, (residual ? w[j] : xm[j]) & 0x7FFF7FFFu);
+  }
+  const uint32_t mb = max(m & 0xFFFFu, m >> 16);
+  const float amax = __uint_as_float(mb << 16);
+  PrepBlock out;
+  out.sfc = ue4m3_rne(div_markstein(__fmul_rn(amax, g), 6.0f, inv6));
+  const bool real = out.sfc > 0 && out.sfc < 127;
+  const float sd = real ? ue4m3_value(out.sfc) : 1.0f;
+  const float sr = real ? __frcp_rn(sd) : 0.0f;
+  float v[16];
+  if (fast) {
+    const float R = __fmul_rn(g, sr);              // exact: g is a power of two in range
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v[2 * j] = snap12(__fmul_rn(bf16_lo(xm[j]), R));
+      v[2 * j + 1] = snap12(__fmul_rn(bf16_hi(xm[j]), R));
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v[2 * j] = div_markstein(__fmul_rn(bf16_lo(xm[j]), g), sd, sr);
+      v[2 * j + 1] = div_markstein(__fmul_rn(bf16_hi(xm[j]), g), sd, sr);
+    }
+  }
+  out.codes0 = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+  out.codes1 = e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+  return out;
+}
+
+template <bool kFuse>
 __global__ void __launch_bounds__(kDThreads, 1)
 splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                              const __grid_constant__ CUtensorMap tmWS, const __grid_constant__ CUtensorMap tmXS,
@@ -118,10 +189,12 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
   float* red = reinterpret_cast<float*>(smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDStages * C::STAGE_BYTES);
   uint64_t* empty = full + kDStages;
-  uint64_t* acc_full = empty + kDStages;
+  uint64_t* xfull = empty + kDStages;              // kFuse: the prepared X / SFX bytes are in the stage
+  uint64_t* acc_full = xfull + kDStages;
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint16_t* pidx = reinterpret_cast<uint16_t*>(tmem_slot + 4);   // kFuse: protected channels, ascending
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = static_cast<int>(ptx::cluster_ctarank());     // K split inside the tile's cluster
@@ -141,18 +214,39 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    for (int s = 0; s < kDStages; ++s) { ptx::mbar_init(full + s, 1); ptx::mbar_init(empty + s, 1); }
+    for (int s = 0; s < kDStages; ++s) {
+      ptx::mbar_init(full + s, 1);
+      ptx::mbar_init(empty + s, 1);
+      ptx::mbar_init(xfull + s, 8 * p.M);          // the 8 M threads of the group preparing it
+    }
     ptx::mbar_init(acc_full, 1);
     ptx::mbar_init(drain, 1);
     ptx::fence_mbar_init();
-    ptx::prefetch_tensormap(&tmW); ptx::prefetch_tensormap(&tmX);
-    if (p.ST > 0) { ptx::prefetch_tensormap(&tmWS); ptx::prefetch_tensormap(&tmXS); }
+    ptx::prefetch_tensormap(&tmW);
+    if constexpr (!kFuse) ptx::prefetch_tensormap(&tmX);
+    if (p.ST > 0) {
+      ptx::prefetch_tensormap(&tmWS);
+      if constexpr (!kFuse) ptx::prefetch_tensormap(&tmXS);
+    }
     if (!p.no_copies)
       for (int kt = kt0; kt < kt1; ++kt) ptx::tma_prefetch_2d(&tmW, kt * 128, n0);
   }
   if (warp == 1) {
     ptx::tmem_alloc<1>(tmem_slot, C::TMEM_COLS);
     ptx::tmem_relinquish<1>();
+  }
+  if constexpr (kFuse) {
+    // The X rows M..15 and the scale bytes that no token row < M owns stay zero, as in a packed
+    // buffer (and as the TMA path's out-of-range fill); the preparing warps rewrite the bytes of
+    // rows 0..M-1 every k-tile.  X and SFX are adjacent in a stage: X_BYTES + SFW_BYTES lie
+    // between them, so the two are cleared separately.
+    constexpr int kX16 = C::X_BYTES / 16, kS16 = C::SFX_BYTES / 16;
+    for (int i = threadIdx.x; i < kDStages * (kX16 + kS16); i += kDThreads) {
+      const int s = i / (kX16 + kS16), o = i % (kX16 + kS16);
+      uint8_t* dst = o < kX16 ? X_at(s) + 16 * o : SFX_at(s) + 16 * (o - kX16);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    ptx::fence_proxy_async_smem();                 // visible to tcgen05.cp
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -169,19 +263,21 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
       uint32_t phase = 0;
       for (int i = 0; i < nk; ++i) {
         if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err, p.wait_ns)) break;
+        // (kFuse: the weight side only; the preparing warps fill X and SFX)
         if (i < nf) {
           const int kt = kt0 + i;
-          ptx::mbar_arrive_expect_tx(full + stage, C::STAGE_BYTES);
+          ptx::mbar_arrive_expect_tx(full + stage, kFuse ? C::W_BYTES + C::SFW_BYTES : C::STAGE_BYTES);
           ptx::tma_load_2d(W_at(stage), &tmW, kt * 128, n0, full + stage);
-          ptx::tma_load_2d(X_at(stage), &tmX, kt * 128, 0, full + stage);
+          if constexpr (!kFuse) ptx::tma_load_2d(X_at(stage), &tmX, kt * 128, 0, full + stage);
           ptx::bulk_load(SFW_at(stage), p.sfw + (static_cast<int64_t>(n0 / kDRows) * p.kb4 + kt * 4) * 512,
                          C::SFW_BYTES, full + stage);
-          ptx::bulk_load(SFX_at(stage), p.sfx + static_cast<int64_t>(kt) * 4 * 512, C::SFX_BYTES, full + stage);
+          if constexpr (!kFuse)
+            ptx::bulk_load(SFX_at(stage), p.sfx + static_cast<int64_t>(kt) * 4 * 512, C::SFX_BYTES, full + stage);
         } else {
           const int sk = i - nf;
-          ptx::mbar_arrive_expect_tx(full + stage, C::W_BYTES + C::X_BYTES);
+          ptx::mbar_arrive_expect_tx(full + stage, kFuse ? C::W_BYTES : C::W_BYTES + C::X_BYTES);
           ptx::tma_load_2d(W_at(stage), &tmWS, sk * 64, n0, full + stage);
-          ptx::tma_load_2d(X_at(stage), &tmXS, sk * 64, 0, full + stage);
+          if constexpr (!kFuse) ptx::tma_load_2d(X_at(stage), &tmXS, sk * 64, 0, full + stage);
         }
         ++issued;
         if (++stage == kDStages) { stage = 0; phase ^= 1; }
@@ -206,6 +302,8 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
       bool ok = true;
       for (int i = 0; i < nk; ++i) {
         if (!wait_bar(full + stage, phase, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
+        if constexpr (kFuse)
+          if (!wait_bar(xfull + stage, phase, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint64_t adesc = ptx::desc_kmajor_sw128(ptx::smem_u32(W_at(stage)));
         const uint64_t bdesc = ptx::desc_kmajor_sw128(ptx::smem_u32(X_at(stage)));
@@ -233,6 +331,116 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
       drain_bar(drain, 0, p.wait_ns);
     }
   } else {
+    if constexpr (kFuse) {
+      // ---------------------------------------------------------------- activation preparation
+      // The 128 threads form R = min(128 / (8 M), stages) groups of 8 M threads; group j prepares
+      // the k-tiles j, j + R, j + 2R, ... of this CTA (FP4 first, then the side k-tiles), so a
+      // small batch issues the loads of several k-tiles at once.  R <= stages keeps every parity
+      // wait within one phase: a group reaches k-tile i (stage i % S) only after its k-tile
+      // i - R passed its own wait, i.e. after the MMAs of k-tile i - R - S >= i - 2S were done,
+      // and its first k-tile is j < S.  In a group, thread (r, c) takes token row r
+      // and the 32 channels c*32 .. c*32+31 of each FP4 k-tile (two scale blocks, one mask word,
+      // four 16-byte loads of X, issued one k-tile ahead) or the side columns c*8 .. c*8+7.
+      __shared__ int warp_tot[4];
+      const int t = threadIdx.x - 64;
+      const int G = 8 * p.M, R = min(128 / G, kDStages);
+      const int grp = t / G, r = (t - grp * G) >> 3, c = t & 7;
+      const uint16_t* xrow = p.x + static_cast<int64_t>(grp < R ? r : 0) * p.ldx;
+      const float g = __ldg(p.gA);
+      const bool fast = pow2_gain_in_fast_range(g);
+      const float inv6 = __frcp_rn(6.0f);
+      const bool residual = p.residual != 0;
+      // X loads of each group's first k-tile and the mask words of the channel list go out
+      // together, so the list's scan waits for the same round trip as the first encode.
+      uint4 cur[4], nxt[4];
+      uint32_t mc = 0, mn = 0;
+      auto load = [&](int kt, uint4 (&v)[4], uint32_t& mw) {
+        const int ch = kt * 256 + c * 32;
+        const uint4* src = reinterpret_cast<const uint4*>(xrow + ch);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = __ldg(src + j);
+        mw = p.p > 0 ? __ldg(p.mask + (ch >> 5)) : 0u;
+      };
+      if (grp < R && grp < nf) load(kt0 + grp, cur, mc);
+      if (nk > nf) {
+        // Protected channel list for the side k-tiles: the set bits of the mask in ascending
+        // order, from contiguous word ranges per thread (up to 4 words kept in registers) and an
+        // exclusive scan of their counts.
+        pidx[t] = 0;
+        pidx[t + 128] = 0;
+        const int nw = p.KT * 8;
+        const int per = (nw + 127) / 128;
+        const int w0 = min(t * per, nw), w1 = min(w0 + per, nw);
+        uint32_t mw4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mw4[j] = w0 + j < w1 ? __ldg(p.mask + w0 + j) : 0u;
+        int cnt = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cnt += __popc(mw4[j]);
+        for (int w = w0 + 4; w < w1; ++w) cnt += __popc(__ldg(p.mask + w));
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (lane == 31) warp_tot[warp - 2] = incl;
+        ptx::named_bar_sync(1, 128);
+        int pos = incl - cnt;
+        for (int q = 0; q < warp - 2; ++q) pos += warp_tot[q];
+        auto scatter = [&](uint32_t mw, int w) {
+          while (mw) {
+            const int b = __ffs(mw) - 1;
+            mw &= mw - 1;
+            if (pos < 256) pidx[pos] = static_cast<uint16_t>(w * 32 + b);
+            ++pos;
+          }
+        };
+#pragma unroll
+        for (int j = 0; j < 4; ++j) scatter(mw4[j], w0 + j);   // words past w1 are zero
+        for (int w = w0 + 4; w < w1; ++w) scatter(__ldg(p.mask + w), w);
+        ptx::named_bar_sync(1, 128);
+      }
+      if (grp < R) {
+        const int xoff = r * 128 + ((c ^ (r & 7)) << 4);   // 128-byte swizzle of the X box
+        const int sfoff = 512 * (c >> 1) + r * 16 + ((2 * c) & 3);
+        bool ok = true;
+        for (int i = grp; i < nf; i += R) {
+          if (i + R < nf) load(kt0 + i + R, nxt, mn);
+          const int stage = i % kDStages;
+          const uint32_t phase = (i / kDStages) & 1;
+          if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
+          const uint32_t wa[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+          const uint32_t wb[8] = {cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
+          const PrepBlock b0 = prep_block(wa, mc & 0xFFFFu, residual, g, fast, inv6);
+          const PrepBlock b1 = prep_block(wb, mc >> 16, residual, g, fast, inv6);
+          *reinterpret_cast<uint4*>(X_at(stage) + xoff) = make_uint4(b0.codes0, b0.codes1, b1.codes0, b1.codes1);
+          *reinterpret_cast<uint16_t*>(SFX_at(stage) + sfoff) = static_cast<uint16_t>(b0.sfc | (b1.sfc << 8));
+          ptx::fence_proxy_async_smem();           // generic writes -> the MMA's async reads
+          ptx::mbar_arrive(xfull + stage);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
+          mc = mn;
+        }
+        // side k-tiles: the indices nf .. nk-1 that fall to this group
+        for (int i = nf + ((grp - nf % R) % R + R) % R; ok && i < nk; i += R) {
+          const int sk = i - nf;
+          const int stage = i % kDStages;
+          const uint32_t phase = (i / kDStages) & 1;
+          if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err, p.wait_ns)) break;
+          uint32_t hv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int col = sk * 64 + c * 8 + e;
+            hv[e] = col < p.p ? static_cast<uint32_t>(__ldg(xrow + pidx[col])) : 0u;
+          }
+          *reinterpret_cast<uint4*>(X_at(stage) + xoff) =
+              make_uint4(hv[0] | (hv[1] << 16), hv[2] | (hv[3] << 16), hv[4] | (hv[5] << 16), hv[6] | (hv[7] << 16));
+          ptx::fence_proxy_async_smem();
+          ptx::mbar_arrive(xfull + stage);
+        }
+      }
+    }
     // ------------------------------------------------------------------ epilogue: TMEM -> partial
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
@@ -295,14 +503,18 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
 
 fs_status launch_splice_gemm_decode_tc(const DecodeParams& d, cudaStream_t s) {
   using C = DCfg;
-  static PerDevice<int> attr;
-  fs_status ast = set_max_dynamic_smem(attr, reinterpret_cast<const void*>(splice_gemm_decode_tc_kernel),
+  using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, DecTcParams);
+  const Kernel kernel = d.fuse ? splice_gemm_decode_tc_kernel<true> : splice_gemm_decode_tc_kernel<false>;
+  const char* who = d.fuse ? "fs_decode_splice_gemm" : "fs_splice_gemm (decode path)";
+  static PerDevice<int> attr, attr_fused;
+  fs_status ast = set_max_dynamic_smem(d.fuse ? attr_fused : attr, reinterpret_cast<const void*>(kernel),
                                        C::SMEM_BYTES, "fs_splice_gemm (decode): smem attribute");
   if (ast != FS_OK) return ast;
   DecTcParams p{};
   p.M = d.M; p.N = d.N; p.KT = d.K / 256; p.ST = static_cast<int>(ceil_div(d.pp, 64)); p.kb4 = d.kb4;
   p.sfw = d.sfw; p.sfx = d.sfx; p.alpha = d.alpha; p.seg = d.seg; p.Y = d.Y; p.ldy = d.ldy; p.out_bf16 = d.out_bf16;
   p.err = d.err; p.wait_ns = d.wait_ns; p.no_copies = d.no_copies;
+  p.x = d.x; p.ldx = d.ldx; p.mask = d.mask; p.p = d.p; p.gA = d.gA; p.residual = d.residual;
   // K split: as many CTAs per 128-row tile as fill the SMs at the resident CTAs per SM, at most 8
   // (a portable cluster);
   // every split keeps at least one FP4 k-tile.
@@ -312,16 +524,19 @@ fs_status launch_splice_gemm_decode_tc(const DecodeParams& d, cudaStream_t s) {
   p.kt_per = static_cast<int>(ceil_div(p.KT, S));
   p.S = static_cast<int>(ceil_div(p.KT, p.kt_per));
 
+  // (the fused kernel reads X itself; its activation maps are placeholders it never uses)
   CUtensorMap tmW, tmX, tmWS, tmXS;
   const uint64_t kbytes = static_cast<uint64_t>(d.K) / 2;
   fs_status st = make_map(&tmW, d.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, d.N, kbytes, 128, kDRows);
-  if (st == FS_OK) st = make_map(&tmX, d.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, d.M, kbytes, 128, kDTok);
+  if (st == FS_OK && !d.fuse) st = make_map(&tmX, d.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, d.M, kbytes, 128, kDTok);
   if (st != FS_OK) return st;
+  if (d.fuse) tmX = tmW;
   if (p.ST > 0) {
     const uint64_t pp = static_cast<uint64_t>(d.pp);
     st = make_map(&tmWS, d.ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, d.N, pp * 2, 64, kDRows);
-    if (st == FS_OK) st = make_map(&tmXS, d.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, d.M, pp * 2, 64, kDTok);
+    if (st == FS_OK && !d.fuse) st = make_map(&tmXS, d.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, d.M, pp * 2, 64, kDTok);
     if (st != FS_OK) return st;
+    if (d.fuse) tmXS = tmWS;
   } else {
     tmWS = tmW;
     tmXS = tmX;
@@ -340,9 +555,9 @@ fs_status launch_splice_gemm_decode_tc(const DecodeParams& d, cudaStream_t s) {
   attrs[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, splice_gemm_decode_tc_kernel, tmW, tmX, tmWS, tmXS, p);
-  if (e != cudaSuccess) return cuda_status(e, "fs_splice_gemm (decode path)");
-  FS_CHECK_LAUNCH("fs_splice_gemm (decode path)");
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tmW, tmX, tmWS, tmXS, p);
+  if (e != cudaSuccess) return cuda_status(e, who);
+  FS_CHECK_LAUNCH(who);
   return FS_OK;
 }
 

@@ -64,6 +64,11 @@ __global__ void __launch_bounds__(kQSThreads, 2) quantize_stats_kernel(const QSA
   __shared__ int sh_bad;
   __shared__ uint4 ring[kQSWarps][kDepth][2][32];   // per warp: kDepth row pairs x 32 lanes x 16 bytes
 
+  // Programmatic dependent launch: the next kernel (the decode GEMM, which streams its weights
+  // into L2 before it waits for this grid) may start now; this grid's own first global access
+  // comes after griddepcontrol.wait, i.e. after the previous kernel has finished and flushed.
+  // Both instructions are no-ops when the launch carries no programmatic dependency.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c0 = blockIdx.x * kSlab + lane * 8;
   const bool active = c0 < a.K;                  // K % 64 == 0: whole 8-lane scale groups
@@ -76,6 +81,7 @@ __global__ void __launch_bounds__(kQSThreads, 2) quantize_stats_kernel(const QSA
   }
   if (threadIdx.x == 0) sh_bad = 0;
   for (int c = threadIdx.x; c < kSlab; c += blockDim.x) { sh_s1[c] = 0; sh_s2[c] = 0; sh_am[c] = 0; }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // Protected lanes of this lane's 8 channels, the words to clear, and the side column of its
   // first protected channel (protected channels below c0).  The count below the slab is shared by
@@ -305,9 +311,19 @@ fs_status launch_quantize_rows(const QSArgs& a, bool with_stats, cudaStream_t s,
   int64_t gy = std::max<int64_t>(1, static_cast<int64_t>(slots) * sm_count() / chunks);
   gy = std::min<int64_t>(gy, std::max<int64_t>(1, ceil_div(a.Mp, 2 * kQSWarps * 16)));
   gy = std::min<int64_t>(gy, 65535);
-  const dim3 grid(chunks, static_cast<unsigned>(gy));
-  if (with_stats) quantize_stats_kernel<true><<<grid, kQSThreads, 0, s>>>(a);
-  else quantize_stats_kernel<false><<<grid, kQSThreads, 0, s>>>(a);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(chunks, static_cast<unsigned>(gy), 1);
+  cfg.blockDim = dim3(kQSThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = with_stats ? cudaLaunchKernelEx(&cfg, quantize_stats_kernel<true>, a)
+                                   : cudaLaunchKernelEx(&cfg, quantize_stats_kernel<false>, a);
+  if (e != cudaSuccess) return cuda_status(e, who);
   FS_CHECK_LAUNCH(who);
   return FS_OK;
 }

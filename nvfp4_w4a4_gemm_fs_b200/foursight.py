@@ -16,7 +16,7 @@ __all__ = [
     "fs_channel_stats", "fs_stats_check", "fs_select_topk", "fs_prepare_weights",
     "fs_quantize_splice", "fs_quantize_splice_grouped", "fs_quantize_splice_stats", "fs_splice_gemm", "fs_splice_gemm_grouped",
     "fs_seq_filter", "Plan", "StatsState", "Packed", "side_cols", "sf_bytes", "grouped_rows", "compact_cols",
-    "fs_splice_gemm_segmented", "stacked_packed", "fs_gemm_bf16", "fs_transpose_bf16", "fs_ste_backward",
+    "fs_splice_gemm_segmented", "fs_decode_splice_gemm", "stacked_packed", "fs_gemm_bf16", "fs_transpose_bf16", "fs_ste_backward",
     "fs_grpo_objective", "fs_k3_kl",
     "alloc_packed", "stream_handle",
 ]
@@ -221,6 +221,31 @@ def fs_splice_gemm_segmented(plan: Plan, xq: Packed, wq: Packed, alpha: torch.Te
                                        _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, len(seg) - 1, arr,
                                        _ptr(alpha), _ptr(Y), Y.stride(0), stream_handle(stream)),
           "fs_splice_gemm_segmented")
+    return Y
+
+
+def fs_decode_splice_gemm(plan: Plan, X: torch.Tensor, mask, p: int, gA: torch.Tensor, wq: Packed,
+                          alpha: torch.Tensor, seg_start=None, xopts: int = 0, Y: torch.Tensor | None = None,
+                          stream=None):
+    """Decode-path SpliceGEMM (M <= 16) with the activation preparation in the same launch: bf16 X
+    [M, K] is masked, quantised and split (as fs_quantize_splice with mask, p, gA, xopts) by the
+    GEMM kernel itself.  seg_start as for fs_splice_gemm_segmented (None: one projection)."""
+    lib = _lib.load()
+    if X.dtype != torch.bfloat16:
+        raise TypeError("fs_decode_splice_gemm takes bf16 activations")
+    M = X.shape[0]
+    if seg_start is None:
+        nseg, arr = 1, None
+    else:
+        seg = [int(v) for v in seg_start]
+        nseg, arr = len(seg) - 1, (C.c_int32 * len(seg))(*seg)
+    if Y is None:
+        dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
+        Y = torch.empty(M, plan.N, dtype=dt, device=X.device)
+    check(lib.fs_decode_splice_gemm(plan.handle, M, p, _ptr(X), X.stride(0), _ptr(mask) if p else None, _ptr(gA),
+                                    xopts, _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, nseg, arr,
+                                    _ptr(alpha), _ptr(Y), Y.stride(0), stream_handle(stream)),
+          "fs_decode_splice_gemm")
     return Y
 
 
