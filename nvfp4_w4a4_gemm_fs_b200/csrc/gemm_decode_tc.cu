@@ -55,9 +55,10 @@ struct DCfg {
   static constexpr int RED_BYTES = kDRows * kDTok * 4;   // partial [token][row], in stage 0 after the MMAs
   static_assert(RED_BYTES <= STAGE_BYTES, "the partial fits in a stage");
   // full, empty, xfull per stage; acc_full; drain; the TMEM slot and abort flag; the protected
-  // channel list of the fused activation preparation (at most 256 uint16)
+  // channel list of the fused activation preparation (at most 256 uint16); the UE4M3 value and
+  // reciprocal tables of the preparation (128 floats each)
   static constexpr int BAR_BYTES = 8 * (3 * kDStages + 2);
-  static constexpr int SMEM_BYTES = 1024 + kDStages * STAGE_BYTES + BAR_BYTES + 16 + 2 * 256;
+  static constexpr int SMEM_BYTES = 1024 + kDStages * STAGE_BYTES + BAR_BYTES + 16 + 2 * 256 + 2 * 128 * 4;
   static constexpr int TMEM_COLS = 128;
   static constexpr int SF_COL = 32;                 // scale buffer b: SFA at SF_COL+32b, SFB at SF_COL+32b+16
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the 128-byte swizzle");
@@ -138,24 +139,32 @@ __device__ __forceinline__ uint32_t dec_vmax_u16x2(uint32_t a, uint32_t b) {
 
 // One 16-element block: w = its 8 bf16 pairs (element 2j in the low half of w[j]), kb = its 16
 // protected-lane bits.
+// sf_val / sf_rcp: per UE4M3 code its value and RN(1 / value) (code 0 and the unused NaN code:
+// 1 and 0, the zero-scale rule).
 __device__ __forceinline__ PrepBlock prep_block(const uint32_t (&w)[8], uint32_t kb, bool residual, float g,
-                                                bool fast, float inv6) {
+                                                bool fast, float inv6, const float* sf_val, const float* sf_rcp) {
   uint32_t xm[8];
   uint32_t m = 0;
+  if (kb == 0) {                                   // no protected lane in the block (the common case)
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t two = (kb >> (2 * j)) & 3u;
-    const uint32_t kill = ((two & 1u) | ((two & 2u) << 15)) * 0xFFFFu;
-    xm[j] = w[j] & ~kill;
-    m = dec_vmax_u16x2(m, (residual ? w[j] : xm[j]) & 0x7FFF7FFFu);
+    for (int j = 0; j < 8; ++j) {
+      xm[j] = w[j];
+      m = dec_vmax_u16x2(m, w[j] & 0x7FFF7FFFu);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t two = (kb >> (2 * j)) & 3u;
+      const uint32_t kill = ((two & 1u) | ((two & 2u) << 15)) * 0xFFFFu;
+      xm[j] = w[j] & ~kill;
+      m = dec_vmax_u16x2(m, (residual ? w[j] : xm[j]) & 0x7FFF7FFFu);
+    }
   }
   const uint32_t mb = max(m & 0xFFFFu, m >> 16);
   const float amax = __uint_as_float(mb << 16);
   PrepBlock out;
   out.sfc = ue4m3_rne(div_markstein(__fmul_rn(amax, g), 6.0f, inv6));
-  const bool real = out.sfc > 0 && out.sfc < 127;
-  const float sd = real ? ue4m3_value(out.sfc) : 1.0f;
-  const float sr = real ? __frcp_rn(sd) : 0.0f;
+  const float sd = sf_val[out.sfc], sr = sf_rcp[out.sfc];
   float v[16];
   if (fast) {
     const float R = __fmul_rn(g, sr);              // exact: g is a power of two in range
@@ -177,7 +186,7 @@ __device__ __forceinline__ PrepBlock prep_block(const uint32_t (&w)[8], uint32_t
 }
 
 template <bool kFuse>
-__global__ void __launch_bounds__(kDThreads, 1)
+__global__ void __launch_bounds__(kDThreads, kDCtasPerSm)
 splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                              const __grid_constant__ CUtensorMap tmWS, const __grid_constant__ CUtensorMap tmXS,
                              const DecTcParams p) {
@@ -195,6 +204,8 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint16_t* pidx = reinterpret_cast<uint16_t*>(tmem_slot + 4);   // kFuse: protected channels, ascending
+  float* sf_val = reinterpret_cast<float*>(pidx + 256);          // kFuse: UE4M3 code -> value
+  float* sf_rcp = sf_val + 128;                                   //        and RN(1 / value)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = static_cast<int>(ptx::cluster_ctarank());     // K split inside the tile's cluster
@@ -236,6 +247,13 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
     ptx::tmem_relinquish<1>();
   }
   if constexpr (kFuse) {
+    if (threadIdx.x < 128) {
+      const int c = threadIdx.x;
+      const bool real = c > 0 && c < 127;
+      const float d = real ? ue4m3_value(c) : 1.0f;
+      sf_val[c] = d;
+      sf_rcp[c] = real ? __frcp_rn(d) : 0.0f;
+    }
     // The X rows M..15 and the scale bytes that no token row < M owns stay zero, as in a packed
     // buffer (and as the TMA path's out-of-range fill); the preparing warps rewrite the bytes of
     // rows 0..M-1 every k-tile.  X and SFX are adjacent in a stage: X_BYTES + SFW_BYTES lie
@@ -340,7 +358,8 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
       // i - R passed its own wait, i.e. after the MMAs of k-tile i - R - S >= i - 2S were done,
       // and its first k-tile is j < S.  In a group, thread (r, c) takes token row r
       // and the 32 channels c*32 .. c*32+31 of each FP4 k-tile (two scale blocks, one mask word,
-      // four 16-byte loads of X, issued one k-tile ahead) or the side columns c*8 .. c*8+7.
+      // four 16-byte loads of X; the next k-tile's are issued right after the current one is handed
+      // over) or the side columns c*8 .. c*8+7.
       __shared__ int warp_tot[4];
       const int t = threadIdx.x - 64;
       const int G = 8 * p.M, R = min(128 / G, kDStages);
@@ -352,8 +371,8 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
       const bool residual = p.residual != 0;
       // X loads of each group's first k-tile and the mask words of the channel list go out
       // together, so the list's scan waits for the same round trip as the first encode.
-      uint4 cur[4], nxt[4];
-      uint32_t mc = 0, mn = 0;
+      uint4 cur[4];
+      uint32_t mc = 0;
       auto load = [&](int kt, uint4 (&v)[4], uint32_t& mw) {
         const int ch = kt * 256 + c * 32;
         const uint4* src = reinterpret_cast<const uint4*>(xrow + ch);
@@ -406,21 +425,18 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
         const int sfoff = 512 * (c >> 1) + r * 16 + ((2 * c) & 3);
         bool ok = true;
         for (int i = grp; i < nf; i += R) {
-          if (i + R < nf) load(kt0 + i + R, nxt, mn);
           const int stage = i % kDStages;
           const uint32_t phase = (i / kDStages) & 1;
           if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
           const uint32_t wa[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
           const uint32_t wb[8] = {cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
-          const PrepBlock b0 = prep_block(wa, mc & 0xFFFFu, residual, g, fast, inv6);
-          const PrepBlock b1 = prep_block(wb, mc >> 16, residual, g, fast, inv6);
+          const PrepBlock b0 = prep_block(wa, mc & 0xFFFFu, residual, g, fast, inv6, sf_val, sf_rcp);
+          const PrepBlock b1 = prep_block(wb, mc >> 16, residual, g, fast, inv6, sf_val, sf_rcp);
           *reinterpret_cast<uint4*>(X_at(stage) + xoff) = make_uint4(b0.codes0, b0.codes1, b1.codes0, b1.codes1);
           *reinterpret_cast<uint16_t*>(SFX_at(stage) + sfoff) = static_cast<uint16_t>(b0.sfc | (b1.sfc << 8));
           ptx::fence_proxy_async_smem();           // generic writes -> the MMA's async reads
           ptx::mbar_arrive(xfull + stage);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
-          mc = mn;
+          if (i + R < nf) load(kt0 + i + R, cur, mc);   // after the handover (it is a release)
         }
         // side k-tiles: the indices nf .. nk-1 that fall to this group
         for (int i = nf + ((grp - nf % R) % R + R) % R; ok && i < nk; i += R) {
