@@ -28,6 +28,7 @@ struct TcParams {
   int64_t M;
   int N, K, KT, ST, BN, n_tiles, E, kb4;
   int n_fast;         // tile order: 1 = N-tiles vary fastest (B stays in L2), 0 = M-tiles fastest
+  int64_t a_groups;   // 128-row groups of the activation buffers (scale atoms past them are not read)
   const int64_t* offsets;
   const uint8_t* sfa;
   const uint8_t* sfb;

@@ -97,7 +97,7 @@ struct Cfg {
   // unit slot; drain
   static constexpr int NUM_BARS = 3 * STAGES + 2 * ACC_SLOTS + 2 * SF_UNITS + 1;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + 8 * NUM_BARS + 16 +
-                                    4 * (kMaxExperts + 1);
+                                    2 * 4 * (kMaxExperts + 1);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 };
 
@@ -141,12 +141,13 @@ struct TileMap {
   int n0;          // first output column
 };
 
-// Tile t -> rows / columns.  cum_m[e] counts the (kBM * CG)-row M-tiles before expert e.  The
+// Tile t -> rows / columns.  cum_m[e] counts the (kBM * CG)-row M-tiles before expert e, cum_g[e]
+// the 128-row groups before it (expert e's packed rows start at row 128 cum_g[e]).  The
 // operand whose tiles vary fastest is read whole by every wave of CTAs, so the order keeps the
 // smaller operand there (it stays in L2) and streams the larger one once: M-tiles fastest when A
 // is the smaller, N-tiles fastest otherwise and for experts.
 template <int CG>
-__device__ __forceinline__ TileMap map_tile(int t, const TcParams& p, const int* cum_m, int rank) {
+__device__ __forceinline__ TileMap map_tile(int t, const TcParams& p, const int* cum_m, const int* cum_g, int rank) {
   TileMap m;
   const int total_m = cum_m[p.E];
   const int mt = p.n_fast ? t / p.n_tiles : t % total_m;
@@ -158,13 +159,17 @@ __device__ __forceinline__ TileMap map_tile(int t, const TcParams& p, const int*
   }
   m.e = lo;
   const int local = mt - cum_m[lo];
-  m.arow = static_cast<int64_t>(mt) * (kBM * CG) + rank * kBM;   // experts start at 128-row boundaries
   if (p.offsets) {
+    // A pair's second CTA may start past the expert's last row: it then has no valid rows, reads
+    // zero fill (or a following expert's rows) and stores nothing.
     const int64_t r0 = p.offsets[lo], r1 = p.offsets[lo + 1];
-    m.yrow = r0 + static_cast<int64_t>(local) * kBM;
+    const int64_t off = static_cast<int64_t>(local) * (kBM * CG) + rank * kBM;
+    m.arow = static_cast<int64_t>(cum_g[lo]) * kBM + off;
+    m.yrow = r0 + off;
     const int64_t left = r1 - m.yrow;
     m.rows = static_cast<int>(left < kBM ? left : kBM);
   } else {
+    m.arow = static_cast<int64_t>(mt) * (kBM * CG) + rank * kBM;
     m.yrow = m.arow;
     const int64_t left = p.M - m.arow;
     m.rows = static_cast<int>(left < kBM ? (left < 0 ? 0 : left) : kBM);
@@ -196,6 +201,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* cum_m = reinterpret_cast<int*>(tmem_slot + 4);
+  int* cum_g = cum_m + (kMaxExperts + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = CG == 2 ? static_cast<int>(ptx::cluster_ctarank()) : 0;
@@ -211,10 +217,12 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     cum_m[0] = 0;
+    cum_g[0] = 0;
     if (p.offsets) {
       for (int e = 0; e < p.E; ++e) {
         const int64_t rows = p.offsets[e + 1] - p.offsets[e];
-        cum_m[e + 1] = cum_m[e] + static_cast<int>((rows + kBM - 1) / kBM);
+        cum_m[e + 1] = cum_m[e] + static_cast<int>((rows + kBM * CG - 1) / (kBM * CG));
+        cum_g[e + 1] = cum_g[e] + static_cast<int>((rows + kBM - 1) / kBM);
       }
     } else {
       cum_m[1] = static_cast<int>((p.M + kBM * CG - 1) / (kBM * CG));
@@ -242,7 +250,8 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   const uint32_t tmem = *tmem_slot;
   const int total_tiles = cum_m[p.E] * p.n_tiles;
   const int ktiles = p.KT + p.ST;
-  const int m_groups = static_cast<int>((p.M + kBM - 1) / kBM);   // 128-row scale groups (dense)
+  // 128-row scale groups of the activation buffer (for experts: the padded rows it holds)
+  const int64_t m_groups = p.offsets ? p.a_groups : (p.M + kBM - 1) / kBM;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -254,10 +263,11 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
       uint32_t sfl_bits = 0, last_fp4 = 0;   // per stage: parity of its next FP4 use; last use was FP4
       bool ok = true;
       for (int t = unit; t < total_tiles && ok; t += nunits) {
-        const TileMap m = map_tile<CG>(t, p, cum_m, rank);
-        // Scale atoms of rows past the end of a dense problem are not in the buffer: skip them
-        // (those output rows are discarded).
-        const bool sfa_ok = p.offsets || (m.arow / kBM) < m_groups;
+        const TileMap m = map_tile<CG>(t, p, cum_m, cum_g, rank);
+        // Scale atoms of rows past the end of the activation buffer (a dense problem's last pair,
+        // an expert's last pair at the end of the buffer) are not there: skip them (those output
+        // rows are discarded).
+        const bool sfa_ok = (m.arow / kBM) < m_groups;
         const int64_t brow = m.brow + rank * C::B_ROWS;
         for (int kt = 0; kt < ktiles; ++kt) {
           if (!wait_bar(empty + stage, phase ^ 1, abort_flag, p.err, p.wait_ns)) { ok = false; break; }
@@ -420,7 +430,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     int acc = 0, nbuf = 0, i = 0;
     uint32_t acc_phase = 0;
     for (int t = unit; t < total_tiles; t += nunits, ++i) {
-      const TileMap m = map_tile<CG>(t, p, cum_m, rank);
+      const TileMap m = map_tile<CG>(t, p, cum_m, cum_g, rank);
       if (!wait_bar(acc_full + acc, acc_phase, abort_flag, p.err, p.wait_ns)) break;
       ptx::tc_fence_after();
       const float alpha = p.alpha ? __ldg(p.alpha + (p.offsets ? m.e : segment_of(m.n0, p.seg))) : 1.0f;
@@ -602,6 +612,7 @@ fs_status launch_cfg(const TcLaunch& L, TcParams prm, int units, cudaStream_t s)
   // then the tiles in flight belong to a few consecutive experts, whose weights stay in L2 while
   // each of their 128-row activation tiles meets every N-tile.
   prm.n_fast = (prm.offsets || (prm.E == 1 && static_cast<int64_t>(prm.N) <= L.a_rows)) ? 1 : 0;
+  prm.a_groups = ceil_div(L.a_rows, kBM);
   CUtensorMap tmA, tmB, tmSA, tmSB;
   const uint64_t kbytes = static_cast<uint64_t>(prm.K) / 2;
   if (prm.KT > 0) {
@@ -694,11 +705,12 @@ fs_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, u
 fs_status launch_splice_gemm_tc(const TcLaunch& L, const TcParams& prm, cudaStream_t s) {
   if (prm.E > kMaxExperts) return fail(FS_ERR_UNSUPPORTED, "fs_splice_gemm: at most %d experts", kMaxExperts);
   const int64_t m_tiles = ceil_div(L.a_rows, kBM);
-  // Dense problems with N % 256 == 0 and at least two 128-row tiles run on CTA pairs.
-  if (L.bn == 256 && !prm.offsets && m_tiles >= 2) {
+  // Problems with N % 256 == 0 and at least two 128-row tiles run on CTA pairs (experts: each
+  // expert's rows in 256-row pair tiles, at most one more pair tile per expert than dense).
+  if (L.bn == 256 && m_tiles >= 2) {
     const int slots = pair_slots();
     if (slots > 0) {
-      const int64_t tiles = ceil_div(L.a_rows, 2 * kBM) * (prm.N / 256);
+      const int64_t tiles = (ceil_div(L.a_rows, 2 * kBM) + (prm.offsets ? prm.E : 0)) * (prm.N / 256);
       const int units = static_cast<int>(std::min<int64_t>(tiles, slots));
       return launch_cfg<256, 2>(L, prm, units, s);
     }
