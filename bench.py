@@ -53,7 +53,7 @@ DECODE_LAYERS = 36
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch per shape of the current kernel, summed
 # over the step's launches (qkv, o, gate_up, down).  None where no capture of the current kernel
 # exists (the one-launch-per-projection form, --unfused).
-GEMM_DRAM_BYTES_PER_STEP = {"fused": 1368882176, "unfused": None}
+GEMM_DRAM_BYTES_PER_STEP = {"fused": 1361701376, "unfused": None}
 
 
 # Issue rate of this kernel's block-scaled MMA alone (kind::mxf4nvf4, 256 x 256 x 64 on CTA pairs and
@@ -838,7 +838,10 @@ def kernel_case(F, args, device):
     xq = F.fs_quantize_splice(X, mask[0], args.p, g)
     plan = F.Plan(N, K, max(args.p, 1))
     Y = torch.empty(M, N, dtype=torch.float32, device=device)
-    if len(rows) == 1:
+    if args.case == "decode" and args.decode_prep == "fused":
+        run = lambda: F.fs_decode_splice_gemm(plan, X, mask[0], args.p, g, wall, alpha,
+                                              seg_start=seg if len(rows) > 1 else None, Y=Y)
+    elif len(rows) == 1:
         run = lambda: F.fs_splice_gemm(plan, xq, wall, alpha, Y=Y)
     else:
         run = lambda: F.fs_splice_gemm_segmented(plan, xq, wall, alpha, seg, Y=Y)
@@ -847,6 +850,7 @@ def kernel_case(F, args, device):
     ms = timed(run, args.steps) / args.steps
     plan.check()
     print(json.dumps({"case": args.case, "shape": args.shape, "M": M, "N": N, "K": K, "p": args.p,
+                      "decode_prep": args.decode_prep if args.case == "decode" else None,
                       "us": ms * 1000.0, "tflops": 2.0 * M * N * K / (ms * 1e-3) / 1e12}))
 
 
@@ -868,6 +872,9 @@ def main():
     ap.add_argument("--shape", default="q", choices=[name for name, _, _, _ in PROJ] + list(GROUP_NAMES[::2]),
                     help="projection shape of --case gemm / decode")
     ap.add_argument("--decode-m", type=int, default=16, help="tokens of --case decode (1..16)")
+    ap.add_argument("--decode-prep", default="packed", choices=["packed", "fused"],
+                    help="--case decode: GEMM on prepared activations, or fs_decode_splice_gemm (preparation "
+                         "inside the launch)")
     ap.add_argument("--prep", default="separate", choices=["fused", "separate"],
                     help="fused: reselect from the previous step's moments, then one pass over X for the "
                          "quantise and the next moments (fs_quantize_splice_stats); separate: statistics, "
