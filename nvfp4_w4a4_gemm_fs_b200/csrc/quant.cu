@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
   __shared__ uint16_t sh_col[16384 / 16];               // side-buffer column of each block's first protected lane
   __shared__ uint16_t sh_pidx[256];                     // channel of each side-buffer column (p <= 256)
   __shared__ float sh_val[128], sh_rcp[128];            // UE4M3 value and RN(1/value) per code
+  __shared__ int sh_wsum[kQThreads / 32];               // per-warp totals of the mask scan
   __shared__ int64_t sh_pad[kGrouped ? kMaxGroupedExperts + 1 : 1];   // padded start of each expert
   __shared__ int64_t sh_off[kGrouped ? kMaxGroupedExperts + 1 : 1];   // row offsets of the experts
 
@@ -221,25 +222,38 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
       if (a.p > 0) {
         __syncthreads();                           // previous expert's tables no longer read
         // per block: its 16 mask bits and the side column of its first protected lane
-        // (protected channels before it), by a block-wide scan in 32-block steps
+        // (protected channels before it).  Thread t takes the contiguous blocks
+        // [t*per, t*per + per) (per <= 4 for K <= 16384): all mask words are loaded in one round
+        // trip, then an exclusive scan of the per-thread counts over the CTA.
         const int nb = a.nb;
-        int carry = 0;
-        for (int b0 = 0; b0 < nb; b0 += 32) {
-          if (tid < 32) {
-            const int b = b0 + tid;
-            const uint32_t mb = (b < nb) ? ((__ldg(mask + (b >> 1)) >> ((b & 1) * 16)) & 0xFFFFu) : 0u;
-            const int cnt = __popc(mb);
-            int incl = cnt;
+        const int per = (nb + kQThreads - 1) / kQThreads;
+        const int bt0 = tid * per;
+        uint32_t mbv[4];
+        int cnt = 0;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const int y = __shfl_up_sync(0xffffffffu, incl, o);
-              if (tid >= o) incl += y;
-            }
-            if (b < nb) {
-              sh_mbits[b] = static_cast<uint16_t>(mb);
-              sh_col[b] = static_cast<uint16_t>(carry + incl - cnt);
-            }
-            carry += __shfl_sync(0xffffffffu, incl, 31);
+        for (int j = 0; j < 4; ++j) {
+          const int b = bt0 + j;
+          mbv[j] = (j < per && b < nb) ? ((__ldg(mask + (b >> 1)) >> ((b & 1) * 16)) & 0xFFFFu) : 0u;
+          cnt += __popc(mbv[j]);
+        }
+        const int lane = tid & 31, wid = tid >> 5;
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (lane == 31) sh_wsum[wid] = incl;
+        __syncthreads();
+        int col = incl - cnt;
+        for (int w = 0; w < wid; ++w) col += sh_wsum[w];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int b = bt0 + j;
+          if (j < per && b < nb) {
+            sh_mbits[b] = static_cast<uint16_t>(mbv[j]);
+            sh_col[b] = static_cast<uint16_t>(col);
+            col += __popc(mbv[j]);
           }
         }
         __syncthreads();
@@ -255,7 +269,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
         }
         if constexpr (sizeof(T) == 2) {
           for (int b = tid; b < nb; b += kQThreads) {
-            const uint32_t mb = (__ldg(mask + (b >> 1)) >> ((b & 1) * 16)) & 0xFFFFu;
+            const uint32_t mb = sh_mbits[b];
             uint32_t k[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
