@@ -1040,7 +1040,7 @@ def main():
                      "kernel": f"splice_gemm_tc_kernel ({len(gemm_names)} launches: {', '.join(gemm_names)}; "
                                "sum 2MNK / sum of CUDA-event times)",
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x 4 (nominal fp4/bf16 ratio), "
-                                    "of measured",
+                                    f"of {peaks['source']}",
                      "peak_fp4_mma_only_tflops": FP4_MMA_ONLY_TFLOPS,
                      "frac_vs_mma_only": gemm_tflops / FP4_MMA_ONLY_TFLOPS},
         "gemm_us": per_proj,
