@@ -15,6 +15,10 @@
 //               before its MMAs) and issues the MMAs
 //   warps 2..5  epilogue: TMEM -> shared-memory partial; after a cluster barrier each CTA sums a
 //               contiguous share of the tile's outputs over all CTAs of the cluster, x alpha, store
+// The kFuse form (fs_decode_splice_gemm) takes bf16 activations instead of packed ones: the
+// producer loads only the weight side, and warps 2..5, before their epilogue, encode this CTA's K
+// range of the tokens into each stage (Mask S->0, FP4 Quant, Extract X_S of §5.1 "Data
+// preparation") and hand it to the MMA thread through a second per-stage barrier.
 // Every mbarrier wait is bounded; on expiry the kernel records a timeout in the error word and
 // still reaches both cluster barriers and releases TMEM.
 #include <cudaTypedefs.h>

@@ -74,3 +74,36 @@ def test_stats_range_flag_is_reported():
     ref = stats.accumulate(stats.new_state(K), x)
     assert ref["flags"] == 1
     assert np.array_equal(st.s1[0].cpu().numpy(), ref["s1"]) and np.array_equal(st.s2[0].cpu().numpy(), ref["s2"])
+
+
+def test_fused_decode_wait_runs_out_then_context_still_computes():
+    """The decode kernel with the activation preparation inside (fs_decode_splice_gemm): with no
+    weight copies issued, the MMA thread's waits run out while the preparing warps, which fill the
+    first stages and then wait for a stage to be released, give up theirs; the launch reports
+    FS_ERR_TIMEOUT and a normal fused launch afterwards matches the oracle.  K = 8192 gives every
+    CTA of the cluster four FP4 k-tiles, more than its three stages."""
+    M, N, K, p = 4, 256, 8192, 64
+    x, _ = synth.outlier_activations(71, M, K)
+    w = synth.gaussian_weights(72, N, K)
+    X, W = splice.as_f32(x, True), splice.as_f32(w, True)
+    st = stats.accumulate(stats.new_state(K), X)
+    P = stats.select_topk(st, p)
+    gA = stats.next_gain(st, P)
+    mask = mask_tensor(stats.protect_mask(P, K))
+    g = torch.tensor([float(gA)], device="cuda")
+    wq, _, alpha = F.fs_prepare_weights(bf16_tensor(w), mask, p, g)
+    Xt = bf16_tensor(x)
+    starved = F.Plan(N, K, p, F.FS_PATH_DECODE | F.FS_FAULT_NO_COPIES)
+    F.fs_decode_splice_gemm(starved, Xt, mask, p, g, wq, alpha)
+    with pytest.raises(F.FoursightError) as exc:
+        starved.check()
+    assert exc.value.status == 5, str(exc.value)
+    good = F.Plan(N, K, p, F.FS_PATH_DECODE)
+    Y = F.fs_decode_splice_gemm(good, Xt, mask, p, g, wq, alpha,
+                                Y=torch.full((M, N), float("nan"), device="cuda"))
+    good.check()
+    xr = splice.quantize_splice(X, P, gA)
+    wr = splice.prepare_weights(W, P, gA)
+    Yr, mag = splice.splice_gemm(xr, wr, wr["alpha"])
+    got = Y.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - Yr) <= 1e-5 * mag)
