@@ -6,7 +6,8 @@
 // the advantage (A' = f A) and keeps the original 1/G loss denominator.  §2.1 gives the group
 // advantage A = (r - mu) / sigma.
 //
-// One CTA per sequence.  Each thread summarises a contiguous chunk of tokens as
+// One CTA per sequence, plus one warp that computes the group advantage meanwhile.  Each of the
+// kFThreads scanning threads summarises a contiguous chunk of tokens as
 // (length, count, leading run, trailing run, longest run); the summaries combine associatively
 // in token order, first within a warp with shuffles, then across warps in shared memory.
 #include "common.cuh"
@@ -53,13 +54,39 @@ __device__ __forceinline__ RunSum shfl_down(const RunSum& s, int o) {
   return r;
 }
 
-__global__ void __launch_bounds__(kFThreads)
+__global__ void __launch_bounds__(kFThreads + 32)
 seq_filter_kernel(const float* __restrict__ logp, int64_t ld, const int32_t* __restrict__ lengths, int T,
                   float log_tau, int K1, int K2, int G, const float* __restrict__ rewards, float* adv,
                   uint8_t* keep, int32_t* tail_count, int32_t* max_run, bool vec_rows) {
   __shared__ RunSum sh[kFThreads / 32];
+  __shared__ float sh_adv;
   const int s = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // The group advantage (§2.1) does not depend on the tokens: an extra warp computes it while the
+  // kFThreads others scan (one thread, sequential float64 order, as the oracle sums).
+  // Barrier 1 joins the scanning warps and, when it works, the extra warp (whole warps only).
+  const uint32_t nbar = kFThreads + (rewards ? 32 : 0);
+  auto bar_sync = [&]() { asm volatile("bar.sync 1, %0;" ::"r"(nbar) : "memory"); };
+  if (warp == kFThreads / 32) {
+    if (!rewards) return;                          // the whole warp: not counted in nbar
+    if (lane == 0) {
+      const int g0 = (s / G) * G;
+      double sum = 0.0;
+      for (int i = 0; i < G; ++i) sum = __dadd_rn(sum, static_cast<double>(__ldg(rewards + g0 + i)));
+      const double mu = __ddiv_rn(sum, static_cast<double>(G));
+      double q = 0.0;
+      for (int i = 0; i < G; ++i) {
+        const double d = __dsub_rn(static_cast<double>(__ldg(rewards + g0 + i)), mu);
+        q = __dadd_rn(q, __dmul_rn(d, d));
+      }
+      const double sigma = __dsqrt_rn(__ddiv_rn(q, static_cast<double>(G)));
+      float A = 0.0f;
+      if (sigma > 0.0) A = __double2float_rn(__ddiv_rn(__dsub_rn(static_cast<double>(__ldg(rewards + s)), mu), sigma));
+      sh_adv = A;
+    }
+    bar_sync();
+    return;
+  }
   int L = lengths ? __ldg(lengths + s) : T;
   L = L < 0 ? 0 : (L > T ? T : L);
   const float* row = logp + static_cast<int64_t>(s) * ld;
@@ -88,7 +115,7 @@ seq_filter_kernel(const float* __restrict__ logp, int64_t ld, const int32_t* __r
     if (lane + o < 32 && (lane & (2 * o - 1)) == 0) acc = combine(acc, other);
   }
   if (lane == 0) sh[warp] = acc;
-  __syncthreads();
+  bar_sync();
   if (tid == 0) {
     RunSum tot = sh[0];
     for (int w = 1; w < kFThreads / 32; ++w) tot = combine(tot, sh[w]);
@@ -97,19 +124,7 @@ seq_filter_kernel(const float* __restrict__ logp, int64_t ld, const int32_t* __r
     tail_count[s] = tot.cnt;
     max_run[s] = tot.best;
     if (rewards) {
-      const int g0 = (s / G) * G;
-      double sum = 0.0;
-      for (int i = 0; i < G; ++i) sum = __dadd_rn(sum, static_cast<double>(__ldg(rewards + g0 + i)));
-      const double mu = __ddiv_rn(sum, static_cast<double>(G));
-      double q = 0.0;
-      for (int i = 0; i < G; ++i) {
-        const double d = __dsub_rn(static_cast<double>(__ldg(rewards + g0 + i)), mu);
-        q = __dadd_rn(q, __dmul_rn(d, d));
-      }
-      const double sigma = __dsqrt_rn(__ddiv_rn(q, static_cast<double>(G)));
-      float A = 0.0f;
-      if (sigma > 0.0) A = __double2float_rn(__ddiv_rn(__dsub_rn(static_cast<double>(__ldg(rewards + s)), mu), sigma));
-      adv[s] = k ? A : 0.0f;
+      adv[s] = k ? sh_adv : 0.0f;                  // written before the barrier above
     } else if (adv) {
       adv[s] = k ? adv[s] : 0.0f;
     }
@@ -134,7 +149,7 @@ extern "C" fs_status fs_seq_filter(const float* logp, int64_t ld, const int32_t*
     if (!adv) return fail(FS_ERR_INVALID_ARGUMENT, "fs_seq_filter: rewards given without adv output");
     if (G < 1 || S % G != 0) return fail(FS_ERR_INVALID_ARGUMENT, "fs_seq_filter: need G >= 1 and S %% G == 0 with rewards");
   }
-  seq_filter_kernel<<<S, kFThreads, 0, static_cast<cudaStream_t>(stream)>>>(logp, ld, lengths, T, log_tau, K1, K2, G,
+  seq_filter_kernel<<<S, kFThreads + 32, 0, static_cast<cudaStream_t>(stream)>>>(logp, ld, lengths, T, log_tau, K1, K2, G,
                                                                            rewards, adv, keep, tail_count, max_run, vec_rows);
   FS_CHECK_LAUNCH("fs_seq_filter");
   return FS_OK;
