@@ -300,13 +300,19 @@ __global__ void __launch_bounds__(kQSThreads, 2) quantize_stats_kernel(const QSA
 // One wave: as many row groups per slab as fill the resident CTA slots, each with at least 16 row
 // pairs per warp when the batch is large enough.
 fs_status launch_quantize_rows(const QSArgs& a, bool with_stats, cudaStream_t s, const char* who) {
-  static PerDevice<int> occ;
+  // resident CTAs per SM of the instantiation that runs (the moments take twice the registers)
+  static PerDevice<int> occ_stats, occ_plain;
   int slots = 1;
-  if (!occ.get(current_device(), &slots, [](int* v) {
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, quantize_stats_kernel<true>, kQSThreads, 0) ==
-                   cudaSuccess && *v >= 1;
-      }))
-    slots = 1;
+  const bool got = with_stats
+      ? occ_stats.get(current_device(), &slots, [](int* v) {
+          return cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, quantize_stats_kernel<true>, kQSThreads, 0) ==
+                     cudaSuccess && *v >= 1;
+        })
+      : occ_plain.get(current_device(), &slots, [](int* v) {
+          return cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, quantize_stats_kernel<false>, kQSThreads, 0) ==
+                     cudaSuccess && *v >= 1;
+        });
+  if (!got) slots = 1;
   const int chunks = static_cast<int>(ceil_div(a.K, kSlab));
   int64_t gy = std::max<int64_t>(1, static_cast<int64_t>(slots) * sm_count() / chunks);
   gy = std::min<int64_t>(gy, std::max<int64_t>(1, ceil_div(a.Mp, 2 * kQSWarps * 16)));
