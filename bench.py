@@ -730,6 +730,15 @@ def cpu_baseline(rows=M_PREFILL):
             "seconds": dt}
 
 
+def step_config(world, p, prep):
+    """The `config` of both arms' JSON lines: the workload the metric is quoted on."""
+    return {"workload": "Qwen3-8B-shaped prefill layer: M=8192 bf16 tokens (8x1024), 7 projections, P=64; "
+                        "per step stats + top-64 reselect + weight pre-split + quantise + SpliceGEMM",
+            "global_batch": world * M_PREFILL, "seq_len": 1024, "parallelism": f"dp{world}",
+            "p": p, "prep": prep,
+            "l2": "inputs larger than L2 (0.85 GB of bf16 activations and weights per step)"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -746,8 +755,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * tot / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "Qwen3-8B-shaped prefill, M=8192 bf16, P=64 (oracle sample: the q projection, all 8192 rows)",
-                       "global_batch": M_PREFILL, "seq_len": 1024, "parallelism": "cpu"},
+            "config": step_config(args.gpus, args.p, args.prep),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                              "sample": "q projection 4096x4096 of all 8192 tokens per step, P=64: stats, select, "
                                        "weight pre-split, quantise, float64 SpliceGEMM"},
@@ -1026,11 +1034,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4 e2m1/ue4m3 + bf16 side, fp32 accumulate and output",
         "data": "synthetic (seeded N(0,1) activations with 1% channels x30, N(0,0.02) weights)",
-        "config": {"workload": "Qwen3-8B-shaped prefill layer: M=8192 bf16 tokens (8x1024), 7 projections, P=64; "
-                               "per step stats + top-64 reselect + weight pre-split + quantise + SpliceGEMM",
-                   "global_batch": world * M_PREFILL, "seq_len": 1024, "parallelism": f"dp{world}",
-                   "p": p, "prep": args.prep,
-                   "l2": "inputs larger than L2 (0.85 GB of bf16 activations and weights per step)"},
+        "config": step_config(world, p, args.prep),
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_STEP[fkey],
                      "traffic_unit": f"DRAM bytes per step (the {len(gemm_names)} GEMM launches; ncu "
