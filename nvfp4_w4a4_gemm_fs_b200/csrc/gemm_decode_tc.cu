@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "moments.cuh"
 #include "ptx.cuh"
 
 namespace fs {
@@ -172,10 +173,13 @@ __device__ __forceinline__ PrepBlock prep_block(const uint32_t (&w)[8], uint32_t
   float v[16];
   if (fast) {
     const float R = __fmul_rn(g, sr);              // exact: g is a power of two in range
+    // two elements per packed multiply (each lane the IEEE RN product of the scalar form)
+    const uint64_t R2 = moments::pack_f32x2(R, R);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      v[2 * j] = snap12(__fmul_rn(bf16_lo(xm[j]), R));
-      v[2 * j + 1] = snap12(__fmul_rn(bf16_hi(xm[j]), R));
+      const uint64_t pr = moments::mul_f32x2(moments::pack_f32x2(bf16_lo(xm[j]), bf16_hi(xm[j])), R2);
+      v[2 * j] = snap12(__uint_as_float(static_cast<uint32_t>(pr)));
+      v[2 * j + 1] = snap12(__uint_as_float(static_cast<uint32_t>(pr >> 32)));
     }
   } else {
 #pragma unroll
