@@ -247,7 +247,9 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
       ptx::prefetch_tensormap(&tmWS);
       if constexpr (!kFuse) ptx::prefetch_tensormap(&tmXS);
     }
-    if (!p.no_copies)
+    // (not in the fused form, whose preparing warps read X meanwhile: measured faster without it
+    // at 16 tokens and equal at 1)
+    if (!kFuse && !p.no_copies)
       for (int kt = kt0; kt < kt1; ++kt) ptx::tma_prefetch_2d(&tmW, kt * 128, n0);
   }
   if (warp == 1) {
