@@ -251,6 +251,18 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr) {
   return v;
 }
 
+// 32-bit load from a CTA of the cluster; same ordering rule as ld_shared_cluster_v4.
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+// Atomic max into a 32-bit word in the shared memory of a CTA of the cluster (no return value);
+// made visible to the owner by the next cluster barrier (arrive.release / wait.acquire).
+__device__ __forceinline__ void red_max_shared_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.max.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 // Instruction descriptor: kind::mxf4nvf4 with E2M1 A/B, UE4M3 scales (16-element blocks), K-major.
 __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
   return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (0u << 23) |

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "moments.cuh"
+#include "ptx.cuh"
 
 namespace fs {
 namespace {
@@ -181,10 +182,13 @@ channel_stats_kernel(const T* __restrict__ X, int64_t M, int K, int64_t ldx, int
 }
 
 // ------------------------------------------------------------------------------------------
-// Reselection: one CTA per problem.
+// Reselection: one cluster of kSelCluster CTAs per problem.
 // ------------------------------------------------------------------------------------------
-constexpr int kSelThreads = 1024;
-constexpr int kMaxK = 16384;
+constexpr int kSelCluster = 8;
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelMaxR = 4;                   // rounds of 32 channels per warp
+constexpr int kMaxK = kSelCluster * kSelThreads * kSelMaxR;   // 16384
 
 // Map a double key to an unsigned integer with the same order (-0 folded onto +0 first).
 __device__ __forceinline__ unsigned long long order_bits(double k) {
@@ -193,70 +197,138 @@ __device__ __forceinline__ unsigned long long order_bits(double k) {
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
-__device__ __forceinline__ double channel_key(long long n, long long s1, long long s2, bool m2_only) {
-  if (n == 0) return 0.0;
-  const double dn = __ll2double_rn(n);
-  const double m2 = __ddiv_rn(__ll2double_rn(s2) / kS2Scale, dn);   // /2^14 exact
+// Correctly rounded y / d in fp64 from r = RN(1/d), by Markstein's correction (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev.
+// 34(1), 1990), the fp64 counterpart of the library's fp32 division: q0 = RN(y*r) is within two
+// ulps; the first remainder step makes it faithful (pre-rounding error below 4u^2 |y/d|, u = 2^-53),
+// after which the remainder y - d*q1 is exact in one fused multiply-add and the second step
+// rounds correctly.  Used with d = n >= 1 and y a scaled integer moment, so nothing underflows.
+__device__ __forceinline__ double div_rn_by(double y, double d, double r) {
+  const double q0 = __dmul_rn(y, r);
+  const double e0 = __fma_rn(-q0, d, y);
+  const double q1 = __fma_rn(e0, r, q0);
+  const double e1 = __fma_rn(-q1, d, y);
+  return __fma_rn(e1, r, q1);
+}
+
+// Key of one channel: fl64(m2 - fl64(m1 * m1)) with m1 = fl64(fl64(s1 / 2^16) / n),
+// m2 = fl64(fl64(s2 / 2^14) / n); dn = n and rn = RN(1/n) are the problem's (n > 0).
+__device__ __forceinline__ double channel_key(double dn, double rn, long long s1, long long s2, bool m2_only) {
+  const double m2 = div_rn_by(__ll2double_rn(s2) / kS2Scale, dn, rn);   // /2^14 exact
   if (m2_only) return m2;
-  const double m1 = __ddiv_rn(__ll2double_rn(s1) / kS1Scale, dn);   // /2^16 exact
+  const double m1 = div_rn_by(__ll2double_rn(s1) / kS1Scale, dn, rn);   // /2^16 exact
   return __dsub_rn(m2, __dmul_rn(m1, m1));
 }
 
-__global__ void __launch_bounds__(kSelThreads)
-select_topk_kernel(int K, long long* n_all, long long* s1_all, long long* s2_all, uint32_t* amax_all,
+// The cluster's CTAs split the channels: CTA c takes [c*chunk, (c+1)*chunk), chunk = 512*R, and
+// its warp w the 32*R channels from c*chunk + 32*R*w, one round of 32 consecutive channels (one
+// mask word) per step, so every thread holds at most kSelMaxR keys in registers.
+//
+// The p-th largest key is found by a radix select over the cluster, 8 bits at a time from the top:
+// each CTA histograms its keys that match the prefix so far (warp-aggregated shared atomics), and
+// after a cluster barrier every CTA sums the 8 histograms through distributed shared memory and
+// takes the same decision.  Histograms are double-buffered, so one barrier per pass suffices: a
+// CTA rewrites a buffer only after the next pass's barrier, which every other CTA reaches after
+// reading it.  Once the bin holding the p-th key is taken whole (its count equals the keys still
+// needed) every key from the bin's prefix up is selected and the passes stop.
+//
+// Selected: key > T, plus the `need` lowest-index channels with key == T.  The CTAs exchange
+// their counts of keys > T and == T (one barrier), which fixes each warp's first tie rank and
+// first output slot; the warps then walk their rounds with ballots, writing P in ascending order
+// and one mask word per round.  The maximum of the unprotected channels' amax goes to CTA 0 by
+// remote atomics; after the last barrier CTA 0 writes the gain.
+__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThreads)
+select_topk_kernel(int K, int R, long long* n_all, long long* s1_all, long long* s2_all, uint32_t* amax_all,
                    uint32_t* flags_all, int p, uint32_t opts, int32_t* P_all, uint32_t* mask_all,
                    float* gA_all, int reset) {
-  extern __shared__ unsigned long long sh_keys[];         // [K]
-  __shared__ unsigned int hist[256];
+  __shared__ unsigned int hist[2][256];          // this CTA's histogram of the pass (double-buffered)
+  __shared__ unsigned int tot[256];              // the cluster's histogram of the pass
   __shared__ unsigned long long sh_prefix;
-  __shared__ int sh_need, sh_binc, sh_ties;
-  __shared__ int sh_scan[kSelThreads / 32];
-  __shared__ uint32_t sh_amax[kSelThreads / 32];
+  __shared__ int sh_need, sh_binc;
+  __shared__ int sh_wgt[kSelWarps], sh_weq[kSelWarps];
+  __shared__ int sh_cnt[2];                      // this CTA's keys > T and == T (read by the cluster)
+  __shared__ uint32_t sh_wam[kSelWarps];
+  __shared__ uint32_t sh_am_cluster;             // CTA 0: maximum over the cluster
 
-  const int prob = blockIdx.x;
+  const int prob = blockIdx.x / kSelCluster;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
   const long long n = n_all[prob];
-  const long long* s1 = s1_all + static_cast<int64_t>(prob) * K;
-  const long long* s2 = s2_all + static_cast<int64_t>(prob) * K;
-  const uint32_t* amax = amax_all + static_cast<int64_t>(prob) * K;
+  long long* s1 = s1_all + static_cast<int64_t>(prob) * K;
+  long long* s2 = s2_all + static_cast<int64_t>(prob) * K;
+  uint32_t* amax = amax_all + static_cast<int64_t>(prob) * K;
   int32_t* P = P_all + static_cast<int64_t>(prob) * p;
   const int words = (K + 31) / 32;
   uint32_t* mask = mask_all + static_cast<int64_t>(prob) * words;
   const bool m2_only = opts & FS_KEY_M2;
-  const int tid = threadIdx.x;
+  const int j_warp = static_cast<int>(rank) * kSelThreads * R + warp * 32 * R;   // first channel of the warp
 
-  for (int j = tid; j < K; j += blockDim.x) sh_keys[j] = order_bits(channel_key(n, s1[j], s2[j], m2_only));
-  if (tid == 0) { sh_prefix = 0; sh_need = p; }
-  __syncthreads();
+  if (tid == 0) sh_am_cluster = 0;               // ordered before any remote access by a cluster barrier
 
-  // Radix select of the p-th largest ordered key, 8 bits at a time from the top.  Histogram
-  // updates are aggregated per warp (lanes with the same digit add once), and warp 0 finds the
-  // threshold digit with a suffix scan over 8 bins per lane.  Once the bin holding the p-th key
-  // is taken whole (its count equals the keys still needed), every key at or above the bin's
-  // prefix is selected: the passes stop with T = that prefix and `need` = the keys equal to it.
-  unsigned long long prefix = 0;
-  int need = p;
-  const int lane = tid & 31, warp_id = tid >> 5;
+  // Keys and maxima into registers, every load in flight at once; the moments are cleared (reset)
+  // by the thread that read them.
+  const double dn = __ll2double_rn(n);
+  const double rn = n > 0 ? __drcp_rn(dn) : 0.0;
+  unsigned long long key[kSelMaxR];
+  uint32_t am[kSelMaxR];
+  bool valid[kSelMaxR];
+  {
+    long long a1[kSelMaxR], a2[kSelMaxR];
+#pragma unroll
+    for (int r = 0; r < kSelMaxR; ++r) {
+      const int j = j_warp + r * 32 + lane;
+      valid[r] = r < R && j < K;
+      a1[r] = 0; a2[r] = 0; am[r] = 0;
+      if (valid[r]) { a1[r] = __ldcg(s1 + j); a2[r] = __ldcg(s2 + j); am[r] = __ldcg(amax + j); }
+    }
+#pragma unroll
+    for (int r = 0; r < kSelMaxR; ++r) {
+      key[r] = order_bits(n == 0 ? 0.0 : channel_key(dn, rn, a1[r], a2[r], m2_only));
+      if (valid[r] && reset) {
+        const int j = j_warp + r * 32 + lane;
+        s1[j] = 0; s2[j] = 0; amax[j] = 0;
+      }
+    }
+  }
+
+  // Threshold T and the number of keys equal to T to take (p = 0: nothing is selected).
+  unsigned long long T = ~0ull;
+  int need = 0;
   if (p > 0) {
-    for (int shift = 56; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    unsigned long long prefix = 0;
+    need = p;
+    int buf = 0;
+    for (int shift = 56; shift >= 0; shift -= 8, buf ^= 1) {
+      for (int i = tid; i < 256; i += kSelThreads) hist[buf][i] = 0;
       __syncthreads();
       const unsigned long long hi_mask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
-      for (int j0 = 0; j0 < K; j0 += blockDim.x) {
-        const int j = j0 + tid;
-        int bin = -1;
-        if (j < K) {
-          const unsigned long long k = sh_keys[j];
-          if ((k & hi_mask) == prefix) bin = static_cast<int>((k >> shift) & 0xFF);
+#pragma unroll
+      for (int r = 0; r < kSelMaxR; ++r) {
+        if (r < R) {                                  // uniform
+          const int bin = (valid[r] && (key[r] & hi_mask) == prefix) ? static_cast<int>((key[r] >> shift) & 0xFF) : -1;
+          const unsigned peers = __match_any_sync(0xffffffffu, bin);
+          if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[buf][bin], static_cast<unsigned>(__popc(peers)));
         }
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<unsigned>(__popc(peers)));
+      }
+      ptx::cluster_sync();                            // every CTA's histogram of this pass is complete
+      if (tid < 256) {
+        const uint32_t addr = ptx::smem_u32(&hist[buf][tid]);
+        unsigned int part[kSelCluster];
+#pragma unroll
+        for (int c = 0; c < kSelCluster; ++c) part[c] = ptx::ld_shared_cluster_u32(ptx::mapa_shared(addr, c));
+        unsigned int sum = 0;
+#pragma unroll
+        for (int c = 0; c < kSelCluster; ++c) sum += part[c];
+        tot[tid] = sum;
       }
       __syncthreads();
-      if (warp_id == 0) {
+      if (warp == 0) {
+        // suffix scan over 8 bins per lane: the digit holding the need-th largest remaining key
         int c[8], local = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { c[i] = static_cast<int>(hist[8 * lane + i]); local += c[i]; }
-        int incl = local;                                  // sum over lanes >= this lane
+        for (int i = 0; i < 8; ++i) { c[i] = static_cast<int>(tot[8 * lane + i]); local += c[i]; }
+        int incl = local;                                  // keys in the bins of lanes >= this lane
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int y = __shfl_down_sync(0xffffffffu, incl, o);
@@ -264,121 +336,95 @@ select_topk_kernel(int K, long long* n_all, long long* s1_all, long long* s2_all
         }
         const int above = incl - local;
         if (above < need && need <= incl) {
-          int r = need - above, d = 8 * lane, bc = 0;
+          int rem = need - above, d = 8 * lane, bc = 0;
 #pragma unroll
           for (int i = 7; i >= 0; --i) {
-            if (c[i] >= r) { d = 8 * lane + i; bc = c[i]; break; }
-            r -= c[i];
+            if (c[i] >= rem) { d = 8 * lane + i; bc = c[i]; break; }
+            rem -= c[i];
           }
           sh_prefix = prefix | (static_cast<unsigned long long>(d) << shift);
-          sh_need = r;
+          sh_need = rem;
           sh_binc = bc;
         }
       }
-      if (tid == 0) sh_ties = 0;
       __syncthreads();
       prefix = sh_prefix;
       need = sh_need;
-      if (shift > 0 && sh_binc == need) {          // uniform: the whole bin is selected
-        int eq = 0;
-        for (int j = tid; j < K; j += blockDim.x) eq += sh_keys[j] == prefix;
-        if (eq) atomicAdd(&sh_ties, eq);
-        __syncthreads();
-        need = sh_ties;
+      const bool whole_bin = shift > 0 && sh_binc == need;   // uniform over the cluster
+      if (whole_bin || shift == 0) {
+        T = prefix;
+        if (whole_bin) need = p;                     // every key == T lies in the bin: take them all
         break;
       }
-      __syncthreads();
     }
   }
-  // Selected: key > T, plus the `need` lowest-index channels with key == T (T = prefix).
-  // Channels are visited in index order, chunk per thread, with block-wide exclusive scans.
-  const int per = (K + blockDim.x - 1) / blockDim.x;
-  const int j0 = tid * per, j1 = min(K, j0 + per);
-  int n_gt = 0, n_eq = 0;
-  if (p > 0) {
-    for (int j = j0; j < j1; ++j) {
-      n_gt += sh_keys[j] > prefix;
-      n_eq += sh_keys[j] == prefix;
-    }
-  }
-  // exclusive scan of n_eq over threads (to rank ties by index)
-  auto block_exclusive_scan = [&](int v) -> int {
-    const int lane = tid & 31, warp = tid >> 5;
-    int x = v;
+
+  // Per warp: keys > T and == T; per CTA: their sums, exchanged over the cluster.
+  int gt = 0, eq = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) sh_scan[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int s = (lane < (int)(blockDim.x >> 5)) ? sh_scan[lane] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, s, o);
-        if (lane >= o) s += y;
-      }
-      if (lane < (int)(blockDim.x >> 5)) sh_scan[lane] = s;
-    }
-    __syncthreads();
-    const int excl = x - v + (warp > 0 ? sh_scan[warp - 1] : 0);
-    __syncthreads();
-    return excl;
-  };
-  const int eq_before = block_exclusive_scan(n_eq);
-  // count selected in this chunk
-  int n_sel = 0;
-  if (p > 0) {
-    int eq_seen = eq_before;
-    for (int j = j0; j < j1; ++j) {
-      const unsigned long long k = sh_keys[j];
-      if (k > prefix || (k == prefix && eq_seen++ < need)) ++n_sel;
-    }
+  for (int r = 0; r < kSelMaxR; ++r) {
+    gt += __popc(__ballot_sync(0xffffffffu, valid[r] && key[r] > T));
+    eq += __popc(__ballot_sync(0xffffffffu, valid[r] && key[r] == T));
   }
-  const int sel_before = block_exclusive_scan(n_sel);
-  // write P (ascending) and the mask; unselected amax feed the gain
-  float am_unprot = 0.0f;
-  {
-    int eq_seen = eq_before, out = sel_before;
-    for (int j = j0; j < j1; ++j) {
-      const unsigned long long k = sh_keys[j];
-      const bool sel = p > 0 && (k > prefix || (k == prefix && eq_seen++ < need));
-      if (sel) P[out++] = j;
-      const float a = __uint_as_float(amax[j]);
-      if (!sel || (opts & FS_RESIDUAL)) am_unprot = fmaxf(am_unprot, a);
-      sh_keys[j] = sel ? 1ull : 0ull;       // reuse as the selection flag
-    }
-  }
+  if (lane == 0) { sh_wgt[warp] = gt; sh_weq[warp] = eq; }
   __syncthreads();
-  for (int w = tid; w < words; w += blockDim.x) {
-    uint32_t bits = 0;
-    for (int b = 0; b < 32; ++b) {
-      const int j = w * 32 + b;
-      if (j < K && sh_keys[j]) bits |= 1u << b;
-    }
-    mask[w] = bits;
+  if (tid == 0) {
+    int cg = 0, ce = 0;
+    for (int w = 0; w < kSelWarps; ++w) { cg += sh_wgt[w]; ce += sh_weq[w]; }
+    sh_cnt[0] = cg;
+    sh_cnt[1] = ce;
   }
-  // block max of the unprotected amax
-  uint32_t am = __float_as_uint(am_unprot);
+  ptx::cluster_sync();                               // every CTA's counts are visible
+  // Ties of lower-ranked CTAs and warps come first; a group with `e_before` ties before it and
+  // g, e of its own takes g + clamp(need - e_before, 0, e) channels.
+  int cta_g = 0, cta_e = 0;
+  if (lane < kSelCluster) {
+    const uint32_t base = ptx::smem_u32(&sh_cnt[0]);
+    cta_g = static_cast<int>(ptx::ld_shared_cluster_u32(ptx::mapa_shared(base, lane)));
+    cta_e = static_cast<int>(ptx::ld_shared_cluster_u32(ptx::mapa_shared(base + 4, lane)));
+  }
+  auto taken = [&](int g, int e, int e_before) { return g + min(max(need - e_before, 0), e); };
+  int e_before = 0, out = 0;
+  for (int c = 0; c < static_cast<int>(rank); ++c) {
+    const int g = __shfl_sync(0xffffffffu, cta_g, c), e = __shfl_sync(0xffffffffu, cta_e, c);
+    out += taken(g, e, e_before);
+    e_before += e;
+  }
+  for (int w = 0; w < warp; ++w) {
+    out += taken(sh_wgt[w], sh_weq[w], e_before);
+    e_before += sh_weq[w];
+  }
+  // The warp's rounds in channel order: P entries, mask words, the unprotected maximum.
+  uint32_t am_unprot = 0;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
-  if ((tid & 31) == 0) sh_amax[tid >> 5] = am;
+  for (int r = 0; r < kSelMaxR; ++r) {
+    if (r < R) {                                      // uniform
+      const uint32_t eqb = __ballot_sync(0xffffffffu, valid[r] && key[r] == T);
+      const bool sel = valid[r] && (key[r] > T || (key[r] == T && e_before + __popc(eqb & lt) < need));
+      const uint32_t selb = __ballot_sync(0xffffffffu, sel);
+      const int j = j_warp + r * 32 + lane;
+      const int slot = out + __popc(selb & lt);
+      if (sel && slot < p) P[slot] = j;
+      const int word = (j_warp + r * 32) >> 5;
+      if (lane == 0 && word < words) mask[word] = selb;
+      if (valid[r] && (!sel || (opts & FS_RESIDUAL))) am_unprot = max(am_unprot, am[r]);   // floats >= 0 order as uints
+      out += __popc(selb);
+      e_before += __popc(eqb);
+    }
+  }
+  am_unprot = __reduce_max_sync(0xffffffffu, am_unprot);
+  if (lane == 0) sh_wam[warp] = am_unprot;
   __syncthreads();
   if (tid == 0) {
     uint32_t m = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = max(m, sh_amax[w]);
-    const float a = __uint_as_float(m);
-    gA_all[prob] = (opts & FS_GAIN_EXACT) ? gain_exact(a) : gain_pow2(a);
+    for (int w = 0; w < kSelWarps; ++w) m = max(m, sh_wam[w]);
+    ptx::red_max_shared_cluster_u32(ptx::mapa_shared(ptx::smem_u32(&sh_am_cluster), 0), m);
   }
-  if (reset) {
-    __syncthreads();
-    for (int j = tid; j < K; j += blockDim.x) {
-      s1_all[static_cast<int64_t>(prob) * K + j] = 0;
-      s2_all[static_cast<int64_t>(prob) * K + j] = 0;
-      amax_all[static_cast<int64_t>(prob) * K + j] = 0;
-    }
-    if (tid == 0) { n_all[prob] = 0; flags_all[prob] = 0; }
+  ptx::cluster_sync();                               // the maxima have arrived; no CTA reads another's memory after this
+  if (rank == 0 && tid == 0) {
+    const float a = __uint_as_float(sh_am_cluster);
+    gA_all[prob] = (opts & FS_GAIN_EXACT) ? gain_exact(a) : gain_pow2(a);
+    if (reset) { n_all[prob] = 0; flags_all[prob] = 0; }   // every CTA read n before the first barrier
   }
 }
 
@@ -452,14 +498,10 @@ extern "C" fs_status fs_select_topk(int32_t nprob, int32_t K, int64_t* n, int64_
   if (nprob == 0) return FS_OK;
   if (!n || !s1 || !s2 || !amax || !flags || !mask || !gA || (p > 0 && !P)) return fail(FS_ERR_INVALID_ARGUMENT, "fs_select_topk: null pointer");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t smem = static_cast<size_t>(K) * sizeof(unsigned long long);
-  static PerDevice<int> attr;
-  fs_status ast = set_max_dynamic_smem(attr, reinterpret_cast<const void*>(select_topk_kernel), kMaxK * 8,
-                                       "fs_select_topk: smem attribute");
-  if (ast != FS_OK) return ast;
-  select_topk_kernel<<<nprob, kSelThreads, smem, s>>>(K, reinterpret_cast<long long*>(n), reinterpret_cast<long long*>(s1),
-                                                     reinterpret_cast<long long*>(s2), amax, flags, p, opts,
-                                                     P, mask, gA, reset);
+  const int R = static_cast<int>(ceil_div(K, kSelCluster * kSelThreads));   // 1..kSelMaxR
+  select_topk_kernel<<<static_cast<unsigned>(nprob) * kSelCluster, kSelThreads, 0, s>>>(
+      K, R, reinterpret_cast<long long*>(n), reinterpret_cast<long long*>(s1), reinterpret_cast<long long*>(s2), amax,
+      flags, p, opts, P, mask, gA, reset);
   FS_CHECK_LAUNCH("fs_select_topk");
   return FS_OK;
 }

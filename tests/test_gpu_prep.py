@@ -93,6 +93,47 @@ def test_select_topk_ties_and_empty_state():
     assert P2[0].cpu().tolist() == [0, 1, 2, 3] and g2.item() == 1.0
 
 
+@pytest.mark.parametrize("K,p", [(16384, 256), (16384, 1), (8256, 64), (1000, 17), (96, 96), (96, 5)])
+def test_select_topk_ranges_of_the_cluster(K, p):
+    """The selection splits K over the CTAs of a cluster (512 channels per CTA per round, up to 4
+    rounds): K = 16384 fills every round, 8256 leaves the last CTAs partly or wholly empty, 1000
+    ends inside a mask word, 96 sits inside the first CTA."""
+    nprob = 2
+    st = F.StatsState(nprob, K)
+    refs = []
+    for i in range(nprob):
+        X, T = _x(300 + i + K, 129, K, "bf16")
+        F.fs_channel_stats(T, st, group=i)
+        refs.append(stats.accumulate(stats.new_state(K), X))
+    P, mask, gA = F.fs_select_topk(st, p, reset=True)
+    for i in range(nprob):
+        Pr = stats.select_topk(refs[i], p)
+        assert np.array_equal(P[i].cpu().numpy(), Pr)
+        assert np.array_equal(mask[i].cpu().numpy().view(np.uint32), stats.protect_mask(Pr, K))
+        assert gA[i].item() == float(stats.next_gain(refs[i], Pr))
+    assert int(st.n.abs().sum()) == 0 and int(st.s1.abs().sum()) == 0 and int(st.flags.abs().sum()) == 0
+
+
+@pytest.mark.parametrize("p", [2, 5, 8])
+def test_select_topk_ties_across_ctas(p):
+    """Equal variances at channels that fall to different CTAs (K = 8192: 1024 channels per CTA):
+    two larger keys come first, then the tied channels in index order until p are taken."""
+    K = 8192
+    tied = [100, 1500, 3000, 5000, 7000, 8100]
+    x = np.zeros((2, K), np.float32)
+    x[0, tied] = 2.0; x[1, tied] = -2.0
+    x[0, [4000, 6500]] = 3.0; x[1, [4000, 6500]] = -3.0
+    x[:, 2000] = 1.5                                                     # zero variance, largest mean
+    st = F.StatsState(1, K)
+    F.fs_channel_stats(f32_tensor(x), st)
+    P, mask, gA = F.fs_select_topk(st, p)
+    ref_state = stats.accumulate(stats.new_state(K), x)
+    ref = stats.select_topk(ref_state, p)
+    assert P[0].cpu().tolist() == ref.tolist() == sorted([4000, 6500] + tied[:p - 2])
+    assert np.array_equal(mask[0].cpu().numpy().view(np.uint32), stats.protect_mask(ref, K))
+    assert gA.item() == float(stats.next_gain(ref_state, ref))
+
+
 # ----------------------------------------------------------------------------- quantisation
 def _prep_inputs(seed, M, K, p, dtype):
     X, T = _x(seed, M, K, dtype)
