@@ -189,14 +189,19 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
   if constexpr (kSide == Side::Weight) alpha_v = __ldg(a.alpha);
   const float inv6 = __frcp_rn(6.0f);
 
-  // General chunks: block i of the chunk is (row i / nb, block i % nb).  kRowPasses (nb a multiple
-  // of the CTA size): every pass covers kQThreads blocks of one row, its row and first block kept
-  // incrementally, so a pass costs no division and its row addresses are uniform.
+  // General chunks: block i of the chunk is (row i / nb, block i % nb), the quotient taken as
+  // trunc((i + 1/2) / nb) in fp32: i < 2^19 and nb <= 1024, so (i + 1/2) / nb lies at least 1/(2 nb)
+  // from every integer while the fp32 product errs by under 2^-23 of it, and the result is exact.
+  // kRowPasses (nb a multiple of the CTA size): every pass covers kQThreads blocks of one row, its
+  // row and first block kept incrementally, so a pass costs no division and its row addresses
+  // are uniform.
+  const float inv_nb = 1.0f / static_cast<float>(a.nb);
+  auto row_of = [&](int i) { return static_cast<int>((static_cast<float>(i) + 0.5f) * inv_nb); };
   auto load_one = [&](const ChunkLoc& L, int i0, RawBlock<T>& x) {
     const int i = i0 + tid;
-    const int r = i / a.nb;
+    const int r = row_of(i);
     if (L.e >= 0 && i < total && r < L.valid) {
-      const int b = i % a.nb;
+      const int b = i - r * a.nb;
       load_raw<T>(X + (L.src_row0 + r) * a.ldx + static_cast<int64_t>(b) * 16, x);
     }
   };
@@ -204,7 +209,17 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
     if (L.e >= 0 && r < L.valid) load_raw<T>(X + (L.src_row0 + r) * a.ldx + static_cast<int64_t>(b0 + tid) * 16, x);
   };
 
-  ChunkLoc L = locate(blockIdx.x);
+  // Chunks per CTA: grouped problems take a contiguous range (consecutive chunks mostly share an
+  // expert, so the expert's mask tables are built once per range instead of once per chunk); the
+  // plain call deals them round-robin (every wave of CTAs sweeps the matrix in order).
+  int64_t c_first = blockIdx.x, c_end = nchunks, c_step = gridDim.x;
+  if constexpr (kGrouped) {
+    const int64_t per = (nchunks + gridDim.x - 1) / gridDim.x;
+    c_first = static_cast<int64_t>(blockIdx.x) * per;
+    c_end = c_first + per < nchunks ? c_first + per : nchunks;
+    c_step = 1;
+  }
+  ChunkLoc L = locate(c_first < c_end ? c_first : nchunks);
   RawBlock<T> xc;
   if constexpr (kRowPasses) load_pass(L, 0, 0, xc);
   else load_one(L, 0, xc);
@@ -213,7 +228,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
   float g = 1.0f;
   bool fast = false;                               // snap12 path (bf16 input, power-of-two gain)
 
-  for (int64_t chunk = blockIdx.x; chunk < nchunks && L.e >= 0; chunk += gridDim.x) {
+  for (int64_t chunk = c_first; chunk < c_end && L.e >= 0; chunk += c_step) {
     if (L.e != cur_e) {                            // uniform across the CTA
       cur_e = L.e;
       mask = (a.p > 0) ? a.masks + static_cast<int64_t>(cur_e) * words : nullptr;
@@ -283,7 +298,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
         __syncthreads();
       }
     }
-    const ChunkLoc Ln = locate(chunk + gridDim.x);
+    const ChunkLoc Ln = locate(chunk + c_step < c_end ? chunk + c_step : nchunks);
     int r_cur = 0, b_cur = 0;                      // kRowPasses: row and first block of this pass
     for (int i0 = 0; i0 < total; i0 += kQThreads) {
       RawBlock<T> xn;
@@ -304,8 +319,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantArgs a, int64_
       } else {
         const int i = i0 + tid;
         in_range = i < total;
-        r = in_range ? i / a.nb : 0;
-        b = in_range ? i % a.nb : 0;
+        r = in_range ? row_of(i) : 0;
+        b = in_range ? i - r * a.nb : 0;
       }
       const int64_t prow = L.prow0 + r;
       const bool has_data = in_range && r < L.valid;
