@@ -16,6 +16,8 @@ using namespace fs;
 namespace {
 
 constexpr uint32_t kPathMask = FS_PATH_TENSOR | FS_PATH_DECODE;
+constexpr int kDecodeRows = 16;        // token columns of the decode kernel's MMA
+constexpr int kDecodeAvgRows = 64;     // grouped: below this many rows per expert, small experts take the decode kernel
 
 fs_status check_operands(const char* who, const fs_plan_s* pl, int32_t p, const uint8_t* xq, const uint8_t* sfx,
                          const uint16_t* xs, const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,
@@ -227,11 +229,30 @@ extern "C" fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64
   prm.seg = one_segment(plan->N);
   prm.Y = Y; prm.ldy = ldy; prm.out_bf16 = (plan->opts & FS_OUT_BF16) ? 1 : 0; prm.err = plan->err;
   prm.wait_ns = wait_limit_ns(plan->opts); prm.no_copies = (plan->opts & FS_FAULT_NO_COPIES) ? 1 : 0;
-  TcLaunch L{};
-  L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = a_rows; L.b_rows = static_cast<int64_t>(E) * plan->N; L.y_rows = max_rows; L.pp = pp;
-  L.bn = (plan->N % 256 == 0) ? 256 : 128;
-  L.max_tiles = ceil_div(a_rows, 128) * (plan->N / L.bn);
-  return launch_splice_gemm_tc(L, prm, static_cast<cudaStream_t>(stream));
+  // Experts of at most kDecodeRows rows go to the weight-streaming decode kernel (their 128-row
+  // weight tiles streamed once against up to 16 token columns) and the tensor-core kernel gives
+  // them no tiles, when the plan asks for it (FS_PATH_DECODE) or, unless it forces the tensor
+  // path, when the batch is small: fewer than kDecodeAvgRows rows per expert on average.  With
+  // max_rows <= kDecodeRows every expert is small and only the decode kernel runs.
+  const bool split = !(plan->opts & FS_PATH_TENSOR) &&
+                     ((plan->opts & FS_PATH_DECODE) || max_rows < kDecodeAvgRows * static_cast<int64_t>(E));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!split || max_rows > kDecodeRows) {
+    prm.skip_small = split ? kDecodeRows : 0;
+    TcLaunch L{};
+    L.xq = xq; L.wq = wq; L.xs = xs; L.ws = ws; L.a_rows = a_rows; L.b_rows = static_cast<int64_t>(E) * plan->N; L.y_rows = max_rows; L.pp = pp;
+    L.bn = (plan->N % 256 == 0) ? 256 : 128;
+    L.max_tiles = ceil_div(a_rows, 128) * (plan->N / L.bn);
+    st = launch_splice_gemm_tc(L, prm, s);
+    if (st != FS_OK || !split) return st;
+  }
+  DecodeParams d{};
+  d.M = 0; d.N = plan->N; d.K = plan->K; d.pp = pp; d.kb4 = static_cast<int>(round_up(plan->K / 16, 4) / 4);
+  d.xq = xq; d.sfx = sfx; d.xs = xs; d.wq = wq; d.sfw = sfw; d.ws = ws; d.alpha = alpha; d.seg = one_segment(plan->N);
+  d.Y = Y; d.ldy = ldy; d.out_bf16 = prm.out_bf16; d.err = plan->err;
+  d.wait_ns = prm.wait_ns; d.no_copies = prm.no_copies;
+  d.offsets = row_offsets; d.E = E; d.small_max = kDecodeRows; d.a_rows = a_rows;
+  return launch_splice_gemm_decode_tc(d, s);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -30,6 +30,7 @@ struct TcParams {
   int n_fast;         // tile order: 1 = N-tiles vary fastest (B stays in L2), 0 = M-tiles fastest
   int64_t a_groups;   // 128-row groups of the activation buffers (scale atoms past them are not read)
   const int64_t* offsets;
+  int skip_small;     // experts: those with at most this many rows get no tiles (the decode kernel's)
   const uint8_t* sfa;
   const uint8_t* sfb;
   const float* alpha;     // [E] for experts, else [segments]
@@ -87,6 +88,13 @@ struct DecodeParams {
   int p;
   const float* gA;
   int residual;
+  // grouped (offsets != null): experts with 1..small_max rows, E stacked weight operands of N rows,
+  // packed activations in the grouped layout (each expert's rows from a 128-row boundary) with
+  // a_rows rows in all; xq, sfx, xs, wq, sfw, ws, alpha as for fs_splice_gemm_grouped
+  const int64_t* offsets;
+  int E;
+  int small_max;
+  int64_t a_rows;
 };
 
 // Wait limits: the normal bound, and the short one of the failure-detection test option

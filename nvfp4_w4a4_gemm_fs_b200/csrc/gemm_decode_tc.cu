@@ -92,6 +92,9 @@ struct DecTcParams {
   int p;
   const float* gA;
   int residual;
+  // grouped (offsets != null): blockIdx.x = expert * n_tiles + tile; experts with 1..small_max rows
+  const int64_t* offsets;
+  int n_tiles, small_max;
 };
 
 __device__ __forceinline__ uint64_t now_ns() {
@@ -217,7 +220,11 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = static_cast<int>(ptx::cluster_ctarank());     // K split inside the tile's cluster
-  const int n0 = static_cast<int>(blockIdx.x) * kDRows;
+  // Output columns n0.. of the tile; its weight rows start at wrow0 (grouped: expert e's weights
+  // are rows e*N .. e*N + N - 1 of the stacked operand).
+  const int expert = p.offsets ? static_cast<int>(blockIdx.x) / p.n_tiles : 0;
+  const int n0 = (static_cast<int>(blockIdx.x) - expert * (p.offsets ? p.n_tiles : 0)) * kDRows;
+  const int wrow0 = expert * p.N + n0;
   const int kt0 = rank * p.kt_per;
   const int kt1 = kt0 + p.kt_per < p.KT ? kt0 + p.kt_per : p.KT;
   const int nf = kt1 - kt0;                                       // FP4 k-tiles of this CTA (>= 1)
@@ -249,8 +256,9 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
     }
     // (not in the fused form, whose preparing warps read X meanwhile: measured faster without it
     // at 16 tokens and equal at 1)
-    if (!kFuse && !p.no_copies)
-      for (int kt = kt0; kt < kt1; ++kt) ptx::tma_prefetch_2d(&tmW, kt * 128, n0);
+    // (nor in the grouped form, which learns only after the wait whether its expert is its own)
+    if (!kFuse && !p.no_copies && !p.offsets)
+      for (int kt = kt0; kt < kt1; ++kt) ptx::tma_prefetch_2d(&tmW, kt * 128, wrow0);
   }
   if (warp == 1) {
     ptx::tmem_alloc<1>(tmem_slot, C::TMEM_COLS);
@@ -281,6 +289,36 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
   ptx::tc_fence_after();
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
+  // Token rows: the problem's M, or expert e's rows r0 .. r1 - 1 of the output, packed from row
+  // xrow0 of the grouped activations (every expert's rows start at a 128-row boundary).  A cluster
+  // whose expert has no rows, or more than small_max (the tensor-core kernel's), leaves at once:
+  // all its CTAs decide alike and none has touched another's memory.
+  int M = p.M;
+  int64_t yrow0 = 0, xrow0 = 0;
+  if (p.offsets) {
+    const int64_t r0 = __ldg(p.offsets + expert), r1 = __ldg(p.offsets + expert + 1);
+    if (r1 - r0 <= 0 || r1 - r0 > p.small_max) {
+      ptx::tc_fence_before();
+      __syncthreads();
+      if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc<1>(tmem, C::TMEM_COLS);
+      }
+      return;
+    }
+    M = static_cast<int>(r1 - r0);
+    yrow0 = r0;
+    if (warp == 0) {
+      int64_t pad = 0;
+      for (int i = lane; i < expert; i += 32) {
+        const int64_t n = __ldg(p.offsets + i + 1) - __ldg(p.offsets + i);
+        pad += (n + 127) / 128 * 128;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) pad += __shfl_xor_sync(0xffffffffu, pad, o);
+      xrow0 = pad;
+    }
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -295,17 +333,18 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
         if (i < nf) {
           const int kt = kt0 + i;
           ptx::mbar_arrive_expect_tx(full + stage, kFuse ? C::W_BYTES + C::SFW_BYTES : C::STAGE_BYTES);
-          ptx::tma_load_2d(W_at(stage), &tmW, kt * 128, n0, full + stage);
-          if constexpr (!kFuse) ptx::tma_load_2d(X_at(stage), &tmX, kt * 128, 0, full + stage);
-          ptx::bulk_load(SFW_at(stage), p.sfw + (static_cast<int64_t>(n0 / kDRows) * p.kb4 + kt * 4) * 512,
+          ptx::tma_load_2d(W_at(stage), &tmW, kt * 128, wrow0, full + stage);
+          if constexpr (!kFuse) ptx::tma_load_2d(X_at(stage), &tmX, kt * 128, static_cast<int32_t>(xrow0), full + stage);
+          ptx::bulk_load(SFW_at(stage), p.sfw + (static_cast<int64_t>(wrow0 / kDRows) * p.kb4 + kt * 4) * 512,
                          C::SFW_BYTES, full + stage);
           if constexpr (!kFuse)
-            ptx::bulk_load(SFX_at(stage), p.sfx + static_cast<int64_t>(kt) * 4 * 512, C::SFX_BYTES, full + stage);
+            ptx::bulk_load(SFX_at(stage), p.sfx + ((xrow0 / kDRows) * p.kb4 + static_cast<int64_t>(kt) * 4) * 512,
+                           C::SFX_BYTES, full + stage);
         } else {
           const int sk = i - nf;
           ptx::mbar_arrive_expect_tx(full + stage, kFuse ? C::W_BYTES : C::W_BYTES + C::X_BYTES);
-          ptx::tma_load_2d(W_at(stage), &tmWS, sk * 64, n0, full + stage);
-          if constexpr (!kFuse) ptx::tma_load_2d(X_at(stage), &tmXS, sk * 64, 0, full + stage);
+          ptx::tma_load_2d(W_at(stage), &tmWS, sk * 64, wrow0, full + stage);
+          if constexpr (!kFuse) ptx::tma_load_2d(X_at(stage), &tmXS, sk * 64, static_cast<int32_t>(xrow0), full + stage);
         }
         ++issued;
         if (++stage == kDStages) { stage = 0; phase ^= 1; }
@@ -495,11 +534,11 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
     const int share = ((kOut + p.S - 1) / p.S + 3) & ~3;
     const int v0 = rank * share;
     const int v1 = v0 + share < kOut ? v0 + share : kOut;
-    const float alpha = __ldg(p.alpha + segment_of(n0, p.seg));
+    const float alpha = __ldg(p.alpha + (p.offsets ? expert : segment_of(n0, p.seg)));
     const uint32_t red_addr = ptx::smem_u32(red);
     for (int v = v0 + 4 * e; v < v1; v += 4 * 128) {
       const int t = v / kDRows, rr = v - t * kDRows;   // 4 rows rr..rr+3 of token t
-      if (t >= p.M || n0 + rr >= p.N) continue;
+      if (t >= M || n0 + rr >= p.N) continue;
       float4 part[kDMaxSplit];
 #pragma unroll
       for (int s2 = 0; s2 < kDMaxSplit; ++s2)
@@ -509,7 +548,7 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
       for (int s2 = 0; s2 < kDMaxSplit; ++s2)
         if (s2 < p.S) { sum.x += part[s2].x; sum.y += part[s2].y; sum.z += part[s2].z; sum.w += part[s2].w; }
       const float y[4] = {sum.x * alpha, sum.y * alpha, sum.z * alpha, sum.w * alpha};
-      const int64_t off = static_cast<int64_t>(t) * p.ldy + n0 + rr;
+      const int64_t off = (yrow0 + t) * p.ldy + n0 + rr;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         if (n0 + rr + q >= p.N) break;
@@ -541,10 +580,15 @@ fs_status launch_splice_gemm_decode_tc(const DecodeParams& d, cudaStream_t s) {
   p.sfw = d.sfw; p.sfx = d.sfx; p.alpha = d.alpha; p.seg = d.seg; p.Y = d.Y; p.ldy = d.ldy; p.out_bf16 = d.out_bf16;
   p.err = d.err; p.wait_ns = d.wait_ns; p.no_copies = d.no_copies;
   p.x = d.x; p.ldx = d.ldx; p.mask = d.mask; p.p = d.p; p.gA = d.gA; p.residual = d.residual;
+  if (d.offsets && d.fuse) return fail(FS_ERR_UNSUPPORTED, "%s: the grouped form takes packed activations", who);
+  const int n_tiles = static_cast<int>(ceil_div(d.N, kDRows));
+  p.offsets = d.offsets; p.n_tiles = n_tiles; p.small_max = d.small_max;
+  const int64_t w_rows = d.offsets ? static_cast<int64_t>(d.E) * d.N : d.N;   // weight operand rows
+  const int64_t x_rows = d.offsets ? d.a_rows : d.M;                          // activation operand rows
   // K split: as many CTAs per 128-row tile as fill the SMs at the resident CTAs per SM, at most 8
   // (a portable cluster);
   // every split keeps at least one FP4 k-tile.
-  const int tiles = static_cast<int>(ceil_div(d.N, kDRows));
+  const int tiles = n_tiles * (d.offsets ? d.E : 1);
   int S = static_cast<int>(std::max<int64_t>(1, (kDCtasPerSm * static_cast<int64_t>(sm_count())) / tiles));
   S = std::min(S, std::min(kDMaxSplit, p.KT));
   p.kt_per = static_cast<int>(ceil_div(p.KT, S));
@@ -553,14 +597,14 @@ fs_status launch_splice_gemm_decode_tc(const DecodeParams& d, cudaStream_t s) {
   // (the fused kernel reads X itself; its activation maps are placeholders it never uses)
   CUtensorMap tmW, tmX, tmWS, tmXS;
   const uint64_t kbytes = static_cast<uint64_t>(d.K) / 2;
-  fs_status st = make_map(&tmW, d.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, d.N, kbytes, 128, kDRows);
-  if (st == FS_OK && !d.fuse) st = make_map(&tmX, d.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, d.M, kbytes, 128, kDTok);
+  fs_status st = make_map(&tmW, d.wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, w_rows, kbytes, 128, kDRows);
+  if (st == FS_OK && !d.fuse) st = make_map(&tmX, d.xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, x_rows, kbytes, 128, kDTok);
   if (st != FS_OK) return st;
   if (d.fuse) tmX = tmW;
   if (p.ST > 0) {
     const uint64_t pp = static_cast<uint64_t>(d.pp);
-    st = make_map(&tmWS, d.ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, d.N, pp * 2, 64, kDRows);
-    if (st == FS_OK && !d.fuse) st = make_map(&tmXS, d.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, d.M, pp * 2, 64, kDTok);
+    st = make_map(&tmWS, d.ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, w_rows, pp * 2, 64, kDRows);
+    if (st == FS_OK && !d.fuse) st = make_map(&tmXS, d.xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pp, x_rows, pp * 2, 64, kDTok);
     if (st != FS_OK) return st;
     if (d.fuse) tmXS = tmWS;
   } else {

@@ -221,7 +221,7 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     if (p.offsets) {
       for (int e = 0; e < p.E; ++e) {
         const int64_t rows = p.offsets[e + 1] - p.offsets[e];
-        cum_m[e + 1] = cum_m[e] + static_cast<int>((rows + kBM * CG - 1) / (kBM * CG));
+        cum_m[e + 1] = cum_m[e] + (rows <= p.skip_small ? 0 : static_cast<int>((rows + kBM * CG - 1) / (kBM * CG)));
         cum_g[e + 1] = cum_g[e] + static_cast<int>((rows + kBM - 1) / kBM);
       }
     } else {
