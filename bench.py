@@ -438,6 +438,32 @@ def moe_case(F, p, device, reps=10):
             res[tag] = {"us": ms * 1000.0, "TFLOPs": flops / (ms * 1e-3) / 1e12}
             del g
         plan.check()
+        # Decode steps of the same layer (the protected sets and packed weights above): 16 and 64
+        # tokens routed top-8 (128 / 512 rows; with 16 tokens no expert can exceed 16 rows).  Every
+        # expert on the tensor-core kernel (the default) against FS_PATH_DECODE, which sends
+        # experts of at most 16 rows to the weight-streaming decode kernel.  GB/s counts the
+        # packed weights of the experts with rows, the packed activations and the fp32 outputs.
+        pw = N * K // 2 + N * (K // 16) + N * pp * 2
+        for tokens in (16, 64):
+            dc = synth.moe_routing_counts(1, tokens=tokens)
+            dtot = int(dc.sum())
+            doffs = torch.tensor(np.concatenate([[0], np.cumsum(dc)]), dtype=torch.int64, device=device)
+            Xd = make_activations(dtot, K, 33, device)
+            xqd = F.fs_quantize_splice_grouped(Xd, doffs, masks, p, gA, max_rows=dtot)
+            Yd = torch.empty(dtot, N, dtype=torch.float32, device=device)
+            dbytes = int((dc > 0).sum()) * pw + F.grouped_rows(dtot, E) * (K // 2 + K // 16 + pp * 2) + dtot * N * 4
+            dres = {"rows": dtot, "experts_with_rows": int((dc > 0).sum()), "max_rows_per_expert": int(dc.max())}
+            for tag, popts in (("tensor_only", 0), ("small_experts_on_decode", F.FS_PATH_DECODE)):
+                dplan = F.Plan(N, K, max(p, 1), popts)
+                g = capture(lambda: F.fs_splice_gemm_grouped(dplan, doffs, dtot, xqd, wq, alpha, Y=Yd))
+                for _ in range(3):
+                    g.replay()
+                ms = timed(g.replay, reps) / reps
+                dplan.check()
+                dres[tag] = {"us": ms * 1000.0, "GBps": dbytes / (ms * 1e-3) / 1e9}
+                del g
+            res[f"decode_{tokens}_tokens"] = dres
+            del Xd, xqd, Yd
         out[name] = res
         del X, xq, wq, Y, st
         torch.cuda.empty_cache()

@@ -296,12 +296,12 @@ fs_status fs_decode_splice_gemm(fs_plan plan, int64_t M, int32_t p, const void* 
  * weights are rows [e*N, (e+1)*N) of stacked wq [E*N][K/2], sfw (tiled over E*N rows) and
  * ws [E*N][Pp]; alpha [E].  Y [row_offsets[E]][ldy] in the original (unpadded) row order.
  * Needs N % 128 == 0 and E <= 256.  Experts run on the tensor-core kernel (256-row CTA-pair
- * tiles, or 128-row tiles), except that experts of 1..16 rows run on the weight-streaming decode
- * kernel (each 128-row weight tile streamed once against the expert's tokens as 16 columns) when
- * the plan has FS_PATH_DECODE, or, unless it has FS_PATH_TENSOR, when max_rows < 64 * E; with
- * max_rows <= 16 only the decode kernel is launched.  Each expert's rows are read from the
- * device offsets inside the kernels, so the split needs no host synchronisation; the results of
- * the two kernels differ only in the fp32 summation order. */
+ * tiles, or 128-row tiles).  With FS_PATH_DECODE in the plan's opts, experts of 1..16 rows run on
+ * the weight-streaming decode kernel instead (each 128-row weight tile streamed once against the
+ * expert's tokens as 16 columns) and the tensor-core kernel skips them; with max_rows <= 16 only
+ * the decode kernel is launched.  Each expert's rows are read from the device offsets inside the
+ * kernels, so the split needs no host synchronisation; the results of the two kernels differ
+ * only in the fp32 summation order. */
 fs_status fs_splice_gemm_grouped(fs_plan plan, int32_t E, const int64_t* row_offsets, int64_t max_rows,
                                  int32_t p, const uint8_t* xq, const uint8_t* sfx, const uint16_t* xs,
                                  const uint8_t* wq, const uint8_t* sfw, const uint16_t* ws,

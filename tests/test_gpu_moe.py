@@ -149,22 +149,24 @@ def test_grouped_partial_tiles_bf16_output(N):
 
 # ---------------------------------------------------------------- small experts on the decode kernel
 @pytest.mark.parametrize("counts,N,K,p", [
-    ([0, 1, 3, 16, 17, 40, 200, 5, 0, 9], 256, 1024, 64),     # mixed: both kernels (64 rows/expert > avg)
+    ([0, 1, 3, 16, 17, 40, 200, 5, 0, 9], 256, 1024, 64),     # mixed: both kernels
     ([1, 0, 4, 2, 5, 0, 3, 1], 384, 2048, 64),                # max_rows <= 16: the decode kernel alone
     ([16, 16, 2, 7], 256, 512, 256),                          # K split over a cluster, four side k-tiles
     ([3, 11, 0, 16, 1], 128, 4096, 0),                        # P = {} (no side k-tiles), one 128-row tile
 ])
 def test_grouped_small_experts_take_the_decode_kernel(counts, N, K, p):
-    """Fewer than 64 rows per expert on average: experts of 1..16 rows run on the weight-streaming
-    decode kernel (their tokens as the 16 MMA columns, read from the expert's padded rows), larger
-    ones on the tensor-core kernel.  Every expert's rows are checked against the oracle."""
+    """FS_PATH_DECODE: experts of 1..16 rows run on the weight-streaming decode kernel (their
+    tokens as the 16 MMA columns, read from the expert's padded rows), larger ones on the
+    tensor-core kernel.  Every expert's rows are checked against the oracle, and the default
+    (every expert on the tensor-core kernel) against it too."""
     E, offs, Xs, Ws, Ps, gAs = _build(counts, N, K, p, seed=6)
-    _, Y = _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p)
-    _check_expert_outputs(offs, Xs, Ws, Ps, gAs, Y)
+    for opts in (F.FS_PATH_DECODE, 0):
+        _, Y = _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p, plan_opts=opts)
+        _check_expert_outputs(offs, Xs, Ws, Ps, gAs, Y)
 
 
 def test_grouped_decode_routing_forced_and_bf16():
-    """FS_PATH_DECODE sends the small experts of a large batch to the decode kernel too, and
+    """FS_PATH_DECODE sends the small experts of a large batch to the decode kernel, and
     FS_PATH_TENSOR keeps every expert on the tensor-core kernel; both match the oracle, with bf16
     output on the decode path."""
     counts = [0, 1, 127, 128, 129, 300, 5, 16, 17]
@@ -184,5 +186,5 @@ def test_grouped_decode_moe_batch():
     assert max(counts) > 16 and min(counts) == 0
     N, K, p = 4096, 4096, 64
     E, offs, Xs, Ws, Ps, gAs = _build(counts, N, K, p, seed=8)
-    _, Y = _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p)
+    _, Y = _run_gpu(E, offs, Xs, Ws, Ps, gAs, N, K, p, plan_opts=F.FS_PATH_DECODE)
     _check_expert_outputs(offs, Xs, Ws, Ps, gAs, Y, rows_per_expert=4)
