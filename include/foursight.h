@@ -74,7 +74,8 @@ enum {
   FS_GAIN_EXACT = 1u << 2, /* encode gain fl32(2688/amax) instead of the power-of-two gain */
   FS_OUT_BF16 = 1u << 3,   /* fs_splice_gemm writes bf16 Y instead of fp32 */
   FS_PATH_TENSOR = 1u << 4, /* plan option: always use the tcgen05 tensor-core kernel */
-  FS_PATH_DECODE = 1u << 5, /* plan option: always use the weight-streaming decode kernel (M <= 16) */
+  FS_PATH_DECODE = 1u << 5, /* plan option: always use the weight-streaming decode kernel (M <= 16);
+                              fs_splice_gemm_grouped: experts of at most 16 rows on it */
   FS_COMPACT_K = 1u << 7,   /* fs_quantize_splice / fs_prepare_weights: compacted-K operand (below) */
   FS_FAULT_NO_COPIES = 1u << 6 /* plan (and fs_splice_gemm_noalloc) option for tests of failure detection:
                               the GEMM kernels' producers issue no copies and every bounded wait is
