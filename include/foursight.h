@@ -144,7 +144,7 @@ fs_status fs_stats_check(const uint32_t* flags, int32_t nprob, void* stream);
  *         (over all channels with FS_RESIDUAL): the largest power of two g with amax*g <= 2688
  *         (exponent clamped to [-126,127]; 1 when amax == 0), or fl32(2688/amax) with FS_GAIN_EXACT.
  * reset != 0 zeroes the state after it has been read (start of the next window).
- * Requirements: 0 <= p <= K <= 16384, p <= 256.  Runs one CTA per problem.
+ * Requirements: 0 <= p <= K <= 16384, p <= 256.  Runs one cluster of 8 CTAs per problem.
  * ---------------------------------------------------------------------------------------- */
 fs_status fs_select_topk(int32_t nprob, int32_t K, int64_t* n, int64_t* s1, int64_t* s2,
                          uint32_t* amax, uint32_t* flags, int32_t p, uint32_t opts,
