@@ -112,3 +112,17 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert "workload" in d["config"] and "model" not in d["config"]
+
+
+def test_moe_routing_workloads():
+    """The routed-row counts bench.py times: top-8 of 4096 tokens over 64 experts sums to 32768
+    rows, and the decode batches (16 / 64 tokens) to 128 / 512 rows; a token picks 8 distinct
+    experts, so with 16 tokens no expert holds more than 16 rows (every expert fits the decode
+    kernel's 16 token columns)."""
+    import synth
+    c = synth.moe_routing_counts(0)
+    assert c.sum() == 32768 and len(c) == 64
+    for tokens in (16, 64):
+        d = synth.moe_routing_counts(1, tokens=tokens)
+        assert d.sum() == 8 * tokens and d.max() <= tokens and d.min() >= 0
+    assert synth.moe_routing_counts(1, tokens=16).max() <= 16
