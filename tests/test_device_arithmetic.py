@@ -1,0 +1,176 @@
+"""CPU checks of the arithmetic shortcuts the kernels take, against the plain IEEE definitions.
+
+The kernels replace a few correctly rounded operations by cheaper sequences whose equality with
+the definition rests on an argument written beside them in the sources:
+
+- multiply-and-snap (``snap12`` in csrc/common.cuh): for bf16 x, a power-of-two gain g and a UE4M3
+  block scale sf, the E2M1 code of snap12(RN(x * RN(g * RN(1/sf)))) equals the code of
+  RN(RN(x * g) / sf), the quantiser's element rule;
+- Markstein's division with two remainder steps (``div_markstein`` in csrc/common.cuh, fp32;
+  ``div_rn_by`` in csrc/stats.cu, fp64): RN(y / d) from r = RN(1/d) and fused multiply-adds;
+- the quantiser's row quotient (csrc/quant.cu): trunc(RN(RN(i + 1/2) * RN(1/nb))) == i // nb.
+
+Each is re-derived here with numpy's IEEE float32 / float64 operations, fused multiply-adds
+emulated exactly with fractions, and compared with the definition, exhaustively where the domain
+is small.  No GPU is needed; the GPU parity tests then hold the kernels to the oracle.
+"""
+from fractions import Fraction
+import math
+
+import numpy as np
+import pytest
+
+# ------------------------------------------------------------------------------- helpers
+E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float64)   # between the 8 magnitudes
+
+
+def e2m1_code(v: np.ndarray) -> np.ndarray:
+    """E2M1 code (sign in bit 3) of float32 values: round to nearest, ties to the even code,
+    saturating at 6; -0 keeps its sign."""
+    a = np.abs(v.astype(np.float64))
+    k = np.searchsorted(E2M1_MIDS, a, side="left")          # midpoints strictly below a
+    tie = (k < len(E2M1_MIDS)) & (a == E2M1_MIDS[np.minimum(k, len(E2M1_MIDS) - 1)])
+    idx = np.where(tie & (k % 2 == 1), k + 1, k)             # a tie goes to the even code
+    sign = np.signbit(v).astype(np.int64) << 3
+    return idx.astype(np.int64) | sign
+
+
+def ue4m3_values() -> np.ndarray:
+    """Values of the UE4M3 codes 1..126 (subnormals m * 2^-9, normals (1 + m/8) 2^(e-7))."""
+    out = []
+    for c in range(1, 127):
+        e, m = c >> 3, c & 7
+        out.append(m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+    return np.array(out, np.float32)
+
+
+def snap12(p: np.ndarray) -> np.ndarray:
+    b = p.view(np.uint32)
+    return ((b + np.uint32(0x800)) & np.uint32(0xFFFFF000)).view(np.float32)
+
+
+def all_finite_bf16() -> np.ndarray:
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    x = (bits << 16).view(np.float32)
+    return x[np.isfinite(x)]
+
+
+def rn32(q: Fraction) -> np.float32:
+    """Correct round-to-nearest-even of a rational to float32 (normal range)."""
+    if q == 0:
+        return np.float32(0.0)
+    s = -1 if q < 0 else 1
+    a = abs(q)
+    e = math.floor(math.log2(a.numerator) - math.log2(a.denominator))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    scaled = a * Fraction(2) ** (23 - e)                      # in [2^23, 2^24)
+    n, rem = divmod(scaled.numerator, scaled.denominator)
+    twice = 2 * rem
+    if twice > scaled.denominator or (twice == scaled.denominator and n % 2 == 1):
+        n += 1
+    return np.float32(s * float(Fraction(n) * Fraction(2) ** (e - 23)))
+
+
+def fma32(a, b, c) -> np.float32:
+    return rn32(Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c)))
+
+
+def fma64(a: float, b: float, c: float) -> float:
+    return float(Fraction(a) * Fraction(b) + Fraction(c))     # float(Fraction) rounds correctly
+
+
+# ------------------------------------------------------------------------------- multiply-and-snap
+@pytest.mark.parametrize("log2g", [-8, 0, 7])
+def test_multiply_and_snap_gives_the_e2m1_code_of_the_two_step_division(log2g):
+    """Every finite bf16 x, every UE4M3 scale, power-of-two gains: the fast path's code equals the
+    element rule's code wherever the kernel uses it (|x g| <= 2688 = 6 * 448, the encode gain's
+    bound, so x g / sf stays finite)."""
+    g = np.float32(2.0 ** log2g)
+    x = all_finite_bf16()
+    x = x[np.abs(x.astype(np.float64) * float(g)) <= 2688.0]
+    for sf in ue4m3_values():
+        sr = np.float32(1.0) / sf                                  # RN(1/sf)
+        exact = (x * g) / sf                                       # RN(RN(x g) / sf)
+        fast = snap12(x * (g * sr))                                # RN(g sr) is exact for g = 2^k
+        got, want = e2m1_code(fast), e2m1_code(exact)
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, f"sf={sf}: x={x[bad[:4]]} codes {got[bad[:4]]} != {want[bad[:4]]}"
+
+
+def test_e2m1_reference_rounding():
+    """The reference rounding above: midpoints go to the even code, values at or above 5 beyond
+    the 4..6 midpoint saturate at 6, -0 keeps its sign."""
+    v = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 5.01, 7.0, 1e30, -0.0, -0.26, 0.24], np.float32)
+    assert e2m1_code(v).tolist() == [0, 2, 2, 4, 4, 6, 6, 7, 7, 7, 8, 9, 0]
+
+
+# ------------------------------------------------------------------------------- row quotient
+def test_fp32_row_quotient_is_exact():
+    """trunc(RN(RN(i + 1/2) * RN(1/nb))) == i // nb for every nb = K/16 with K % 64 == 0 up to
+    K = 16384, and every block index i of a chunk (below 2^18)."""
+    i = np.arange(1 << 18, dtype=np.int64)
+    fi = i.astype(np.float32) + np.float32(0.5)
+    for nb in range(4, 1025, 4):
+        inv = np.float32(1.0) / np.float32(nb)
+        q = (fi * inv).astype(np.int64)                            # float -> int truncates
+        assert np.array_equal(q, i // nb), f"nb={nb}"
+
+
+# ------------------------------------------------------------------------------- Markstein division
+def div_markstein32(y, d, r):
+    q0 = np.float32(y * r)
+    e0 = fma32(-q0, d, y)
+    q1 = fma32(e0, r, q0)
+    e1 = fma32(-q1, d, y)
+    q2 = fma32(e1, r, q1)
+    return np.float32(math.copysign(abs(float(q2)), float(y)))
+
+
+def div_rn_by64(y: float, d: float, r: float) -> float:
+    q0 = y * r
+    e0 = fma64(-q0, d, y)
+    q1 = fma64(e0, r, q0)
+    e1 = fma64(-q1, d, y)
+    return fma64(e1, r, q1)
+
+
+def test_markstein_fp32_block_scale_and_element_division():
+    """RN(y / d) for the divisors the quantiser uses: d = 6 (block scale t = fl32(a g) / 6) and
+    every UE4M3 value (element v = fl32(x g) / sf), on random and near-tie dividends."""
+    rng = np.random.default_rng(5)
+    divisors = [np.float32(6.0)] + list(ue4m3_values()[::5])
+    for d in divisors:
+        r = np.float32(1.0) / d
+        ys = list(rng.standard_normal(60).astype(np.float32) * np.float32(rng.uniform(0.01, 300)))
+        # dividends whose quotient is (next to) a midpoint of float32 values: y = RN(d * m) for
+        # m halfway between neighbours
+        for m in rng.uniform(0.1, 10.0, 20).astype(np.float32):
+            mid = (Fraction(float(m)) + Fraction(float(np.nextafter(m, np.float32(20))))) / 2
+            ys.append(rn32(mid * Fraction(float(d))))
+        ys += [np.float32(-0.0), np.float32(0.0)]
+        for y in ys:
+            got = div_markstein32(y, d, r)
+            want = rn32(Fraction(float(y)) / Fraction(float(d))) if y != 0 else y
+            assert got == want and np.signbit(got) == np.signbit(want), (float(y), float(d))
+
+
+def test_markstein_fp64_selection_key_division():
+    """The selection's m = fl64(fl64(s / 2^k) / n) with n the row count: two remainder steps from
+    RN(1/n) give the correctly rounded quotient, on random moments and counts and on exact
+    quotients."""
+    rng = np.random.default_rng(9)
+    cases = []
+    for _ in range(3000):
+        n = int(rng.integers(1, 1 << 22))
+        s = int(rng.integers(-(1 << 62), 1 << 62))
+        cases.append((float(s) / 2.0 ** 14, float(n)))
+    for _ in range(500):                                           # exact quotients
+        n = int(rng.integers(1, 1 << 20))
+        q = int(rng.integers(-(1 << 30), 1 << 30))
+        cases.append((float(q * n) / 2.0 ** 16, float(n)))
+    for y, d in cases:
+        r = 1.0 / d                                                # RN(1/d) in IEEE double
+        assert div_rn_by64(y, d, r) == float(Fraction(y) / Fraction(d)), (y, d)
