@@ -8,7 +8,9 @@ the definition rests on an argument written beside them in the sources:
   RN(RN(x * g) / sf), the quantiser's element rule;
 - Markstein's division with two remainder steps (``div_markstein`` in csrc/common.cuh, fp32;
   ``div_rn_by`` in csrc/stats.cu, fp64): RN(y / d) from r = RN(1/d) and fused multiply-adds;
-- the quantiser's row quotient (csrc/quant.cu): trunc(RN(RN(i + 1/2) * RN(1/nb))) == i // nb.
+- the quantiser's row quotient (csrc/quant.cu): trunc(RN(RN(i + 1/2) * RN(1/nb))) == i // nb;
+- the bit-level roundings of csrc/common.cuh: ``ue4m3_rne`` (block scale to UE4M3, ties to even,
+  saturating) and ``gain_pow2`` (largest power-of-two gain with amax * g <= 2688).
 
 Each is re-derived here with numpy's IEEE float32 / float64 operations, fused multiply-adds
 emulated exactly with fractions, and compared with the definition, exhaustively where the domain
@@ -174,3 +176,68 @@ def test_markstein_fp64_selection_key_division():
     for y, d in cases:
         r = 1.0 / d                                                # RN(1/d) in IEEE double
         assert div_rn_by64(y, d, r) == float(Fraction(y) / Fraction(d)), (y, d)
+
+
+# ------------------------------------------------------------------------------- UE4M3 and gain bits
+def ue4m3_rne_bits(t: np.ndarray) -> np.ndarray:
+    """The block-scale rounding of csrc/common.cuh (``ue4m3_rne``) step by step on float32 bits:
+    saturate at 448, subnormals as rint(t * 512), otherwise round the fraction to 3 bits (ties to
+    even) with one integer add and rebias the exponent."""
+    t = t.astype(np.float32)
+    b = t.view(np.uint32).astype(np.int64)
+    b = b + 0x7FFFF + ((b >> 20) & 1)
+    normal = ((((b >> 23) - 120) << 3) | ((b >> 20) & 7))
+    normal = np.minimum(normal, 0x7E)
+    sub = np.rint((t * np.float32(512.0)).astype(np.float64)).astype(np.int64)   # rint: ties to even
+    return np.where(t >= np.float32(448.0), 0x7E, np.where(t < np.float32(0.015625), sub, normal))
+
+
+def test_ue4m3_bit_rounding_matches_the_definition_on_every_float32_scale():
+    """Every float32 t from 2^-12 up to 2^9 (and 0), binade by binade: the bit-level rounding
+    equals round-to-nearest-even onto the UE4M3 values, saturating at 448."""
+    from oracle import nvfp4
+    mant = np.arange(1 << 23, dtype=np.uint32)
+    for e in range(127 - 12, 127 + 9):
+        t = ((np.uint32(e) << np.uint32(23)) | mant).view(np.float32)
+        assert np.array_equal(ue4m3_rne_bits(t), nvfp4.ue4m3_encode(t)), f"binade 2^{e - 127}"
+    z = np.zeros(1, np.float32)
+    assert ue4m3_rne_bits(z)[0] == 0 == nvfp4.ue4m3_encode(z)[0]
+
+
+def gain_pow2_bits(amax: np.ndarray) -> np.ndarray:
+    """The encode gain of csrc/common.cuh (``gain_pow2``) on float32 bits, for finite amax > 0."""
+    a = amax.astype(np.float32)
+    b = a.view(np.uint32).astype(np.int64)
+    subn = (b >> 23) == 0
+    bias = np.where(subn, 64, 0)
+    with np.errstate(over="ignore"):                           # evaluated for normal a too, unused there
+        scaled = (a * np.float32(2.0 ** 64)).view(np.uint32).astype(np.int64)
+    b = np.where(subn, scaled, b)
+    e = (b >> 23) - 126 - bias
+    frac = b & 0x7FFFFF
+    E = np.where(frac <= 0x280000, 12 - e, 11 - e)
+    E = np.clip(E, -126, 127)
+    return E
+
+
+def test_pow2_gain_bits_give_the_largest_fitting_power():
+    """For amax over every float32 binade (normal and subnormal) with mantissas at and around
+    the 0.65625 boundary plus random ones: g = 2^E is the largest power of two with
+    amax * g <= 2688, E clamped to [-126, 127] (products with powers of two are exact in float64)."""
+    rng = np.random.default_rng(3)
+    mants = np.unique(np.concatenate([
+        np.array([0, 1, 0x27FFFF, 0x280000, 0x280001, 0x7FFFFE, 0x7FFFFF, 0x400000], np.int64),
+        rng.integers(0, 1 << 23, 64)]))
+    amax = []
+    for e in range(0, 255):
+        for m in mants:
+            if e == 0 and m == 0:
+                continue
+            amax.append((e << 23) | int(m))
+    a = np.array(amax, np.uint32).view(np.float32)
+    E = gain_pow2_bits(a)
+    a64 = a.astype(np.float64)
+    fits = a64 * np.exp2(E.astype(np.float64)) <= 2688.0
+    next_fits = a64 * np.exp2(E.astype(np.float64) + 1) <= 2688.0
+    assert np.all(fits | (E == -126)), "gain too large"
+    assert np.all(~next_fits | (E == 127)), "a larger power of two would fit"
