@@ -10,7 +10,9 @@ the definition rests on an argument written beside them in the sources:
   ``div_rn_by`` in csrc/stats.cu, fp64): RN(y / d) from r = RN(1/d) and fused multiply-adds;
 - the quantiser's row quotient (csrc/quant.cu): trunc(RN(RN(i + 1/2) * RN(1/nb))) == i // nb;
 - the bit-level roundings of csrc/common.cuh: ``ue4m3_rne`` (block scale to UE4M3, ties to even,
-  saturating) and ``gain_pow2`` (largest power-of-two gain with amax * g <= 2688).
+  saturating) and ``gain_pow2`` (largest power-of-two gain with amax * g <= 2688);
+- the statistics' integer moments (csrc/moments.cuh): magic-number roundings give rint(x 2^16) and
+  rint(x^2 2^14) for every in-range bf16 x, and raw-bit sums survive 32-bit wrap-around.
 
 Each is re-derived here with numpy's IEEE float32 / float64 operations, fused multiply-adds
 emulated exactly with fractions, and compared with the definition, exhaustively where the domain
@@ -241,3 +243,61 @@ def test_pow2_gain_bits_give_the_largest_fitting_power():
     next_fits = a64 * np.exp2(E.astype(np.float64) + 1) <= 2688.0
     assert np.all(fits | (E == -126)), "gain too large"
     assert np.all(~next_fits | (E == 127)), "a larger power of two would fit"
+
+
+# ------------------------------------------------------------------------------- integer moments
+MAGIC = np.float32(12582912.0)          # 1.5 * 2^23
+MAGIC8 = np.float32(3221225472.0)       # 1.5 * 2^31
+MAGIC_BITS, MAGIC8_BITS = 0x4B400000, 0x4F400000
+
+
+def moment_raw_terms(x: np.ndarray):
+    """The four raw-bit terms csrc/moments.cuh (``add_bf16``) adds per in-range element, as
+    uint32: fp32 additions with the magic constants round to integers (ties to even); the
+    multiply-adds are an exact product plus one rounding, as numpy's float32 add reproduces."""
+    x = x.astype(np.float32)
+    t1 = x + MAGIC
+    frac = x - (t1 - MAGIC)
+    b1 = frac * np.float32(65536.0) + MAGIC
+    y = x * x
+    u = y + MAGIC8
+    yl = y - (u - MAGIC8)
+    d2 = yl * np.float32(16384.0) + MAGIC
+    return [v.view(np.uint32).astype(np.int64) for v in (t1, b1, u, d2)]
+
+
+def rint_even(num: int, den: int) -> int:
+    q, r = divmod(num, den)
+    return q + (1 if 2 * r > den or (2 * r == den and q % 2 == 1) else 0)
+
+
+def test_integer_moment_terms_of_every_bf16_value():
+    """For every bf16 x with |x| < 2^15: the recovered terms give s1 = rint(x 2^16) and
+    s2 = rint(x^2 2^14) exactly (ties to even), the statistics' fixed-point definition."""
+    x = all_finite_bf16()
+    x = x[np.abs(x) < 32768.0]
+    a1, b1, c2, d2 = moment_raw_terms(x)
+    s1 = (a1 - MAGIC_BITS) * 65536 + (b1 - MAGIC_BITS)
+    s2 = (c2 - MAGIC8_BITS) * 4194304 + (d2 - MAGIC_BITS)
+    for xi, g1, g2 in zip(x.tolist(), s1.tolist(), s2.tolist()):
+        f = Fraction(xi)
+        assert g1 == rint_even(f.numerator * 65536, f.denominator), xi
+        assert g2 == rint_even(f.numerator ** 2 * 16384, f.denominator ** 2), xi
+
+
+def test_integer_moments_survive_wrapping_32_bit_sums_of_256_rows():
+    """Raw-bit terms of 256 rows summed modulo 2^32, minus 256 magic patterns, give the exact sums
+    of the terms, for rows at the range limit (the largest terms) and random rows."""
+    rng = np.random.default_rng(7)
+    cases = [np.full(256, np.float32(32512.0)), np.full(256, np.float32(-32512.0)),
+             (rng.standard_normal(256) * 3000).astype(np.float32),
+             (rng.standard_normal(256) * 0.01).astype(np.float32)]
+    for rows in cases:
+        rows = (rows.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)   # bf16 values
+        terms = moment_raw_terms(rows)
+        magics = (MAGIC_BITS, MAGIC_BITS, MAGIC8_BITS, MAGIC_BITS)
+        for t, m in zip(terms, magics):
+            wrapped = int(t.sum()) % (1 << 32)
+            small = (wrapped - 256 * m) % (1 << 32)
+            small = small - (1 << 32) if small >= (1 << 31) else small    # back to int32
+            assert small == int((t - m).sum())
