@@ -12,7 +12,8 @@ the definition rests on an argument written beside them in the sources:
 - the bit-level roundings of csrc/common.cuh: ``ue4m3_rne`` (block scale to UE4M3, ties to even,
   saturating) and ``gain_pow2`` (largest power-of-two gain with amax * g <= 2688);
 - the statistics' integer moments (csrc/moments.cuh): magic-number roundings give rint(x 2^16) and
-  rint(x^2 2^14) for every in-range bf16 x, and raw-bit sums survive 32-bit wrap-around.
+  rint(x^2 2^14) for every in-range bf16 x, and raw-bit sums survive 32-bit wrap-around;
+- the selection's key map (``order_bits`` in csrc/stats.cu) preserves the order of doubles.
 
 Each is re-derived here with numpy's IEEE float32 / float64 operations, fused multiply-adds
 emulated exactly with fractions, and compared with the definition, exhaustively where the domain
@@ -301,3 +302,29 @@ def test_integer_moments_survive_wrapping_32_bit_sums_of_256_rows():
             small = (wrapped - 256 * m) % (1 << 32)
             small = small - (1 << 32) if small >= (1 << 31) else small    # back to int32
             assert small == int((t - m).sum())
+
+
+def order_bits(k: np.ndarray) -> np.ndarray:
+    """The selection's key map of csrc/stats.cu (``order_bits``): -0 folded onto +0, then
+    negative doubles' bits inverted and positive ones' sign bit set."""
+    k = np.where(k == 0.0, 0.0, k)
+    b = k.view(np.uint64)
+    return np.where((b >> np.uint64(63)) == 1, ~b, b | np.uint64(1 << 63))
+
+
+def test_selection_key_map_preserves_the_order_of_doubles():
+    """Sorting by the mapped integers sorts the keys (ties exactly where the keys are equal, -0
+    equal to +0), over random doubles of both signs and magnitudes and the special values the
+    keys can take (zero of both signs, subnormals, the largest finite)."""
+    rng = np.random.default_rng(13)
+    k = np.concatenate([rng.standard_normal(4000) * 10.0 ** rng.integers(-30, 30, 4000),
+                        np.array([0.0, -0.0, 5e-324, -5e-324, 1.7976931348623157e308,
+                                  -1.7976931348623157e308, 1.0, -1.0, 1.0])])
+    m = order_bits(k)
+    i, j = rng.integers(0, len(k), (2, 200000))
+    assert np.array_equal(m[i] < m[j], k[i] < k[j])
+    assert np.array_equal(m[i] == m[j], k[i] == k[j])
+    sp = k[-9:]                                                    # every pair of the special values
+    ms = order_bits(sp)
+    assert np.array_equal(ms[:, None] < ms[None, :], sp[:, None] < sp[None, :])
+    assert np.array_equal(ms[:, None] == ms[None, :], sp[:, None] == sp[None, :])
