@@ -14,7 +14,9 @@ one pass of the per-step path over one layer:
 `value` is the whole-step throughput in TFLOP/s, counting 2*M*N*K per projection (the same
 numerator for every P).  Inputs (activations and bf16 weights, about 0.85 GB) are larger than the
 126 MB L2 and are resident in HBM when timing starts.  Extra keys report the decode path (M in
-{1,4,16}, 36 distinct layers per CUDA-graph replay) in GB/s and the overhead against P = 0.
+{1,4,16}, 36 distinct layers per CUDA-graph replay) in GB/s and the overhead against P = 0, and
+the mixture-of-experts projections (64 experts: a 32768-row prefill batch in TFLOP/s, decode
+batches of 16 and 64 tokens in GB/s).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extras]
                   [--case step|gemm|decode|prep|moe] [--shape ...] [--unfused]
