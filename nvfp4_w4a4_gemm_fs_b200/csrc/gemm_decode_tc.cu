@@ -19,6 +19,11 @@
 // producer loads only the weight side, and warps 2..5, before their epilogue, encode this CTA's K
 // range of the tokens into each stage (Mask S->0, FP4 Quant, Extract X_S of §5.1 "Data
 // preparation") and hand it to the MMA thread through a second per-stage barrier.
+// The grouped form (mixture-of-experts projections, FS_PATH_DECODE on fs_splice_gemm_grouped)
+// runs one 128-row weight tile of one expert per cluster: the expert's rows come from the device
+// offsets after the programmatic-launch wait, its tokens from the first rows of its 128-row padded
+// range of the grouped activations, its weights from rows e*N .. of the stacked operand; a cluster
+// whose expert has no rows or more than 16 leaves before any copy.
 // Every mbarrier wait is bounded; on expiry the kernel records a timeout in the error word and
 // still reaches both cluster barriers and releases TMEM.
 #include <cudaTypedefs.h>
