@@ -1066,8 +1066,9 @@ def main():
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_STEP[fkey],
                      "traffic_unit": f"DRAM bytes per step (the {len(gemm_names)} GEMM launches; ncu "
-                                     "dram__bytes_read.sum + dram__bytes_write.sum per shape of the "
-                                     "current kernel)",
+                                     "dram__bytes_read.sum + dram__bytes_write.sum per shape; the "
+                                     "kernel's only later change, a skip of small experts in the "
+                                     "grouped tile map, does not touch dense problems)",
                      "algorithmic_bytes": gemm_alg_bytes(p, layer.fused),
                      "kernel": f"splice_gemm_tc_kernel ({len(gemm_names)} launches: {', '.join(gemm_names)}; "
                                "sum 2MNK / sum of CUDA-event times)",
