@@ -1,0 +1,83 @@
+"""The grouped (mixture-of-experts) tile map of the tensor-core kernel (csrc/gemm_tc.cu: the
+prologue's prefix sums and ``map_tile``), restated on the CPU and checked on random routings.
+
+Per expert e with n_e routed rows: cum_m counts its pair (or single) tiles, 0 for an expert the
+kernel skips (n_e <= skip_small: those run on the decode kernel with FS_PATH_DECODE), and cum_g
+its 128-row groups in the packed activations (every expert padded to 128 rows, whether skipped or
+not: the packed layout is fixed by the grouped quantiser).  Tile mt belongs to the last expert with
+cum_m[e] <= mt; rank r of a CTA pair takes rows local * 128 CG + 128 r of the expert.
+
+Checked: every row of every expert the kernel does not skip is written exactly once, by a CTA
+whose packed A row is the same row of the expert's padded range; skipped and empty experts get no
+rows; every CTA with rows reads scale atoms inside the packed buffer.
+"""
+import numpy as np
+import pytest
+
+KBM = 128
+
+
+def prologue(counts, CG, skip_small):
+    cum_m, cum_g = [0], [0]
+    for n in counts:
+        cum_m.append(cum_m[-1] + (0 if n <= skip_small else -(-n // (KBM * CG))))
+        cum_g.append(cum_g[-1] + -(-n // KBM))
+    return cum_m, cum_g
+
+
+def map_tile(mt, rank, CG, offsets, cum_m, cum_g):
+    E = len(offsets) - 1
+    lo, hi = 0, E - 1
+    while lo < hi:
+        mid = (lo + hi + 1) >> 1
+        if cum_m[mid] <= mt:
+            lo = mid
+        else:
+            hi = mid - 1
+    local = mt - cum_m[lo]
+    off = local * (KBM * CG) + rank * KBM
+    arow = cum_g[lo] * KBM + off
+    yrow = offsets[lo] + off
+    rows = min(offsets[lo + 1] - yrow, KBM)                 # <= 0: a pair's CTA past the expert
+    return lo, arow, yrow, rows
+
+
+def check(counts, CG, skip_small):
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64).tolist()
+    cum_m, cum_g = prologue(counts, CG, skip_small)
+    # the packed layout of the grouped quantiser: expert e's rows from pad[e], a 128-row boundary
+    pad = np.concatenate([[0], np.cumsum([-(-n // KBM) * KBM for n in counts])]).astype(np.int64).tolist()
+    written = np.zeros(offsets[-1], np.int64)
+    for mt in range(cum_m[-1]):
+        for rank in range(CG):
+            e, arow, yrow, rows = map_tile(mt, rank, CG, offsets, cum_m, cum_g)
+            assert counts[e] > skip_small, "a skipped or empty expert got a tile"
+            if rows <= 0:
+                continue
+            assert offsets[e] <= yrow and yrow + rows <= offsets[e + 1]
+            assert arow - pad[e] == yrow - offsets[e]               # the same row of the expert
+            assert arow + rows <= pad[e + 1]                        # inside its padded range
+            assert arow // KBM < pad[-1] // KBM                     # its scale atoms exist
+            written[yrow:yrow + rows] += 1
+    for e, n in enumerate(counts):
+        want = 1 if n > skip_small else 0
+        assert np.all(written[offsets[e]:offsets[e + 1]] == want), (e, n)
+
+
+@pytest.mark.parametrize("CG", [1, 2])
+@pytest.mark.parametrize("skip_small", [0, 16])
+def test_grouped_tile_map_covers_every_row_once(CG, skip_small):
+    rng = np.random.default_rng(100 * CG + skip_small)
+    fixed = [[0], [1], [16], [17], [127, 128, 129, 255, 256, 257], [0, 0, 5, 0, 300, 0, 16, 17, 0]]
+    for counts in fixed:
+        check(counts, CG, skip_small)
+    for _ in range(300):
+        E = int(rng.integers(1, 65))
+        kind = rng.integers(0, 3)
+        if kind == 0:
+            counts = rng.integers(0, 40, E)                          # decode-like: small experts
+        elif kind == 1:
+            counts = rng.integers(0, 700, E)                         # prefill-like
+        else:
+            counts = np.where(rng.random(E) < 0.5, 0, rng.integers(1, 300, E))   # many empty
+        check([int(c) for c in counts], CG, skip_small)
