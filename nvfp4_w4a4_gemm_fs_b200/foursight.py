@@ -81,6 +81,49 @@ def alloc_packed(rows: int, K: int, p: int, device="cuda") -> Packed:
     return Packed(q, sf, side if pp else side, rows, K, p)
 
 
+# ------------------------------------------------------------------ extents the C ABI cannot see
+# The library takes plain pointers, so it cannot tell how many bytes stand behind them; these
+# checks compare the tensors' shapes with what a call will read or write before anything is
+# launched (a short buffer would otherwise be read or written past its end on the GPU).
+def _need(ok: bool, who: str, what: str) -> None:
+    if not ok:
+        raise ValueError(f"{who}: {what}")
+
+
+def _check_packed(who: str, name: str, pk: Packed, rows: int, K: int, p: int) -> None:
+    """pk holds at least `rows` rows of the packed layout: E2M1 codes with a row pitch of K/2
+    bytes, the tiled scales of those rows, and (p > 0) bf16 side columns with a pitch of Pp."""
+    q = pk.q
+    _need(q.dim() == 2 and q.dtype == torch.uint8 and q.shape[1] * 2 == K and q.stride(1) == 1
+          and (q.shape[0] <= 1 or q.stride(0) == K // 2), who, f"{name}.q must be uint8 rows of K/2 = {K // 2} bytes")
+    _need(q.shape[0] >= rows, who, f"{name} has {q.shape[0]} rows, {rows} are read or written")
+    _need(pk.sf.dtype == torch.uint8 and pk.sf.is_contiguous() and pk.sf.numel() >= sf_bytes(rows, K), who,
+          f"{name}.sf must hold the {sf_bytes(rows, K)} tiled scale bytes of {rows} rows")
+    if p > 0:
+        pp, sd = side_cols(p), pk.side
+        _need(sd is not None and sd.dim() == 2 and sd.dtype == torch.bfloat16 and sd.shape[0] >= rows
+              and sd.shape[1] >= pp and sd.stride(1) == 1 and (sd.shape[0] <= 1 or sd.stride(0) == pp), who,
+              f"{name}.side must be bf16 rows of Pp = {pp} columns")
+
+
+def _check_out(who: str, Y: torch.Tensor, rows: int, cols: int, bf16: bool) -> None:
+    _need(Y.dim() == 2 and Y.shape[0] >= rows and Y.shape[1] >= cols and Y.stride(1) == 1, who,
+          f"Y must have at least {rows} rows of {cols} columns, unit column stride")
+    _need(Y.dtype == (torch.bfloat16 if bf16 else torch.float32), who,
+          f"Y must be {'bfloat16' if bf16 else 'float32'} for this plan")
+
+
+def _check_floats(who: str, name: str, t: torch.Tensor, n: int) -> None:
+    _need(t.dtype == torch.float32 and t.numel() >= n, who, f"{name} must hold {n} float32 values")
+
+
+def _check_gemm_operands(who: str, plan: "Plan", xq: Packed, wq: Packed, alpha, w_rows: int, n_alpha: int) -> None:
+    _need(xq.p == wq.p, who, "activations and weights must share p")
+    _check_packed(who, "xq", xq, xq.rows, plan.K, xq.p)
+    _check_packed(who, "wq", wq, w_rows, plan.K, wq.p)
+    _check_floats(who, "alpha", alpha, n_alpha)
+
+
 def fs_channel_stats(X: torch.Tensor, state: StatsState, group: int = 0, row_stride: int = 1, stream=None):
     lib = _lib.load()
     n, s1, s2, amax, flags = state.group(group)
@@ -123,6 +166,9 @@ def fs_prepare_weights(W: torch.Tensor, mask, p: int, gA: torch.Tensor, opts: in
     out = alloc_packed(N, _packed_cols(K, p, opts), p, W.device) if out is None else out
     gW = torch.empty(1, dtype=torch.float32, device=W.device) if gW is None else gW
     alpha = torch.empty(1, dtype=torch.float32, device=W.device) if alpha is None else alpha
+    _check_packed("fs_prepare_weights", "out", out, N, _packed_cols(K, p, opts), p)
+    _check_floats("fs_prepare_weights", "gW", gW, 1)
+    _check_floats("fs_prepare_weights", "alpha", alpha, 1)
     check(lib.fs_prepare_weights(_ptr(W), _dtype_code(W), N, K, W.stride(0), _ptr(mask) if p else None, p, opts,
                                  _ptr(gA), _ptr(out.q), _ptr(out.sf), _ptr(out.side) if p else None, _ptr(gW),
                                  _ptr(alpha), stream_handle(stream)), "fs_prepare_weights")
@@ -134,6 +180,7 @@ def fs_quantize_splice(X: torch.Tensor, mask, p: int, gA: torch.Tensor, opts: in
     lib = _lib.load()
     M, K = X.shape
     out = alloc_packed(M, _packed_cols(K, p, opts), p, X.device) if out is None else out
+    _check_packed("fs_quantize_splice", "out", out, M, _packed_cols(K, p, opts), p)
     check(lib.fs_quantize_splice(_ptr(X), _dtype_code(X), M, K, X.stride(0), _ptr(mask) if p else None, p,
                                  _ptr(gA), opts, _ptr(out.q), _ptr(out.sf), _ptr(out.side) if p else None,
                                  stream_handle(stream)), "fs_quantize_splice")
@@ -147,6 +194,8 @@ def fs_quantize_splice_stats(X: torch.Tensor, mask, p: int, gA: torch.Tensor, st
     lib = _lib.load()
     M, K = X.shape
     out = alloc_packed(M, K, p, X.device) if out is None else out
+    _check_packed("fs_quantize_splice_stats", "out", out, M, K, p)
+    _need(state.K == K, "fs_quantize_splice_stats", f"statistics state of K = {state.K} for K = {K}")
     n, s1, s2, amax, flags = state.group(group)
     check(lib.fs_quantize_splice_stats(_ptr(X), _dtype_code(X), M, K, X.stride(0), _ptr(mask) if p else None, p,
                                        _ptr(gA), opts, _ptr(out.q), _ptr(out.sf), _ptr(out.side) if p else None,
@@ -162,6 +211,7 @@ def fs_quantize_splice_grouped(X: torch.Tensor, row_offsets: torch.Tensor, masks
     E = row_offsets.numel() - 1
     max_rows = rows if max_rows is None else max_rows
     out = alloc_packed(grouped_rows(max_rows, E), K, p, X.device) if out is None else out
+    _check_packed("fs_quantize_splice_grouped", "out", out, grouped_rows(max_rows, E), K, p)
     check(lib.fs_quantize_splice_grouped(_ptr(X), _dtype_code(X), E, _ptr(row_offsets), max_rows, K, X.stride(0),
                                          _ptr(masks) if p else None, p, _ptr(gA), opts, _ptr(out.q), _ptr(out.sf),
                                          _ptr(out.side) if p else None, stream_handle(stream)),
@@ -200,6 +250,8 @@ def fs_splice_gemm(plan: Plan, xq: Packed, wq: Packed, alpha: torch.Tensor, Y: t
     if Y is None:
         dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
         Y = torch.empty(M, plan.N, dtype=dt, device=xq.q.device)
+    _check_gemm_operands("fs_splice_gemm", plan, xq, wq, alpha, plan.N, 1)
+    _check_out("fs_splice_gemm", Y, M, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
     check(lib.fs_splice_gemm(plan.handle, M, xq.p, _ptr(xq.q), _ptr(xq.sf), _ptr(xq.side) if xq.p else None,
                              _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, _ptr(alpha), _ptr(Y),
                              Y.stride(0), stream_handle(stream)), "fs_splice_gemm")
@@ -217,6 +269,8 @@ def fs_splice_gemm_segmented(plan: Plan, xq: Packed, wq: Packed, alpha: torch.Te
     if Y is None:
         dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
         Y = torch.empty(M, plan.N, dtype=dt, device=xq.q.device)
+    _check_gemm_operands("fs_splice_gemm_segmented", plan, xq, wq, alpha, plan.N, max(len(seg) - 1, 1))
+    _check_out("fs_splice_gemm_segmented", Y, M, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
     check(lib.fs_splice_gemm_segmented(plan.handle, M, xq.p, _ptr(xq.q), _ptr(xq.sf), _ptr(xq.side) if xq.p else None,
                                        _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, len(seg) - 1, arr,
                                        _ptr(alpha), _ptr(Y), Y.stride(0), stream_handle(stream)),
@@ -242,6 +296,16 @@ def fs_decode_splice_gemm(plan: Plan, X: torch.Tensor, mask, p: int, gA: torch.T
     if Y is None:
         dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
         Y = torch.empty(M, plan.N, dtype=dt, device=X.device)
+    who = "fs_decode_splice_gemm"
+    _need(X.dim() == 2 and X.shape[1] == plan.K and X.stride(1) == 1, who, f"X must be [M, K = {plan.K}] rows")
+    _need(wq.p == p, who, "the weights must be prepared with the same p")
+    _check_packed(who, "wq", wq, plan.N, plan.K, p)
+    _check_floats(who, "alpha", alpha, nseg)
+    _check_floats(who, "gA", gA, 1)
+    if p > 0:
+        _need(mask is not None and mask.numel() * mask.element_size() >= 4 * ((plan.K + 31) // 32), who,
+              "mask must hold ceil(K/32) words")
+    _check_out(who, Y, M, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
     check(lib.fs_decode_splice_gemm(plan.handle, M, p, _ptr(X), X.stride(0), _ptr(mask) if p else None, _ptr(gA),
                                     xopts, _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, nseg, arr,
                                     _ptr(alpha), _ptr(Y), Y.stride(0), stream_handle(stream)),
@@ -273,6 +337,13 @@ def fs_splice_gemm_grouped(plan: Plan, row_offsets: torch.Tensor, max_rows: int,
     if Y is None:
         dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
         Y = torch.empty(max_rows, plan.N, dtype=dt, device=xq.q.device)
+    who = "fs_splice_gemm_grouped"
+    _need(row_offsets.dtype == torch.int64 and E >= 1, who, "row_offsets must be E + 1 int64 values")
+    _need(xq.p == wq.p, who, "activations and weights must share p")
+    _check_packed(who, "xq", xq, grouped_rows(max_rows, E), plan.K, xq.p)
+    _check_packed(who, "wq", wq, E * plan.N, plan.K, wq.p)
+    _check_floats(who, "alpha", alpha, E)
+    _check_out(who, Y, max_rows, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
     check(lib.fs_splice_gemm_grouped(plan.handle, E, _ptr(row_offsets), max_rows, xq.p, _ptr(xq.q), _ptr(xq.sf),
                                      _ptr(xq.side) if xq.p else None, _ptr(wq.q), _ptr(wq.sf),
                                      _ptr(wq.side) if wq.p else None, _ptr(alpha), _ptr(Y), Y.stride(0),

@@ -1,0 +1,125 @@
+"""The Python binding's extent checks: the C ABI takes plain pointers, so the binding compares the
+tensors' shapes with what each call reads or writes and refuses a short or mistyped buffer before
+anything is launched.
+
+These run on the CPU: the library's launching entries are replaced by no-ops (the host-only size
+helpers stay real), so the bench's own step, with its real buffers, passes through every check,
+and each kind of wrong buffer raises ValueError without reaching the library.
+"""
+import pytest
+import torch
+
+import bench
+import nvfp4_w4a4_gemm_fs_b200 as F
+from nvfp4_w4a4_gemm_fs_b200 import _lib
+
+HOST_ONLY = {"fs_sf_bytes", "fs_side_cols", "fs_grouped_rows", "fs_compact_cols", "fs_status_string",
+             "fs_last_error", "fs_version"}
+
+
+@pytest.fixture
+def no_launch(monkeypatch):
+    real = _lib.load()
+    calls = []
+
+    class Fake:
+        def __getattr__(self, name):
+            if name in HOST_ONLY:
+                return getattr(real, name)
+
+            def fn(*args):
+                calls.append(name)
+                return 0                                        # FS_OK, nothing launched
+            return fn
+    monkeypatch.setattr(_lib, "load", lambda: Fake())
+    monkeypatch.setattr(F.foursight, "stream_handle", lambda stream=None: 0)   # no CUDA stream here
+    return calls
+
+
+@pytest.mark.parametrize("fused,compact,p,out_bf16,fused_prep", [(True, False, 64, False, False),
+                                                                 (False, False, 64, False, False),
+                                                                 (True, True, 256, False, False),
+                                                                 (True, False, 0, True, False),
+                                                                 (True, False, 64, False, True)])
+def test_the_bench_step_passes_every_check(no_launch, fused, compact, p, out_bf16, fused_prep):
+    lay = bench.PrefillLayer(F, 256, p, seed=1, device="cpu", out_bf16=out_bf16, fused=fused, compact=compact,
+                             fused_prep=fused_prep)
+    lay.step()
+    assert "fs_splice_gemm_segmented" in no_launch or "fs_splice_gemm" in no_launch
+
+
+def test_decode_shaped_calls_pass_every_check(no_launch):
+    K, p, M = 4096, 64, 16
+    rows = [4096, 1024, 1024]
+    wall, views = F.stacked_packed(rows, K, p, "cpu")
+    alpha = torch.zeros(3)
+    mask = torch.zeros(K // 32, dtype=torch.int32)
+    gA = torch.ones(1)
+    X = torch.zeros(M, K, dtype=torch.bfloat16)
+    plan = F.Plan(sum(rows), K, p)
+    xq = F.fs_quantize_splice(X, mask, p, gA)
+    F.fs_splice_gemm_segmented(plan, xq, wall, alpha, [0, 4096, 5120, 6144])
+    F.fs_decode_splice_gemm(plan, X, mask, p, gA, wall, alpha, seg_start=[0, 4096, 5120, 6144])
+    wide = torch.zeros(M, K + 192, dtype=torch.bfloat16)
+    F.fs_decode_splice_gemm(F.Plan(4096, K, p), wide[:, 64:64 + K], mask, p, gA, views[0], alpha[:1])
+
+
+def _gemm_inputs(M=32, N=256, K=512, p=16):
+    mask = torch.zeros(K // 32, dtype=torch.int32)
+    gA = torch.ones(1)
+    xq = F.fs_quantize_splice(torch.zeros(M, K, dtype=torch.bfloat16), mask, p, gA)
+    wq, _, alpha = F.fs_prepare_weights(torch.zeros(N, K, dtype=torch.bfloat16), mask, p, gA)
+    return xq, wq, alpha, mask, gA
+
+
+def test_short_or_mistyped_buffers_are_refused(no_launch):
+    M, N, K, p = 32, 256, 512, 16
+    xq, wq, alpha, mask, gA = _gemm_inputs(M, N, K, p)
+    plan = F.Plan(N, K, p)
+    plan16 = F.Plan(N, K, p, F.FS_OUT_BF16)
+    F.fs_splice_gemm(plan, xq, wq, alpha)                                   # well-formed: accepted
+    bad = [
+        lambda: F.fs_splice_gemm(plan, xq, wq, alpha, Y=torch.empty(M - 1, N)),             # short Y
+        lambda: F.fs_splice_gemm(plan, xq, wq, alpha, Y=torch.empty(M, N - 16)),            # narrow Y
+        lambda: F.fs_splice_gemm(plan, xq, wq, alpha, Y=torch.empty(M, N, dtype=torch.bfloat16)),   # dtype
+        lambda: F.fs_splice_gemm(plan16, xq, wq, alpha, Y=torch.empty(M, N)),
+        lambda: F.fs_splice_gemm(plan, xq, wq, alpha, Y=torch.empty(N, M).t()),             # strided columns
+        lambda: F.fs_splice_gemm(F.Plan(2 * N, K, p), xq, wq, alpha),                       # weights too short
+        lambda: F.fs_splice_gemm(F.Plan(N, 2 * K, p), xq, wq, alpha),                       # K differs
+        lambda: F.fs_splice_gemm(plan, xq, F.Packed(wq.q, wq.sf[:100], wq.side, N, K, p), alpha),   # scales
+        lambda: F.fs_splice_gemm(plan, xq, F.Packed(wq.q, wq.sf, wq.side[:, :8], N, K, p), alpha),  # side
+        lambda: F.fs_splice_gemm(plan, F.alloc_packed(M, K, 32, "cpu"), wq, alpha),               # p differs
+        lambda: F.fs_splice_gemm_segmented(plan, xq, wq, alpha, [0, 128, 256]),             # one alpha, two segments
+        lambda: F.fs_decode_splice_gemm(plan, torch.zeros(4, K // 2, dtype=torch.bfloat16), mask, p, gA, wq, alpha),
+        lambda: F.fs_decode_splice_gemm(plan, torch.zeros(4, K, dtype=torch.bfloat16), mask[:2], p, gA, wq, alpha),
+        lambda: F.fs_quantize_splice(torch.zeros(M, K, dtype=torch.bfloat16), mask, p, gA,
+                                     out=F.alloc_packed(M - 1, K, p, "cpu")),                      # short out
+        lambda: F.fs_prepare_weights(torch.zeros(N, K, dtype=torch.bfloat16), mask, p, gA,
+                                     out=F.alloc_packed(N, 2 * K, p, "cpu")),                      # wrong width
+    ]
+    for call in bad:
+        n = len(no_launch)
+        with pytest.raises(ValueError):
+            call()
+        assert all(name == "fs_plan_create" for name in no_launch[n:]), no_launch[n:]   # nothing launched
+
+
+def test_grouped_buffers_are_checked(no_launch):
+    E, N, K, p, total = 4, 256, 512, 16, 100
+    offs = torch.tensor([0, 10, 40, 70, 100], dtype=torch.int64)
+    X = torch.zeros(total, K, dtype=torch.bfloat16)
+    masks = torch.zeros(E, K // 32, dtype=torch.int32)
+    gA = torch.ones(E)
+    xq = F.fs_quantize_splice_grouped(X, offs, masks, p, gA)
+    wq = F.alloc_packed(E * N, K, p, "cpu")
+    alpha = torch.zeros(E)
+    plan = F.Plan(N, K, p)
+    F.fs_splice_gemm_grouped(plan, offs, total, xq, wq, alpha)              # well-formed: accepted
+    with pytest.raises(ValueError):
+        F.fs_splice_gemm_grouped(plan, offs, total, F.alloc_packed(total, K, p, "cpu"), wq, alpha)   # not padded
+    with pytest.raises(ValueError):
+        F.fs_splice_gemm_grouped(plan, offs, total, xq, F.alloc_packed(N, K, p, "cpu"), alpha)       # one expert's rows
+    with pytest.raises(ValueError):
+        F.fs_splice_gemm_grouped(plan, offs, total, xq, wq, alpha[:2])
+    with pytest.raises(ValueError):
+        F.fs_splice_gemm_grouped(plan, offs.to(torch.int32), total, xq, wq, alpha)
