@@ -18,7 +18,7 @@ __all__ = [
     "fs_seq_filter", "Plan", "StatsState", "Packed", "side_cols", "sf_bytes", "grouped_rows", "compact_cols",
     "fs_splice_gemm_segmented", "fs_decode_splice_gemm", "stacked_packed", "fs_gemm_bf16", "fs_transpose_bf16", "fs_ste_backward",
     "fs_grpo_objective", "fs_k3_kl",
-    "alloc_packed", "stream_handle",
+    "alloc_packed", "stream_handle", "ArgumentError",
 ]
 
 
@@ -85,9 +85,18 @@ def alloc_packed(rows: int, K: int, p: int, device="cuda") -> Packed:
 # The library takes plain pointers, so it cannot tell how many bytes stand behind them; these
 # checks compare the tensors' shapes with what a call will read or write before anything is
 # launched (a short buffer would otherwise be read or written past its end on the GPU).
+class ArgumentError(_lib.FoursightError, ValueError):
+    """An argument the binding refuses before calling the library: status FS_ERR_INVALID_ARGUMENT,
+    as the library reports its own argument errors (and a ValueError)."""
+
+    def __init__(self, who: str, what: str):
+        RuntimeError.__init__(self, f"{who}: invalid argument: {what}")
+        self.status = _lib.FS_ERR_INVALID_ARGUMENT
+
+
 def _need(ok: bool, who: str, what: str) -> None:
     if not ok:
-        raise ValueError(f"{who}: {what}")
+        raise ArgumentError(who, what)
 
 
 def _check_packed(who: str, name: str, pk: Packed, rows: int, K: int, p: int) -> None:
@@ -250,8 +259,9 @@ def fs_splice_gemm(plan: Plan, xq: Packed, wq: Packed, alpha: torch.Tensor, Y: t
     if Y is None:
         dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
         Y = torch.empty(M, plan.N, dtype=dt, device=xq.q.device)
-    _check_gemm_operands("fs_splice_gemm", plan, xq, wq, alpha, plan.N, 1)
-    _check_out("fs_splice_gemm", Y, M, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
+    if M > 0:                                       # an empty batch reads no operand
+        _check_gemm_operands("fs_splice_gemm", plan, xq, wq, alpha, plan.N, 1)
+        _check_out("fs_splice_gemm", Y, M, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
     check(lib.fs_splice_gemm(plan.handle, M, xq.p, _ptr(xq.q), _ptr(xq.sf), _ptr(xq.side) if xq.p else None,
                              _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, _ptr(alpha), _ptr(Y),
                              Y.stride(0), stream_handle(stream)), "fs_splice_gemm")
@@ -269,8 +279,9 @@ def fs_splice_gemm_segmented(plan: Plan, xq: Packed, wq: Packed, alpha: torch.Te
     if Y is None:
         dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
         Y = torch.empty(M, plan.N, dtype=dt, device=xq.q.device)
-    _check_gemm_operands("fs_splice_gemm_segmented", plan, xq, wq, alpha, plan.N, max(len(seg) - 1, 1))
-    _check_out("fs_splice_gemm_segmented", Y, M, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
+    if M > 0:
+        _check_gemm_operands("fs_splice_gemm_segmented", plan, xq, wq, alpha, plan.N, max(len(seg) - 1, 1))
+        _check_out("fs_splice_gemm_segmented", Y, M, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
     check(lib.fs_splice_gemm_segmented(plan.handle, M, xq.p, _ptr(xq.q), _ptr(xq.sf), _ptr(xq.side) if xq.p else None,
                                        _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, len(seg) - 1, arr,
                                        _ptr(alpha), _ptr(Y), Y.stride(0), stream_handle(stream)),
@@ -297,15 +308,16 @@ def fs_decode_splice_gemm(plan: Plan, X: torch.Tensor, mask, p: int, gA: torch.T
         dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
         Y = torch.empty(M, plan.N, dtype=dt, device=X.device)
     who = "fs_decode_splice_gemm"
-    _need(X.dim() == 2 and X.shape[1] == plan.K and X.stride(1) == 1, who, f"X must be [M, K = {plan.K}] rows")
-    _need(wq.p == p, who, "the weights must be prepared with the same p")
-    _check_packed(who, "wq", wq, plan.N, plan.K, p)
-    _check_floats(who, "alpha", alpha, nseg)
-    _check_floats(who, "gA", gA, 1)
-    if p > 0:
-        _need(mask is not None and mask.numel() * mask.element_size() >= 4 * ((plan.K + 31) // 32), who,
-              "mask must hold ceil(K/32) words")
-    _check_out(who, Y, M, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
+    if M > 0:
+        _need(X.dim() == 2 and X.shape[1] == plan.K and X.stride(1) == 1, who, f"X must be [M, K = {plan.K}] rows")
+        _need(wq.p == p, who, "the weights must be prepared with the same p")
+        _check_packed(who, "wq", wq, plan.N, plan.K, p)
+        _check_floats(who, "alpha", alpha, nseg)
+        _check_floats(who, "gA", gA, 1)
+        if p > 0:
+            _need(mask is not None and mask.numel() * mask.element_size() >= 4 * ((plan.K + 31) // 32), who,
+                  "mask must hold ceil(K/32) words")
+        _check_out(who, Y, M, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
     check(lib.fs_decode_splice_gemm(plan.handle, M, p, _ptr(X), X.stride(0), _ptr(mask) if p else None, _ptr(gA),
                                     xopts, _ptr(wq.q), _ptr(wq.sf), _ptr(wq.side) if wq.p else None, nseg, arr,
                                     _ptr(alpha), _ptr(Y), Y.stride(0), stream_handle(stream)),
@@ -338,12 +350,13 @@ def fs_splice_gemm_grouped(plan: Plan, row_offsets: torch.Tensor, max_rows: int,
         dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
         Y = torch.empty(max_rows, plan.N, dtype=dt, device=xq.q.device)
     who = "fs_splice_gemm_grouped"
-    _need(row_offsets.dtype == torch.int64 and E >= 1, who, "row_offsets must be E + 1 int64 values")
-    _need(xq.p == wq.p, who, "activations and weights must share p")
-    _check_packed(who, "xq", xq, grouped_rows(max_rows, E), plan.K, xq.p)
-    _check_packed(who, "wq", wq, E * plan.N, plan.K, wq.p)
-    _check_floats(who, "alpha", alpha, E)
-    _check_out(who, Y, max_rows, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
+    if max_rows > 0:                                # no routed rows: nothing is read or written
+        _need(row_offsets.dtype == torch.int64 and E >= 1, who, "row_offsets must be E + 1 int64 values")
+        _need(xq.p == wq.p, who, "activations and weights must share p")
+        _check_packed(who, "xq", xq, grouped_rows(max_rows, E), plan.K, xq.p)
+        _check_packed(who, "wq", wq, E * plan.N, plan.K, wq.p)
+        _check_floats(who, "alpha", alpha, E)
+        _check_out(who, Y, max_rows, plan.N, bool(plan.opts & _lib.FS_OUT_BF16))
     check(lib.fs_splice_gemm_grouped(plan.handle, E, _ptr(row_offsets), max_rows, xq.p, _ptr(xq.q), _ptr(xq.sf),
                                      _ptr(xq.side) if xq.p else None, _ptr(wq.q), _ptr(wq.sf),
                                      _ptr(wq.side) if wq.p else None, _ptr(alpha), _ptr(Y), Y.stride(0),

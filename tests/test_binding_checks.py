@@ -104,6 +104,20 @@ def test_short_or_mistyped_buffers_are_refused(no_launch):
         assert all(name == "fs_plan_create" for name in no_launch[n:]), no_launch[n:]   # nothing launched
 
 
+def test_refusals_are_library_argument_errors_and_empty_batches_read_nothing(no_launch):
+    """A refused buffer raises the library's invalid-argument status (callers that expect the
+    library's FoursightError see it), and an empty batch is passed through unchecked, as the
+    library reads no operand then."""
+    M, N, K, p = 32, 256, 512, 16
+    xq, wq, alpha, mask, gA = _gemm_inputs(M, N, K, p)
+    with pytest.raises(F.FoursightError) as exc:
+        F.fs_splice_gemm(F.Plan(2 * N, K, p), xq, wq, alpha)
+    assert exc.value.status == 1                                            # FS_ERR_INVALID_ARGUMENT
+    empty = F.fs_quantize_splice(torch.zeros(0, K, dtype=torch.bfloat16), mask, p, gA)
+    F.fs_splice_gemm(F.Plan(N, K, p), empty, wq, alpha)
+    F.fs_splice_gemm_grouped(F.Plan(N, K, p), torch.zeros(3, dtype=torch.int64), 0, empty, wq, alpha.repeat(2))
+
+
 def test_grouped_buffers_are_checked(no_launch):
     E, N, K, p, total = 4, 256, 512, 16, 100
     offs = torch.tensor([0, 10, 40, 70, 100], dtype=torch.int64)
