@@ -103,11 +103,13 @@ def _check_packed(who: str, name: str, pk: Packed, rows: int, K: int, p: int) ->
     """pk holds at least `rows` rows of the packed layout: E2M1 codes with a row pitch of K/2
     bytes, the tiled scales of those rows, and (p > 0) bf16 side columns with a pitch of Pp."""
     q = pk.q
-    _need(q.dim() == 2 and q.dtype == torch.uint8 and q.shape[1] * 2 == K and q.stride(1) == 1
-          and (q.shape[0] <= 1 or q.stride(0) == K // 2), who, f"{name}.q must be uint8 rows of K/2 = {K // 2} bytes")
-    _need(q.shape[0] >= rows, who, f"{name} has {q.shape[0]} rows, {rows} are read or written")
-    _need(pk.sf.dtype == torch.uint8 and pk.sf.is_contiguous() and pk.sf.numel() >= sf_bytes(rows, K), who,
-          f"{name}.sf must hold the {sf_bytes(rows, K)} tiled scale bytes of {rows} rows")
+    if K > 0:                                       # (a compacted operand of no columns has no codes)
+        _need(q.dim() == 2 and q.dtype == torch.uint8 and q.shape[1] * 2 == K and q.stride(1) == 1
+              and (q.shape[0] <= 1 or q.stride(0) == K // 2), who,
+              f"{name}.q must be uint8 rows of K/2 = {K // 2} bytes")
+        _need(q.shape[0] >= rows, who, f"{name} has {q.shape[0]} rows, {rows} are read or written")
+        _need(pk.sf.dtype == torch.uint8 and pk.sf.is_contiguous() and pk.sf.numel() >= sf_bytes(rows, K), who,
+              f"{name}.sf must hold the {sf_bytes(rows, K)} tiled scale bytes of {rows} rows")
     if p > 0:
         pp, sd = side_cols(p), pk.side
         _need(sd is not None and sd.dim() == 2 and sd.dtype == torch.bfloat16 and sd.shape[0] >= rows

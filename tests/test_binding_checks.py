@@ -48,6 +48,19 @@ def test_the_bench_step_passes_every_check(no_launch, fused, compact, p, out_bf1
     assert "fs_splice_gemm_segmented" in no_launch or "fs_splice_gemm" in no_launch
 
 
+@pytest.mark.parametrize("M,K,p", [(8, 512, 64), (3, 256, 256), (5, 256, 0), (0, 512, 16), (16, 12288, 256)])
+def test_quantise_and_pre_split_outputs_pass_every_check(no_launch, M, K, p):
+    """The binding's own outputs in every form: split and compacted K, p = 0, p = K (a compacted
+    operand of no NVFP4 columns), an empty batch."""
+    mask = torch.zeros((K + 31) // 32, dtype=torch.int32)
+    gA = torch.ones(1)
+    for opts in (0, F.FS_COMPACT_K):
+        F.fs_quantize_splice(torch.zeros(M, K, dtype=torch.bfloat16), mask, p, gA, opts=opts)
+        F.fs_quantize_splice(torch.zeros(M, K, dtype=torch.float32), mask, p, gA, opts=opts)
+        F.fs_prepare_weights(torch.zeros(max(M, 128), K, dtype=torch.bfloat16), mask, p, gA, opts=opts)
+    F.fs_quantize_splice_stats(torch.zeros(M, K, dtype=torch.bfloat16), mask, p, gA, F.StatsState(1, K, device="cpu"))
+
+
 def test_decode_shaped_calls_pass_every_check(no_launch):
     K, p, M = 4096, 64, 16
     rows = [4096, 1024, 1024]
