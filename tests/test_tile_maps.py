@@ -81,3 +81,24 @@ def test_grouped_tile_map_covers_every_row_once(CG, skip_small):
         else:
             counts = np.where(rng.random(E) < 0.5, 0, rng.integers(1, 300, E))   # many empty
         check([int(c) for c in counts], CG, skip_small)
+
+
+@pytest.mark.parametrize("i", [0, 1, 2, 3])
+def test_overlapping_accumulator_epilogue_writes_every_column_once(i):
+    """BN = 256 with overlapping accumulators (csrc/gemm_tc.cu, epilogue): tile i accumulates in
+    TMEM columns [base, base + 256), base = 128 (i & 1), so consecutive tiles share [128, 256).
+    Part 1 reads those shared columns (released at once), part 2 the others; every TMEM column read
+    maps to output column (column - base), and each of the 256 output columns is written once."""
+    base = 128 * (i & 1)
+    p1_tcol, p1_ocol = 128, 128 - base
+    p2_tcol, p2_ocol = (0, 0) if base == 0 else (256, 128)
+    written = []
+    for tcol0, ocol0 in ((p1_tcol, p1_ocol), (p2_tcol, p2_ocol)):
+        for c in range(4):                                   # 32-column chunks
+            tcol, ocol = tcol0 + 32 * c, ocol0 + 32 * c
+            assert base <= tcol < base + 256 and tcol - base == ocol
+            written += range(ocol, ocol + 32)
+    assert sorted(written) == list(range(256))
+    shared = set(range(128, 256))                            # the next tile's accumulator overlaps these
+    assert set(range(p1_tcol, p1_tcol + 128)) == shared      # part 1 frees exactly the shared half
+    assert base + 256 <= 384                                 # inside the 384 accumulator columns
