@@ -100,3 +100,46 @@ def test_fused_preparation_x_swizzle_is_the_128_byte_pattern():
     for r in range(KD_TOK):
         offs = sorted(128 * r + 16 * (c ^ (r & 7)) for c in range(8))
         assert offs == [128 * r + 16 * j for j in range(8)]
+
+
+def _protected_list_like_the_decode_prep(words, KT):
+    """The fused preparation's channel list: 128 threads take contiguous ranges of the K/32 mask
+    words (ceil(nw / 128) each), count their set bits, scan the counts in thread order and write
+    their channels in ascending order from that position (positions past 256 dropped)."""
+    nw = KT * 8
+    per = -(-nw // 128)
+    counts, ranges = [], []
+    for t in range(128):
+        w0 = min(t * per, nw)
+        w1 = min(w0 + per, nw)
+        ranges.append((w0, w1))
+        counts.append(sum(bin(int(words[w])).count("1") for w in range(w0, w1)))
+    pidx = [0] * 256
+    pos = 0
+    for t in range(128):
+        w0, w1 = ranges[t]
+        for w in range(w0, w1):
+            mw = int(words[w])
+            while mw:
+                b = (mw & -mw).bit_length() - 1
+                mw &= mw - 1
+                if pos < 256:
+                    pidx[pos] = w * 32 + b
+                pos += 1
+    assert pos == sum(counts)
+    return pidx, pos
+
+
+def test_decode_prep_protected_channel_list():
+    """The list equals the protected channels in ascending order (the side columns' order) for
+    random sets of up to 256 channels, K from 256 to 16384 (per-thread ranges of 1 to 4 words)."""
+    import numpy as np
+    rng = np.random.default_rng(21)
+    for K in (256, 512, 4096, 12288, 16384):
+        for p in (0, 1, 17, 64, 256):
+            P = np.sort(rng.choice(K, p, replace=False))
+            words = np.zeros(K // 32, np.uint64)
+            for j in P:
+                words[j // 32] |= np.uint64(1) << np.uint64(j % 32)
+            pidx, n = _protected_list_like_the_decode_prep(words, K // 256)
+            assert n == p and pidx[:p] == P.tolist()

@@ -122,3 +122,56 @@ def test_grouped_quantiser_rows_land_in_the_padded_layout(K):
                 for j in range(pad[e], pad[e + 1]):
                     want = offs[e] + (j - pad[e]) if j - pad[e] < counts[e] else None
                     assert written.get(j, "missing") == want, (e, j)
+
+
+def _mask_tables_like_the_quantiser(words, nb):
+    """The per-CTA tables: thread t takes blocks [t per, t per + per), per = ceil(nb / 256); each
+    block's 16 mask bits; the side column of its first protected lane from an exclusive scan of the
+    per-thread counts; the channel of every side column; per block eight words of lanes to clear."""
+    per = -(-nb // THREADS)
+    mbits = [(int(words[b >> 1]) >> ((b & 1) * 16)) & 0xFFFF for b in range(nb)]
+    col, c = [0] * nb, 0
+    for t in range(THREADS):
+        for b in range(t * per, min(t * per + per, nb)):
+            col[b] = c
+            c += bin(mbits[b]).count("1")
+    pidx = [0] * 256
+    for b in range(nb):
+        mb, k = mbits[b], col[b]
+        while mb:
+            j = (mb & -mb).bit_length() - 1
+            mb &= mb - 1
+            pidx[k] = b * 16 + j
+            k += 1
+    kill = []
+    for b in range(nb):
+        ws = []
+        for j in range(8):
+            two = (mbits[b] >> (2 * j)) & 3
+            ws.append(((two & 1) | ((two & 2) << 15)) * 0xFFFF)
+        kill.append(ws)
+    return mbits, col, pidx, kill
+
+
+def test_quantiser_mask_tables():
+    """Side columns, channel list and lane kills equal their definitions: the side column of a
+    block is the count of protected channels before it, the list is the protected channels in
+    ascending order, and the kill words clear exactly the protected bf16 lanes of a block."""
+    rng = np.random.default_rng(23)
+    for K in (64, 512, 4096, 12288, 16384):
+        nb = K // 16
+        for p in (0, 1, 16, 64, 256):
+            P = np.sort(rng.choice(K, min(p, K), replace=False))
+            words = np.zeros(K // 32, np.uint64)
+            for j in P:
+                words[j // 32] |= np.uint64(1) << np.uint64(j % 32)
+            mbits, col, pidx, kill = _mask_tables_like_the_quantiser(words, nb)
+            assert col == [int(np.sum(P < 16 * b)) for b in range(nb)]
+            assert pidx[:len(P)] == P.tolist()
+            for b in rng.integers(0, nb, 20):
+                lanes = rng.integers(1, 0xFFFF, 16)              # bf16 bit patterns, none zero
+                wordsb = [int(lanes[2 * j]) | (int(lanes[2 * j + 1]) << 16) for j in range(8)]
+                cleared = [w & ~k & 0xFFFFFFFF for w, k in zip(wordsb, kill[b])]
+                out = [(cleared[j // 2] >> (16 * (j % 2))) & 0xFFFF for j in range(16)]
+                prot = {int(j) - 16 * int(b) for j in P if 16 * b <= j < 16 * b + 16}
+                assert [out[j] == 0 for j in range(16)] == [j in prot for j in range(16)]
