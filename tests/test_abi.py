@@ -98,3 +98,34 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.fs_seq_filter(dummy, 64, None, 4, 64, -9.0, 0, 5, 0, None, None, dummy, dummy, dummy, None) == 1
     assert lib.fs_seq_filter(dummy, 64, None, 4, 64, -9.0, 3, 5, 3, dummy, dummy, dummy, dummy, dummy, None) == 1
     assert lib.fs_seq_filter(dummy, 64, None, 0, 64, -9.0, 3, 5, 0, None, None, dummy, dummy, dummy, None) == 0
+
+
+def test_host_validation_of_the_later_entries(lib):
+    """The grouped quantiser, the fused statistics + quantise pass, the fused decode GEMM and the
+    selection refuse bad arguments on the host, before any device call."""
+    dummy = C.c_void_p(256)
+    # grouped quantise: E out of range, null offsets; no routed rows is a no-op
+    assert lib.fs_quantize_splice_grouped(dummy, 0, 0, dummy, 8, 64, 64, None, 0, dummy, 0, dummy, dummy, None,
+                                          None) == 1
+    assert lib.fs_quantize_splice_grouped(dummy, 0, 257, dummy, 8, 64, 64, None, 0, dummy, 0, dummy, dummy, None,
+                                          None) == 1
+    assert lib.fs_quantize_splice_grouped(dummy, 0, 4, None, 8, 64, 64, None, 0, dummy, 0, dummy, dummy, None,
+                                          None) == 1
+    assert lib.fs_quantize_splice_grouped(dummy, 0, 4, dummy, 0, 64, 64, None, 0, dummy, 0, dummy, dummy, None,
+                                          None) == 0
+    # fused statistics + quantise: fp32 activations unsupported (2), row_stride 0, K % 64
+    stats = [dummy] * 5
+    assert lib.fs_quantize_splice_stats(dummy, 1, 4, 64, 64, None, 0, dummy, 0, dummy, dummy, None, 1, *stats,
+                                        None) == 2
+    assert lib.fs_quantize_splice_stats(dummy, 0, 4, 64, 64, None, 0, dummy, 0, dummy, dummy, None, 0, *stats,
+                                        None) == 1
+    assert lib.fs_quantize_splice_stats(dummy, 0, 4, 96, 96, None, 0, dummy, 0, dummy, dummy, None, 1, *stats,
+                                        None) == 1
+    # fused decode GEMM: a plan is required
+    assert lib.fs_decode_splice_gemm(None, 4, 0, dummy, 64, None, dummy, 0, dummy, dummy, None, 1, None, dummy,
+                                     dummy, 256, None) == 1
+    # selection: K above 16384
+    assert lib.fs_select_topk(1, 16416, dummy, dummy, dummy, dummy, dummy, 8, 0, dummy, dummy, dummy, 0, None) == 1
+    # grouped GEMM: a plan is required; E must be positive
+    assert lib.fs_splice_gemm_grouped(None, 4, dummy, 8, 0, dummy, dummy, None, dummy, dummy, None, dummy, dummy,
+                                      256, None) == 1
