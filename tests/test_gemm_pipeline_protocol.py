@@ -1,4 +1,5 @@
-"""The tensor-core SpliceGEMM's pipeline (csrc/gemm_tc.cu, one CTA) as a protocol model.
+"""The tensor-core SpliceGEMM's pipeline (csrc/gemm_tc.cu) as a protocol model, for one CTA and
+for a CTA pair (cta_group::2).
 
 Roles and barriers as in the kernel:
 * the producer waits on a stage's ``empty`` barrier, then issues the stage's scale atoms (FP4
@@ -22,7 +23,8 @@ the MMAs and scale warps that read its previous contents, a scale slot for the M
 previous unit, an accumulator column for the epilogue read of the previous tile that wrote it;
 and that every MMA reads its own k-tile and scale unit, every epilogue read its own finished tile,
 and nothing deadlocks.  Variants with a known mistake (the scale-atom parity taken from the ring's
-phase, the shared columns released before they are read, the wrong half read back) must fail.
+phase, the shared columns released before they are read, the wrong half read back; in a pair, the
+leader's stage barrier expecting only its own bytes, the scale barrier counting one CTA) must fail.
 """
 import random
 
@@ -66,71 +68,79 @@ ACC_MODES = {
 }
 
 
-def play(S, KT, ST, tiles, sf_bufs, sf_split, acc_mode, seed, sfl_global=False):
+def play(S, KT, ST, tiles, sf_bufs, sf_split, acc_mode, seed, cg=1, sfl_global=False, leader_tx=None,
+         sf_count=None):
+    """One random schedule of a CTA (cg = 1) or a CTA pair (cg = 2); returns (problems, finished).
+
+    In a pair the leader (CTA 0) holds the `full`, `sf_full` and `acc_empty` barriers that count
+    both CTAs; the other barriers are per CTA and the leader's commits arrive on both copies.
+    `leader_tx` (copies the leader's `full` expects) and `sf_count` plant pair mistakes."""
     rng = random.Random(seed)
     ktiles = KT + ST
     units = sf_bufs * sf_split
     slots, writes, part1, part2 = ACC_MODES[acc_mode]
-    full = [Bar() for _ in range(S)]
-    sfl = [Bar() for _ in range(S)]
-    empty = [Bar() for _ in range(S)]
-    sf_full = [Bar(QUADS) for _ in range(units)]
-    sf_empty = [Bar() for _ in range(units)]
-    acc_full = [Bar() for _ in range(slots)]
-    acc_empty = [Bar(QUADS) for _ in range(slots)]
+    ctas = range(cg)
+    full = [Bar() for _ in range(S)]                                  # the leader's
+    sfl = [[Bar() for _ in range(S)] for _ in ctas]
+    empty = [[Bar() for _ in range(S)] for _ in ctas]
+    sf_full = [Bar(sf_count or QUADS * cg) for _ in range(units)]     # the leader's
+    sf_empty = [[Bar() for _ in range(units)] for _ in ctas]
+    acc_full = [[Bar() for _ in range(slots)] for _ in ctas]
+    acc_empty = [Bar(QUADS * cg) for _ in range(slots)]               # the leader's
 
-    stage_ab = [None] * S                     # k-tile whose A/B bytes have landed in a stage
-    stage_sf = [None] * S                     # k-tile whose scale atoms have landed in a stage
-    ab_issued = [None] * S                    # k-tile whose copies were last issued to a stage
-    ab_released = [None] * S                  # k-tile whose MMAs' commit on `empty` completed
-    atoms_read = [[None] * S for _ in range(QUADS)]   # k-tile whose atoms each scale warp read
-    slot = [[None] * units for _ in range(QUADS)]     # scale unit each quadrant of a slot holds
-    slot_released = [None] * units            # unit whose MMAs' commit on `sf_empty` completed
-    writer = [dict() for _ in range(QUADS)]   # accumulator column block -> tile that last wrote it
-    read = [dict() for _ in range(QUADS)]     # accumulator column block -> tile last read from it
-    tiles_done = [-1]                         # last tile whose `acc_full` commit completed
+    stage_ab = [[None] * S for _ in ctas]     # k-tile whose A/B bytes have landed in a stage
+    stage_sf = [[None] * S for _ in ctas]     # k-tile whose scale atoms have landed in a stage
+    ab_issued = [[None] * S for _ in ctas]    # k-tile whose copies were last issued to a stage
+    ab_released = [[None] * S for _ in ctas]  # k-tile whose MMAs' commit on `empty` completed
+    atoms_read = [[[None] * S for _ in range(QUADS)] for _ in ctas]   # k-tile each scale warp read
+    slot = [[[None] * units for _ in range(QUADS)] for _ in ctas]     # unit each quadrant of a slot holds
+    slot_released = [[None] * units for _ in ctas]   # unit whose MMAs' commit on `sf_empty` completed
+    writer = [[dict() for _ in range(QUADS)] for _ in ctas]   # accumulator column block -> tile that wrote it
+    read = [[dict() for _ in range(QUADS)] for _ in ctas]     # accumulator column block -> tile last read
+    tiles_done = [-1] * cg                    # last tile whose `acc_full` commit completed
     copies, commits, bad = [], [], []
 
-    def producer():
+    def producer(c):
         stage, phase = 0, 0
         for t in range(tiles):
             for kt in range(ktiles):
                 s, ph = stage, phase
-                yield lambda: empty[s].ok(ph ^ 1)
-                prev = ab_issued[s]
-                if prev is not None and ab_released[s] != prev:
-                    bad.append(("stage overwritten before its MMAs completed", (t, kt), prev))
+                yield lambda: empty[c][s].ok(ph ^ 1)
+                prev = ab_issued[c][s]
+                if prev is not None and ab_released[c][s] != prev:
+                    bad.append(("stage overwritten before its MMAs completed", c, (t, kt), prev))
                 if kt < KT:
-                    if prev is not None and prev[1] < KT and any(atoms_read[q][s] != prev for q in range(QUADS)):
-                        bad.append(("atoms overwritten before the scale warps read them", (t, kt), prev))
-                    sfl[s].arrive(copies=2)                                 # SFA and SFB atoms
-                    copies.extend([("sf", s, (t, kt)), ("sf", s, (t, kt))])
-                full[s].arrive(copies=2)                                    # A and B tiles
-                copies.extend([("ab", s, (t, kt)), ("ab", s, (t, kt))])
-                ab_issued[s] = (t, kt)
+                    if prev is not None and prev[1] < KT and any(atoms_read[c][q][s] != prev for q in range(QUADS)):
+                        bad.append(("atoms overwritten before the scale warps read them", c, (t, kt), prev))
+                    sfl[c][s].arrive(copies=2)                              # SFA and SFB atoms
+                    copies.extend([("sf", c, s, (t, kt))] * 2)
+                if c == 0:                                                  # the leader counts both CTAs' bytes
+                    full[s].arrive(copies=leader_tx or 2 * cg)
+                copies.extend([("ab", c, s, (t, kt))] * 2)                  # A and B tiles
+                ab_issued[c][s] = (t, kt)
                 stage += 1
                 if stage == S:
                     stage, phase = 0, phase ^ 1
 
-    def scale_warp(q):
+    def scale_warp(c, q):
         stage, phase, unit, bits = 0, 0, 0, 0
         for t in range(tiles):
             for kt in range(ktiles):
                 s = stage
                 if kt < KT:
                     par = phase if sfl_global else (bits >> s) & 1
-                    yield lambda: sfl[s].ok(par)
+                    yield lambda: sfl[c][s].ok(par)
                     bits ^= 1 << s
-                    if stage_sf[s] != (t, kt):
-                        bad.append(("scale warp read another k-tile's atoms", (t, kt), stage_sf[s]))
-                    atoms_read[q][s] = (t, kt)
+                    if stage_sf[c][s] != (t, kt):
+                        bad.append(("scale warp read another k-tile's atoms", c, (t, kt), stage_sf[c][s]))
+                    atoms_read[c][q][s] = (t, kt)
                     for h in range(sf_split):
                         u, up = unit % units, ((unit // units) & 1) ^ 1
-                        yield lambda: sf_empty[u].ok(up)
-                        prev = slot[q][u]
-                        if prev is not None and slot_released[u] != prev:
-                            bad.append(("scale slot overwritten before its MMAs completed", (t, kt, h), prev))
-                        slot[q][u] = (t, kt, h)
+                        yield lambda: sf_empty[c][u].ok(up)
+                        prev = slot[c][q][u]
+                        if prev is not None and slot_released[c][u] != prev:
+                            bad.append(("scale slot overwritten before its MMAs completed", c, (t, kt, h), prev))
+                        slot[c][q][u] = (t, kt, h)
                         sf_full[u].arrive()
                         unit += 1
                 stage += 1
@@ -138,12 +148,13 @@ def play(S, KT, ST, tiles, sf_bufs, sf_split, acc_mode, seed, sfl_global=False):
                     stage, phase = 0, phase ^ 1
 
     def mma_writes(i):
-        for q in range(QUADS):
-            for c in writes(i):
-                w = writer[q].get(c)
-                if w is not None and w != i and read[q].get(c) != w:
-                    bad.append(("accumulator overwritten before the epilogue read it", i, w))
-                writer[q][c] = i
+        for c in ctas:
+            for q in range(QUADS):
+                for col in writes(i):
+                    w = writer[c][q].get(col)
+                    if w is not None and w != i and read[c][q].get(col) != w:
+                        bad.append(("accumulator overwritten before the epilogue read it", c, i, w))
+                    writer[c][q][col] = i
 
     def mma():
         stage, phase, acc, acc_phase, unit = 0, 0, 0, 0, 0
@@ -153,14 +164,16 @@ def play(S, KT, ST, tiles, sf_bufs, sf_split, acc_mode, seed, sfl_global=False):
             for kt in range(ktiles):
                 s, ph = stage, phase
                 yield lambda: full[s].ok(ph)
-                if stage_ab[s] != (i, kt):
-                    bad.append(("MMA read another k-tile's operands", (i, kt), stage_ab[s]))
+                for c in ctas:
+                    if stage_ab[c][s] != (i, kt):
+                        bad.append(("MMA read another k-tile's operands", c, (i, kt), stage_ab[c][s]))
                 if kt < KT:
                     for h in range(sf_split):
                         u, up = unit % units, (unit // units) & 1
                         yield lambda: sf_full[u].ok(up)
-                        if any(slot[q][u] != (i, kt, h) for q in range(QUADS)):
-                            bad.append(("MMA read another unit's scales", (i, kt, h), [slot[q][u] for q in range(QUADS)]))
+                        held = [slot[c][q][u] for c in ctas for q in range(QUADS)]
+                        if any(x != (i, kt, h) for x in held):
+                            bad.append(("MMA read another unit's scales", (i, kt, h), held))
                         mma_writes(i)
                         commits.append(("sf", u, (i, kt, h)))
                         unit += 1
@@ -175,28 +188,29 @@ def play(S, KT, ST, tiles, sf_bufs, sf_split, acc_mode, seed, sfl_global=False):
             if acc == slots:
                 acc, acc_phase = 0, acc_phase ^ 1
 
-    def epilogue(q):
+    def epilogue(c, q):
         acc, acc_phase = 0, 0
         for i in range(tiles):
             a, ap = acc, acc_phase
-            yield lambda: acc_full[a].ok(ap)
+            yield lambda: acc_full[c][a].ok(ap)
 
-            def take(c):
-                if writer[q].get(c) != i or tiles_done[0] < i:
-                    bad.append(("epilogue read an unfinished or another tile", i, writer[q].get(c), tiles_done[0]))
-                read[q][c] = i
+            def take(col):
+                if writer[c][q].get(col) != i or tiles_done[c] < i:
+                    bad.append(("epilogue read an unfinished or another tile", c, i, writer[c][q].get(col)))
+                read[c][q][col] = i
 
-            for c in part1(i):
-                take(c)
+            for col in part1(i):
+                take(col)
             acc_empty[a].arrive()
-            for c in part2(i):
+            for col in part2(i):
                 yield lambda: True                        # the next tile's MMAs may run meanwhile
-                take(c)
+                take(col)
             acc += 1
             if acc == slots:
                 acc, acc_phase = 0, acc_phase ^ 1
 
-    roles = [producer(), mma()] + [scale_warp(q) for q in range(QUADS)] + [epilogue(q) for q in range(QUADS)]
+    roles = [mma()] + [producer(c) for c in ctas]
+    roles += [scale_warp(c, q) for c in ctas for q in range(QUADS)] + [epilogue(c, q) for c in ctas for q in range(QUADS)]
     waits = [None] * len(roles)
     alive = [True] * len(roles)
     for _ in range(1000000):
@@ -215,24 +229,25 @@ def play(S, KT, ST, tiles, sf_bufs, sf_split, acc_mode, seed, sfl_global=False):
             break
         pick = rng.choice(choices)
         if pick == "copy":
-            kind, s, ident = copies.pop(rng.randrange(len(copies)))
+            kind, c, s, ident = copies.pop(rng.randrange(len(copies)))
             if kind == "sf":
-                stage_sf[s] = ident
-                sfl[s].land()
+                stage_sf[c][s] = ident
+                sfl[c][s].land()
             else:
-                stage_ab[s] = ident
+                stage_ab[c][s] = ident
                 full[s].land()
         elif pick == "commit":
             kind, k, ident = commits.pop(0)                # tensor-core work completes in order
-            if kind == "sf":
-                slot_released[k] = ident
-                sf_empty[k].arrive()
-            elif kind == "stage":
-                ab_released[k] = ident
-                empty[k].arrive()
-            else:
-                tiles_done[0] = ident
-                acc_full[k].arrive()
+            for c in ctas:                                 # the commit arrives on both CTAs' barriers
+                if kind == "sf":
+                    slot_released[c][k] = ident
+                    sf_empty[c][k].arrive()
+                elif kind == "stage":
+                    ab_released[c][k] = ident
+                    empty[c][k].arrive()
+                else:
+                    tiles_done[c] = ident
+                    acc_full[c][k].arrive()
         else:
             waits[pick] = None                            # the wait passed; run to the next one
     finished = not any(alive) and not copies and not commits
@@ -275,3 +290,26 @@ def test_releasing_the_shared_columns_before_reading_them_races():
 
 def test_reading_back_the_wrong_half_is_caught():
     assert _fails(S=3, KT=2, ST=1, tiles=3, sf_bufs=2, sf_split=1, acc_mode="wrong_half")
+
+
+@pytest.mark.parametrize("acc_mode", ["overlap256", "plain256"])
+@pytest.mark.parametrize("S", [3, 5])
+def test_cta_pairs_read_both_halves_of_their_own_k_tiles(acc_mode, S):
+    """cta_group::2: the leader's MMAs read both CTAs' stages and scale slots and write both
+    CTAs' accumulators; the peer's copies may land on the leader's barrier before the leader
+    has armed it for that phase (its byte count runs below zero until then)."""
+    rng = random.Random(S)
+    for KT, ST in MIXES:
+        for tiles in (1, 2, 4):
+            for seed in range(10):
+                sf_bufs, sf_split = rng.choice([(2, 1), (1, 1), (2, 2)])
+                bad, finished = play(S, KT, ST, tiles, sf_bufs, sf_split, acc_mode, seed, cg=2)
+                assert bad == [] and finished, (acc_mode, S, KT, ST, tiles, sf_bufs, sf_split, seed, bad[:2])
+
+
+def test_a_pair_whose_leader_counts_only_its_own_bytes_races():
+    assert _fails(S=3, KT=2, ST=1, tiles=2, sf_bufs=2, sf_split=1, acc_mode="overlap256", cg=2, leader_tx=2)
+
+
+def test_a_pair_whose_scale_barrier_counts_one_cta_races():
+    assert _fails(S=3, KT=3, ST=0, tiles=2, sf_bufs=2, sf_split=1, acc_mode="overlap256", cg=2, sf_count=QUADS)
