@@ -354,8 +354,12 @@ splice_gemm_decode_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __gr
         ++issued;
         if (++stage == kDStages) { stage = 0; phase ^= 1; }
       }
-      if (*abort_flag) {
-        // copies issued but possibly not landed: the last min(issued, stages) stages
+      {
+        // Copies issued but possibly not landed: the last min(issued, stages) stages, drained
+        // whether or not a wait has given up yet (another role may give up later, and the CTA
+        // must not exit with a copy landing in its shared memory).  The waits replay the
+        // (stage, parity) pairs the MMA waits on; on the normal path they are met before the
+        // epilogue starts.
         int s = stage;
         uint32_t ph = phase;
         for (int i = 0; i < kDStages && i < issued; ++i) {

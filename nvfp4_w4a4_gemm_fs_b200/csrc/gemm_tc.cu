@@ -299,9 +299,14 @@ splice_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
-      if (!ok) {
-        // Copies issued but possibly not landed: the last min(issued, STAGES) stages.  The leader
-        // can observe both CTAs' A/B bytes; every CTA observes its own scale atoms.
+      {
+        // Copies issued but possibly not landed: the last min(issued, STAGES) stages.  Drained
+        // whether this loop finished or gave up, since another role may still give up after it
+        // finished, and the CTA must not exit with a copy landing in its shared memory.  The
+        // waits replay the (stage, parity) pairs the consumers wait on, and no later phase can
+        // complete once nothing more is issued; on the normal path they are met before the last
+        // tile's epilogue starts.  The leader can observe both CTAs' A/B bytes; every CTA
+        // observes its own scale atoms.
         int s = stage;
         uint32_t ph = phase;
         for (int i = 0; i < C::STAGES && i < issued; ++i) {

@@ -313,3 +313,179 @@ def test_a_pair_whose_leader_counts_only_its_own_bytes_races():
 
 def test_a_pair_whose_scale_barrier_counts_one_cta_races():
     assert _fails(S=3, KT=3, ST=0, tiles=2, sf_bufs=2, sf_split=1, acc_mode="overlap256", cg=2, sf_count=QUADS)
+
+
+def play_abort(S, KT, ST, tiles, seed, abort_at, drain):
+    """One CTA's pipeline in which a wait gives up at step `abort_at` (the kernel's timeout): the
+    flag is raised, every role's pending wait returns false unless its barrier is ready, and each
+    role leaves; the producer drains its last min(issued, S) stages by the rule `drain`
+    ("always": after its loop, however it ended; "own_failure": only when its own wait gave up;
+    "flag_at_finish": only when the flag is up as its loop ends), and the MMA thread waits for all
+    it issued.  Returns what is still in flight into the CTA's memory when every role has left."""
+    rng = random.Random(seed)
+    ktiles = KT + ST
+    units = 2
+    full, sfl, empty = ([Bar() for _ in range(S)] for _ in range(3))
+    sf_full = [Bar(QUADS) for _ in range(units)]
+    sf_empty = [Bar() for _ in range(units)]
+    acc_full, acc_empty = Bar(), Bar(QUADS)
+    copies, commits = [], []
+    flag = [False]
+
+    def until(cond):                          # the kernel's wait: ready, or give up once flagged
+        return lambda: cond() or flag[0]
+
+    def producer():
+        stage, phase, issued, bits, last_fp4 = 0, 0, 0, 0, 0
+        ok = True
+        for t in range(tiles):
+            for kt in range(ktiles):
+                s, ph = stage, phase
+                ready = lambda: empty[s].ok(ph ^ 1)
+                yield until(ready)
+                if not ready():
+                    ok = False
+                    break
+                fp4 = kt < KT
+                last_fp4 = (last_fp4 & ~(1 << s)) | (int(fp4) << s)
+                if fp4:
+                    bits ^= 1 << s
+                    sfl[s].arrive(copies=2)
+                    copies.extend([("sf", s)] * 2)
+                full[s].arrive(copies=2)
+                copies.extend([("ab", s)] * 2)
+                issued += 1
+                stage += 1
+                if stage == S:
+                    stage, phase = 0, phase ^ 1
+            if not ok:
+                break
+        if drain == "always" or (drain == "own_failure" and not ok) or (drain == "flag_at_finish" and flag[0]):
+            s, ph = stage, phase
+            for _ in range(min(S, issued)):
+                s -= 1
+                if s < 0:
+                    s, ph = S - 1, ph ^ 1
+                yield (lambda s=s, ph=ph: full[s].ok(ph))
+                if (last_fp4 >> s) & 1:
+                    yield (lambda s=s, par=((bits >> s) & 1) ^ 1: sfl[s].ok(par))
+
+    def mma():
+        stage, phase, acc_phase, unit = 0, 0, 0, 0
+        ok = True
+        for _ in range(tiles):
+            ap = acc_phase
+            ready = lambda: acc_empty.ok(ap ^ 1)
+            yield until(ready)
+            if not ready():
+                break
+            for kt in range(ktiles):
+                s, ph = stage, phase
+                ready = lambda: full[s].ok(ph)
+                yield until(ready)
+                if not ready():
+                    ok = False
+                    break
+                if kt < KT:
+                    u, up = unit % units, (unit // units) & 1
+                    ready = lambda: sf_full[u].ok(up)
+                    yield until(ready)
+                    if not ready():
+                        ok = False
+                        break
+                    commits.append(sf_empty[u])
+                    unit += 1
+                commits.append(empty[s])
+                stage += 1
+                if stage == S:
+                    stage, phase = 0, phase ^ 1
+            if not ok:
+                break
+            commits.append(acc_full)
+            acc_phase ^= 1
+        done = Bar()                          # the drain commit: all MMAs issued so far are done
+        commits.append(done)
+        yield lambda: done.done > 0
+
+    def scale_warp():
+        stage, unit, bits = 0, 0, 0
+        for _ in range(tiles):
+            for kt in range(ktiles):
+                s = stage
+                if kt < KT:
+                    par = (bits >> s) & 1
+                    ready = lambda: sfl[s].ok(par)
+                    yield until(ready)
+                    if not ready():
+                        return
+                    bits ^= 1 << s
+                    u, up = unit % units, ((unit // units) & 1) ^ 1
+                    ready = lambda: sf_empty[u].ok(up)
+                    yield until(ready)
+                    if not ready():
+                        return
+                    sf_full[u].arrive()
+                    unit += 1
+                stage = (stage + 1) % S
+
+    def epilogue():
+        acc_phase = 0
+        for _ in range(tiles):
+            ap = acc_phase
+            ready = lambda: acc_full.ok(ap)
+            yield until(ready)
+            if not ready():
+                return
+            acc_empty.arrive()
+            acc_phase ^= 1
+
+    roles = [producer(), mma()] + [scale_warp() for _ in range(QUADS)] + [epilogue() for _ in range(QUADS)]
+    waits = [None] * len(roles)
+    alive = [True] * len(roles)
+    for step in range(1, 1000000):
+        for r, role in enumerate(roles):
+            if alive[r] and waits[r] is None:
+                try:
+                    waits[r] = next(role)
+                except StopIteration:
+                    alive[r] = False
+        if not any(alive):
+            break
+        if step == abort_at:
+            flag[0] = True
+        choices = [r for r in range(len(roles)) if alive[r] and waits[r]()]
+        if copies:
+            choices.append("copy")
+        if commits:
+            choices.append("commit")
+        assert choices, "deadlock"
+        pick = rng.choice(choices)
+        if pick == "copy":
+            kind, s = copies.pop(rng.randrange(len(copies)))
+            (sfl if kind == "sf" else full)[s].land()
+        elif pick == "commit":
+            commits.pop(0).arrive()
+        else:
+            waits[pick] = None
+    return len(copies), len(commits)
+
+
+def _abort_cases(n):
+    rng = random.Random(2024)
+    for seed in range(n):
+        KT, ST = rng.choice([(2, 1), (4, 0), (1, 3), (3, 3), (5, 2)])
+        yield rng.choice([3, 4, 5]), KT, ST, rng.choice([1, 2, 3]), seed, rng.randrange(1, 90)
+
+
+def test_after_a_timeout_nothing_is_in_flight_when_the_cta_exits():
+    """Both kernels' producers drain after their loop however it ended, so a CTA that gave up
+    exits with no copy landing in its shared memory and no MMA running, wherever the timeout
+    fell (also after the producer had issued everything, or before anything was issued)."""
+    for S, KT, ST, tiles, seed, abort_at in _abort_cases(1500):
+        assert play_abort(S, KT, ST, tiles, seed, abort_at, "always") == (0, 0), (S, KT, ST, tiles, seed, abort_at)
+
+
+@pytest.mark.parametrize("drain", ["own_failure", "flag_at_finish"])
+def test_draining_only_on_the_producers_own_failure_can_leave_copies_in_flight(drain):
+    """The narrower rules miss a timeout that falls after the producer's loop has ended."""
+    assert any(play_abort(*case, drain)[0] for case in _abort_cases(1500))
