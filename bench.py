@@ -1067,8 +1067,10 @@ def main():
                      "frac": gemm_tflops / fp4_peak, "traffic": GEMM_DRAM_BYTES_PER_STEP[fkey],
                      "traffic_unit": f"DRAM bytes per step (the {len(gemm_names)} GEMM launches; ncu "
                                      "dram__bytes_read.sum + dram__bytes_write.sum per shape; the "
-                                     "kernel's only later change, a skip of small experts in the "
-                                     "grouped tile map, does not touch dense problems)",
+                                     "kernel's later changes move no bytes on this path: a skip of "
+                                     "small experts in the grouped tile map, which dense problems "
+                                     "never take, and the producer's drain of its copies in flight "
+                                     "at loop end, which only waits on barriers)",
                      "algorithmic_bytes": gemm_alg_bytes(p, layer.fused),
                      "kernel": f"splice_gemm_tc_kernel ({len(gemm_names)} launches: {', '.join(gemm_names)}; "
                                "sum 2MNK / sum of CUDA-event times)",
