@@ -24,9 +24,9 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg may import this package.  It shares no code with the CUDA library and never
 imports it.  Every function is pinned by ``-m "not gpu"`` tests to facts the
 paper fixes (value sets, worked examples, closed forms, bounds, brute force);
-the two readings that no page fact can pin are marked "parity unpinned" where
-they live: the MoE routing synthesis (a workload choice, not a result) and the
-absolute accumulation error of the tensor cores (covered only by the stated
-tolerance).
+the one reading that no page fact can pin is marked "parity unpinned" where it
+lives: the absolute accumulation error of the tensor cores (covered only by the
+stated tolerance).  The MoE routing synthesis is an input drawn by ``synth``,
+not a result, and is pinned there to the law of its reading.
 """
 from . import nvfp4, splice, stats, seqfilter, bounds, train  # noqa: F401

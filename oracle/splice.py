@@ -119,7 +119,10 @@ def splice_gemm(xq, wq, alpha, rows=None):
     ``xq`` and ``wq`` are the dicts returned above.  The NVFP4 part runs over all K
     lanes (protected lanes hold code 0).  ``rows`` optionally restricts the output to a
     subset of M rows.  Returns (Y float64 [m,N], absolute-product sums float64 [m,N]),
-    the latter being sum_k |x_hat_k w_hat_k| for the parity tolerance.
+    the latter being sum_k |x_hat_k w_hat_k| for the parity tolerance.  Y itself is
+    pinned; the tensor cores' own accumulation error against it is parity unpinned
+    (the pages fix no accumulation order or width, so only the stated tolerance,
+    1e-5 of this sum, covers it).
     """
     xc, xsf, xs = xq["codes"], xq["sf"], xq["xs"]
     if rows is not None:
