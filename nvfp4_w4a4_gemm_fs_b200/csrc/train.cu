@@ -18,9 +18,9 @@ namespace {
 constexpr int kTile = 64;
 
 // dst[c][r] = src[r][c] for a 64 x 64 tile per CTA: 16-byte loads along src rows into shared
-// memory, 16-byte stores along dst rows.  Rows of the tile are padded to 66 elements (33 words),
-// so the column reads of the store phase (8 consecutive rows per thread, 8 threads 8 rows apart)
-// fall in distinct banks.
+// memory, 16-byte stores along dst rows.  Rows of the tile are padded to 66 elements (33 words):
+// the load phase's writes are then free of bank conflicts (4-way unpadded) and the store phase's
+// column reads (8 threads 8 rows apart) at most 2-way (8-way unpadded; rows 4 x 8 apart share a bank).
 __global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t* __restrict__ src, int64_t lds, uint16_t* dst,
                                                              int64_t ldd, int64_t R, int64_t C, bool vec) {
   __shared__ uint16_t tile[kTile][kTile + 2];

@@ -254,7 +254,7 @@ def play(S, KT, ST, tiles, sf_bufs, sf_split, acc_mode, seed, cg=1, sfl_global=F
     return bad, finished
 
 
-MIXES = [(1, 0), (2, 1), (5, 0), (4, 4), (1, 4), (3, 2)]     # (FP4 k-tiles, BF16 k-tiles)
+MIXES = [(1, 0), (2, 1), (5, 0), (4, 4), (1, 4), (3, 2), (0, 1), (0, 5)]   # (FP4, BF16 k-tiles); no FP4: the BF16 GEMM
 
 
 @pytest.mark.parametrize("acc_mode", ["overlap256", "plain256", "bn128"])
