@@ -65,6 +65,29 @@ class StatsState:
     def group(self, i: int):
         return self.n[i:i + 1], self.s1[i], self.s2[i], self.amax[i], self.flags[i:i + 1]
 
+    _FIELDS = (("n", torch.int64), ("s1", torch.int64), ("s2", torch.int64), ("amax", torch.int32),
+               ("flags", torch.int32))
+
+    def state_dict(self) -> dict:
+        """A checkpoint of the state as host tensors.  The moments are integer sums, so a state
+        restored with load_state_dict continues bit-exactly where it stopped (row subsampling
+        restarts at row 0 of each call, as it does without a checkpoint)."""
+        d = {name: getattr(self, name).detach().to("cpu", copy=True) for name, _ in self._FIELDS}
+        d["K"], d["nprob"] = self.K, self.nprob
+        return d
+
+    def load_state_dict(self, d: dict) -> None:
+        """Restores a checkpoint taken from a state of the same nprob and K (any device)."""
+        who = "StatsState.load_state_dict"
+        _need(d.get("K") == self.K and d.get("nprob") == self.nprob, who,
+              f"checkpoint of nprob={d.get('nprob')}, K={d.get('K')} for a state of nprob={self.nprob}, K={self.K}")
+        for name, dtype in self._FIELDS:
+            src, dst = d.get(name), getattr(self, name)
+            _need(isinstance(src, torch.Tensor) and src.dtype == dtype and tuple(src.shape) == tuple(dst.shape), who,
+                  f"field {name} must be {dtype} of shape {tuple(dst.shape)}")
+        for name, _ in self._FIELDS:
+            getattr(self, name).copy_(d[name])
+
 
 class Packed:
     """Packed NVFP4 operand: q [R,K/2] u8, sf (tiled) u8, side [R,Pp] bf16."""
