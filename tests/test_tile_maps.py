@@ -102,3 +102,43 @@ def test_overlapping_accumulator_epilogue_writes_every_column_once(i):
     shared = set(range(128, 256))                            # the next tile's accumulator overlaps these
     assert set(range(p1_tcol, p1_tcol + 128)) == shared      # part 1 frees exactly the shared half
     assert base + 256 <= 384                                 # inside the 384 accumulator columns
+
+
+def epilogue_parts(BN, overlap, i):
+    """The epilogue's (TMEM column, output column, width) parts for tile i, as the kernel forms
+    them, and the TMEM column the MMAs of tile i start at."""
+    base = (i & 1) * 128 if overlap else 0
+    d = base
+    p1_tcol = 128 if BN == 256 else base
+    p1_ocol = 128 - base if BN == 256 else 0
+    p2_tcol = 0 if base == 0 else 256
+    p2_ocol = 0 if base == 0 else 128
+    parts = [(p1_tcol, p1_ocol, 128)]
+    if BN == 256:
+        parts.append((p2_tcol, p2_ocol, 128))
+    return d, parts
+
+
+@pytest.mark.parametrize("BN,overlap", [(256, True), (256, False), (128, True)])
+def test_epilogue_reads_each_output_column_from_its_accumulator_column(BN, overlap):
+    """The MMAs of tile i write output column c at TMEM column d + c; the epilogue's parts must
+    read exactly those, once each.  With overlapping accumulators (BN = 256) part 1 is the 128
+    columns the next tile also writes, so it must be the columns the two tiles share; a part read
+    after the release must lie outside the next tile's columns."""
+    for i in range(4):
+        d, parts = epilogue_parts(BN, overlap, i)
+        seen = []
+        for tcol, ocol, w in parts:
+            for c in range(w):
+                assert tcol + c == d + ocol + c
+                seen.append(ocol + c)
+        assert sorted(seen) == list(range(BN))
+        assert d + BN <= (384 if (BN == 256 and overlap) else 256)      # inside the accumulator span
+        if BN == 256 and overlap:
+            d_next = epilogue_parts(BN, overlap, i + 1)[0]
+            nxt = set(range(d_next, d_next + BN))
+            assert set(range(parts[0][0], parts[0][0] + 128)) == set(range(d, d + BN)) & nxt
+            assert not set(range(parts[1][0], parts[1][0] + 128)) & nxt
+        if BN == 128:
+            d_next = epilogue_parts(BN, overlap, i + 1)[0]
+            assert not set(range(d, d + BN)) & set(range(d_next, d_next + BN))   # two disjoint buffers
