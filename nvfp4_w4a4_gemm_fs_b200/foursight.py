@@ -158,8 +158,25 @@ def _check_gemm_operands(who: str, plan: "Plan", xq: Packed, wq: Packed, alpha, 
     _check_floats(who, "alpha", alpha, n_alpha)
 
 
+def _check_matrix(who: str, name: str, t: torch.Tensor, rows: int, cols: int, dtypes) -> None:
+    """t is a 2-D tensor of one of `dtypes` with at least rows x cols and unit column stride (its
+    row pitch is passed to the library, which checks it against the width)."""
+    _need(t.dim() == 2 and t.dtype in dtypes and t.shape[0] >= rows and t.shape[1] >= cols
+          and (t.shape[1] <= 1 or t.stride(1) == 1), who,
+          f"{name} must be {'/'.join(str(d) for d in dtypes)} [>= {rows}, >= {cols}] with unit column stride")
+
+
+def _check_vector(who: str, name: str, t, n: int, dtype) -> None:
+    if t is not None:
+        _need(t.dtype == dtype and t.is_contiguous() and t.numel() >= n, who, f"{name} must hold {n} {dtype} values")
+
+
 def fs_channel_stats(X: torch.Tensor, state: StatsState, group: int = 0, row_stride: int = 1, stream=None):
     lib = _lib.load()
+    who = "fs_channel_stats"
+    _need(0 <= group < state.nprob, who, f"group {group} outside the state's {state.nprob}")
+    _need(X.dim() == 2 and X.shape[1] == state.K, who, f"X must be [M, K = {state.K}] (the state's K)")
+    _check_matrix(who, "X", X, X.shape[0], state.K, (torch.bfloat16, torch.float32))
     n, s1, s2, amax, flags = state.group(group)
     M, K = X.shape
     check(lib.fs_channel_stats(_ptr(X), _dtype_code(X), M, K, X.stride(0), row_stride, _ptr(n), _ptr(s1),
@@ -178,6 +195,13 @@ def fs_select_topk(state: StatsState, p: int, opts: int = 0, reset: bool = False
     P = torch.empty(nprob, max(p, 1), dtype=torch.int32, device=dev)[:, :p] if P is None else P
     mask = torch.empty(nprob, (K + 31) // 32, dtype=torch.int32, device=dev) if mask is None else mask
     gA = torch.empty(nprob, dtype=torch.float32, device=dev) if gA is None else gA
+    who, nw = "fs_select_topk", (K + 31) // 32
+    if p > 0:
+        _check_matrix(who, "P", P, nprob, p, (torch.int32,))
+        _need(nprob <= 1 or P.stride(0) == p, who, f"P rows must be p = {p} apart")
+    _check_matrix(who, "mask", mask, nprob, nw, (torch.int32,))
+    _need(mask.shape[1] == nw and (nprob <= 1 or mask.stride(0) == nw), who, f"mask rows must be {nw} words")
+    _check_vector(who, "gA", gA, nprob, torch.float32)
     check(lib.fs_select_topk(nprob, K, _ptr(state.n), _ptr(state.s1), _ptr(state.s2), _ptr(state.amax),
                              _ptr(state.flags), p, opts, _ptr(P), _ptr(mask), _ptr(gA), int(reset),
                              stream_handle(stream)), "fs_select_topk")
@@ -393,6 +417,11 @@ def fs_seq_filter(logp: torch.Tensor, log_tau: float, K1: int, K2: int, lengths=
                   adv=None, stream=None):
     lib = _lib.load()
     S, T = logp.shape
+    who = "fs_seq_filter"
+    _check_matrix(who, "logp", logp, S, T, (torch.float32,))
+    _check_vector(who, "lengths", lengths, S, torch.int32)
+    _check_vector(who, "rewards", rewards, S, torch.float32)
+    _check_vector(who, "adv", adv, S, torch.float32)
     dev = logp.device
     keep = torch.empty(max(S, 1), dtype=torch.uint8, device=dev)[:S]
     cnt = torch.empty(max(S, 1), dtype=torch.int32, device=dev)[:S]
@@ -418,9 +447,15 @@ def fs_gemm_bf16(plan: Plan, A: torch.Tensor, B: torch.Tensor, alpha: torch.Tens
     lib = _lib.load()
     M, K = A.shape
     N = B.shape[0]
+    dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
     if Y is None:
-        dt = torch.bfloat16 if plan.opts & _lib.FS_OUT_BF16 else torch.float32
         Y = torch.empty(M, N, dtype=dt, device=A.device)
+    who = "fs_gemm_bf16"
+    _check_matrix(who, "A", A, M, K, (torch.bfloat16,))
+    _need(B.dim() == 2 and B.shape[1] == K, who, f"B must be [N, K = {K}]")
+    _check_matrix(who, "B", B, N, K, (torch.bfloat16,))
+    _check_matrix(who, "Y", Y, M, N, (dt,))
+    _check_vector(who, "alpha", alpha, 1, torch.float32)
     check(lib.fs_gemm_bf16(plan.handle, M, N, K, _ptr(_bits16(A)), A.stride(0), _ptr(_bits16(B)), B.stride(0),
                            _ptr(alpha), _ptr(Y), Y.stride(0), stream_handle(stream)), "fs_gemm_bf16")
     return Y
@@ -430,6 +465,8 @@ def fs_transpose_bf16(src: torch.Tensor, dst: torch.Tensor | None = None, stream
     lib = _lib.load()
     R, C_ = src.shape
     dst = torch.empty(C_, R, dtype=torch.bfloat16, device=src.device) if dst is None else dst
+    _check_matrix("fs_transpose_bf16", "src", src, R, C_, (torch.bfloat16,))
+    _check_matrix("fs_transpose_bf16", "dst", dst, C_, R, (torch.bfloat16,))
     check(lib.fs_transpose_bf16(R, C_, _ptr(_bits16(src)), src.stride(0), _ptr(dst), dst.stride(0),
                                 stream_handle(stream)), "fs_transpose_bf16")
     return dst
@@ -446,6 +483,14 @@ def fs_ste_backward(plan: Plan, dY: torch.Tensor, X: torch.Tensor, W: torch.Tens
     work = torch.empty(nbytes, dtype=torch.uint8, device=dY.device) if work is None else work
     dX = torch.empty(M, K, dtype=dt, device=dY.device) if dX is None else dX
     dW = torch.empty(N, K, dtype=dt, device=dY.device) if dW is None else dW
+    who = "fs_ste_backward"
+    _check_matrix(who, "dY", dY, M, N, (torch.bfloat16,))
+    _check_matrix(who, "X", X, M, K, (torch.bfloat16,))
+    _need(W.dim() == 2 and W.shape[1] == K, who, f"W must be [N, K = {K}]")
+    _check_matrix(who, "W", W, N, K, (torch.bfloat16,))
+    _check_matrix(who, "dX", dX, M, K, (dt,))
+    _check_matrix(who, "dW", dW, N, K, (dt,))
+    _check_vector(who, "work", work, nbytes, torch.uint8)
     check(lib.fs_ste_backward(plan.handle, M, N, K, _ptr(_bits16(dY)), dY.stride(0), _ptr(_bits16(X)), X.stride(0),
                               _ptr(_bits16(W)), W.stride(0), _ptr(work), work.numel(), _ptr(dX), dX.stride(0),
                               _ptr(dW), dW.stride(0), stream_handle(stream)), "fs_ste_backward")
@@ -457,6 +502,12 @@ def fs_grpo_objective(logp: torch.Tensor, logp_old: torch.Tensor, adv: torch.Ten
     """Eq. 4 with filtered advantages: returns (J [1], seq_obj [S], grad [S, T] or None)."""
     lib = _lib.load()
     S, T = logp.shape
+    who = "fs_grpo_objective"
+    _check_matrix(who, "logp", logp, S, T, (torch.float32,))
+    _check_matrix(who, "logp_old", logp_old, S, T, (torch.float32,))
+    _need(S <= 1 or logp_old.stride(0) == logp.stride(0), who, "logp and logp_old must share their row pitch")
+    _check_vector(who, "adv", adv, S, torch.float32)
+    _check_vector(who, "lengths", lengths, S, torch.int32)
     seq = torch.empty(max(S, 1), dtype=torch.float32, device=logp.device)[:S]
     J = torch.empty(1, dtype=torch.float32, device=logp.device)
     grad = torch.empty(S, T, dtype=torch.float32, device=logp.device) if with_grad else None
@@ -470,6 +521,11 @@ def fs_k3_kl(logp_train: torch.Tensor, logp_roll: torch.Tensor, lengths=None, st
     """K3 estimates of KL(pi_rollout || pi_train): (per-sequence means [S], batch mean [1])."""
     lib = _lib.load()
     S, T = logp_train.shape
+    who = "fs_k3_kl"
+    _check_matrix(who, "logp_train", logp_train, S, T, (torch.float32,))
+    _check_matrix(who, "logp_roll", logp_roll, S, T, (torch.float32,))
+    _need(S <= 1 or logp_roll.stride(0) == logp_train.stride(0), who, "both log-prob arrays must share their row pitch")
+    _check_vector(who, "lengths", lengths, S, torch.int32)
     seq = torch.empty(max(S, 1), dtype=torch.float32, device=logp_train.device)[:S]
     batch = torch.empty(1, dtype=torch.float32, device=logp_train.device)
     work = torch.empty(max(lib.fs_k3_work_bytes(S), 8), dtype=torch.uint8, device=logp_train.device)

@@ -14,7 +14,7 @@ import nvfp4_w4a4_gemm_fs_b200 as F
 from nvfp4_w4a4_gemm_fs_b200 import _lib
 
 HOST_ONLY = {"fs_sf_bytes", "fs_side_cols", "fs_grouped_rows", "fs_compact_cols", "fs_status_string",
-             "fs_last_error", "fs_version"}
+             "fs_last_error", "fs_version", "fs_ste_backward_work_bytes", "fs_k3_work_bytes"}
 
 
 @pytest.fixture
@@ -150,3 +150,59 @@ def test_grouped_buffers_are_checked(no_launch):
         F.fs_splice_gemm_grouped(plan, offs, total, xq, wq, alpha[:2])
     with pytest.raises(ValueError):
         F.fs_splice_gemm_grouped(plan, offs.to(torch.int32), total, xq, wq, alpha)
+
+
+def _refused(calls, fn):
+    n = len(calls)
+    with pytest.raises(F.ArgumentError):
+        fn()
+    assert calls[n:] == [], calls[n:]                                       # nothing reached the library
+
+
+def test_statistics_selection_and_filter_buffers_are_checked(no_launch):
+    K = 256
+    st = F.StatsState(2, K, device="cpu")
+    X = torch.zeros(10, K, dtype=torch.bfloat16)
+    F.fs_channel_stats(X, st, group=1)
+    F.fs_channel_stats(X[:0], st)                                           # an empty batch
+    F.fs_select_topk(st, 16)
+    F.fs_select_topk(st, 0)
+    P = torch.empty(2, 16, dtype=torch.int32)
+    F.fs_select_topk(st, 16, P=P, mask=torch.empty(2, K // 32, dtype=torch.int32), gA=torch.empty(2))
+    _refused(no_launch, lambda: F.fs_channel_stats(torch.zeros(10, 2 * K, dtype=torch.bfloat16), st))   # wider than K
+    _refused(no_launch, lambda: F.fs_channel_stats(X, st, group=2))                                 # no such group
+    _refused(no_launch, lambda: F.fs_channel_stats(torch.zeros(K, 10, dtype=torch.bfloat16).t(), st))   # strided columns
+    _refused(no_launch, lambda: F.fs_select_topk(st, 16, P=torch.empty(1, 16, dtype=torch.int32)))      # one row for two
+    _refused(no_launch, lambda: F.fs_select_topk(st, 16, P=torch.empty(2, 32, dtype=torch.int32)[:, :16]))  # pitch
+    _refused(no_launch, lambda: F.fs_select_topk(st, 16, mask=torch.empty(2, 4, dtype=torch.int32)))    # short mask
+    _refused(no_launch, lambda: F.fs_select_topk(st, 16, gA=torch.empty(1)))
+    S, T = 8, 64
+    lp = torch.zeros(S, T)
+    F.fs_seq_filter(lp, -9.0, 9, 5, lengths=torch.full((S,), T, dtype=torch.int32), G=4, rewards=torch.zeros(S))
+    _refused(no_launch, lambda: F.fs_seq_filter(lp.double(), -9.0, 9, 5))
+    _refused(no_launch, lambda: F.fs_seq_filter(lp, -9.0, 9, 5, lengths=torch.full((S,), T)))         # int64 lengths
+    _refused(no_launch, lambda: F.fs_seq_filter(lp, -9.0, 9, 5, G=4, rewards=torch.zeros(S - 1)))
+    _refused(no_launch, lambda: F.fs_seq_filter(lp, -9.0, 9, 5, adv=torch.zeros(S, dtype=torch.float64)))
+
+
+def test_training_side_buffers_are_checked(no_launch):
+    M, N, K = 64, 32, 48
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    plan = F.Plan(256, 256, 1)
+    F.fs_gemm_bf16(plan, bf(M, K), bf(N, K), Y=torch.empty(M, N))
+    F.fs_transpose_bf16(bf(M, K))
+    F.fs_ste_backward(plan, bf(M, N), bf(M, K), bf(N, K))
+    S, T = 4, 16
+    lp, lo = torch.zeros(S, T), torch.zeros(S, T)
+    F.fs_grpo_objective(lp, lo, torch.zeros(S), 0.2, lengths=torch.full((S,), T, dtype=torch.int32))
+    F.fs_k3_kl(lp, lo)
+    _refused(no_launch, lambda: F.fs_gemm_bf16(plan, bf(M, K), bf(N, K + 16)))                     # K differs
+    _refused(no_launch, lambda: F.fs_gemm_bf16(plan, bf(M, K), bf(N, K), Y=torch.empty(M, N - 1)))
+    _refused(no_launch, lambda: F.fs_gemm_bf16(plan, bf(M, K), bf(N, K), Y=bf(M, N)))              # dtype of the plan
+    _refused(no_launch, lambda: F.fs_transpose_bf16(bf(M, K), dst=bf(K, M - 1)))
+    _refused(no_launch, lambda: F.fs_ste_backward(plan, bf(M, N), bf(M - 1, K), bf(N, K)))
+    _refused(no_launch, lambda: F.fs_ste_backward(plan, bf(M, N), bf(M, K), bf(N, K), work=torch.empty(8, dtype=torch.uint8)))
+    _refused(no_launch, lambda: F.fs_ste_backward(plan, bf(M, N), bf(M, K), bf(N, K), dW=torch.empty(N, K - 1)))
+    _refused(no_launch, lambda: F.fs_grpo_objective(lp, torch.zeros(S, 2 * T)[:, :T], torch.zeros(S), 0.2))   # pitch
+    _refused(no_launch, lambda: F.fs_grpo_objective(lp, lo, torch.zeros(S - 1), 0.2))
+    _refused(no_launch, lambda: F.fs_k3_kl(lp, torch.zeros(S - 1, T)))
