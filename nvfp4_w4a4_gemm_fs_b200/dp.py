@@ -56,9 +56,34 @@ def _broadcast_bytes(t: torch.Tensor, src: int, group) -> None:
         t.copy_(tmp)
 
 
+_MAX_PARTS = 8
+
+
+def _agree_on_sizes(tensors, src: int, group) -> None:
+    """Every rank compares its tensor count and byte counts with rank ``src``'s before any data
+    moves, and all ranks learn the outcome together (a broadcast of ``src``'s fixed-size header,
+    then a MAX all-reduce of the mismatch flag), so a wrong receiver buffer raises on every rank
+    instead of leaving ranks in broadcasts of different sizes."""
+    if len(tensors) > _MAX_PARTS:
+        raise ValueError(f"broadcast_packed: at most {_MAX_PARTS} tensors")
+    dev = tensors[0].device
+    head = [len(tensors)] + [t.numel() * t.element_size() for t in tensors]
+    mine = torch.tensor(head + [0] * (_MAX_PARTS + 1 - len(head)), dtype=torch.int64, device=dev)
+    ref = mine.clone()
+    dist.broadcast(ref, src=src, group=group)
+    bad = torch.tensor([0 if torch.equal(ref, mine) else 1], dtype=torch.int64, device=dev)
+    dist.all_reduce(bad, op=dist.ReduceOp.MAX, group=group)
+    if int(bad.item()):
+        raise ValueError(f"broadcast_packed: buffer sizes differ between ranks (rank {dist.get_rank(group)}: "
+                         f"{mine.tolist()}, rank {src}: {ref.tolist()})")
+
+
 def broadcast_packed(packed, gW=None, alpha=None, src: int = 0, group=None) -> None:
     """Send rank ``src``'s packed weights (q, sf, side) and, when given, its gW and alpha to every
     rank of ``group`` in place.  Receivers must hold buffers of the same shapes (alloc_packed with the
-    same N, K, p); their contents are overwritten byte for byte."""
-    for t in packed_tensors(packed, gW, alpha):
+    same N, K, p); their contents are overwritten byte for byte.  The sizes are compared first on
+    every rank; a mismatch raises ValueError on all ranks and nothing is sent."""
+    tensors = packed_tensors(packed, gW, alpha)
+    _agree_on_sizes(tensors, src, group)
+    for t in tensors:
         _broadcast_bytes(t, src, group)

@@ -157,3 +157,37 @@ def test_packed_weight_broadcast_without_requantisation(tmp_path):
         assert np.array_equal(d["side"].view(np.uint16), nvfp4.bf16_bits(ref["ws"]))
         assert d["gW"][0] == ref["gW"] and d["alpha"][0] == ref["alpha"]
         assert np.array_equal(d["Y"], Yfull[r::world])           # rank r's rows of the full batch
+
+
+def _mismatch_worker(rank, world, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    from datetime import timedelta
+
+    from nvfp4_w4a4_gemm_fs_b200 import dp
+    from nvfp4_w4a4_gemm_fs_b200 import foursight as Fs
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    pp = 64 if rank == 0 else 16                                   # rank 1 holds side columns of another p
+    packed = Fs.Packed(torch.zeros(N_W, K // 2, dtype=torch.uint8), torch.zeros(1024, dtype=torch.uint8),
+                       torch.zeros(N_W, pp, dtype=torch.bfloat16), N_W, K, pp)
+    try:
+        dp.broadcast_packed(packed, torch.zeros(1), torch.zeros(1), src=0)
+        outcome = "sent"
+    except ValueError:
+        outcome = "refused"
+    with open(os.path.join(out_dir, f"mm{rank}.txt"), "w") as f:
+        f.write(outcome)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_packed_weight_broadcast_refuses_mismatched_buffers_on_every_rank(tmp_path):
+    """A receiver whose buffers differ in size from the sender's makes every rank raise before any
+    weight bytes move (no rank is left in a broadcast of another size)."""
+    world = 2
+    mp.spawn(_mismatch_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    for r in range(world):
+        assert open(os.path.join(tmp_path, f"mm{r}.txt")).read() == "refused"
